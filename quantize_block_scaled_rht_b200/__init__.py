@@ -1,0 +1,228 @@
+"""quantize_block_scaled_rht_b200 -- MXFP4 quantization and block-scaled GEMMs on B200.
+
+A thin Python binding over the C ABI of libmxfp4.so (include/mxfp4.h): every
+function here only marshals arguments (torch tensors -> device pointers, the
+current CUDA stream) and calls the library; all arithmetic runs in the CUDA
+kernels.  PyTorch provides device memory and streams.  There is no CPU
+fallback: without the built library or a CUDA device these calls raise.
+
+The method is the one on "MXFP4" (aiwiki.ai) -- "Format specification",
+"Conversion rules", "Training with MXFP4" -- as used by the ALTO recipe
+("Training an MoE LLM in MXFP4", abstract): 1D blocks for activations and
+gradients, 2D 32x32 blocks for weights, randomized Hadamard transform and
+stochastic rounding.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmxfp4.so")
+
+# enums (include/mxfp4.h)
+MXFP4_OK = 0
+MXFP4_ERR_INVALID_ARG = 1
+MXFP4_ERR_ALIGNMENT = 2
+MXFP4_ERR_UNSUPPORTED = 3
+MXFP4_ERR_CUDA = 4
+MXFP4_ERR_TIMEOUT = 5
+LAYOUT_1D_ROW, LAYOUT_1D_COL, LAYOUT_2D = 0, 1, 2
+ROUND_RNE, ROUND_SR = 0, 1
+SCALES_ROWMAJOR, SCALES_MMA = 0, 1
+OUT_BF16, OUT_F32 = 0, 1
+
+ABI_FUNCTIONS = (
+    "mxfp4_status_string", "mxfp4_version", "mxfp4_mma_scales_bytes", "mxfp4_mma_scale_offset",
+    "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_grouped_gemm", "mxfp4_get_error",
+    "mxfp4_set_wait_limit_ns", "mxfp4_wait_probe",
+)
+
+
+class MXFP4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmxfp4.so from the package directory (built by build.py)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libmxfp4.so not built: run `python -m quantize_block_scaled_rht_b200.build` ({LIB_PATH})")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, u64, i32, vp = ctypes.c_int64, ctypes.c_uint64, ctypes.c_int, ctypes.c_void_p
+        L.mxfp4_status_string.argtypes = [i32]
+        L.mxfp4_status_string.restype = ctypes.c_char_p
+        L.mxfp4_version.restype = i32
+        L.mxfp4_mma_scales_bytes.argtypes = [i64, i64]
+        L.mxfp4_mma_scales_bytes.restype = i64
+        L.mxfp4_mma_scale_offset.argtypes = [i64, i64, i64]
+        L.mxfp4_mma_scale_offset.restype = i64
+        L.mxfp4_quantize.argtypes = [vp, i64, i64, i64, i32, i32, i32, u64, u64, vp, i64, vp, i64, i32,
+                                     vp, i64, vp, i64, vp]
+        L.mxfp4_quantize.restype = i32
+        L.mxfp4_dequantize.argtypes = [vp, i64, vp, i64, i32, i64, i64, i32, i32, u64, vp, i64, i32, vp]
+        L.mxfp4_dequantize.restype = i32
+        L.mxfp4_gemm.argtypes = [vp, i64, vp, vp, i64, vp, i64, i64, i64, vp, i64, vp]
+        L.mxfp4_gemm.restype = i32
+        L.mxfp4_grouped_gemm.argtypes = [vp, i64, vp, i64, vp, vp, i32, vp, i64, vp, i64, i64, vp, i64, vp]
+        L.mxfp4_grouped_gemm.restype = i32
+        L.mxfp4_get_error.argtypes = [vp]
+        L.mxfp4_get_error.restype = i32
+        L.mxfp4_set_wait_limit_ns.argtypes = [u64]
+        L.mxfp4_set_wait_limit_ns.restype = u64
+        L.mxfp4_wait_probe.argtypes = [i32, vp]
+        L.mxfp4_wait_probe.restype = i32
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().mxfp4_status_string(int(status)).decode()
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != MXFP4_OK:
+        raise MXFP4Error(rc, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmxfp4 takes CUDA tensors (device pointers)")
+    return t.data_ptr()
+
+
+def mma_scales_bytes(rows: int, k: int) -> int:
+    """Bytes of the GEMM-ready scale layout of a (rows x k) operand."""
+    return int(lib().mxfp4_mma_scales_bytes(rows, k))
+
+
+def mma_scale_offset(row: int, kb: int, k: int) -> int:
+    return int(lib().mxfp4_mma_scale_offset(row, kb, k))
+
+
+@dataclass
+class Quantized:
+    """Output of mxfp4_quantize: codes/scales (and the 2D transposed copy)."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    rows: int            # rows of the quantized operand (output view)
+    k: int               # elements per row of the quantized operand
+    layout: int
+    scale_layout: int
+    codes_t: Optional[torch.Tensor] = None
+    scales_t: Optional[torch.Tensor] = None
+
+
+def _scale_tensor(rows, k, scale_layout, device, two_d=False):
+    if scale_layout == SCALES_MMA:
+        return torch.empty(mma_scales_bytes(rows, k), dtype=torch.uint8, device=device)
+    if two_d:
+        return torch.empty((rows // 32, k // 32), dtype=torch.uint8, device=device)
+    return torch.empty((rows, k // 32), dtype=torch.uint8, device=device)
+
+
+def mxfp4_quantize(x: torch.Tensor, layout: int = LAYOUT_1D_ROW, rht_size: int = 0, rounding: int = ROUND_RNE,
+                   seed: int = 0, elem_offset: int = 0, scale_layout: int = SCALES_ROWMAJOR,
+                   transposed_copy: bool = False, stream=None, out: Optional[Quantized] = None) -> Quantized:
+    """Quantize a 2-D bf16 CUDA tensor to MXFP4 (see mxfp4_quantize in include/mxfp4.h)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    if out is None:
+        dev = x.device
+        if layout == LAYOUT_1D_COL:
+            orows, k = cols, rows
+        else:
+            orows, k = rows, cols
+        codes = torch.empty((orows, k // 2), dtype=torch.uint8, device=dev)
+        scales = _scale_tensor(orows, k, scale_layout, dev, two_d=(layout == LAYOUT_2D))
+        codes_t = scales_t = None
+        if transposed_copy:
+            codes_t = torch.empty((cols, rows // 2), dtype=torch.uint8, device=dev)
+            scales_t = _scale_tensor(cols, rows, scale_layout, dev, two_d=True)
+        out = Quantized(codes, scales, orows, k, layout, scale_layout, codes_t, scales_t)
+    ld_sc = out.scales.shape[1] if out.scales.dim() == 2 else 0
+    ld_sct = out.scales_t.shape[1] if (out.scales_t is not None and out.scales_t.dim() == 2) else 0
+    rc = lib().mxfp4_quantize(
+        _ptr(x), rows, cols, x.stride(0), layout, rht_size, rounding, seed & 0xFFFFFFFFFFFFFFFF, elem_offset,
+        _ptr(out.codes), out.codes.stride(0), _ptr(out.scales), ld_sc, scale_layout,
+        _ptr(out.codes_t), out.codes_t.stride(0) if out.codes_t is not None else 0,
+        _ptr(out.scales_t), ld_sct, _stream(stream))
+    _check(rc, "mxfp4_quantize")
+    return out
+
+
+def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, rows: int, cols: int, layout: int = LAYOUT_1D_ROW,
+                     rht_size: int = 0, seed: int = 0, scale_layout: int = SCALES_ROWMAJOR,
+                     out_dtype: torch.dtype = torch.bfloat16, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Decode MXFP4 codes/scales of a [rows, cols] tensor (inverse RHT if rht_size)."""
+    if out is None:
+        out = torch.empty((rows, cols), dtype=out_dtype, device=codes.device)
+    od = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    ld_sc = scales.shape[1] if scales.dim() == 2 else 0
+    rc = lib().mxfp4_dequantize(_ptr(codes), codes.stride(0), _ptr(scales), ld_sc, scale_layout, rows, cols,
+                                layout, rht_size, seed & 0xFFFFFFFFFFFFFFFF, _ptr(out), out.stride(0), od,
+                                _stream(stream))
+    _check(rc, "mxfp4_dequantize")
+    return out
+
+
+def mxfp4_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Tensor,
+               K: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """C[M, N] = A[M, K] B[N, K]^T in FP32; scales in the GEMM-ready (MMA) layout."""
+    M, N = a_codes.shape[0], b_codes.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=a_codes.device)
+    rc = lib().mxfp4_gemm(_ptr(a_codes), a_codes.stride(0), _ptr(a_scales), _ptr(b_codes), b_codes.stride(0),
+                          _ptr(b_scales), M, N, K, _ptr(out), out.stride(0), _stream(stream))
+    _check(rc, "mxfp4_gemm")
+    return out
+
+
+def mxfp4_grouped_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, group_offsets: torch.Tensor,
+                       group_sizes: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Tensor, N: int, K: int,
+                       out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per group g: C[rows of g] = A[rows of g] B_g^T.  b_codes is [G, N, K/2]."""
+    a_rows = a_codes.shape[0]
+    G = group_sizes.numel()
+    if out is None:
+        out = torch.empty((a_rows, N), dtype=torch.float32, device=a_codes.device)
+    rc = lib().mxfp4_grouped_gemm(_ptr(a_codes), a_codes.stride(0), _ptr(a_scales), a_rows, _ptr(group_offsets),
+                                  _ptr(group_sizes), G, _ptr(b_codes), b_codes.stride(-2), _ptr(b_scales), N, K,
+                                  _ptr(out), out.stride(0), _stream(stream))
+    _check(rc, "mxfp4_grouped_gemm")
+    return out
+
+
+def mxfp4_get_error(stream=None) -> int:
+    """Synchronize the stream; return and clear the first device-side error."""
+    return int(lib().mxfp4_get_error(_stream(stream)))
+
+
+def mxfp4_set_wait_limit_ns(limit_ns: int) -> int:
+    return int(lib().mxfp4_set_wait_limit_ns(limit_ns))
+
+
+def mxfp4_wait_probe(arrive: bool, stream=None) -> None:
+    _check(lib().mxfp4_wait_probe(1 if arrive else 0, _stream(stream)), "mxfp4_wait_probe")

@@ -1,0 +1,168 @@
+// api.cu -- the extern "C" boundary of libmxfp4 (declared in include/mxfp4.h):
+// argument validation, then one launch on the caller's stream.  No device
+// memory is allocated here; errors come back as status codes.
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace mxfp4 {
+cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rht,
+                            int rounding, uint64_t seed, uint64_t elem_offset, uint8_t *codes, int64_t ld_codes,
+                            uint8_t *scales, int64_t ld_scales, int scale_layout, uint8_t *codes_t,
+                            int64_t ld_codes_t, uint8_t *scales_t, int64_t ld_scales_t, cudaStream_t s);
+cudaError_t launch_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
+                              int scale_layout, int64_t rows, int64_t cols, int layout, int rht, uint64_t seed,
+                              void *out, int64_t ld_out, int out_dtype, cudaStream_t s);
+int launch_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes, int64_t ldb,
+                const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s);
+int launch_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
+                        const int32_t *offsets, const int32_t *sizes, int G, const uint8_t *b_codes, int64_t ldb,
+                        const uint8_t *b_scales, int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s);
+int get_error(cudaStream_t s);
+int launch_wait_probe(int arrive, cudaStream_t s);
+uint64_t set_wait_limit(uint64_t ns);
+}  // namespace mxfp4
+
+namespace {
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+}  // namespace
+
+extern "C" {
+
+const char *mxfp4_status_string(int status) {
+    switch (status) {
+        case MXFP4_OK: return "MXFP4_OK";
+        case MXFP4_ERR_INVALID_ARG: return "MXFP4_ERR_INVALID_ARG";
+        case MXFP4_ERR_ALIGNMENT: return "MXFP4_ERR_ALIGNMENT";
+        case MXFP4_ERR_UNSUPPORTED: return "MXFP4_ERR_UNSUPPORTED";
+        case MXFP4_ERR_CUDA: return "MXFP4_ERR_CUDA";
+        case MXFP4_ERR_TIMEOUT: return "MXFP4_ERR_TIMEOUT";
+        default: return "MXFP4_ERR_UNKNOWN";
+    }
+}
+
+int mxfp4_version(void) { return 100; }
+
+int64_t mxfp4_mma_scales_bytes(int64_t rows, int64_t k) {
+    if (rows <= 0 || k <= 0) return 0;
+    return ((rows + 127) / 128) * mxfp4::mma_katoms(k) * 512;
+}
+
+int64_t mxfp4_mma_scale_offset(int64_t row, int64_t kb, int64_t k) {
+    return mxfp4::mma_scale_off(row, kb, mxfp4::mma_katoms(k));
+}
+
+int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rht_size, int rounding,
+                   uint64_t seed, uint64_t elem_offset, uint8_t *codes, int64_t ld_codes, uint8_t *scales,
+                   int64_t ld_scales, int scale_layout, uint8_t *codes_t, int64_t ld_codes_t, uint8_t *scales_t,
+                   int64_t ld_scales_t, void *stream) {
+    if (!x || !codes || !scales) return MXFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (layout != MXFP4_LAYOUT_1D_ROW && layout != MXFP4_LAYOUT_1D_COL && layout != MXFP4_LAYOUT_2D)
+        return MXFP4_ERR_INVALID_ARG;
+    if (rht_size != 0 && rht_size != 16 && rht_size != 32) return MXFP4_ERR_INVALID_ARG;
+    if (rounding != MXFP4_ROUND_RNE && rounding != MXFP4_ROUND_SR) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout != MXFP4_SCALES_ROWMAJOR && scale_layout != MXFP4_SCALES_MMA) return MXFP4_ERR_INVALID_ARG;
+    if ((elem_offset & 3u) != 0) return MXFP4_ERR_INVALID_ARG;
+    if (layout == MXFP4_LAYOUT_1D_ROW && (cols % 32)) return MXFP4_ERR_INVALID_ARG;
+    if (layout == MXFP4_LAYOUT_1D_COL && (rows % 32)) return MXFP4_ERR_INVALID_ARG;
+    if (layout == MXFP4_LAYOUT_2D && ((rows % 32) || (cols % 32))) return MXFP4_ERR_INVALID_ARG;
+    if (cols % 8) return MXFP4_ERR_INVALID_ARG;
+    if ((codes_t || scales_t) && layout != MXFP4_LAYOUT_2D) return MXFP4_ERR_INVALID_ARG;
+    if (scales_t && !codes_t) return MXFP4_ERR_INVALID_ARG;
+    const int64_t code_cols = layout == MXFP4_LAYOUT_1D_COL ? rows / 2 : cols / 2;
+    if (ld_x < cols || ld_codes < code_cols) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout == MXFP4_SCALES_ROWMAJOR) {
+        const int64_t sc = layout == MXFP4_LAYOUT_1D_COL ? rows / 32 : cols / 32;
+        if (ld_scales < sc) return MXFP4_ERR_INVALID_ARG;
+        if (scales_t && ld_scales_t < rows / 32) return MXFP4_ERR_INVALID_ARG;
+    }
+    if (codes_t && ld_codes_t < rows / 2) return MXFP4_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || (ld_x % 8) || (ld_codes % 16)) return MXFP4_ERR_ALIGNMENT;
+    if (codes_t && (!aligned16(codes_t) || (ld_codes_t % 16))) return MXFP4_ERR_ALIGNMENT;
+    if (scale_layout == MXFP4_SCALES_MMA && (!aligned16(scales) || (scales_t && !aligned16(scales_t))))
+        return MXFP4_ERR_ALIGNMENT;
+    const cudaError_t e = mxfp4::launch_quantize(x, rows, cols, ld_x, layout, rht_size, rounding, seed, elem_offset,
+                                                 codes, ld_codes, scales, ld_scales, scale_layout, codes_t,
+                                                 ld_codes_t, scales_t, ld_scales_t,
+                                                 static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
+}
+
+int mxfp4_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
+                     int scale_layout, int64_t rows, int64_t cols, int layout, int rht_size, uint64_t seed,
+                     void *out, int64_t ld_out, int out_dtype, void *stream) {
+    if (!codes || !scales || !out) return MXFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (layout != MXFP4_LAYOUT_1D_ROW && layout != MXFP4_LAYOUT_1D_COL && layout != MXFP4_LAYOUT_2D)
+        return MXFP4_ERR_INVALID_ARG;
+    if (rht_size != 0 && rht_size != 16 && rht_size != 32) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout != MXFP4_SCALES_ROWMAJOR && scale_layout != MXFP4_SCALES_MMA) return MXFP4_ERR_INVALID_ARG;
+    if (out_dtype != MXFP4_OUT_BF16 && out_dtype != MXFP4_OUT_F32) return MXFP4_ERR_INVALID_ARG;
+    if (layout == MXFP4_LAYOUT_1D_ROW && (cols % 32)) return MXFP4_ERR_INVALID_ARG;
+    if (layout == MXFP4_LAYOUT_1D_COL && (rows % 32)) return MXFP4_ERR_INVALID_ARG;
+    if (layout == MXFP4_LAYOUT_2D && ((rows % 32) || (cols % 32))) return MXFP4_ERR_INVALID_ARG;
+    if (cols % 8) return MXFP4_ERR_INVALID_ARG;
+    const int64_t code_cols = layout == MXFP4_LAYOUT_1D_COL ? rows / 2 : cols / 2;
+    if (ld_codes < code_cols || ld_out < cols) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout == MXFP4_SCALES_ROWMAJOR) {
+        const int64_t sc = layout == MXFP4_LAYOUT_1D_COL ? rows / 32 : cols / 32;
+        if (ld_scales < sc) return MXFP4_ERR_INVALID_ARG;
+    }
+    if (!aligned16(codes) || !aligned16(out) || (ld_codes % 16) || (ld_out % 8)) return MXFP4_ERR_ALIGNMENT;
+    const cudaError_t e = mxfp4::launch_dequantize(codes, ld_codes, scales, ld_scales, scale_layout, rows, cols,
+                                                   layout, rht_size, seed, out, ld_out, out_dtype,
+                                                   static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
+}
+
+static int check_gemm_common(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                             int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, const float *c,
+                             int64_t ldc) {
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !c) return MXFP4_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (K % 32) return MXFP4_ERR_INVALID_ARG;
+    if (K % 64) return MXFP4_ERR_UNSUPPORTED;
+    if (lda < K / 2 || ldb < K / 2 || ldc < N) return MXFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
+        !aligned16(c) || (lda % 16) || (ldb % 16) || (ldc % 4))
+        return MXFP4_ERR_ALIGNMENT;
+    if (N > (int64_t)1 << 31 || K > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    return MXFP4_OK;
+}
+
+int mxfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes, int64_t ldb,
+               const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, float *c, int64_t ldc, void *stream) {
+    if (M <= 0) return MXFP4_ERR_INVALID_ARG;
+    const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc);
+    if (rc != MXFP4_OK) return rc;
+    if (M > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    return mxfp4::launch_gemm(a_codes, lda, a_scales, b_codes, ldb, b_scales, M, N, K, c, ldc,
+                              static_cast<cudaStream_t>(stream));
+}
+
+int mxfp4_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
+                       const int32_t *group_offsets, const int32_t *group_sizes, int num_groups,
+                       const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, float *c,
+                       int64_t ldc, void *stream) {
+    if (!group_offsets || !group_sizes) return MXFP4_ERR_INVALID_ARG;
+    if (num_groups <= 0 || a_rows <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (num_groups > 1024) return MXFP4_ERR_UNSUPPORTED;
+    const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc);
+    if (rc != MXFP4_OK) return rc;
+    if (a_rows > (int64_t)1 << 31 || (int64_t)num_groups * N > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    return mxfp4::launch_grouped_gemm(a_codes, lda, a_scales, a_rows, group_offsets, group_sizes, num_groups,
+                                      b_codes, ldb, b_scales, N, K, c, ldc, static_cast<cudaStream_t>(stream));
+}
+
+int mxfp4_get_error(void *stream) { return mxfp4::get_error(static_cast<cudaStream_t>(stream)); }
+
+uint64_t mxfp4_set_wait_limit_ns(uint64_t limit_ns) { return mxfp4::set_wait_limit(limit_ns); }
+
+int mxfp4_wait_probe(int arrive, void *stream) {
+    return mxfp4::launch_wait_probe(arrive, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,177 @@
+// common.cuh -- device helpers shared by the MXFP4 kernels (sm_100a).
+//
+// Number format: "MXFP4" (aiwiki.ai), "Format specification" (E2M1 elements,
+// E8M0 scale, blocks of 32) and "Conversion rules" (scale = 2^floor(log2 amax)
+// / 4, round-to-nearest-even with saturation).  Random bits: Philox4x32-10 of
+// Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3" (SC'11).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/mxfp4.h"
+
+namespace mxfp4 {
+
+// ---------------------------------------------------------------------------
+// Host/device layout helpers
+// ---------------------------------------------------------------------------
+
+// K-blocks of one MMA scale atom row group and the atom geometry: 128 rows x
+// 4 K-blocks, 512 bytes, (row % 32) * 16 + ((row % 128) / 32) * 4 + kb % 4.
+__host__ __device__ __forceinline__ int64_t mma_katoms(int64_t k) { return (k / 32 + 3) / 4; }
+
+__host__ __device__ __forceinline__ int64_t mma_scale_off(int64_t row, int64_t kb, int64_t katoms) {
+    return (((row >> 7) * katoms + (kb >> 2)) << 9) + ((row & 31) << 4) + (((row >> 5) & 3) << 2) + (kb & 3);
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (SC'11): 10 rounds of two 32x32->64 multiplies; the high
+// halves are xored with the odd counter words and the key, the key advances
+// by the Weyl constants after every round.
+// ---------------------------------------------------------------------------
+struct U4 { uint32_t x, y, z, w; };
+
+__device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                            uint32_t k0, uint32_t k1) {
+    constexpr uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+    constexpr uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t lo0 = M0 * c0, hi0 = __umulhi(M0, c0);
+        const uint32_t lo1 = M1 * c2, hi1 = __umulhi(M1, c2);
+        const uint32_t n0 = hi1 ^ c1 ^ k0;
+        const uint32_t n2 = hi0 ^ c3 ^ k1;
+        c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+        k0 += W0; k1 += W1;
+    }
+    return U4{c0, c1, c2, c3};
+}
+
+// Sign mask of the RHT diagonal for a seed: word 0 of the block with counter
+// (0, 0, 0, 0x52485400).  Computed on the host too (same function body).
+__host__ __device__ inline uint32_t rht_sign_mask_hd(uint64_t seed) {
+    uint32_t c0 = 0, c1 = 0, c2 = 0, c3 = 0x52485400u;
+    uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+    for (int r = 0; r < 10; ++r) {
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        c1 = (uint32_t)p1; c3 = (uint32_t)p0; c0 = n0; c2 = n2;
+        k0 += 0x9E3779B9u; k1 += 0xBB67AE85u;
+    }
+    return c0;
+}
+
+// ---------------------------------------------------------------------------
+// bf16 <-> fp32
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Two fp32 -> packed bf16x2 (round to nearest even), a in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// amax with NaN propagation (max.NaN returns NaN if either input is NaN)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float amax_nan(float acc, float v) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(acc), "f"(fabsf(v)));
+    return r;
+}
+
+// E8M0 scale code of a block from its amax (NaN or Inf -> 0xFF; 0 -> 0):
+// clamp(floor(log2 amax) - 2 + 127, 0, 254).  For a normal amax the biased
+// exponent field E gives floor(log2 amax) = E - 127, so the code is E - 2;
+// a subnormal amax (E = 0) or E <= 2 clamps to 0.
+__device__ __forceinline__ uint32_t scale_code_from_amax(float amax) {
+    const uint32_t b = __float_as_uint(amax);
+    if (b >= 0x7F800000u) return 0xFFu;
+    const int e = (int)(b >> 23) - 2;
+    return e > 0 ? (uint32_t)e : 0u;
+}
+
+// 2^-(code - 127) as fp32 for code in [0, 252]: biased exponent 254 - code.
+__device__ __forceinline__ float inv_scale_from_code(uint32_t code) {
+    return __uint_as_float((254u - code) << 23);
+}
+
+// 2^(code - 127) as fp32 for code in [0, 254] (code 0 is the subnormal 2^-127).
+__device__ __forceinline__ float scale_from_code(uint32_t code) {
+    return code ? __uint_as_float(code << 23) : __uint_as_float(0x00400000u);
+}
+
+// ---------------------------------------------------------------------------
+// E2M1 encoders
+// ---------------------------------------------------------------------------
+
+// Eight scaled fp32 values -> 8 nibbles (round to nearest even, saturate to
+// +-6), element 0 in bits 3:0.  cvt.rn.satfinite.e2m1x2.f32 d, a, b puts a in
+// the high nibble and b in the low nibble of d.
+__device__ __forceinline__ uint32_t e2m1x8_rn(const float *v) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
+// Stochastic rounding of one scaled value with random word r: lo <= |v| < hi
+// neighbouring grid values, up iff r < ceil(f * 2^32) with
+// f = (|v| - lo) / (hi - lo).  On [1, 6] the grid has one mantissa bit, so the
+// lower 22 mantissa bits are f * 2^22; on [0.5, 1) f is the 23-bit mantissa;
+// below 0.5, f * 2^32 = |v| * 2^33 (exact), rounded up to an integer.
+__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
+    const uint32_t sign = (__float_as_uint(v) >> 28) & 8u;
+    const float a = fminf(fabsf(v), 6.0f);
+    const uint32_t ab = __float_as_uint(a);
+    uint32_t t, lo;
+    if (a >= 1.0f) {
+        t = ab << 10;
+        lo = (ab >> 22) - 252u;            // 1 -> 2, 1.5 -> 3, 2 -> 4, 3 -> 5, 4 -> 6, 6 -> 7
+    } else if (a >= 0.5f) {
+        t = ab << 9;
+        lo = 1u;
+    } else {
+        t = __float2uint_ru(a * 8589934592.0f);  // 2^33
+        lo = 0u;
+    }
+    return sign | (lo + (r < t ? 1u : 0u));
+}
+
+// ---------------------------------------------------------------------------
+// In-register fast Walsh-Hadamard butterfly over D values, stages h = 1..D/2,
+// (a, b) -> (a + b, a - b), each rounded in fp32.
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void fwht(float *v) {
+#pragma unroll
+    for (int h = 1; h < D; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < D; ++i) {
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = __fadd_rn(a, b);
+                v[i + h] = __fsub_rn(a, b);
+            }
+        }
+    }
+}
+
+template <int D>
+__device__ __forceinline__ float rht_norm() {
+    return D == 16 ? 0.25f : __uint_as_float(0x3E3504F3u);  // fp32(1/sqrt(32))
+}
+
+}  // namespace mxfp4

@@ -1,0 +1,609 @@
+// quantize.cu -- MXFP4 quantize / dequantize kernels for sm_100a.
+//
+// "MXFP4" (aiwiki.ai): "Format specification" (E2M1 codes, E8M0 scales,
+// 32-element blocks), "Conversion rules" (X = 2^floor(log2 amax) / 4, RNE with
+// saturation), "Training with MXFP4" (random Hadamard transform of size 16/32,
+// stochastic rounding).  "Training an MoE LLM in MXFP4" (ALTO), abstract:
+// 1D blocks for activations/gradients, 2D blocks for weights.
+//
+// All kernels are HBM-bound streaming kernels (2 B read + 0.5 B + 1/32 B
+// written per element): 128-bit loads/stores, in-register Hadamard butterflies,
+// and shared-memory staging only where a transpose is needed.
+#include <cstdint>
+#include <cstdio>
+
+#include "common.cuh"
+
+namespace mxfp4 {
+
+struct QuantParams {
+    const uint16_t *x;
+    int64_t rows, cols, ld_x;
+    uint8_t *codes;
+    int64_t ld_codes;
+    uint8_t *scales;
+    int64_t ld_scales, katoms;      // katoms: MMA layout K-atoms of the output operand
+    uint8_t *codes_t;
+    int64_t ld_codes_t;
+    uint8_t *scales_t;
+    int64_t ld_scales_t, katoms_t;
+    uint32_t seed_lo, seed_hi;
+    uint64_t elem_offset;
+    // RHT signs as xor words: pair[j] flips the bf16 halves of word j of a
+    // 32-element row segment (elements 2j, 2j+1); dup[i] flips both halves of
+    // a word for element i of a column segment.
+    uint32_t sgn_pair[16];
+    uint32_t sgn_dup[32];
+};
+
+// ---------------------------------------------------------------------------
+// Per-block quantization core: 32 fp32 values (already transformed) -> scale
+// code and 16 bytes of codes.  `g0` is the stream index of element 0.
+// ---------------------------------------------------------------------------
+template <bool SR>
+__device__ __forceinline__ uint32_t quantize32(float *v, uint4 &out, uint64_t g0, uint32_t k0, uint32_t k1) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = amax_nan(amax, v[i]);
+    const uint32_t code = scale_code_from_amax(amax);
+    if (code == 0xFFu) {
+        out = make_uint4(0, 0, 0, 0);
+        return code;
+    }
+    const float inv = inv_scale_from_code(code);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], inv);
+    uint32_t p[4];
+    if constexpr (!SR) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) p[q] = e2m1x8_rn(v + 8 * q);
+    } else {
+        const uint64_t blk = g0 >> 2;  // g0 % 4 == 0
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint64_t b0 = blk + 2 * q, b1 = b0 + 1;
+            const U4 r0 = philox4x32_10((uint32_t)b0, (uint32_t)(b0 >> 32), 0u, 0u, k0, k1);
+            const U4 r1 = philox4x32_10((uint32_t)b1, (uint32_t)(b1 >> 32), 0u, 0u, k0, k1);
+            const float *w = v + 8 * q;
+            p[q] = e2m1_sr(w[0], r0.x) | (e2m1_sr(w[1], r0.y) << 4) | (e2m1_sr(w[2], r0.z) << 8) |
+                   (e2m1_sr(w[3], r0.w) << 12) | (e2m1_sr(w[4], r1.x) << 16) | (e2m1_sr(w[5], r1.y) << 20) |
+                   (e2m1_sr(w[6], r1.z) << 24) | (e2m1_sr(w[7], r1.w) << 28);
+        }
+    }
+    out = make_uint4(p[0], p[1], p[2], p[3]);
+    return code;
+}
+
+// Unpack 16 bf16x2 words to 32 fp32 values, with RHT sign flips and butterfly.
+template <int RHT>
+__device__ __forceinline__ void unpack_row32(const uint32_t *w, float *v, const QuantParams &p) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        uint32_t u = w[j];
+        if constexpr (RHT) u ^= p.sgn_pair[j];
+        v[2 * j] = bf16lo(u);
+        v[2 * j + 1] = bf16hi(u);
+    }
+    if constexpr (RHT) {
+#pragma unroll
+        for (int s = 0; s < 32; s += RHT) fwht<RHT>(v + s);
+        const float c = rht_norm<RHT>();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], c);
+    }
+}
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void stg_v4(void *p, uint4 v) {
+    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// 1D row blocks: one thread per 32-element block, grid-stride.
+// ---------------------------------------------------------------------------
+template <int RHT, bool SR, bool MMA>
+__global__ void __launch_bounds__(256) quant_row_kernel(const QuantParams p) {
+    const int64_t nb = p.cols >> 5;
+    const int64_t total = p.rows * nb;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= total) return;
+    int64_t r = b / nb, kb = b - r * nb;
+    const int64_t sr_ = stride / nb, sk_ = stride - sr_ * nb;
+    for (; b < total; b += stride) {
+        const uint16_t *src = p.x + r * p.ld_x + (kb << 5);
+        uint32_t w[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 t = ldg_nc_v4(src + 8 * q);
+            w[4 * q] = t.x; w[4 * q + 1] = t.y; w[4 * q + 2] = t.z; w[4 * q + 3] = t.w;
+        }
+        float v[32];
+        unpack_row32<RHT>(w, v, p);
+        uint4 packed;
+        const uint64_t g0 = (uint64_t)(r * p.cols + (kb << 5)) + p.elem_offset;
+        const uint32_t code = quantize32<SR>(v, packed, g0, p.seed_lo, p.seed_hi);
+        stg_v4(p.codes + r * p.ld_codes + (kb << 4), packed);
+        if constexpr (MMA) p.scales[mma_scale_off(r, kb, p.katoms)] = (uint8_t)code;
+        else p.scales[r * p.ld_scales + kb] = (uint8_t)code;
+        r += sr_;
+        kb += sk_;
+        if (kb >= nb) { kb -= nb; ++r; }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 1D column blocks (output = transposed view).  A CTA stages a 256 x 64 bf16
+// tile in shared memory with coalesced 16-byte copies; warp w quantizes the
+// 32-row block w of the tile, lane l the two columns 2l and 2l+1; the codes of
+// the 64 output rows x 128 bytes go back through shared memory so that the
+// global stores are full 128-byte lines.
+// ---------------------------------------------------------------------------
+constexpr int COL_TR = 256, COL_TC = 64;
+
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <int RHT, bool SR, bool MMA>
+__global__ void __launch_bounds__(256) quant_col_kernel(const QuantParams p) {
+    __shared__ __align__(16) uint32_t tin[COL_TR][COL_TC / 2];   // 32 KB: bf16 pairs
+    __shared__ __align__(16) uint4 tout[COL_TC][COL_TR / 32];    // 8 KB: 64 rows x 128 B
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t tiles_r = (p.rows + COL_TR - 1) / COL_TR;
+    const int64_t tiles_c = (p.cols + COL_TC - 1) / COL_TC;
+    const int64_t ntiles = tiles_r * tiles_c;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        const int64_t r0 = tr * COL_TR, c0 = tc * COL_TC;
+        // load: 256 rows x 8 chunks of 16 B
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int row = (tid >> 3) + 32 * i, ch = tid & 7;
+            const int64_t gr = r0 + row, gc = c0 + 8 * ch;
+            if (gr < p.rows && gc < p.cols) cp_async16(&tin[row][4 * ch], p.x + gr * p.ld_x + gc);
+        }
+        cp_async_wait_all();
+        __syncthreads();
+        const int64_t rb = r0 + 32 * warp;        // first input row of this warp's block
+        const int64_t oc = c0 + 2 * lane;         // first of the two output rows of this lane
+        const bool blk_ok = rb < p.rows;
+        if (blk_ok && oc < p.cols) {
+            float v0[32], v1[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                uint32_t u = tin[32 * warp + i][lane];
+                if constexpr (RHT) u ^= p.sgn_dup[i % RHT];
+                v0[i] = bf16lo(u);
+                v1[i] = bf16hi(u);
+            }
+            if constexpr (RHT) {
+                const float c = rht_norm<RHT>();
+#pragma unroll
+                for (int s = 0; s < 32; s += RHT) { fwht<RHT>(v0 + s); fwht<RHT>(v1 + s); }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) { v0[i] = __fmul_rn(v0[i], c); v1[i] = __fmul_rn(v1[i], c); }
+            }
+            const int64_t kb = rb >> 5;           // output K-block
+            uint4 q0, q1;
+            const uint64_t g0 = (uint64_t)(oc * p.rows + rb) + p.elem_offset;
+            const uint32_t s0 = quantize32<SR>(v0, q0, g0, p.seed_lo, p.seed_hi);
+            const uint32_t s1 = quantize32<SR>(v1, q1, g0 + (uint64_t)p.rows, p.seed_lo, p.seed_hi);
+            const int sw = lane & 7;
+            tout[2 * lane][warp ^ sw] = q0;
+            tout[2 * lane + 1][warp ^ sw] = q1;
+            if constexpr (MMA) {
+                p.scales[mma_scale_off(oc, kb, p.katoms)] = (uint8_t)s0;
+                p.scales[mma_scale_off(oc + 1, kb, p.katoms)] = (uint8_t)s1;
+            } else {
+                p.scales[oc * p.ld_scales + kb] = (uint8_t)s0;
+                p.scales[(oc + 1) * p.ld_scales + kb] = (uint8_t)s1;
+            }
+        }
+        __syncthreads();
+        // store: 64 output rows x 8 chunks of 16 B
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int row = (tid >> 3) + 32 * i, ch = tid & 7;
+            const int64_t orow = c0 + row, rin = r0 + 32 * ch;
+            if (orow < p.cols && rin < p.rows)
+                stg_v4(p.codes + orow * p.ld_codes + (rin >> 1), tout[row][ch ^ ((row >> 1) & 7)]);
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 2D 32x32 blocks.  A CTA covers 32 rows x 256 columns: warp w owns the tile
+// of columns 32w..32w+31, lane l its row l.  amax is a warp max.  The
+// optional transposed copy is built through a byte-transposed 512-byte
+// shared-memory tile per warp.
+// ---------------------------------------------------------------------------
+template <int RHT, bool SR, bool MMA, bool TRANS>
+__global__ void __launch_bounds__(256) quant_2d_kernel(const QuantParams p) {
+    __shared__ __align__(16) uint8_t tb[8][16][32];   // per warp: byte j of row r at [j][r]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t nbr = p.rows >> 5, nbc = p.cols >> 5;
+    const int64_t groups_c = (nbc + 7) >> 3;
+    const int64_t ngroups = nbr * groups_c;
+    for (int64_t t = blockIdx.x; t < ngroups; t += gridDim.x) {
+        const int64_t br = t / groups_c;
+        const int64_t bc = (t - br * groups_c) * 8 + warp;
+        if (bc < nbc) {
+            const int64_t r = (br << 5) + lane, c0 = bc << 5;
+            const uint16_t *src = p.x + r * p.ld_x + c0;
+            uint32_t w[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 u = ldg_nc_v4(src + 8 * q);
+                w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+            }
+            float v[32];
+            unpack_row32<RHT>(w, v, p);
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) amax = amax_nan(amax, v[i]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float other = __shfl_xor_sync(0xFFFFFFFFu, amax, o);
+                asm("max.NaN.f32 %0, %0, %1;" : "+f"(amax) : "f"(other));
+            }
+            const uint32_t code = scale_code_from_amax(amax);
+            uint4 packed = make_uint4(0, 0, 0, 0);
+            if (code != 0xFFu) {
+                const float inv = inv_scale_from_code(code);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], inv);
+                uint32_t pk[4];
+                if constexpr (!SR) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) pk[q] = e2m1x8_rn(v + 8 * q);
+                } else {
+                    const uint64_t blk = ((uint64_t)(r * p.cols + c0) + p.elem_offset) >> 2;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint64_t b0 = blk + 2 * q, b1 = b0 + 1;
+                        const U4 r0 = philox4x32_10((uint32_t)b0, (uint32_t)(b0 >> 32), 0u, 0u, p.seed_lo, p.seed_hi);
+                        const U4 r1 = philox4x32_10((uint32_t)b1, (uint32_t)(b1 >> 32), 0u, 0u, p.seed_lo, p.seed_hi);
+                        const float *x8 = v + 8 * q;
+                        pk[q] = e2m1_sr(x8[0], r0.x) | (e2m1_sr(x8[1], r0.y) << 4) | (e2m1_sr(x8[2], r0.z) << 8) |
+                                (e2m1_sr(x8[3], r0.w) << 12) | (e2m1_sr(x8[4], r1.x) << 16) |
+                                (e2m1_sr(x8[5], r1.y) << 20) | (e2m1_sr(x8[6], r1.z) << 24) |
+                                (e2m1_sr(x8[7], r1.w) << 28);
+                    }
+                }
+                packed = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            stg_v4(p.codes + r * p.ld_codes + (c0 >> 1), packed);
+            if constexpr (MMA) {
+                p.scales[mma_scale_off(r, bc, p.katoms)] = (uint8_t)code;
+            } else {
+                if (lane == 0) p.scales[br * p.ld_scales + bc] = (uint8_t)code;
+            }
+            if constexpr (TRANS) {
+                // byte-transpose through shared memory: tb[j][row] = byte j of row
+                const uint32_t pw[4] = {packed.x, packed.y, packed.z, packed.w};
+#pragma unroll
+                for (int j = 0; j < 16; ++j) tb[warp][j][lane] = (uint8_t)(pw[j >> 2] >> (8 * (j & 3)));
+                __syncwarp();
+                // lane c gathers byte c/2 of every row and keeps nibble c&1
+                const uint4 *rowp = reinterpret_cast<const uint4 *>(&tb[warp][lane >> 1][0]);
+                const uint4 a = rowp[0], b2 = rowp[1];
+                const uint32_t bw[8] = {a.x, a.y, a.z, a.w, b2.x, b2.y, b2.z, b2.w};
+                const int sh = 4 * (lane & 1);
+                uint32_t o[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    // words 2q, 2q+1 hold rows 8q..8q+7 (one byte each)
+                    const uint32_t lo = (bw[2 * q] >> sh) & 0x0F0F0F0Fu;      // nibbles of rows 8q..8q+3
+                    const uint32_t hi = (bw[2 * q + 1] >> sh) & 0x0F0F0F0Fu;  // rows 8q+4..8q+7
+                    // pack row pairs: out byte k = nib(2k) | nib(2k+1) << 4
+                    const uint32_t lo2 = (lo | (lo >> 4)) & 0x00FF00FFu;      // bytes: r0|r1, r2|r3
+                    const uint32_t hi2 = (hi | (hi >> 4)) & 0x00FF00FFu;
+                    o[q] = (lo2 & 0xFFu) | ((lo2 >> 8) & 0xFF00u) | ((hi2 & 0xFFu) << 16) | ((hi2 << 8) & 0xFF000000u);
+                }
+                __syncwarp();
+                const int64_t ct = c0 + lane;       // row of the transposed operand
+                stg_v4(p.codes_t + ct * p.ld_codes_t + (br << 4), make_uint4(o[0], o[1], o[2], o[3]));
+                if (p.scales_t) {
+                    if constexpr (MMA) {
+                        p.scales_t[mma_scale_off(ct, br, p.katoms_t)] = (uint8_t)code;
+                    } else {
+                        if (lane == 0) p.scales_t[bc * p.ld_scales_t + br] = (uint8_t)code;
+                    }
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Dequantize.
+// ---------------------------------------------------------------------------
+struct DequantParams {
+    const uint8_t *codes;
+    int64_t ld_codes;
+    const uint8_t *scales;
+    int64_t ld_scales, katoms;
+    int64_t rows, cols;   // output shape
+    void *out;
+    int64_t ld_out;
+    uint32_t sgn_pair[16];
+    uint32_t sgn_dup[32];
+};
+
+// fp32 bit pattern of an E2M1 magnitude code m (0..7): m >= 2 -> (252 + m) << 22
+// (1.0 .. 6.0), m == 1 -> 0.5, m == 0 -> 0.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+    const uint32_t m = c & 7u;
+    uint32_t b = m >= 2u ? (252u + m) << 22 : (m ? 0x3F000000u : 0u);
+    b |= (c & 8u) << 28;
+    return __uint_as_float(b);
+}
+
+__device__ __forceinline__ void decode32(const uint4 q, uint32_t scode, float *v) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    if (scode == 0xFFu) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(0x7FFFFFFFu);
+        return;
+    }
+    const float X = scale_from_code(scode);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(e2m1_value((w[i >> 3] >> (4 * (i & 7))) & 0xFu), X);
+}
+
+template <int RHT>
+__device__ __forceinline__ void inverse_rht32(float *v, const uint32_t *sgn_pair) {
+    if constexpr (RHT) {
+        const float c = rht_norm<RHT>();
+#pragma unroll
+        for (int s = 0; s < 32; s += RHT) fwht<RHT>(v + s);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], c);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            v[2 * j] = __uint_as_float(__float_as_uint(v[2 * j]) ^ (sgn_pair[j] << 16));
+            v[2 * j + 1] = __uint_as_float(__float_as_uint(v[2 * j + 1]) ^ (sgn_pair[j] & 0x80000000u));
+        }
+    }
+}
+
+// SMODE: 0 = row-major per row [rows, cols/32], 1 = row-major 2D tiles
+// [rows/32, cols/32], 2 = MMA layout per row.
+template <int RHT, bool F32, int SMODE>
+__global__ void __launch_bounds__(256) dequant_row_kernel(const DequantParams p) {
+    const int64_t nb = p.cols >> 5;
+    const int64_t total = p.rows * nb;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < total;
+         b += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = b / nb, kb = b - r * nb;
+        const uint4 q = ldg_nc_v4(p.codes + r * p.ld_codes + (kb << 4));
+        uint32_t sc;
+        if constexpr (SMODE == 0) sc = p.scales[r * p.ld_scales + kb];
+        else if constexpr (SMODE == 1) sc = p.scales[(r >> 5) * p.ld_scales + kb];
+        else sc = p.scales[mma_scale_off(r, kb, p.katoms)];
+        float v[32];
+        decode32(q, sc, v);
+        inverse_rht32<RHT>(v, p.sgn_pair);
+        if constexpr (F32) {
+            float *dst = reinterpret_cast<float *>(p.out) + r * p.ld_out + (kb << 5);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                stg_v4(dst + 4 * i, make_uint4(__float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
+                                               __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3])));
+        } else {
+            uint16_t *dst = reinterpret_cast<uint16_t *>(p.out) + r * p.ld_out + (kb << 5);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                stg_v4(dst + 8 * i, make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                               pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7])));
+        }
+    }
+}
+
+// Transposed-view codes [cols, rows/2] back to out[rows, cols].  A CTA handles
+// 64 code rows (= output columns) x 8 blocks (= 256 output rows): the codes
+// are staged with coalesced 16-byte loads; warp w decodes block w, lane l the
+// output columns 2l and 2l+1, so each output row is written as one contiguous
+// 128-byte (bf16) or 256-byte (fp32) warp store.
+template <int RHT, bool F32, bool MMA>
+__global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p) {
+    __shared__ __align__(16) uint4 tin[COL_TC][8];                 // 8 KB of codes
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t tiles_r = (p.rows + COL_TR - 1) / COL_TR;
+    const int64_t tiles_c = (p.cols + COL_TC - 1) / COL_TC;
+    const int64_t ntiles = tiles_r * tiles_c;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        const int64_t r0 = tr * COL_TR, c0 = tc * COL_TC;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int row = (tid >> 3) + 32 * i, ch = tid & 7;
+            const int64_t crow = c0 + row, rin = r0 + 32 * ch;
+            if (crow < p.cols && rin < p.rows)
+                tin[row][ch] = ldg_nc_v4(p.codes + crow * p.ld_codes + (rin >> 1));
+        }
+        __syncthreads();
+        const int64_t rb = r0 + 32 * warp, oc = c0 + 2 * lane;
+        if (rb < p.rows && oc < p.cols) {
+            const int64_t kb = rb >> 5;
+            uint32_t s0, s1;
+            if constexpr (MMA) {
+                s0 = p.scales[mma_scale_off(oc, kb, p.katoms)];
+                s1 = p.scales[mma_scale_off(oc + 1, kb, p.katoms)];
+            } else {
+                s0 = p.scales[oc * p.ld_scales + kb];
+                s1 = p.scales[(oc + 1) * p.ld_scales + kb];
+            }
+            float v0[32], v1[32];
+            decode32(tin[2 * lane][warp], s0, v0);
+            decode32(tin[2 * lane + 1][warp], s1, v1);
+            if constexpr (RHT) {
+                const float c = rht_norm<RHT>();
+#pragma unroll
+                for (int s = 0; s < 32; s += RHT) { fwht<RHT>(v0 + s); fwht<RHT>(v1 + s); }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const uint32_t fl = p.sgn_dup[i % RHT] & 0x80000000u;
+                    v0[i] = __uint_as_float(__float_as_uint(__fmul_rn(v0[i], c)) ^ fl);
+                    v1[i] = __uint_as_float(__float_as_uint(__fmul_rn(v1[i], c)) ^ fl);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int64_t gr = rb + i;
+                if constexpr (F32) {
+                    float2 *dst = reinterpret_cast<float2 *>(reinterpret_cast<float *>(p.out) + gr * p.ld_out + oc);
+                    *dst = make_float2(v0[i], v1[i]);
+                } else {
+                    uint32_t *dst = reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(p.out) + gr * p.ld_out + oc);
+                    *dst = pack_bf16x2(v0[i], v1[i]);
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (called by the C ABI after validation).
+// ---------------------------------------------------------------------------
+static int g_num_sms = 0;
+
+static int num_sms() {
+    if (g_num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (g_num_sms <= 0) g_num_sms = 148;
+    }
+    return g_num_sms;
+}
+
+static void fill_signs(uint32_t mask, int rht, uint32_t *pair, uint32_t *dup) {
+    for (int j = 0; j < 16; ++j) {
+        const uint32_t e0 = (uint32_t)(2 * j) % (uint32_t)(rht ? rht : 32);
+        const uint32_t e1 = (uint32_t)(2 * j + 1) % (uint32_t)(rht ? rht : 32);
+        const uint32_t s0 = rht ? (mask >> e0) & 1u : 0u;
+        const uint32_t s1 = rht ? (mask >> e1) & 1u : 0u;
+        pair[j] = (s0 << 15) | (s1 << 31);
+    }
+    for (int i = 0; i < 32; ++i) {
+        const uint32_t s = rht ? (mask >> (i % rht)) & 1u : 0u;
+        dup[i] = s ? 0x80008000u : 0u;
+    }
+}
+
+static int64_t grid_for(int64_t items, int threads) {
+    int64_t g = (items + threads - 1) / threads;
+    const int64_t cap = (int64_t)num_sms() * 32;
+    return g < 1 ? 1 : (g > cap ? cap : g);
+}
+
+template <int RHT, bool SR, bool MMA>
+static cudaError_t launch_quant_t(int layout, bool trans, const QuantParams &p, cudaStream_t s) {
+    if (layout == MXFP4_LAYOUT_1D_ROW) {
+        quant_row_kernel<RHT, SR, MMA><<<(unsigned)grid_for(p.rows * (p.cols / 32), 256), 256, 0, s>>>(p);
+    } else if (layout == MXFP4_LAYOUT_1D_COL) {
+        const int64_t tiles = ((p.rows + COL_TR - 1) / COL_TR) * ((p.cols + COL_TC - 1) / COL_TC);
+        const int64_t cap = (int64_t)num_sms() * 8;
+        quant_col_kernel<RHT, SR, MMA><<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, s>>>(p);
+    } else {
+        const int64_t groups = (p.rows / 32) * ((p.cols / 32 + 7) / 8);
+        const int64_t cap = (int64_t)num_sms() * 16;
+        const unsigned g = (unsigned)(groups < cap ? groups : cap);
+        if (trans) quant_2d_kernel<RHT, SR, MMA, true><<<g, 256, 0, s>>>(p);
+        else quant_2d_kernel<RHT, SR, MMA, false><<<g, 256, 0, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+template <int RHT, bool SR>
+static cudaError_t launch_quant_r(int layout, bool trans, bool mma, const QuantParams &p, cudaStream_t s) {
+    return mma ? launch_quant_t<RHT, SR, true>(layout, trans, p, s) : launch_quant_t<RHT, SR, false>(layout, trans, p, s);
+}
+
+template <int RHT>
+static cudaError_t launch_quant_s(int layout, bool trans, bool mma, bool sr, const QuantParams &p, cudaStream_t s) {
+    return sr ? launch_quant_r<RHT, true>(layout, trans, mma, p, s) : launch_quant_r<RHT, false>(layout, trans, mma, p, s);
+}
+
+cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rht,
+                            int rounding, uint64_t seed, uint64_t elem_offset, uint8_t *codes, int64_t ld_codes,
+                            uint8_t *scales, int64_t ld_scales, int scale_layout, uint8_t *codes_t,
+                            int64_t ld_codes_t, uint8_t *scales_t, int64_t ld_scales_t, cudaStream_t s) {
+    QuantParams p{};
+    p.x = static_cast<const uint16_t *>(x);
+    p.rows = rows; p.cols = cols; p.ld_x = ld_x;
+    p.codes = codes; p.ld_codes = ld_codes;
+    p.scales = scales; p.ld_scales = ld_scales;
+    p.codes_t = codes_t; p.ld_codes_t = ld_codes_t;
+    p.scales_t = scales_t; p.ld_scales_t = ld_scales_t;
+    const int64_t k_out = layout == MXFP4_LAYOUT_1D_COL ? rows : cols;
+    p.katoms = mma_katoms(k_out);
+    p.katoms_t = mma_katoms(rows);
+    p.seed_lo = (uint32_t)seed; p.seed_hi = (uint32_t)(seed >> 32);
+    p.elem_offset = elem_offset;
+    fill_signs(rht ? rht_sign_mask_hd(seed) : 0u, rht, p.sgn_pair, p.sgn_dup);
+    const bool mma = scale_layout == MXFP4_SCALES_MMA;
+    const bool sr = rounding == MXFP4_ROUND_SR;
+    const bool trans = codes_t != nullptr;
+    switch (rht) {
+        case 0: return launch_quant_s<0>(layout, trans, mma, sr, p, s);
+        case 16: return launch_quant_s<16>(layout, trans, mma, sr, p, s);
+        default: return launch_quant_s<32>(layout, trans, mma, sr, p, s);
+    }
+}
+
+template <int RHT, bool F32>
+static cudaError_t launch_dequant_t(int layout, int smode, const DequantParams &p, cudaStream_t s) {
+    if (layout == MXFP4_LAYOUT_1D_COL) {
+        const int64_t tiles = ((p.rows + COL_TR - 1) / COL_TR) * ((p.cols + COL_TC - 1) / COL_TC);
+        const int64_t cap = (int64_t)num_sms() * 8;
+        const unsigned g = (unsigned)(tiles < cap ? tiles : cap);
+        if (smode == 2) dequant_col_kernel<RHT, F32, true><<<g, 256, 0, s>>>(p);
+        else dequant_col_kernel<RHT, F32, false><<<g, 256, 0, s>>>(p);
+    } else {
+        const unsigned g = (unsigned)grid_for(p.rows * (p.cols / 32), 256);
+        if (smode == 0) dequant_row_kernel<RHT, F32, 0><<<g, 256, 0, s>>>(p);
+        else if (smode == 1) dequant_row_kernel<RHT, F32, 1><<<g, 256, 0, s>>>(p);
+        else dequant_row_kernel<RHT, F32, 2><<<g, 256, 0, s>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+template <int RHT>
+static cudaError_t launch_dequant_r(int layout, int smode, bool f32, const DequantParams &p, cudaStream_t s) {
+    return f32 ? launch_dequant_t<RHT, true>(layout, smode, p, s) : launch_dequant_t<RHT, false>(layout, smode, p, s);
+}
+
+cudaError_t launch_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
+                              int scale_layout, int64_t rows, int64_t cols, int layout, int rht, uint64_t seed,
+                              void *out, int64_t ld_out, int out_dtype, cudaStream_t s) {
+    DequantParams p{};
+    p.codes = codes; p.ld_codes = ld_codes;
+    p.scales = scales; p.ld_scales = ld_scales;
+    p.rows = rows; p.cols = cols; p.out = out; p.ld_out = ld_out;
+    p.katoms = mma_katoms(layout == MXFP4_LAYOUT_1D_COL ? rows : cols);
+    fill_signs(rht ? rht_sign_mask_hd(seed) : 0u, rht, p.sgn_pair, p.sgn_dup);
+    const int smode = scale_layout == MXFP4_SCALES_MMA ? 2 : (layout == MXFP4_LAYOUT_2D ? 1 : 0);
+    const bool f32 = out_dtype == MXFP4_OUT_F32;
+    switch (rht) {
+        case 0: return launch_dequant_r<0>(layout, smode, f32, p, s);
+        case 16: return launch_dequant_r<16>(layout, smode, f32, p, s);
+        default: return launch_dequant_r<32>(layout, smode, f32, p, s);
+    }
+}
+
+}  // namespace mxfp4

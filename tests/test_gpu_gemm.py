@@ -1,0 +1,181 @@
+"""GPU parity: mxfp4_gemm / mxfp4_grouped_gemm through the C ABI against the fp64 oracle.
+
+Tolerance (block dot products, "Conversion rules" on "MXFP4", FP32 result):
+|C_gpu - C_fp64| <= 1e-5 * sum_k |a_k b_k| element-wise.  The tcgen05 MMA
+accumulates each 64-element K step into FP32, so the FP32 rounding error is at
+most (K/64) * 2^-24 * sum|a b| (<= 5.4e-6 * S for K = 5760) plus the
+rounding inside a step, which the bound leaves room for.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantize_block_scaled_rht_b200 as mx
+import synth
+from mxfp4_testutil import assert_gemm_close, dev_bf16, dev_u8, expand_2d, host, to_mma
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_operand(bits, layout=oracle.LAYOUT_1D_ROW, rht=0, rnd=oracle.ROUND_RNE, seed=0):
+    codes, scales = oracle.quantize(bits, layout, rht, rnd, seed)[:2]
+    return codes, scales
+
+
+def _run_gemm_from_oracle_operands(ca, sa, cb, sb, K):
+    """GEMM on the GPU from oracle-quantized operands (scales moved to the MMA layout)."""
+    out = mx.mxfp4_gemm(dev_u8(ca), dev_u8(to_mma(sa, K)), dev_u8(cb), dev_u8(to_mma(sb, K)), K)
+    torch.cuda.synchronize()
+    return host(out)
+
+
+def test_pr1_256_cube_quantize_and_gemm_on_gpu():
+    """PR1: X, Y 256x256 N(0,1) (seeds 0, 1), 1D RNE, C = X Y^T."""
+    xb, yb = synth.pr1_inputs()
+    qx = mx.mxfp4_quantize(dev_bf16(xb), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    qy = mx.mxfp4_quantize(dev_bf16(yb), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    c = host(mx.mxfp4_gemm(qx.codes, qx.scales, qy.codes, qy.scales, 256))
+    ca, sa = _oracle_operand(xb)
+    cb, sb = _oracle_operand(yb)
+    assert np.array_equal(host(qx.codes), ca) and np.array_equal(host(qy.codes), cb)
+    ref, s = oracle.gemm(ca, sa, cb, sb, 256)
+    assert_gemm_close(c, ref, s)
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 192, 64), (300, 200, 320), (512, 768, 1024), (130, 72, 2880),
+                                   (1, 8, 128), (257, 388, 576)])
+def test_gemm_shapes(M, N, K):
+    a = synth.normal_bf16((M, K), 10 + M)
+    b = synth.normal_bf16((N, K), 20 + N, 0.02)
+    ca, sa = _oracle_operand(a)
+    cb, sb = _oracle_operand(b)
+    c = _run_gemm_from_oracle_operands(ca, sa, cb, sb, K)
+    ref, s = oracle.gemm(ca, sa, cb, sb, K)
+    assert_gemm_close(c, ref, s)
+
+
+def test_gemm_wide_dynamic_range_and_nan():
+    M, N, K = 256, 384, 512
+    g = np.random.default_rng(3)
+    a = synth.bf16_bits((g.standard_normal((M, K)) * 2.0 ** g.integers(-30, 30, (M, 1))).astype(np.float32))
+    b = synth.bf16_bits((g.standard_normal((N, K)) * 2.0 ** g.integers(-30, 30, (1, K))).astype(np.float32))
+    ca, sa = _oracle_operand(a)
+    cb, sb = _oracle_operand(b)
+    sa = sa.copy(); sb = sb.copy()
+    sa[5, 3] = 0xFF
+    sb[7, 0] = 0xFF
+    c = _run_gemm_from_oracle_operands(ca, sa, cb, sb, K)
+    ref, s = oracle.gemm(ca, sa, cb, sb, K)
+    assert np.all(np.isnan(c[5])) and np.all(np.isnan(c[:, 7]))
+    assert_gemm_close(c, ref, s)
+
+
+def test_fprop_dgrad_with_2d_weight_and_transposed_copy():
+    """W quantized once in 2D; fprop uses W's codes, dgrad the transposed copy."""
+    T, H, I = 256, 320, 448
+    x = synth.activations_with_outliers(T, H, seed=2)
+    w = synth.normal_bf16((I, H), 3, 0.02)
+    dy = synth.normal_bf16((T, I), 4, 1e-3)
+    qw = mx.mxfp4_quantize(dev_bf16(w), mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA, transposed_copy=True)
+    qx = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    qdy = mx.mxfp4_quantize(dev_bf16(dy), mx.LAYOUT_1D_ROW, 0, mx.ROUND_SR, 42, scale_layout=mx.SCALES_MMA)
+    y = host(mx.mxfp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, H))
+    dx = host(mx.mxfp4_gemm(qdy.codes, qdy.scales, qw.codes_t, qw.scales_t, I))
+    cw, sw, cwt = oracle.quantize(w, oracle.LAYOUT_2D, transposed_copy=True)
+    cx, sx = _oracle_operand(x)
+    cdy, sdy = _oracle_operand(dy, rnd=oracle.ROUND_SR, seed=42)
+    ref_y, s_y = oracle.gemm(cx, sx, cw, sw, H, 0, 1)
+    ref_dx, s_dx = oracle.gemm(cdy, sdy, cwt, sw, I, 0, 2)
+    assert_gemm_close(y, ref_y, s_y)
+    assert_gemm_close(dx, ref_dx, s_dx)
+
+
+def test_wgrad_rht32_along_tokens():
+    """wgrad: dY^T and X^T quantized along tokens (1D col) with RHT32 and shared signs."""
+    T, H, I = 512, 192, 320
+    x = synth.normal_bf16((T, H), 5)
+    dy = synth.normal_bf16((T, I), 6, 1e-3)
+    qdyt = mx.mxfp4_quantize(dev_bf16(dy), mx.LAYOUT_1D_COL, 32, mx.ROUND_SR, 42, scale_layout=mx.SCALES_MMA)
+    qxt = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_COL, 32, mx.ROUND_RNE, 42, scale_layout=mx.SCALES_MMA)
+    dw = host(mx.mxfp4_gemm(qdyt.codes, qdyt.scales, qxt.codes, qxt.scales, T))
+    ca, sa = oracle.quantize(dy, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_SR, 42)
+    cb, sb = oracle.quantize(x, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_RNE, 42)
+    ref, s = oracle.gemm(ca, sa, cb, sb, T)
+    assert_gemm_close(dw, ref, s)
+
+
+def _grouped_case(sizes, N, K, seed=0):
+    G = len(sizes)
+    sizes = np.asarray(sizes, np.int32)
+    padded = (sizes + 127) // 128 * 128
+    offsets = np.zeros(G + 1, np.int32)
+    offsets[1:] = np.cumsum(padded)
+    rows = int(max(offsets[-1], 128))
+    a = synth.normal_bf16((rows, K), seed + 1)
+    w = synth.normal_bf16((G, N, K), seed + 2, 0.02)
+    return sizes, offsets, rows, a, w
+
+
+@pytest.mark.parametrize("sizes,N,K", [([1, 130, 0, 257, 128], 192, 256), ([300, 5, 64], 384, 576),
+                                       ([17], 224, 128)])
+def test_grouped_gemm(sizes, N, K):
+    sizes, offsets, rows, a, w = _grouped_case(sizes, N, K)
+    G = len(sizes)
+    qa = mx.mxfp4_quantize(dev_bf16(a), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    qw = [mx.mxfp4_quantize(dev_bf16(w[g]), mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA) for g in range(G)]
+    b_codes = torch.stack([q.codes for q in qw])
+    b_scales = torch.cat([q.scales for q in qw])
+    sentinel = 12345.0
+    out = torch.full((rows, N), sentinel, dtype=torch.float32, device="cuda")
+    mx.mxfp4_grouped_gemm(qa.codes, qa.scales, torch.from_numpy(offsets).cuda(), torch.from_numpy(sizes).cuda(),
+                          b_codes, b_scales, N, K, out=out)
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    c = host(out)
+    ca, sa = oracle.quantize(a, oracle.LAYOUT_1D_ROW)
+    for g in range(G):
+        o, n = int(offsets[g]), int(sizes[g])
+        cw, sw = oracle.quantize(w[g], oracle.LAYOUT_2D)
+        if n:
+            ref, s = oracle.gemm(ca[o:o + n], sa[o:o + n], cw, sw, K, 0, 1)
+            assert_gemm_close(c[o:o + n], ref, s)
+        # padding rows of the group are never written
+        assert np.all(c[o + n:int(offsets[g + 1])] == sentinel)
+
+
+def test_grouped_gemm_misaligned_offset_is_reported():
+    sizes, offsets, rows, a, w = _grouped_case([64, 64], 192, 128)
+    offsets = offsets.copy()
+    offsets[1] = 100                                        # not a multiple of 128
+    qa = mx.mxfp4_quantize(dev_bf16(a), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    qw = [mx.mxfp4_quantize(dev_bf16(w[g]), mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA) for g in range(2)]
+    mx.mxfp4_grouped_gemm(qa.codes, qa.scales, torch.from_numpy(offsets).cuda(), torch.from_numpy(sizes).cuda(),
+                          torch.stack([q.codes for q in qw]), torch.cat([q.scales for q in qw]), 192, 128)
+    assert mx.mxfp4_get_error() == mx.MXFP4_ERR_INVALID_ARG
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+
+
+def test_gemm_rejects_bad_k_and_alignment():
+    a = torch.zeros((128, 48), dtype=torch.uint8, device="cuda")
+    s = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    with pytest.raises(mx.MXFP4Error) as e:
+        mx.mxfp4_gemm(a, s, a, s, 96)                       # K % 64 != 0
+    assert e.value.status == mx.MXFP4_ERR_UNSUPPORTED
+    big = torch.zeros((128, 80), dtype=torch.uint8, device="cuda")
+    with pytest.raises(mx.MXFP4Error) as e:
+        mx.mxfp4_gemm(big[:, 8:], s, big[:, 8:], s, 128)    # misaligned pointer
+    assert e.value.status == mx.MXFP4_ERR_ALIGNMENT
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    mx.mxfp4_wait_probe(True)
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    old = mx.mxfp4_set_wait_limit_ns(2_000_000)             # 2 ms
+    try:
+        mx.mxfp4_wait_probe(False)                          # nothing ever arrives
+        assert mx.mxfp4_get_error() == mx.MXFP4_ERR_TIMEOUT
+    finally:
+        mx.mxfp4_set_wait_limit_ns(old)
+    # the context is still usable
+    test_gemm_shapes(128, 192, 64)

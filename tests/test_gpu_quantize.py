@@ -1,0 +1,159 @@
+"""GPU parity: mxfp4_quantize / mxfp4_dequantize through the C ABI against the oracle.
+
+Codes and scales must be bit-exact (including stochastic rounding and the RHT).
+Shapes span several CTA tiles with ragged tails; edge cases cover every bf16
+bit pattern (NaN, Inf, subnormals, zeros, ties, saturation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantize_block_scaled_rht_b200 as mx
+import synth
+from mxfp4_testutil import dev_bf16, expand_2d, from_mma, host
+
+pytestmark = pytest.mark.gpu
+
+LAYOUTS = [mx.LAYOUT_1D_ROW, mx.LAYOUT_1D_COL, mx.LAYOUT_2D]
+SHAPES = {mx.LAYOUT_1D_ROW: (67, 352), mx.LAYOUT_1D_COL: (288, 136), mx.LAYOUT_2D: (96, 288)}
+
+
+def _quantize_both(x_bits, layout, rht, rnd, seed, scale_layout, offset=0, trans=False):
+    x = dev_bf16(x_bits)
+    q = mx.mxfp4_quantize(x, layout, rht, rnd, seed, offset, scale_layout, transposed_copy=trans)
+    torch.cuda.synchronize()
+    ref = oracle.quantize(x_bits, layout, rht, rnd, seed, offset, transposed_copy=trans)
+    return q, ref
+
+
+def _scales_rowmajor(q, layout, ref_scales, rows, cols):
+    s = host(q.scales)
+    if q.scale_layout == mx.SCALES_ROWMAJOR:
+        return s
+    if layout == mx.LAYOUT_2D:
+        return from_mma(s, rows, cols)      # per-row expansion of the tile scales
+    return from_mma(s, q.rows, q.k)
+
+
+@pytest.mark.parametrize("scale_layout", [mx.SCALES_ROWMAJOR, mx.SCALES_MMA])
+@pytest.mark.parametrize("rnd", [mx.ROUND_RNE, mx.ROUND_SR])
+@pytest.mark.parametrize("rht", [0, 16, 32])
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_quantize_bit_exact(layout, rht, rnd, scale_layout):
+    rows, cols = SHAPES[layout]
+    x = synth.student_t_bf16((rows, cols), seed=100 + layout * 7 + rht)
+    trans = layout == mx.LAYOUT_2D
+    q, ref = _quantize_both(x, layout, rht, rnd, 42, scale_layout, trans=trans)
+    assert np.array_equal(host(q.codes), ref[0])
+    got = _scales_rowmajor(q, layout, ref[1], rows, cols)
+    want = expand_2d(ref[1], rows) if (layout == mx.LAYOUT_2D and scale_layout == mx.SCALES_MMA) else ref[1]
+    assert np.array_equal(got, want)
+    if trans:
+        assert np.array_equal(host(q.codes_t), ref[2])
+        st = host(q.scales_t)
+        if scale_layout == mx.SCALES_ROWMAJOR:
+            assert np.array_equal(st, ref[1].T)
+        else:
+            assert np.array_equal(from_mma(st, cols, rows), expand_2d(ref[1].T, cols))
+
+
+@pytest.mark.parametrize("rht", [0, 32])
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_every_bf16_pattern(layout, rht):
+    """All 65536 bf16 bit patterns, in blocks, twice: as they come (each block
+    scaled by its own max) and with a 4.0 in every row block (scale 1)."""
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    g = np.random.default_rng(5)
+    a = g.permutation(allbits).reshape(256, 256)
+    b = a.copy()
+    b[:, ::32] = 0x4080                                   # 4.0
+    x = np.concatenate([a, b], axis=0)
+    for rnd in (mx.ROUND_RNE, mx.ROUND_SR):
+        q, ref = _quantize_both(x, layout, rht, rnd, 9, mx.SCALES_ROWMAJOR, trans=(layout == mx.LAYOUT_2D))
+        assert np.array_equal(host(q.codes), ref[0])
+        assert np.array_equal(host(q.scales), ref[1])
+        if layout == mx.LAYOUT_2D:
+            assert np.array_equal(host(q.codes_t), ref[2])
+
+
+def test_adversarial_blocks():
+    vals = np.zeros((8, 64), np.float32)
+    vals[0, :32] = 7.5; vals[0, 1] = 0.25; vals[0, 2] = -0.75; vals[0, 3] = 5.0
+    vals[1, :32] = np.linspace(-6, 6, 32)
+    vals[1, 32:] = [0.25 * i for i in range(32)]           # ties after scaling
+    vals[2, :] = 3.3895314e38                               # near bf16 max
+    vals[3, :32] = np.float32(2.0 ** -133)                  # bf16 subnormals
+    vals[3, 32:] = -0.0
+    vals[4, :] = [8.0, -8.0] * 32
+    vals[5, :32] = 6.0; vals[5, 32:] = 1e-30
+    x = synth.bf16_bits(vals)
+    x[6, 5] = 0x7FC0                                        # NaN
+    x[7, 40] = 0xFF80                                       # -Inf
+    for layout in (mx.LAYOUT_1D_ROW,):
+        for rht in (0, 16, 32):
+            for rnd in (mx.ROUND_RNE, mx.ROUND_SR):
+                q, ref = _quantize_both(x, layout, rht, rnd, 3, mx.SCALES_ROWMAJOR)
+                assert np.array_equal(host(q.codes), ref[0]), (rht, rnd)
+                assert np.array_equal(host(q.scales), ref[1]), (rht, rnd)
+
+
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_sharded_sr_equals_whole(layout):
+    rows, cols = 256, 192
+    x = synth.student_t_bf16((rows, cols), seed=77)
+    whole = mx.mxfp4_quantize(dev_bf16(x), layout, 32, mx.ROUND_SR, 42)
+    if layout == mx.LAYOUT_1D_COL:
+        pa = mx.mxfp4_quantize(dev_bf16(np.ascontiguousarray(x[:, :96])), layout, 32, mx.ROUND_SR, 42, 0)
+        pb = mx.mxfp4_quantize(dev_bf16(np.ascontiguousarray(x[:, 96:])), layout, 32, mx.ROUND_SR, 42, 96 * rows)
+    else:
+        pa = mx.mxfp4_quantize(dev_bf16(np.ascontiguousarray(x[:128])), layout, 32, mx.ROUND_SR, 42, 0)
+        pb = mx.mxfp4_quantize(dev_bf16(np.ascontiguousarray(x[128:])), layout, 32, mx.ROUND_SR, 42, 128 * cols)
+    assert torch.equal(whole.codes, torch.cat([pa.codes, pb.codes]))
+    assert torch.equal(whole.scales, torch.cat([pa.scales, pb.scales]))
+
+
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rht", [0, 16, 32])
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_dequantize_matches_oracle(layout, rht, out_dtype):
+    rows, cols = SHAPES[layout]
+    x = synth.student_t_bf16((rows, cols), seed=300 + layout)
+    codes, scales = oracle.quantize(x, layout, rht, oracle.ROUND_SR, 11)[:2]
+    scales = scales.copy()
+    scales.reshape(-1)[3] = 0xFF                            # one NaN block
+    f32, b16 = oracle.dequantize(codes, scales, rows, cols, layout, rht, 11)
+    out = mx.mxfp4_dequantize(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), rows, cols,
+                              layout, rht, 11, out_dtype=out_dtype)
+    got = host(out)
+    if out_dtype == torch.float32:
+        assert np.array_equal(np.isnan(got), np.isnan(f32))
+        ok = ~np.isnan(f32)
+        assert np.array_equal(got[ok].view(np.uint32), f32[ok].view(np.uint32))
+    else:
+        nan = np.isnan(synth.bf16_to_f32(b16))
+        assert np.array_equal(np.isnan(synth.bf16_to_f32(got)), nan)
+        assert np.array_equal(got[~nan], b16[~nan])
+
+
+def test_dequantize_mma_scales():
+    rows, cols = 200, 256
+    x = synth.normal_bf16((rows, cols), 4)
+    q = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_ROW, 0, mx.ROUND_RNE, 0, 0, mx.SCALES_MMA)
+    out = mx.mxfp4_dequantize(q.codes, q.scales, rows, cols, mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    codes, scales = oracle.quantize(x, oracle.LAYOUT_1D_ROW)
+    _, b16 = oracle.dequantize(codes, scales, rows, cols, oracle.LAYOUT_1D_ROW)
+    assert np.array_equal(host(out), b16)
+
+
+def test_invalid_arguments_are_rejected():
+    x = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(mx.MXFP4Error) as e:
+        mx.mxfp4_quantize(x[:, :48], mx.LAYOUT_1D_ROW)       # 48 not a multiple of 32
+    assert e.value.status == mx.MXFP4_ERR_INVALID_ARG
+    with pytest.raises(mx.MXFP4Error) as e:
+        mx.mxfp4_quantize(x, mx.LAYOUT_1D_ROW, rht_size=8)
+    assert e.value.status == mx.MXFP4_ERR_INVALID_ARG
+    with pytest.raises(mx.MXFP4Error) as e:
+        mx.mxfp4_quantize(x, mx.LAYOUT_1D_ROW, elem_offset=2)
+    assert e.value.status == mx.MXFP4_ERR_INVALID_ARG
