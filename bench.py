@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""bench.py -- throughput of the MXFP4 training hot path on B200.
+
+One step = the forward and backward MXFP4 pass of one GPT-OSS-20B expert
+linear layer (gate_up: hidden 2880 -> intermediate 5760, 4096 tokens) under the
+ALTO recipe ("Training an MoE LLM in MXFP4", abstract; "MXFP4" (aiwiki.ai),
+"Training with MXFP4"):
+  quantize X   1D row blocks, RNE                        [4096 x 2880]
+  quantize W   2D 32x32 blocks, RNE, + transposed copy   [5760 x 2880]
+  fprop        Y  = X  W^T   (4096 x 5760 x 2880)
+  quantize dY  1D row blocks, stochastic rounding        [4096 x 5760]
+  dgrad        dX = dY W     (4096 x 2880 x 5760, B = W^T copy)
+  quantize dY^T, X^T  1D blocks along tokens, RHT-32 (shared signs), SR / RNE
+  wgrad        dW = dY^T X   (5760 x 2880 x 4096)
+Inputs are synthetic (seeded) with the GPT-OSS-20B shapes; the data and weights
+of the pages' workloads are not available.
+
+`value` is GEMM TFLOP/s of the whole step (3 x 2*4096*5760*2880 FLOP / step
+time); per-kernel GB/s and TFLOP/s with roofline fractions are reported too.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU, weak scaling)
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MXFP4 GEMM TFLOP/s + RHT/SR quantize GB/s, % of B200 roofline"
+TOKENS, HIDDEN, INTER = synth.TOKENS, synth.HIDDEN, synth.INTERMEDIATE
+SR_SEED = synth.SR_SEED
+WORKLOAD = ("gpt-oss-20b expert gate_up linear, MXFP4 fwd+bwd (ALTO recipe): 4096 tokens, 2880->5760; "
+            "X 1D-RNE, W 2D-RNE + W^T copy, dY 1D-SR, dY^T/X^T 1D-col RHT32 (SR/RNE); fprop, dgrad, wgrad")
+GEMMS = {"fprop": (TOKENS, INTER, HIDDEN), "dgrad": (TOKENS, HIDDEN, INTER), "wgrad": (INTER, HIDDEN, TOKENS)}
+STEP_FLOPS = sum(2 * m * n * k for m, n, k in GEMMS.values())
+# algorithmic bytes per quantized element: bf16 read + E2M1 codes + one scale per 32
+Q1D_BYTES = 2 + 0.5 + 1 / 32
+Q2D_T_BYTES = 2 + 0.5 + 0.5 + 1 / 32 + 1 / 32      # 2D with transposed copy, GEMM-ready scales
+QUANT_OPS = {"quant_x_row": TOKENS * HIDDEN * Q1D_BYTES, "quant_w_2d": INTER * HIDDEN * Q2D_T_BYTES,
+             "quant_dy_row_sr": TOKENS * INTER * Q1D_BYTES, "quant_dyt_col_rht_sr": TOKENS * INTER * Q1D_BYTES,
+             "quant_xt_col_rht": TOKENS * HIDDEN * Q1D_BYTES}
+KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sus=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.dev)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the step
+# ---------------------------------------------------------------------------
+class ExpertStep:
+    """Device buffers and the enqueue order of one step (all on the current stream)."""
+
+    def __init__(self, mx, torch, x_bits, w_bits, dy_bits, device):
+        self.mx, self.torch = mx, torch
+        bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
+        self.x, self.w, self.dy = bf(x_bits), bf(w_bits), bf(dy_bits)
+        T, H, I = TOKENS, HIDDEN, INTER
+        u8 = lambda *s: torch.empty(s, dtype=torch.uint8, device=device)
+        f32 = lambda *s: torch.empty(s, dtype=torch.float32, device=device)
+        Q = mx.Quantized
+        msb = mx.mma_scales_bytes
+        self.qx = Q(u8(T, H // 2), u8(msb(T, H)), T, H, mx.LAYOUT_1D_ROW, mx.SCALES_MMA)
+        self.qw = Q(u8(I, H // 2), u8(msb(I, H)), I, H, mx.LAYOUT_2D, mx.SCALES_MMA, u8(H, I // 2), u8(msb(H, I)))
+        self.qdy = Q(u8(T, I // 2), u8(msb(T, I)), T, I, mx.LAYOUT_1D_ROW, mx.SCALES_MMA)
+        self.qdyt = Q(u8(I, T // 2), u8(msb(I, T)), I, T, mx.LAYOUT_1D_COL, mx.SCALES_MMA)
+        self.qxt = Q(u8(H, T // 2), u8(msb(H, T)), H, T, mx.LAYOUT_1D_COL, mx.SCALES_MMA)
+        self.y, self.dx, self.dw = f32(T, I), f32(T, H), f32(I, H)
+
+    def ops(self):
+        mx = self.mx
+        return [
+            ("quant_x_row", lambda: mx.mxfp4_quantize(self.x, mx.LAYOUT_1D_ROW, 0, mx.ROUND_RNE, 0, 0,
+                                                      mx.SCALES_MMA, out=self.qx)),
+            ("quant_w_2d", lambda: mx.mxfp4_quantize(self.w, mx.LAYOUT_2D, 0, mx.ROUND_RNE, 0, 0, mx.SCALES_MMA,
+                                                     out=self.qw)),
+            ("fprop", lambda: mx.mxfp4_gemm(self.qx.codes, self.qx.scales, self.qw.codes, self.qw.scales, HIDDEN,
+                                            out=self.y)),
+            ("quant_dy_row_sr", lambda: mx.mxfp4_quantize(self.dy, mx.LAYOUT_1D_ROW, 0, mx.ROUND_SR, SR_SEED, 0,
+                                                          mx.SCALES_MMA, out=self.qdy)),
+            ("dgrad", lambda: mx.mxfp4_gemm(self.qdy.codes, self.qdy.scales, self.qw.codes_t, self.qw.scales_t,
+                                            INTER, out=self.dx)),
+            ("quant_dyt_col_rht_sr", lambda: mx.mxfp4_quantize(self.dy, mx.LAYOUT_1D_COL, 32, mx.ROUND_SR,
+                                                               SR_SEED, 0, mx.SCALES_MMA, out=self.qdyt)),
+            ("quant_xt_col_rht", lambda: mx.mxfp4_quantize(self.x, mx.LAYOUT_1D_COL, 32, mx.ROUND_RNE, SR_SEED, 0,
+                                                           mx.SCALES_MMA, out=self.qxt)),
+            ("wgrad", lambda: mx.mxfp4_gemm(self.qdyt.codes, self.qdyt.scales, self.qxt.codes, self.qxt.scales,
+                                            TOKENS, out=self.dw)),
+        ]
+
+
+def rank_inputs(rank: int):
+    """Seeded synthetic inputs; rank r draws its own tokens (weak scaling)."""
+    if rank == 0:
+        x, w = synth.fprop_inputs()
+        dy = synth.backward_inputs()
+    else:
+        x = synth.activations_with_outliers(TOKENS, HIDDEN, seed=2 + 1000 * rank)
+        w = synth.normal_bf16((INTER, HIDDEN), 3, 0.02)                # weights replicated
+        dy = synth.normal_bf16((TOKENS, INTER), 4 + 1000 * rank, 1e-3)
+    return x, w, dy
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(x, w, dy, tokens: int, hidden: int, inter: int):
+    """Run the step on a sub-problem (first `tokens` tokens, first hidden/inter
+    features) through the oracle; returns (seconds, GEMM FLOPs of the sample)."""
+    import oracle
+    xs = np.ascontiguousarray(x[:tokens, :hidden])
+    ws = np.ascontiguousarray(w[:inter, :hidden])
+    dys = np.ascontiguousarray(dy[:tokens, :inter])
+    t0 = time.perf_counter()
+    cx, sx = oracle.quantize(xs, oracle.LAYOUT_1D_ROW)
+    cw, sw, cwt = oracle.quantize(ws, oracle.LAYOUT_2D, transposed_copy=True)
+    oracle.gemm(cx, sx, cw, sw, hidden, 0, 1, want_abs=False)
+    cdy, sdy = oracle.quantize(dys, oracle.LAYOUT_1D_ROW, 0, oracle.ROUND_SR, SR_SEED)
+    oracle.gemm(cdy, sdy, cwt, sw, inter, 0, 2, want_abs=False)
+    cdyt, sdyt = oracle.quantize(dys, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_SR, SR_SEED)
+    cxt, sxt = oracle.quantize(xs, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_RNE, SR_SEED)
+    oracle.gemm(cdyt, sdyt, cxt, sxt, tokens, want_abs=False)
+    dt = time.perf_counter() - t0
+    return dt, 3 * 2 * tokens * hidden * inter
+
+
+def cpu_baseline(x, w, dy):
+    import oracle
+    tokens = 64
+    dt, flops = oracle_sample(x, w, dy, tokens, HIDDEN, INTER)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"the step on {tokens} of {TOKENS} tokens (full 2880/5760 features, W quantized in full): "
+                      f"{flops / 1e9:.2f} GFLOP in {dt:.2f} s"}
+
+
+def run_reference(args, rank):
+    """Reference arm: the oracle as it stands on the host cores, each step a
+    bounded sample of the workload, sized so that the run ends in minutes."""
+    if rank != 0:
+        return 0
+    import oracle
+    x, w, dy = rank_inputs(0)
+    # calibrate on the smallest sample, then pick the sub-problem for the budget
+    budget_s = 120.0
+    n_total = args.steps + args.warmup
+    ladder = [(32, 256, 512), (32, 512, 1024), (32, 1024, 2048), (64, 1440, 2880), (64, HIDDEN, INTER)]
+    dt0, fl0 = oracle_sample(x, w, dy, *ladder[0])
+    choice = ladder[0]
+    for cand in ladder[1:]:
+        est = dt0 * (cand[0] * cand[1] * cand[2]) / (ladder[0][0] * ladder[0][1] * ladder[0][2])
+        if est * n_total <= budget_s:
+            choice = cand
+    for _ in range(args.warmup):
+        oracle_sample(x, w, dy, *choice)
+    t_sum, flops = 0.0, 0
+    for _ in range(args.steps):
+        dt, fl = oracle_sample(x, w, dy, *choice)
+        t_sum += dt
+        flops += fl
+    value = flops / t_sum / 1e12
+    sample = (f"per step the step on a {choice[0]} tokens x {choice[1]} hidden x {choice[2]} intermediate "
+              f"sub-problem of the workload ({3 * 2 * choice[0] * choice[1] * choice[2] / 1e6:.1f} MFLOP)")
+    line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000 * t_sum / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens": TOKENS, "hidden": HIDDEN, "intermediate": INTER},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-mib", type=int, default=256)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        sys.exit(run_reference(args, rank))
+
+    import torch
+    import torch.distributed as dist
+    import quantize_block_scaled_rht_b200 as mx
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=device)
+    mx.lib()
+    peaks = load_peaks()
+
+    x, w, dy = rank_inputs(rank)
+    step = ExpertStep(mx, torch, x, w, dy, device)
+    ops = step.ops()
+    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        for _, fn in ops:
+            fn()
+    torch.cuda.synchronize()
+    if mx.mxfp4_get_error() != mx.MXFP4_OK:
+        raise RuntimeError("device-side error during warm-up")
+
+    K = args.steps
+    n_ops = len(ops)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ops + 1)] for _ in range(K)]
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)   # let the sampler start before the load
+    t_wall = time.perf_counter()
+    for i in range(K):
+        flush.zero_()                                   # L2 flush between timed steps (outside the step)
+        e = evs[i]
+        e[0].record(stream)
+        for j, (_, fn) in enumerate(ops):
+            fn()
+            e[j + 1].record(stream)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    err = mx.mxfp4_get_error()
+    if err != mx.MXFP4_OK:
+        raise RuntimeError(f"device-side error in the timed region: {mx.status_string(err)}")
+
+    per_op = np.zeros((K, n_ops))
+    for i in range(K):
+        for j in range(n_ops):
+            per_op[i, j] = evs[i][j].elapsed_time(evs[i][j + 1])     # ms
+    step_ms = per_op.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = STEP_FLOPS * world / (total_ms / K / 1e3) / 1e12
+
+    # per-kernel figures (averaged over the timed launches)
+    names = [n for n, _ in ops]
+    avg_ms = per_op.mean(axis=0)
+    kernels = {}
+    gemm_ms = 0.0
+    quant_ms, quant_bytes = 0.0, 0.0
+    for j, n in enumerate(names):
+        if n in GEMMS:
+            m_, n_, k_ = GEMMS[n]
+            tf = 2 * m_ * n_ * k_ / (avg_ms[j] / 1e3) / 1e12
+            kernels[n] = {"us": avg_ms[j] * 1e3, "TFLOP/s": tf, "frac_fp4_peak": tf / (4 * peaks["bf16"])}
+            gemm_ms += avg_ms[j]
+        else:
+            gbs = QUANT_OPS[n] / (avg_ms[j] / 1e3) / 1e9
+            kernels[n] = {"us": avg_ms[j] * 1e3, "GB/s": gbs, "frac_hbm": gbs / peaks["hbm"]}
+            quant_ms += avg_ms[j]
+            quant_bytes += QUANT_OPS[n]
+    gemm_tf = STEP_FLOPS / (gemm_ms / 1e3) / 1e12
+    fp4_peak = 4 * peaks["bf16"]
+    roofline = {"bound": "tensor", "kernel": "mxfp4_gemm_kernel (fprop+dgrad+wgrad launches)",
+                "achieved": gemm_tf, "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
+                "traffic": None,
+                "peak_note": f"dense FP4 = 4 x {peaks['src']} bf16 burst ({peaks['bf16']} TFLOP/s), "
+                             "the nominal 9 : 2.25 PFLOP/s ratio"}
+    quant_gbs = quant_bytes / (quant_ms / 1e3) / 1e9
+    roofline_q = {"bound": "hbm", "kernel": "mxfp4 quantize kernels (5 launches per step)", "achieved": quant_gbs,
+                  "peak": peaks["hbm"], "unit": "GB/s", "frac": quant_gbs / peaks["hbm"], "traffic": None,
+                  "peak_note": f"{peaks['src']} copy bandwidth"}
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hx = step.x.cpu().pin_memory()
+        hw = step.w.cpu().pin_memory()
+        hdy = step.dy.cpu().pin_memory()
+        hy = torch.empty(step.y.shape, dtype=torch.float32).pin_memory()
+        hdx = torch.empty(step.dx.shape, dtype=torch.float32).pin_memory()
+        hdw = torch.empty(step.dw.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            step.x.copy_(hx, non_blocking=True)
+            step.w.copy_(hw, non_blocking=True)
+            step.dy.copy_(hdy, non_blocking=True)
+            for _, fn in ops:
+                fn()
+            hy.copy_(step.y, non_blocking=True)
+            hdx.copy_(step.dx, non_blocking=True)
+            hdw.copy_(step.dw, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = (hx.numel() + hw.numel() + hdy.numel()) * 2
+        d2h = (hy.numel() + hdx.numel() + hdw.numel()) * 4
+        e2e = {"value": STEP_FLOPS * world / (e2e_ms / args.e2e_steps / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(x, w, dy)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "mxfp4 e2m1/e8m0 operands, fp32 accumulate", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "tokens_per_gpu": TOKENS, "hidden": HIDDEN, "intermediate": INTER,
+                           "parallelism": f"dp{world} (independent tokens per rank, no collective)",
+                           "l2": f"flushed between timed steps ({args.flush_mib} MiB write, outside step events)"},
+                "roofline": roofline, "roofline_quantize": roofline_q, "kernels": kernels,
+                "quantize_GBps": quant_gbs, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": KERNELS_PER_STEP * K, "clocks": clocks, "wall_s_timed_region": t_wall}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
