@@ -8,19 +8,22 @@
 // UE8M0 scale per 32 K-elements from tensor memory, FP32 accumulators in
 // tensor memory (TMEM), 64 K-elements per instruction.
 //
-// Kernel structure (persistent, one CTA per SM, 6 warps):
-//   warp 0      TMA producer: A/B code tiles (128x256 and 192x256 E2M1,
-//               128-byte swizzle) and the matching scale atoms (bulk copies of
-//               the GEMM-ready scale layout) into a 4-stage shared-memory ring;
-//   warp 1      MMA issuer: copies the stage's scale atoms to TMEM
-//               (tcgen05.cp 32x128b.warpx4), issues 4 MMAs per stage into one
-//               of two TMEM accumulators (128 x 192 FP32 each), releases the
-//               stage with tcgen05.commit;
-//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld) -> swizzled smem ->
-//               TMA store of FP32 C, overlapping the next tile's MMAs.
+// Kernel structure: persistent, clusters of two CTAs (one per SM) that share
+// one 256 x BN output tile with the pair MMA (cta_group::2): each CTA holds 128
+// rows of A and BN/2 rows of B, so every SM streams 128 + BN/2 operand rows per
+// K step instead of 128 + BN.  Per CTA, 6 warps:
+//   warp 0      TMA producer: its A rows, its half of B and the scale atoms
+//               (A: its own 128 rows; B: all BN rows) into a 6-stage ring;
+//               every load completes on the even CTA's stage barrier;
+//   warp 1      TMEM owner; in the even CTA also the MMA issuer: scale atoms
+//               to TMEM (tcgen05.cp, both CTAs), 4 pair MMAs per stage into one
+//               of two accumulators, stage release by a commit to both CTAs;
+//   warps 2..5  epilogue: TMEM -> registers -> swizzled smem -> TMA store of
+//               this CTA's 128 rows, overlapping the next tile's MMAs, then an
+//               arrive on the even CTA's accumulator-empty barrier.
 // Every barrier wait is bounded by the GPU global timer; a wait that runs out
-// records MXFP4_ERR_TIMEOUT, raises a CTA-wide abort flag and every role
-// drains its own in-flight copies / MMAs before the CTA exits.
+// records MXFP4_ERR_TIMEOUT, raises the CTA's abort flag, and each role drains
+// what it has in flight before both CTAs meet at the final cluster barrier.
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -34,41 +37,58 @@
 
 namespace mxfp4 {
 
-constexpr int BM = 128, BN = 192, BKB = 128;          // tile rows, tile cols, K bytes per stage (256 E2M1)
-constexpr int STAGES = 4;
+constexpr int BM = 128, BKB = 128;                    // rows per CTA, K bytes per stage (256 E2M1)
 constexpr int A_BYTES = BM * BKB;                     // 16 KB
-constexpr int B_BYTES = BN * BKB;                     // 24 KB
-constexpr int SFA_BYTES = 2 * 512;                    // 2 K-atoms of 128 rows
-constexpr int SFB_BYTES = 2 * 2 * 512;                // 2 row tiles x 2 K-atoms
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;   // 44032 = 43 KB
+constexpr int SFA_BYTES = 2 * 512;                    // 2 K-atoms of this CTA's 128 rows
 constexpr int EPI_WARPS = 4;
 constexpr int EPI_BUF = 32 * 32 * 4;                  // 32 rows x 32 FP32
 constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_STRIDE = 256;                  // accumulator b at column 256 b
-constexpr uint32_t SF_COL = 192;                      // scale factors: [192, 240)
 constexpr int MAX_GROUPS = 1024;
+constexpr int MAX_STAGES = 8;
 
-// Instruction descriptor, kind::mxf4 block-scaled: A/B E2M1 (1), K-major,
-// N >> 3 at bit 17, UE8M0 scales (bit 23), M >> 4 at bit 24, scale-factor
-// byte selectors at bits 4 (B) and 29 (A).
-constexpr uint32_t IDESC_BASE = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
-                                ((uint32_t)(BM >> 4) << 24);
+// Tile configuration: a pair tile is 256 x BN; STAGES-deep smem ring per CTA.
+template <int BN_, int STAGES_>
+struct TileCfg {
+    static constexpr int BN = BN_;
+    static constexpr int STAGES = STAGES_;
+    // B scale atoms span one 128-row tile when BN = 128, two when BN = 192
+    // (a 192-column tile starts at 0 or 64 within a 128-row scale tile).
+    static constexpr int NRT = BN == 128 ? 1 : 2;
+    static constexpr int B_BYTES = (BN / 2) * BKB;    // this CTA's half of the B tile
+    static constexpr int SFB_BYTES = NRT * 2 * 512;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr uint32_t STAGE_TX = 2u * STAGE_BYTES;   // both CTAs complete on the even CTA's barrier
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+    // TMEM (per CTA): accumulators at columns 0 and 256; scale factors of two
+    // consecutive stages right after the first accumulator.
+    static constexpr uint32_t SF_COL = BN;
+    static constexpr uint32_t SF_STAGE_COLS = 8 + 8 * NRT;
+    // Instruction descriptor, kind::mxf4 block-scaled: A/B E2M1 (1), K-major,
+    // N >> 3 at bit 17, UE8M0 scales (bit 23), M >> 4 at bit 24 (M = 256 for
+    // the pair), scale-factor byte selectors at bits 4 (B) and 29 (A).
+    static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
+                                      ((uint32_t)(256 >> 4) << 24);
+    static_assert(BN == 128 || BN == 192, "tile width");
+    static_assert(STAGES <= MAX_STAGES, "stages");
+    static_assert(SF_COL + 2 * SF_STAGE_COLS <= ACC_STRIDE, "TMEM layout");
+    static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle alignment");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+using DefaultCfg = TileCfg<192, 6>;
 
 __device__ unsigned int g_error_code;
 
 __device__ __forceinline__ void record_error(unsigned int code) { atomicCAS(&g_error_code, 0u, code); }
 
 struct GemmParams {
-    const uint8_t *a_scales;
-    const uint8_t *b_scales;
     int64_t M, N, K;
     int64_t katoms;            // ceil(K / 128): scale atoms per 128-row tile
-    int64_t b_rowtiles;        // ceil(N / 128)
-    int64_t b_group_sf_bytes;  // grouped: MMA scale bytes of one expert
+    int64_t b_rowtiles;        // ceil(N / 128): 128-row scale tiles of one B operand
     float *c;
     int64_t ldc;
     const int32_t *group_offsets;
@@ -78,7 +98,7 @@ struct GemmParams {
 };
 
 struct Shared {
-    uint64_t full[STAGES], empty[STAGES];
+    uint64_t full[MAX_STAGES], empty[MAX_STAGES];
     uint64_t tmem_full[2], tmem_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -89,7 +109,8 @@ struct Shared {
 // Bounded wait: true once the phase of `parity` has completed; false if the
 // CTA aborted or the wait ran past the limit (which records the timeout and
 // aborts the CTA).  `hard` waits ignore the abort flag (used while draining).
-__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, Shared *sh, uint64_t limit, bool hard = false) {
+__device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, Shared *sh, uint64_t limit,
+                                           bool hard = false) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
@@ -107,26 +128,35 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, Share
     }
 }
 
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < ns) {
+    }
+}
+
 struct TileInfo {
-    int64_t row0;       // first A/C row
-    int rows_valid;     // rows of this tile that belong to the problem (grouped: to the group)
+    int64_t row0;       // first A/C row of this CTA's half
+    int rows_valid;     // rows of this CTA's half that belong to the problem (grouped: to the group)
     int64_t n0;         // first C column
-    int64_t b_row;      // TMA row coordinate of the first B row
-    const uint8_t *sfb; // scale base of this B operand (expert)
+    int64_t b_row;      // TMA row coordinate of the first B row of the pair tile
+    int64_t sfb_atom0;  // first scale atom row (128-row tile * katoms) of this B operand
 };
 
-template <bool GROUPED>
-__device__ __forceinline__ TileInfo get_tile(int t, const GemmParams &p, const int *cum, int tiles_n) {
+// Pair tile t -> coordinates.  Dense: M in steps of 256 (fastest), then N.
+// Grouped: group g owns cum[g+1] - cum[g] pair tiles.
+template <int BN, bool GROUPED>
+__device__ __forceinline__ TileInfo get_tile(int t, uint32_t rank, const GemmParams &p, const int *cum,
+                                             int tiles_n) {
     TileInfo ti;
     if constexpr (!GROUPED) {
-        const int tiles_m = (int)((p.M + BM - 1) / BM);
+        const int tiles_m = (int)((p.M + 255) / 256);
         const int tm = t % tiles_m, tn = t / tiles_m;
-        ti.row0 = (int64_t)tm * BM;
+        ti.row0 = (int64_t)tm * 256 + 128 * rank;
         const int64_t left = p.M - ti.row0;
-        ti.rows_valid = left < BM ? (int)left : BM;
+        ti.rows_valid = left <= 0 ? 0 : (left < BM ? (int)left : BM);
         ti.n0 = (int64_t)tn * BN;
         ti.b_row = ti.n0;
-        ti.sfb = p.b_scales;
+        ti.sfb_atom0 = 0;
     } else {
         int g = 0;
         while (g + 1 < p.num_groups && cum[g + 1] <= t) ++g;
@@ -134,20 +164,68 @@ __device__ __forceinline__ TileInfo get_tile(int t, const GemmParams &p, const i
         const int tiles_g = (cum[g + 1] - cum[g]) / tiles_n;
         const int tm = local % tiles_g, tn = local / tiles_g;
         const int64_t size = p.group_sizes[g];
-        ti.row0 = (int64_t)p.group_offsets[g] + (int64_t)tm * BM;
-        const int64_t left = size - (int64_t)tm * BM;
-        ti.rows_valid = left < BM ? (int)left : BM;
+        const int64_t r_in = (int64_t)tm * 256 + 128 * rank;
+        ti.row0 = (int64_t)p.group_offsets[g] + r_in;
+        const int64_t left = size - r_in;
+        ti.rows_valid = left <= 0 ? 0 : (left < BM ? (int)left : BM);
         ti.n0 = (int64_t)tn * BN;
         ti.b_row = (int64_t)g * p.N + ti.n0;
-        ti.sfb = p.b_scales + (int64_t)g * p.b_group_sf_bytes;
+        ti.sfb_atom0 = (int64_t)g * p.b_rowtiles * p.katoms;
     }
     return ti;
 }
 
-template <bool GROUPED>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// One K stage of the pair tile, issued by the converged MMA warp: the stage's
+// scale atoms go to tensor memory (A: NATOMS atoms of this pair's rows; B: NRT
+// 128-row tiles x NATOMS atoms), then NK MMAs of K = 64 walk the 128-byte
+// swizzled rows 32 bytes at a time.  Scale selector k & 1 picks bytes 0-1 or
+// 2-3 of each 32-bit scale word (two 32-element blocks per MMA).
+template <class Cfg, int NATOMS, int NK>
+__device__ __forceinline__ void issue_stage(uint32_t d_tmem, uint32_t st, uint32_t sfa_col, uint32_t b_shift,
+                                            bool first) {
+    constexpr int NRT = Cfg::NRT;
+    const uint32_t sfb_col = sfa_col + 8u;
+    const uint64_t sf_desc = smem_desc(st + A_BYTES + Cfg::B_BYTES, 0, 128, 0);
+#pragma unroll
+    for (int a = 0; a < NATOMS; ++a) {
+        tc_cp_32x128_warpx4_pair_elect(sfa_col + 4u * a, sf_desc + (uint64_t)((512 * a) >> 4));
+#pragma unroll
+        for (int rt = 0; rt < NRT; ++rt)
+            tc_cp_32x128_warpx4_pair_elect(sfb_col + 4u * NRT * a + 4u * rt,
+                                           sf_desc + (uint64_t)((SFA_BYTES + 1024 * rt + 512 * a) >> 4));
+    }
+    const uint64_t adesc = smem_desc(st, 16, 1024, 2);
+    const uint64_t bdesc = adesc + (uint64_t)(A_BYTES >> 4);
+#pragma unroll
+    for (int k = 0; k < NK; ++k) {
+        constexpr uint32_t sel0 = 0u, sel1 = 2u;
+        const uint32_t idesc = (k & 1) ? (Cfg::IDESC | (sel1 << 29) | (sel1 << 4)) : (Cfg::IDESC | (sel0 << 29) | sel0);
+        mma_mxf4_pair_elect(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
+                            sfa_col + 4u * (uint32_t)(k >> 1), sfb_col + 4u * NRT * (uint32_t)(k >> 1) + b_shift,
+                            (k == 0 && first) ? 0u : 1u);
+    }
+}
+
+// Partial last K stage (K not a multiple of 256): runtime atom and MMA counts.
+template <class Cfg>
+__device__ __noinline__ void issue_stage_tail(uint32_t d_tmem, uint32_t st, uint32_t sfa_col, uint32_t b_shift,
+                                              bool first, int natoms, int nk) {
+    switch (natoms * 8 + nk) {
+        case 2 * 8 + 4: issue_stage<Cfg, 2, 4>(d_tmem, st, sfa_col, b_shift, first); break;
+        case 2 * 8 + 3: issue_stage<Cfg, 2, 3>(d_tmem, st, sfa_col, b_shift, first); break;
+        case 1 * 8 + 2: issue_stage<Cfg, 1, 2>(d_tmem, st, sfa_col, b_shift, first); break;
+        case 1 * 8 + 1: issue_stage<Cfg, 1, 1>(d_tmem, st, sfa_col, b_shift, first); break;
+        default: break;   // unreachable: K % 64 == 0 gives (2,4), (2,3), (1,2) or (1,1)
+    }
+}
+
+template <class Cfg, bool GROUPED>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     mxfp4_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                      const __grid_constant__ CUtensorMap tma_c, const GemmParams p) {
+                      const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ CUtensorMap tma_sfa,
+                      const __grid_constant__ CUtensorMap tma_sfb, const GemmParams p) {
+    constexpr int BN = Cfg::BN, STAGES = Cfg::STAGES, NRT = Cfg::NRT;
+    constexpr int B_BYTES = Cfg::B_BYTES, STAGE_BYTES = Cfg::STAGE_BYTES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stage_base = smem;
@@ -156,13 +234,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __shared__ int cum[GROUPED ? MAX_GROUPS + 1 : 1];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();               // 0 = MMA issuer of the pair
+    const int pair = (int)cluster_id_x(), npairs = (int)nclusters_x();
     const int tiles_n = (int)((p.N + BN - 1) / BN);
     const int ktiles = (int)((p.K / 2 + BKB - 1) / BKB);
     const uint64_t limit = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(&sh->full[s], 1); mbar_init(&sh->empty[s], 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(&sh->tmem_full[b], 1); mbar_init(&sh->tmem_empty[b], EPI_WARPS); }
+        for (int b = 0; b < 2; ++b) { mbar_init(&sh->tmem_full[b], 1); mbar_init(&sh->tmem_empty[b], 2 * EPI_WARPS); }
         mbar_init(&sh->drain, 1);
         sh->abort = 0;
         fence_barrier_init();
@@ -170,10 +250,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         prefetch_tmap(&tma_a);
         prefetch_tmap(&tma_b);
         prefetch_tmap(&tma_c);
+        prefetch_tmap(&tma_sfa);
+        prefetch_tmap(&tma_sfb);
     }
     if (warp == 1) {
-        tmem_alloc(&sh->tmem_base, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(&sh->tmem_base, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     if constexpr (GROUPED) {
         if (threadIdx.x == 32 * 2) {
@@ -181,12 +263,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int g = 0; g < p.num_groups; ++g) {
                 cum[g] = acc;
                 const int64_t off = p.group_offsets[g], nxt = p.group_offsets[g + 1];
-                int64_t size = p.group_sizes[g];
+                const int64_t size = p.group_sizes[g];
                 int tm = 0;
-                if ((off % BM) != 0 || size < 0 || off + size > nxt) {
-                    record_error(MXFP4_ERR_INVALID_ARG);
+                if ((off % BM) != 0 || size < 0 || off + size > nxt || nxt > p.M) {
+                    if (rank == 0) record_error(MXFP4_ERR_INVALID_ARG);
                 } else {
-                    tm = (int)((size + BM - 1) / BM);
+                    tm = (int)((size + 255) / 256);
                 }
                 acc += tm * tiles_n;
             }
@@ -194,59 +276,74 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             sh->ntiles = acc;
         }
     } else {
-        if (threadIdx.x == 0) sh->ntiles = (int)((p.M + BM - 1) / BM) * tiles_n;
+        if (threadIdx.x == 0) sh->ntiles = (int)((p.M + 255) / 256) * tiles_n;
     }
+    // barriers of both CTAs initialized before any cross-CTA traffic
     __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem = sh->tmem_base;
     const int ntiles = sh->ntiles;
+    bool aborted_any = false;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            uint32_t armed = 0, armed_par = 0;   // per stage: armed at least once, parity of last arm
+        // ------------------------------------------------------------ producer (both CTAs)
+        // The whole warp runs the loop; one elected lane issues the copies.
+        const bool issuer = elect_one();
+        {
+            uint32_t armed = 0, armed_par = 0;   // even CTA: stages armed, parity of the last arm
             int s = 0;
             uint32_t ph = 0;
-            for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
-                const TileInfo ti = get_tile<GROUPED>(t, p, cum, tiles_n);
+            for (int t = pair; t < ntiles && !sh->abort; t += npairs) {
+                const TileInfo ti = get_tile<BN, GROUPED>(t, rank, p, cum, tiles_n);
                 const int64_t rt0 = ti.n0 / 128;
-                const int nrt = (rt0 + 1 < p.b_rowtiles) ? 2 : 1;
-                const uint8_t *sfa_src = p.a_scales + ((ti.row0 / 128) * p.katoms) * 512;
+                const int64_t sfa_atom = (ti.row0 / 128) * p.katoms;
                 bool ok = true;
                 for (int kt = 0; kt < ktiles; ++kt) {
                     if (!wait_phase(&sh->empty[s], ph ^ 1u, sh, limit)) { ok = false; break; }
-                    const int natoms = (int)((p.katoms - 2 * kt) < 2 ? (p.katoms - 2 * kt) : 2);
-                    const uint32_t sf_bytes = (uint32_t)natoms * 512u;
                     uint8_t *st = stage_base + s * STAGE_BYTES;
-                    mbar_arrive_expect_tx(&sh->full[s], A_BYTES + B_BYTES + sf_bytes * (1 + nrt));
-                    tma_load_2d(st, &tma_a, kt * BKB, (int32_t)ti.row0, &sh->full[s]);
-                    tma_load_2d(st + A_BYTES, &tma_b, kt * BKB, (int32_t)ti.b_row, &sh->full[s]);
-                    bulk_load(st + A_BYTES + B_BYTES, sfa_src + (int64_t)(2 * kt) * 512, sf_bytes, &sh->full[s]);
-                    for (int rt = 0; rt < nrt; ++rt)
-                        bulk_load(st + A_BYTES + B_BYTES + SFA_BYTES + rt * 1024,
-                                  ti.sfb + ((rt0 + rt) * p.katoms + 2 * kt) * 512, sf_bytes, &sh->full[s]);
-                    armed |= 1u << s;
-                    armed_par = (armed_par & ~(1u << s)) | (ph << s);
+                    const uint32_t full_leader = mapa_shared(smem_u32(&sh->full[s]), 0);
+                    if (rank == 0) {
+                        armed |= 1u << s;
+                        armed_par = (armed_par & ~(1u << s)) | (ph << s);
+                    }
+                    if (issuer) {
+                        if (rank == 0) mbar_arrive_expect_tx(&sh->full[s], Cfg::STAGE_TX);
+                        tma_load_2d_pair(st, &tma_a, kt * BKB, (int32_t)ti.row0, full_leader);
+                        tma_load_2d_pair(st + A_BYTES, &tma_b, kt * BKB, (int32_t)(ti.b_row + rank * (BN / 2)),
+                                         full_leader);
+                        tma_load_2d_pair(st + A_BYTES + B_BYTES, &tma_sfa, 0, (int32_t)(sfa_atom + 2 * kt),
+                                         full_leader);
+#pragma unroll
+                        for (int rt = 0; rt < NRT; ++rt)
+                            tma_load_2d_pair(st + A_BYTES + B_BYTES + SFA_BYTES + rt * 1024, &tma_sfb, 0,
+                                             (int32_t)(ti.sfb_atom0 + (rt0 + rt) * p.katoms + 2 * kt), full_leader);
+                    }
+                    __syncwarp();
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
             }
-            // drain: every armed stage's last load must have landed before exit
-            for (int i = 0; i < STAGES; ++i)
-                if (armed & (1u << i)) wait_phase(&sh->full[i], (armed_par >> i) & 1u, sh, limit, true);
+            if (rank == 0) {
+                // drain: the last load of every armed stage (both CTAs' bytes) has landed
+                for (int i = 0; i < STAGES; ++i)
+                    if (armed & (1u << i)) wait_phase(&sh->full[i], (armed_par >> i) & 1u, sh, limit, true);
+            }
+            if (sh->abort) aborted_any = true;
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        // The whole warp runs the loop (warp-uniform operands); one elected
+        // lane issues each tcgen05 instruction.
+        if (rank == 0) {
             bool issued = false;
             int s = 0;
             uint32_t ph = 0, kglobal = 0;
             int acc = 0;
             uint32_t acc_ph = 0;
-            for (int t = blockIdx.x; t < ntiles && !sh->abort; t += gridDim.x) {
-                const TileInfo ti = get_tile<GROUPED>(t, p, cum, tiles_n);
+            for (int t = pair; t < ntiles && !sh->abort; t += npairs) {
+                const TileInfo ti = get_tile<BN, GROUPED>(t, 0, p, cum, tiles_n);
                 const int64_t rt0 = ti.n0 / 128;
-                const int nrt = (rt0 + 1 < p.b_rowtiles) ? 2 : 1;
                 const uint32_t b_shift = (uint32_t)((ti.n0 - rt0 * 128) / 32);
                 if (!wait_phase(&sh->tmem_empty[acc], acc_ph ^ 1u, sh, limit)) break;
                 tc_fence_after();
@@ -258,49 +355,39 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const int natoms = (int)((p.katoms - 2 * kt) < 2 ? (p.katoms - 2 * kt) : 2);
                     const int64_t kleft = p.K - (int64_t)kt * 256;
                     const int nk = kleft >= 256 ? 4 : (int)(kleft / 64);
-                    const uint32_t sfa_col = SF_COL + 24u * (kglobal & 1u);
-                    const uint32_t sfb_col = sfa_col + 8u;
+                    const uint32_t sfa_col = tmem + Cfg::SF_COL + Cfg::SF_STAGE_COLS * (kglobal & 1u);
                     const uint32_t st = smem_u32(stage_base + s * STAGE_BYTES);
-                    const uint32_t sfa_s = st + A_BYTES + B_BYTES, sfb_s = sfa_s + SFA_BYTES;
-                    for (int a = 0; a < natoms; ++a) {
-                        tc_cp_32x128_warpx4(tmem + sfa_col + 4u * a, smem_desc(sfa_s + 512u * a, 0, 128, 0));
-                        for (int rt = 0; rt < nrt; ++rt)
-                            tc_cp_32x128_warpx4(tmem + sfb_col + 8u * a + 4u * rt,
-                                                smem_desc(sfb_s + 1024u * rt + 512u * a, 0, 128, 0));
-                    }
-                    const uint64_t adesc = smem_desc(st, 16, 1024, 2);
-                    const uint64_t bdesc = smem_desc(st + A_BYTES, 16, 1024, 2);
-                    for (int k = 0; k < nk; ++k) {
-                        const uint32_t sel = 2u * (uint32_t)(k & 1);
-                        const uint32_t idesc = IDESC_BASE | (sel << 29) | (sel << 4);
-                        mma_mxf4(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
-                                 tmem + sfa_col + 4u * (uint32_t)(k >> 1),
-                                 tmem + sfb_col + 8u * (uint32_t)(k >> 1) + b_shift, (kt | k) != 0);
-                    }
+                    if (natoms == 2 && nk == 4)
+                        issue_stage<Cfg, 2, 4>(d_tmem, st, sfa_col, b_shift, kt == 0);
+                    else
+                        issue_stage_tail<Cfg>(d_tmem, st, sfa_col, b_shift, kt == 0, natoms, nk);
                     issued = true;
-                    tc_commit(&sh->empty[s]);
+                    tc_commit_pair_elect(&sh->empty[s]);
                     ++kglobal;
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
                 }
                 if (!ok) break;
-                tc_commit(&sh->tmem_full[acc]);
+                tc_commit_pair_elect(&sh->tmem_full[acc]);
                 if (++acc == 2) { acc = 0; acc_ph ^= 1u; }
             }
             if (issued) {
-                // drain: all MMAs / copies of this thread complete before TMEM is freed
-                tc_commit(&sh->drain);
+                // drain: all MMAs / copies of this thread complete before TMEM or smem go away
+                tc_commit_pair_elect(&sh->drain);
                 wait_phase(&sh->drain, 0, sh, limit, true);
             }
+            if (sh->abort) aborted_any = true;
         }
     } else {
-        // ------------------------------------------------------------ epilogue
+        // ------------------------------------------------------------ epilogue (both CTAs)
         const int q = warp & 3;                 // TMEM lane quarter of this warp
         const int ew = warp - 2;                // epilogue warp index
+        const uint32_t empty_leader0 = mapa_shared(smem_u32(&sh->tmem_empty[0]), 0);
+        const uint32_t empty_leader1 = mapa_shared(smem_u32(&sh->tmem_empty[1]), 0);
         int acc = 0;
         uint32_t acc_ph = 0;
         uint32_t buf_i = 0;
-        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-            const TileInfo ti = get_tile<GROUPED>(t, p, cum, tiles_n);
+        for (int t = pair; t < ntiles; t += npairs) {
+            const TileInfo ti = get_tile<BN, GROUPED>(t, rank, p, cum, tiles_n);
             if (!wait_phase(&sh->tmem_full[acc], acc_ph, sh, limit)) break;
             tc_fence_after();
             const int row_lo = 32 * q;
@@ -313,7 +400,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 if (j == BN / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sh->tmem_empty[acc]);
+                    if (lane == 0) mbar_arrive_cluster(acc ? empty_leader1 : empty_leader0);
                 }
                 if (!any_row) continue;
                 const int64_t col0 = ti.n0 + 32 * j;
@@ -356,11 +443,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();
+        if (sh->abort) aborted_any = true;
     }
+    // After an abort, loads issued by this CTA may still be landing in its
+    // shared memory with nobody waiting for them: give them time to finish.
+    if (aborted_any) spin_ns(200000);
     __syncthreads();
+    cluster_sync();   // neither CTA leaves while the pair may still touch its smem or TMEM
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc_pair(tmem, TMEM_COLS);
     }
 }
 
@@ -405,16 +497,15 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
-                     uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+                     uint64_t stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {stride_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 static int sm_count() {
@@ -424,64 +515,76 @@ static int sm_count() {
     return n > 0 ? n : 148;
 }
 
-template <bool GROUPED>
+template <class Cfg, bool GROUPED>
 static cudaError_t set_smem_attr() {
-    // per device: cudaFuncSetAttribute is cheap, but keep it off the hot path
+    // once per device and instantiation: keep cudaFuncSetAttribute off the hot path
     static int done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<GROUPED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<Cfg, GROUPED>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
     return e;
 }
 
+struct GemmArgs {
+    const uint8_t *a_codes, *a_scales, *b_codes, *b_scales;
+    int64_t lda, ldb, M, N, K, ldc;
+    float *c;
+    const int32_t *offsets, *sizes;
+    int G;
+};
+
 // Returns 0 on success, MXFP4_ERR_CUDA when a map or launch fails.
+template <class Cfg, bool GROUPED>
+static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
+    constexpr int BN = Cfg::BN;
+    const int G = GROUPED ? g.G : 1;
+    const int64_t katoms = mma_katoms(g.K);
+    const int64_t a_tiles = (g.M + 127) / 128, b_tiles = (g.N + 127) / 128;
+    CUtensorMap ta, tb, tc, tsa, tsb;
+    if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a_codes, (uint64_t)(g.K / 2), (uint64_t)g.M,
+                  (uint64_t)g.lda, BKB, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b_codes, (uint64_t)(g.K / 2), (uint64_t)G * g.N,
+                  (uint64_t)g.ldb, BKB, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.c, (uint64_t)g.N, (uint64_t)g.M, (uint64_t)g.ldc * 4, 32,
+                  32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        // scale atoms: rows of 512 bytes (128 x 32-bit), two consecutive atoms per load
+        !make_map(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.a_scales, 128, (uint64_t)(a_tiles * katoms), 512, 128, 2,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b_scales, 128, (uint64_t)(G * b_tiles * katoms), 512, 128,
+                  2, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return MXFP4_ERR_CUDA;
+    if (set_smem_attr<Cfg, GROUPED>() != cudaSuccess) return MXFP4_ERR_CUDA;
+    GemmParams p{};
+    p.M = g.M; p.N = g.N; p.K = g.K;
+    p.katoms = katoms;
+    p.b_rowtiles = b_tiles;
+    p.c = g.c; p.ldc = g.ldc;
+    p.group_offsets = g.offsets; p.group_sizes = g.sizes; p.num_groups = g.G;
+    p.wait_limit_ns = g_wait_limit_ns;
+    const int pairs_max = sm_count() / 2;
+    int pairs = pairs_max;
+    if (!GROUPED) {
+        const int64_t tiles = ((g.M + 255) / 256) * ((g.N + BN - 1) / BN);
+        pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
+    }
+    mxfp4_gemm_kernel<Cfg, GROUPED><<<(unsigned)(2 * pairs), NUM_THREADS, Cfg::SMEM_BYTES, s>>>(ta, tb, tc, tsa, tsb, p);
+    return cudaGetLastError() == cudaSuccess ? 0 : MXFP4_ERR_CUDA;
+}
+
 int launch_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes, int64_t ldb,
                 const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s) {
-    CUtensorMap ta, tb, tc;
-    if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)(K / 2), (uint64_t)M, (uint64_t)lda, BKB, BM) ||
-        !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)ldb, BKB, BN) ||
-        !make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c, (uint64_t)N, (uint64_t)M, (uint64_t)ldc * 4, 32, 32))
-        return MXFP4_ERR_CUDA;
-    if (set_smem_attr<false>() != cudaSuccess) return MXFP4_ERR_CUDA;
-    GemmParams p{};
-    p.a_scales = a_scales; p.b_scales = b_scales;
-    p.M = M; p.N = N; p.K = K;
-    p.katoms = mma_katoms(K);
-    p.b_rowtiles = (N + 127) / 128;
-    p.c = c; p.ldc = ldc;
-    p.wait_limit_ns = g_wait_limit_ns;
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const int sms = sm_count();
-    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    mxfp4_gemm_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tc, p);
-    return cudaGetLastError() == cudaSuccess ? 0 : MXFP4_ERR_CUDA;
+    GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, M, N, K, ldc, c, nullptr, nullptr, 1};
+    return launch_cfg<DefaultCfg, false>(g, s);
 }
 
 int launch_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
                         const int32_t *offsets, const int32_t *sizes, int G, const uint8_t *b_codes, int64_t ldb,
                         const uint8_t *b_scales, int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s) {
-    CUtensorMap ta, tb, tc;
-    if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)(K / 2), (uint64_t)a_rows, (uint64_t)lda, BKB,
-                  BM) ||
-        !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, b_codes, (uint64_t)(K / 2), (uint64_t)(G * N), (uint64_t)ldb,
-                  BKB, BN) ||
-        !make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, c, (uint64_t)N, (uint64_t)a_rows, (uint64_t)ldc * 4, 32, 32))
-        return MXFP4_ERR_CUDA;
-    if (set_smem_attr<true>() != cudaSuccess) return MXFP4_ERR_CUDA;
-    GemmParams p{};
-    p.a_scales = a_scales; p.b_scales = b_scales;
-    p.M = a_rows; p.N = N; p.K = K;
-    p.katoms = mma_katoms(K);
-    p.b_rowtiles = (N + 127) / 128;
-    p.b_group_sf_bytes = ((N + 127) / 128) * p.katoms * 512;
-    p.c = c; p.ldc = ldc;
-    p.group_offsets = offsets; p.group_sizes = sizes; p.num_groups = G;
-    p.wait_limit_ns = g_wait_limit_ns;
-    mxfp4_gemm_kernel<true><<<(unsigned)sm_count(), NUM_THREADS, SMEM_BYTES, s>>>(ta, tb, tc, p);
-    return cudaGetLastError() == cudaSuccess ? 0 : MXFP4_ERR_CUDA;
+    GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, a_rows, N, K, ldc, c, offsets, sizes, G};
+    return launch_cfg<DefaultCfg, true>(g, s);
 }
 
 int get_error(cudaStream_t s) {
