@@ -37,49 +37,57 @@
 
 namespace mxfp4 {
 
-constexpr int BM = 128, BKB = 128;                    // rows per CTA, K bytes per stage (256 E2M1)
-constexpr int A_BYTES = BM * BKB;                     // 16 KB
-constexpr int SFA_BYTES = 2 * 512;                    // 2 K-atoms of this CTA's 128 rows
+constexpr int BM = 128;                               // rows per CTA
+constexpr int CHUNK = 128;                            // K bytes per swizzled chunk (256 E2M1 = 8 scale blocks)
 constexpr int EPI_WARPS = 4;
 constexpr int EPI_BUF = 32 * 32 * 4;                  // 32 rows x 32 FP32
 constexpr int EPI_BYTES = EPI_WARPS * 2 * EPI_BUF;
 constexpr int BAR_BYTES = 256;
 constexpr int NUM_THREADS = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC_STRIDE = 256;                  // accumulator b at column 256 b
 constexpr int MAX_GROUPS = 1024;
 constexpr int MAX_STAGES = 8;
 
-// Tile configuration: a pair tile is 256 x BN; STAGES-deep smem ring per CTA.
-template <int BN_, int STAGES_>
+// Tile configuration: a pair tile is 256 x BN; each stage of the STAGES-deep
+// smem ring holds KCH chunks of K (KCH * 256 E2M1 elements, 4 * KCH MMAs).
+template <int BN_, int STAGES_, int KCH_>
 struct TileCfg {
     static constexpr int BN = BN_;
     static constexpr int STAGES = STAGES_;
+    static constexpr int KCH = KCH_;
+    static constexpr int KSTEP = 256 * KCH;           // E2M1 elements of K per stage
+    static constexpr int NATOM = 2 * KCH;             // 4-block scale atoms per row tile per stage
     // B scale atoms span one 128-row tile when BN = 128, two when BN = 192
     // (a 192-column tile starts at 0 or 64 within a 128-row scale tile).
     static constexpr int NRT = BN == 128 ? 1 : 2;
-    static constexpr int B_BYTES = (BN / 2) * BKB;    // this CTA's half of the B tile
-    static constexpr int SFB_BYTES = NRT * 2 * 512;
+    static constexpr int A_CHUNK = BM * CHUNK;               // 16 KB per chunk
+    static constexpr int B_CHUNK = (BN / 2) * CHUNK;         // this CTA's half of the B tile
+    static constexpr int A_BYTES = KCH * A_CHUNK;
+    static constexpr int B_BYTES = KCH * B_CHUNK;
+    static constexpr int SFA_BYTES = NATOM * 512;
+    static constexpr int SFB_BYTES = NRT * NATOM * 512;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr uint32_t STAGE_TX = 2u * STAGE_BYTES;   // both CTAs complete on the even CTA's barrier
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
-    // TMEM (per CTA): accumulators at columns 0 and 256; scale factors of two
-    // consecutive stages right after the first accumulator.
+    // TMEM columns (per CTA): accumulator 0 at [0, BN), the scale factors of
+    // two consecutive stages after it, accumulator 1 at the top.
     static constexpr uint32_t SF_COL = BN;
-    static constexpr uint32_t SF_STAGE_COLS = 8 + 8 * NRT;
+    static constexpr uint32_t SF_STAGE_COLS = 4 * NATOM * (1 + NRT);
+    static constexpr uint32_t ACC1_COL = TMEM_COLS - BN;
     // Instruction descriptor, kind::mxf4 block-scaled: A/B E2M1 (1), K-major,
     // N >> 3 at bit 17, UE8M0 scales (bit 23), M >> 4 at bit 24 (M = 256 for
     // the pair), scale-factor byte selectors at bits 4 (B) and 29 (A).
     static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
                                       ((uint32_t)(256 >> 4) << 24);
     static_assert(BN == 128 || BN == 192, "tile width");
+    static_assert(KCH == 1 || KCH == 2, "chunks per stage");
     static_assert(STAGES <= MAX_STAGES, "stages");
-    static_assert(SF_COL + 2 * SF_STAGE_COLS <= ACC_STRIDE, "TMEM layout");
-    static_assert(STAGE_BYTES % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle alignment");
+    static_assert(SF_COL + 2 * SF_STAGE_COLS <= ACC1_COL, "TMEM layout");
+    static_assert(A_CHUNK % 1024 == 0 && B_CHUNK % 1024 == 0 && STAGE_BYTES % 1024 == 0, "swizzle alignment");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
-using DefaultCfg = TileCfg<192, 6>;
+using DefaultCfg = TileCfg<192, 3, 2>;
 
 __device__ unsigned int g_error_code;
 
@@ -139,7 +147,7 @@ struct TileInfo {
     int rows_valid;     // rows of this CTA's half that belong to the problem (grouped: to the group)
     int64_t n0;         // first C column
     int64_t b_row;      // TMA row coordinate of the first B row of the pair tile
-    int64_t sfb_atom0;  // first scale atom row (128-row tile * katoms) of this B operand
+    int64_t sfb_rt_base;  // first 128-row scale tile of this B operand (expert)
 };
 
 // Pair tile t -> coordinates.  Dense: M in steps of 256 (fastest), then N.
@@ -156,7 +164,7 @@ __device__ __forceinline__ TileInfo get_tile(int t, uint32_t rank, const GemmPar
         ti.rows_valid = left <= 0 ? 0 : (left < BM ? (int)left : BM);
         ti.n0 = (int64_t)tn * BN;
         ti.b_row = ti.n0;
-        ti.sfb_atom0 = 0;
+        ti.sfb_rt_base = 0;
     } else {
         int g = 0;
         while (g + 1 < p.num_groups && cum[g + 1] <= t) ++g;
@@ -170,7 +178,7 @@ __device__ __forceinline__ TileInfo get_tile(int t, uint32_t rank, const GemmPar
         ti.rows_valid = left <= 0 ? 0 : (left < BM ? (int)left : BM);
         ti.n0 = (int64_t)tn * BN;
         ti.b_row = (int64_t)g * p.N + ti.n0;
-        ti.sfb_atom0 = (int64_t)g * p.b_rowtiles * p.katoms;
+        ti.sfb_rt_base = (int64_t)g * p.b_rowtiles;
     }
     return ti;
 }
@@ -178,44 +186,49 @@ __device__ __forceinline__ TileInfo get_tile(int t, uint32_t rank, const GemmPar
 // One K stage of the pair tile, issued by the converged MMA warp: the stage's
 // scale atoms go to tensor memory (A: NATOMS atoms of this pair's rows; B: NRT
 // 128-row tiles x NATOMS atoms), then NK MMAs of K = 64 walk the 128-byte
-// swizzled rows 32 bytes at a time.  Scale selector k & 1 picks bytes 0-1 or
-// 2-3 of each 32-bit scale word (two 32-element blocks per MMA).
+// swizzled chunk rows 32 bytes at a time (4 MMAs per chunk).  The scale
+// selector k & 1 picks bytes 0-1 or 2-3 of each 32-bit scale word (two
+// 32-element blocks per MMA); k >> 1 steps to the next 4-block atom.
 template <class Cfg, int NATOMS, int NK>
 __device__ __forceinline__ void issue_stage(uint32_t d_tmem, uint32_t st, uint32_t sfa_col, uint32_t b_shift,
                                             bool first) {
-    constexpr int NRT = Cfg::NRT;
-    const uint32_t sfb_col = sfa_col + 8u;
-    const uint64_t sf_desc = smem_desc(st + A_BYTES + Cfg::B_BYTES, 0, 128, 0);
+    constexpr int NRT = Cfg::NRT, NATOM = Cfg::NATOM;
+    const uint32_t sfb_col = sfa_col + 4u * NATOM;
+    const uint64_t sf_desc = smem_desc(st + Cfg::A_BYTES + Cfg::B_BYTES, 0, 128, 0);
 #pragma unroll
     for (int a = 0; a < NATOMS; ++a) {
         tc_cp_32x128_warpx4_pair_elect(sfa_col + 4u * a, sf_desc + (uint64_t)((512 * a) >> 4));
 #pragma unroll
         for (int rt = 0; rt < NRT; ++rt)
             tc_cp_32x128_warpx4_pair_elect(sfb_col + 4u * NRT * a + 4u * rt,
-                                           sf_desc + (uint64_t)((SFA_BYTES + 1024 * rt + 512 * a) >> 4));
+                                           sf_desc + (uint64_t)((Cfg::SFA_BYTES + NATOM * 512 * rt + 512 * a) >> 4));
     }
     const uint64_t adesc = smem_desc(st, 16, 1024, 2);
-    const uint64_t bdesc = adesc + (uint64_t)(A_BYTES >> 4);
+    const uint64_t bdesc = smem_desc(st + Cfg::A_BYTES, 16, 1024, 2);
 #pragma unroll
     for (int k = 0; k < NK; ++k) {
-        constexpr uint32_t sel0 = 0u, sel1 = 2u;
-        const uint32_t idesc = (k & 1) ? (Cfg::IDESC | (sel1 << 29) | (sel1 << 4)) : (Cfg::IDESC | (sel0 << 29) | sel0);
-        mma_mxf4_pair_elect(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc,
-                            sfa_col + 4u * (uint32_t)(k >> 1), sfb_col + 4u * NRT * (uint32_t)(k >> 1) + b_shift,
-                            (k == 0 && first) ? 0u : 1u);
+        const uint32_t idesc = (k & 1) ? (Cfg::IDESC | (2u << 29) | (2u << 4)) : Cfg::IDESC;
+        const uint64_t a_off = (uint64_t)(((k >> 2) * Cfg::A_CHUNK + (k & 3) * 32) >> 4);
+        const uint64_t b_off = (uint64_t)(((k >> 2) * Cfg::B_CHUNK + (k & 3) * 32) >> 4);
+        mma_mxf4_pair_elect(d_tmem, adesc + a_off, bdesc + b_off, idesc, sfa_col + 4u * (uint32_t)(k >> 1),
+                            sfb_col + 4u * NRT * (uint32_t)(k >> 1) + b_shift, (k == 0 && first) ? 0u : 1u);
     }
 }
 
-// Partial last K stage (K not a multiple of 256): runtime atom and MMA counts.
+// Partial last K stage (K not a multiple of the stage depth): NK = kleft / 64
+// MMAs and ceil(NK / 2) scale atoms.
 template <class Cfg>
 __device__ __noinline__ void issue_stage_tail(uint32_t d_tmem, uint32_t st, uint32_t sfa_col, uint32_t b_shift,
-                                              bool first, int natoms, int nk) {
-    switch (natoms * 8 + nk) {
-        case 2 * 8 + 4: issue_stage<Cfg, 2, 4>(d_tmem, st, sfa_col, b_shift, first); break;
-        case 2 * 8 + 3: issue_stage<Cfg, 2, 3>(d_tmem, st, sfa_col, b_shift, first); break;
-        case 1 * 8 + 2: issue_stage<Cfg, 1, 2>(d_tmem, st, sfa_col, b_shift, first); break;
-        case 1 * 8 + 1: issue_stage<Cfg, 1, 1>(d_tmem, st, sfa_col, b_shift, first); break;
-        default: break;   // unreachable: K % 64 == 0 gives (2,4), (2,3), (1,2) or (1,1)
+                                              bool first, int nk) {
+    switch (nk) {
+        case 1: issue_stage<Cfg, 1, 1>(d_tmem, st, sfa_col, b_shift, first); break;
+        case 2: issue_stage<Cfg, 1, 2>(d_tmem, st, sfa_col, b_shift, first); break;
+        case 3: issue_stage<Cfg, 2, 3>(d_tmem, st, sfa_col, b_shift, first); break;
+        case 4: issue_stage<Cfg, 2, 4>(d_tmem, st, sfa_col, b_shift, first); break;
+        case 5: issue_stage<Cfg, 3, 5>(d_tmem, st, sfa_col, b_shift, first); break;
+        case 6: issue_stage<Cfg, 3, 6>(d_tmem, st, sfa_col, b_shift, first); break;
+        case 7: issue_stage<Cfg, 4, 7>(d_tmem, st, sfa_col, b_shift, first); break;
+        default: break;   // a full stage never takes this path
     }
 }
 
@@ -225,7 +238,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                       const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ CUtensorMap tma_sfa,
                       const __grid_constant__ CUtensorMap tma_sfb, const GemmParams p) {
     constexpr int BN = Cfg::BN, STAGES = Cfg::STAGES, NRT = Cfg::NRT;
-    constexpr int B_BYTES = Cfg::B_BYTES, STAGE_BYTES = Cfg::STAGE_BYTES;
+    constexpr int A_BYTES = Cfg::A_BYTES, B_BYTES = Cfg::B_BYTES, SFA_BYTES = Cfg::SFA_BYTES;
+    constexpr int STAGE_BYTES = Cfg::STAGE_BYTES, KCH = Cfg::KCH, NATOM = Cfg::NATOM;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stage_base = smem;
@@ -237,7 +251,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     const uint32_t rank = cluster_ctarank();               // 0 = MMA issuer of the pair
     const int pair = (int)cluster_id_x(), npairs = (int)nclusters_x();
     const int tiles_n = (int)((p.N + BN - 1) / BN);
-    const int ktiles = (int)((p.K / 2 + BKB - 1) / BKB);
+    const int ktiles = (int)((p.K + Cfg::KSTEP - 1) / Cfg::KSTEP);
     const uint64_t limit = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
@@ -296,8 +310,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             uint32_t ph = 0;
             for (int t = pair; t < ntiles && !sh->abort; t += npairs) {
                 const TileInfo ti = get_tile<BN, GROUPED>(t, rank, p, cum, tiles_n);
-                const int64_t rt0 = ti.n0 / 128;
-                const int64_t sfa_atom = (ti.row0 / 128) * p.katoms;
+                const int32_t sfa_rt = (int32_t)(ti.row0 / 128);
+                const int32_t sfb_rt = (int32_t)(ti.sfb_rt_base + ti.n0 / 128);
                 bool ok = true;
                 for (int kt = 0; kt < ktiles; ++kt) {
                     if (!wait_phase(&sh->empty[s], ph ^ 1u, sh, limit)) { ok = false; break; }
@@ -309,15 +323,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     }
                     if (issuer) {
                         if (rank == 0) mbar_arrive_expect_tx(&sh->full[s], Cfg::STAGE_TX);
-                        tma_load_2d_pair(st, &tma_a, kt * BKB, (int32_t)ti.row0, full_leader);
-                        tma_load_2d_pair(st + A_BYTES, &tma_b, kt * BKB, (int32_t)(ti.b_row + rank * (BN / 2)),
-                                         full_leader);
-                        tma_load_2d_pair(st + A_BYTES + B_BYTES, &tma_sfa, 0, (int32_t)(sfa_atom + 2 * kt),
-                                         full_leader);
 #pragma unroll
-                        for (int rt = 0; rt < NRT; ++rt)
-                            tma_load_2d_pair(st + A_BYTES + B_BYTES + SFA_BYTES + rt * 1024, &tma_sfb, 0,
-                                             (int32_t)(ti.sfb_atom0 + (rt0 + rt) * p.katoms + 2 * kt), full_leader);
+                        for (int c = 0; c < KCH; ++c) {
+                            const int32_t kx = (kt * KCH + c) * CHUNK;
+                            tma_load_2d_pair(st + c * Cfg::A_CHUNK, &tma_a, kx, (int32_t)ti.row0, full_leader);
+                            tma_load_2d_pair(st + A_BYTES + c * Cfg::B_CHUNK, &tma_b, kx,
+                                             (int32_t)(ti.b_row + rank * (BN / 2)), full_leader);
+                        }
+                        // scale atoms: NATOM consecutive K atoms of one (A) or NRT (B) 128-row tiles
+                        tma_load_3d_pair(st + A_BYTES + B_BYTES, &tma_sfa, 0, kt * NATOM, sfa_rt, full_leader);
+                        tma_load_3d_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &tma_sfb, 0, kt * NATOM, sfb_rt,
+                                         full_leader);
                     }
                     __syncwarp();
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -347,20 +363,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const uint32_t b_shift = (uint32_t)((ti.n0 - rt0 * 128) / 32);
                 if (!wait_phase(&sh->tmem_empty[acc], acc_ph ^ 1u, sh, limit)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)acc * ACC_STRIDE;
+                const uint32_t d_tmem = tmem + (acc ? Cfg::ACC1_COL : 0u);
                 bool ok = true;
                 for (int kt = 0; kt < ktiles; ++kt) {
                     if (!wait_phase(&sh->full[s], ph, sh, limit)) { ok = false; break; }
                     tc_fence_after();
-                    const int natoms = (int)((p.katoms - 2 * kt) < 2 ? (p.katoms - 2 * kt) : 2);
-                    const int64_t kleft = p.K - (int64_t)kt * 256;
-                    const int nk = kleft >= 256 ? 4 : (int)(kleft / 64);
+                    const int64_t kleft = p.K - (int64_t)kt * Cfg::KSTEP;
                     const uint32_t sfa_col = tmem + Cfg::SF_COL + Cfg::SF_STAGE_COLS * (kglobal & 1u);
                     const uint32_t st = smem_u32(stage_base + s * STAGE_BYTES);
-                    if (natoms == 2 && nk == 4)
-                        issue_stage<Cfg, 2, 4>(d_tmem, st, sfa_col, b_shift, kt == 0);
+                    if (kleft >= Cfg::KSTEP)
+                        issue_stage<Cfg, NATOM, 4 * KCH>(d_tmem, st, sfa_col, b_shift, kt == 0);
                     else
-                        issue_stage_tail<Cfg>(d_tmem, st, sfa_col, b_shift, kt == 0, natoms, nk);
+                        issue_stage_tail<Cfg>(d_tmem, st, sfa_col, b_shift, kt == 0, (int)(kleft / 64));
                     issued = true;
                     tc_commit_pair_elect(&sh->empty[s]);
                     ++kglobal;
@@ -395,7 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const bool any_row = row_lo < ti.rows_valid;
             for (int j = 0; j < BN / 32; ++j) {
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)acc * ACC_STRIDE + 32u * j, v);
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (acc ? Cfg::ACC1_COL : 0u) + 32u * j, v);
                 tmem_ld_wait();
                 if (j == BN / 32 - 1) {
                     tc_fence_before();
@@ -508,6 +522,21 @@ static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, u
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Scale atoms of the GEMM-ready layout: 512-byte atoms, katoms per 128-row
+// tile, `tiles` row tiles; boxes of `box_k` atoms x `box_t` tiles.
+static bool make_map_3d(CUtensorMap *m, const void *base, uint64_t katoms, uint64_t tiles, uint32_t box_k,
+                        uint32_t box_t) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {128, katoms, tiles};
+    const cuuint64_t strides[2] = {512, 512 * katoms};
+    const cuuint32_t box[3] = {128, box_k, box_t};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int sm_count() {
     int dev = 0, n = 0;
     cudaGetDevice(&dev);
@@ -545,16 +574,15 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
     const int64_t a_tiles = (g.M + 127) / 128, b_tiles = (g.N + 127) / 128;
     CUtensorMap ta, tb, tc, tsa, tsb;
     if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a_codes, (uint64_t)(g.K / 2), (uint64_t)g.M,
-                  (uint64_t)g.lda, BKB, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                  (uint64_t)g.lda, CHUNK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b_codes, (uint64_t)(g.K / 2), (uint64_t)G * g.N,
-                  (uint64_t)g.ldb, BKB, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                  (uint64_t)g.ldb, CHUNK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.c, (uint64_t)g.N, (uint64_t)g.M, (uint64_t)g.ldc * 4, 32,
                   32, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        // scale atoms: rows of 512 bytes (128 x 32-bit), two consecutive atoms per load
-        !make_map(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.a_scales, 128, (uint64_t)(a_tiles * katoms), 512, 128, 2,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.b_scales, 128, (uint64_t)(G * b_tiles * katoms), 512, 128,
-                  2, CU_TENSOR_MAP_SWIZZLE_NONE))
+        // scale atoms as a 3D tensor [128-row tile][K atom][512 bytes = 128 x 32-bit]:
+        // one box holds NATOM consecutive atoms of one (A) or NRT (B) row tiles
+        !make_map_3d(&tsa, g.a_scales, (uint64_t)katoms, (uint64_t)a_tiles, Cfg::NATOM, 1) ||
+        !make_map_3d(&tsb, g.b_scales, (uint64_t)katoms, (uint64_t)(G * b_tiles), Cfg::NATOM, Cfg::NRT))
         return MXFP4_ERR_CUDA;
     if (set_smem_attr<Cfg, GROUPED>() != cudaSuccess) return MXFP4_ERR_CUDA;
     GemmParams p{};
