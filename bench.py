@@ -5,12 +5,13 @@ One step = the forward and backward MXFP4 pass of one GPT-OSS-20B expert
 linear layer (gate_up: hidden 2880 -> intermediate 5760, 4096 tokens) under the
 ALTO recipe ("Training an MoE LLM in MXFP4", abstract; "MXFP4" (aiwiki.ai),
 "Training with MXFP4"):
-  quantize X   1D row blocks, RNE                        [4096 x 2880]
-  quantize W   2D 32x32 blocks, RNE, + transposed copy   [5760 x 2880]
+  quantize X   one read: 1D row blocks (RNE) and 1D blocks along tokens with
+               RHT-32 (RNE)                                [4096 x 2880]
+  quantize W   2D 32x32 blocks, RNE, + transposed copy     [5760 x 2880]
   fprop        Y  = X  W^T   (4096 x 5760 x 2880)
-  quantize dY  1D row blocks, stochastic rounding        [4096 x 5760]
+  quantize dY  one read: 1D row blocks with stochastic rounding and 1D blocks
+               along tokens with RHT-32 (same signs as X) + SR  [4096 x 5760]
   dgrad        dX = dY W     (4096 x 2880 x 5760, B = W^T copy)
-  quantize dY^T, X^T  1D blocks along tokens, RHT-32 (shared signs), SR / RNE
   wgrad        dW = dY^T X   (5760 x 2880 x 4096)
 Inputs are synthetic (seeded) with the GPT-OSS-20B shapes; the data and weights
 of the pages' workloads are not available.
@@ -49,9 +50,10 @@ STEP_FLOPS = sum(2 * m * n * k for m, n, k in GEMMS.values())
 # algorithmic bytes per quantized element: bf16 read + E2M1 codes + one scale per 32
 Q1D_BYTES = 2 + 0.5 + 1 / 32
 Q2D_T_BYTES = 2 + 0.5 + 0.5 + 1 / 32 + 1 / 32      # 2D with transposed copy, GEMM-ready scales
-QUANT_OPS = {"quant_x_row": TOKENS * HIDDEN * Q1D_BYTES, "quant_w_2d": INTER * HIDDEN * Q2D_T_BYTES,
-             "quant_dy_row_sr": TOKENS * INTER * Q1D_BYTES, "quant_dyt_col_rht_sr": TOKENS * INTER * Q1D_BYTES,
-             "quant_xt_col_rht": TOKENS * HIDDEN * Q1D_BYTES}
+# dual quantizers: one bf16 read, two sets of codes and GEMM-ready scales
+QDUAL_BYTES = 2 + 2 * (0.5 + 1 / 32)
+QUANT_OPS = {"quant_x_dual": TOKENS * HIDDEN * QDUAL_BYTES, "quant_w_2d": INTER * HIDDEN * Q2D_T_BYTES,
+             "quant_dy_dual_sr": TOKENS * INTER * QDUAL_BYTES}
 KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 
 
@@ -140,20 +142,18 @@ class ExpertStep:
     def ops(self):
         mx = self.mx
         return [
-            ("quant_x_row", lambda: mx.mxfp4_quantize(self.x, mx.LAYOUT_1D_ROW, 0, mx.ROUND_RNE, 0, 0,
-                                                      mx.SCALES_MMA, out=self.qx)),
+            # X: row blocks (fprop) and blocks along tokens with RHT-32 (wgrad), one read
+            ("quant_x_dual", lambda: mx.mxfp4_quantize_dual(self.x, 32, mx.ROUND_RNE, SR_SEED, 0, 0, mx.SCALES_MMA,
+                                                            out_row=self.qx, out_col=self.qxt)),
             ("quant_w_2d", lambda: mx.mxfp4_quantize(self.w, mx.LAYOUT_2D, 0, mx.ROUND_RNE, 0, 0, mx.SCALES_MMA,
                                                      out=self.qw)),
             ("fprop", lambda: mx.mxfp4_gemm(self.qx.codes, self.qx.scales, self.qw.codes, self.qw.scales, HIDDEN,
                                             out=self.y)),
-            ("quant_dy_row_sr", lambda: mx.mxfp4_quantize(self.dy, mx.LAYOUT_1D_ROW, 0, mx.ROUND_SR, SR_SEED, 0,
-                                                          mx.SCALES_MMA, out=self.qdy)),
+            # dY: row blocks with SR (dgrad) and blocks along tokens with RHT-32 + SR (wgrad), one read
+            ("quant_dy_dual_sr", lambda: mx.mxfp4_quantize_dual(self.dy, 32, mx.ROUND_SR, SR_SEED, 0, 0,
+                                                                mx.SCALES_MMA, out_row=self.qdy, out_col=self.qdyt)),
             ("dgrad", lambda: mx.mxfp4_gemm(self.qdy.codes, self.qdy.scales, self.qw.codes_t, self.qw.scales_t,
                                             INTER, out=self.dx)),
-            ("quant_dyt_col_rht_sr", lambda: mx.mxfp4_quantize(self.dy, mx.LAYOUT_1D_COL, 32, mx.ROUND_SR,
-                                                               SR_SEED, 0, mx.SCALES_MMA, out=self.qdyt)),
-            ("quant_xt_col_rht", lambda: mx.mxfp4_quantize(self.x, mx.LAYOUT_1D_COL, 32, mx.ROUND_RNE, SR_SEED, 0,
-                                                           mx.SCALES_MMA, out=self.qxt)),
             ("wgrad", lambda: mx.mxfp4_gemm(self.qdyt.codes, self.qdyt.scales, self.qxt.codes, self.qxt.scales,
                                             TOKENS, out=self.dw)),
         ]
@@ -354,7 +354,7 @@ def main():
                 "peak_note": f"dense FP4 = 4 x {peaks['src']} bf16 burst ({peaks['bf16']} TFLOP/s), "
                              "the nominal 9 : 2.25 PFLOP/s ratio"}
     quant_gbs = quant_bytes / (quant_ms / 1e3) / 1e9
-    roofline_q = {"bound": "hbm", "kernel": "mxfp4 quantize kernels (5 launches per step)", "achieved": quant_gbs,
+    roofline_q = {"bound": "hbm", "kernel": "mxfp4 quantize kernels (3 launches per step)", "achieved": quant_gbs,
                   "peak": peaks["hbm"], "unit": "GB/s", "frac": quant_gbs / peaks["hbm"], "traffic": None,
                   "peak_note": f"{peaks['src']} copy bandwidth"}
 

@@ -142,6 +142,29 @@ MXFP4_API int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t 
                    void *stream);
 
 /*
+ * mxfp4_quantize_dual -- both 1D layouts of one bf16 tensor x[rows, cols] from
+ * a single read: row blocks (32 along cols, no RHT) into row_codes /
+ * row_scales, exactly as mxfp4_quantize with MXFP4_LAYOUT_1D_ROW, and column
+ * blocks (32 along rows, RHT of col_rht_size along rows) into col_codes /
+ * col_scales, exactly as mxfp4_quantize with MXFP4_LAYOUT_1D_COL.  The ALTO
+ * recipe ("Training an MoE LLM in MXFP4", abstract) quantizes activations and
+ * gradients in both orientations: row blocks for the forward and data-gradient
+ * GEMMs, blocks along tokens (with RHT) for the weight-gradient GEMM.  Both
+ * outputs use `rounding` and `seed`; each output's SR stream index is the
+ * element's index in its own output view plus row_elem_offset /
+ * col_elem_offset.  Either output may be skipped by passing NULL codes.
+ * Requirements: rows % 32 == 0, cols % 32 == 0, alignment as mxfp4_quantize.
+ */
+MXFP4_API int mxfp4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
+                                  int col_rht_size, int rounding, uint64_t seed,
+                                  uint64_t row_elem_offset, uint64_t col_elem_offset,
+                                  uint8_t *row_codes, int64_t ld_row_codes,
+                                  uint8_t *row_scales, int64_t ld_row_scales,
+                                  uint8_t *col_codes, int64_t ld_col_codes,
+                                  uint8_t *col_scales, int64_t ld_col_scales,
+                                  int scale_layout, void *stream);
+
+/*
  * mxfp4_dequantize -- MXFP4 codes and scales back to a [rows, cols] tensor.
  * ("Format specification": value = E2M1(code) * 2^(scale - 127), the whole
  * block NaN for scale 0xFF.)  If rht_size != 0 the inverse transform

@@ -38,7 +38,7 @@ OUT_BF16, OUT_F32 = 0, 1
 
 ABI_FUNCTIONS = (
     "mxfp4_status_string", "mxfp4_version", "mxfp4_mma_scales_bytes", "mxfp4_mma_scale_offset",
-    "mxfp4_quantize", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_grouped_gemm", "mxfp4_get_error",
+    "mxfp4_quantize", "mxfp4_quantize_dual", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_grouped_gemm", "mxfp4_get_error",
     "mxfp4_set_wait_limit_ns", "mxfp4_wait_probe",
 )
 
@@ -70,6 +70,9 @@ def lib() -> ctypes.CDLL:
         L.mxfp4_quantize.argtypes = [vp, i64, i64, i64, i32, i32, i32, u64, u64, vp, i64, vp, i64, i32,
                                      vp, i64, vp, i64, vp]
         L.mxfp4_quantize.restype = i32
+        L.mxfp4_quantize_dual.argtypes = [vp, i64, i64, i64, i32, i32, u64, u64, u64, vp, i64, vp, i64, vp, i64,
+                                          vp, i64, i32, vp]
+        L.mxfp4_quantize_dual.restype = i32
         L.mxfp4_dequantize.argtypes = [vp, i64, vp, i64, i32, i64, i64, i32, i32, u64, vp, i64, i32, vp]
         L.mxfp4_dequantize.restype = i32
         L.mxfp4_gemm.argtypes = [vp, i64, vp, vp, i64, vp, i64, i64, i64, vp, i64, vp]
@@ -170,6 +173,35 @@ def mxfp4_quantize(x: torch.Tensor, layout: int = LAYOUT_1D_ROW, rht_size: int =
         _ptr(out.scales_t), ld_sct, _stream(stream))
     _check(rc, "mxfp4_quantize")
     return out
+
+
+def mxfp4_quantize_dual(x: torch.Tensor, col_rht_size: int = 0, rounding: int = ROUND_RNE, seed: int = 0,
+                        row_elem_offset: int = 0, col_elem_offset: int = 0, scale_layout: int = SCALES_ROWMAJOR,
+                        row: bool = True, col: bool = True, stream=None, out_row: Optional[Quantized] = None,
+                        out_col: Optional[Quantized] = None):
+    """Row blocks and column blocks (RHT along rows) of one bf16 tensor from a
+    single read (see mxfp4_quantize_dual in include/mxfp4.h).  Returns
+    (row Quantized or None, column Quantized or None)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    dev = x.device
+    if row and out_row is None:
+        out_row = Quantized(torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                            _scale_tensor(rows, cols, scale_layout, dev), rows, cols, LAYOUT_1D_ROW, scale_layout)
+    if col and out_col is None:
+        out_col = Quantized(torch.empty((cols, rows // 2), dtype=torch.uint8, device=dev),
+                            _scale_tensor(cols, rows, scale_layout, dev), cols, rows, LAYOUT_1D_COL, scale_layout)
+    r = out_row if row else None
+    c = out_col if col else None
+    ld = lambda q: (q.scales.shape[1] if q.scales.dim() == 2 else 0) if q is not None else 0
+    rc = lib().mxfp4_quantize_dual(
+        _ptr(x), rows, cols, x.stride(0), col_rht_size, rounding, seed & 0xFFFFFFFFFFFFFFFF, row_elem_offset,
+        col_elem_offset, _ptr(r.codes) if r else None, r.codes.stride(0) if r else 0, _ptr(r.scales) if r else None,
+        ld(r), _ptr(c.codes) if c else None, c.codes.stride(0) if c else 0, _ptr(c.scales) if c else None, ld(c),
+        scale_layout, _stream(stream))
+    _check(rc, "mxfp4_quantize_dual")
+    return r, c
 
 
 def mxfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, rows: int, cols: int, layout: int = LAYOUT_1D_ROW,

@@ -12,6 +12,11 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, int64_t l
                             int rounding, uint64_t seed, uint64_t elem_offset, uint8_t *codes, int64_t ld_codes,
                             uint8_t *scales, int64_t ld_scales, int scale_layout, uint8_t *codes_t,
                             int64_t ld_codes_t, uint8_t *scales_t, int64_t ld_scales_t, cudaStream_t s);
+cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int col_rht, int rounding,
+                                 uint64_t seed, uint64_t row_offset, uint64_t col_offset, uint8_t *rcodes,
+                                 int64_t ld_rcodes, uint8_t *rscales, int64_t ld_rscales, uint8_t *ccodes,
+                                 int64_t ld_ccodes, uint8_t *cscales, int64_t ld_cscales, int scale_layout,
+                                 cudaStream_t s);
 cudaError_t launch_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
                               int scale_layout, int64_t rows, int64_t cols, int layout, int rht, uint64_t seed,
                               void *out, int64_t ld_out, int out_dtype, cudaStream_t s);
@@ -88,6 +93,35 @@ int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int 
                                                  codes, ld_codes, scales, ld_scales, scale_layout, codes_t,
                                                  ld_codes_t, scales_t, ld_scales_t,
                                                  static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
+}
+
+int mxfp4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int col_rht_size, int rounding,
+                        uint64_t seed, uint64_t row_elem_offset, uint64_t col_elem_offset, uint8_t *row_codes,
+                        int64_t ld_row_codes, uint8_t *row_scales, int64_t ld_row_scales, uint8_t *col_codes,
+                        int64_t ld_col_codes, uint8_t *col_scales, int64_t ld_col_scales, int scale_layout,
+                        void *stream) {
+    if (!x || (!row_codes && !col_codes)) return MXFP4_ERR_INVALID_ARG;
+    if ((row_codes && !row_scales) || (col_codes && !col_scales)) return MXFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0 || (rows % 32) || (cols % 32)) return MXFP4_ERR_INVALID_ARG;
+    if (col_rht_size != 0 && col_rht_size != 16 && col_rht_size != 32) return MXFP4_ERR_INVALID_ARG;
+    if (rounding != MXFP4_ROUND_RNE && rounding != MXFP4_ROUND_SR) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout != MXFP4_SCALES_ROWMAJOR && scale_layout != MXFP4_SCALES_MMA) return MXFP4_ERR_INVALID_ARG;
+    if ((row_elem_offset & 3u) || (col_elem_offset & 3u)) return MXFP4_ERR_INVALID_ARG;
+    if (ld_x < cols) return MXFP4_ERR_INVALID_ARG;
+    if (row_codes && ld_row_codes < cols / 2) return MXFP4_ERR_INVALID_ARG;
+    if (col_codes && ld_col_codes < rows / 2) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout == MXFP4_SCALES_ROWMAJOR) {
+        if (row_codes && ld_row_scales < cols / 32) return MXFP4_ERR_INVALID_ARG;
+        if (col_codes && ld_col_scales < rows / 32) return MXFP4_ERR_INVALID_ARG;
+    }
+    if (!aligned16(x) || (ld_x % 8)) return MXFP4_ERR_ALIGNMENT;
+    if (row_codes && (!aligned16(row_codes) || (ld_row_codes % 16))) return MXFP4_ERR_ALIGNMENT;
+    if (col_codes && (!aligned16(col_codes) || (ld_col_codes % 16))) return MXFP4_ERR_ALIGNMENT;
+    const cudaError_t e = mxfp4::launch_quantize_dual(
+        x, rows, cols, ld_x, col_rht_size, rounding, seed, row_elem_offset, col_elem_offset, row_codes, ld_row_codes,
+        row_scales, ld_row_scales, col_codes, ld_col_codes, col_scales, ld_col_scales, scale_layout,
+        static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
 }
 

@@ -134,17 +134,17 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float *v) {
 // below 0.5, f * 2^32 = |v| * 2^33 (exact), rounded up to an integer.
 __device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
     const uint32_t sign = (__float_as_uint(v) >> 28) & 8u;
-    const float a = fminf(fabsf(v), 6.0f);
-    const uint32_t ab = __float_as_uint(a);
+    const uint32_t ab = __float_as_uint(fminf(fabsf(v), 6.0f));
     uint32_t t, lo;
-    if (a >= 1.0f) {
-        t = ab << 10;
-        lo = (ab >> 22) - 252u;            // 1 -> 2, 1.5 -> 3, 2 -> 4, 3 -> 5, 4 -> 6, 6 -> 7
-    } else if (a >= 0.5f) {
-        t = ab << 9;
-        lo = 1u;
-    } else {
-        t = __float2uint_ru(a * 8589934592.0f);  // 2^33
+    if (ab >= 0x3F000000u) {                 // |v| >= 0.5: one mantissa bit on the grid
+        const uint32_t big = ab >= 0x3F800000u ? 1u : 0u;
+        t = ab << (9u + big);                // 22 (or 23) fraction bits, scaled to 2^32
+        lo = big ? (ab >> 22) - 252u : 1u;   // 1 -> 2, 1.5 -> 3, 2 -> 4, 3 -> 5, 4 -> 6, 6 -> 7
+    } else if (ab >= 0x3A800000u) {          // 2^-10 <= |v| < 0.5: |v| * 2^33 is an integer
+        t = ((ab & 0x007FFFFFu) | 0x00800000u) << ((ab >> 23) - 117u);
+        lo = 0u;
+    } else {                                 // tiny or zero: ceil(|v| * 2^33), exact in fp32
+        t = __float2uint_ru(__uint_as_float(ab) * 8589934592.0f);
         lo = 0u;
     }
     return sign | (lo + (r < t ? 1u : 0u));

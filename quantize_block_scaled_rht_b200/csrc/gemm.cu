@@ -237,7 +237,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     mxfp4_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                       const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ CUtensorMap tma_sfa,
                       const __grid_constant__ CUtensorMap tma_sfb, const GemmParams p) {
-    constexpr int BN = Cfg::BN, STAGES = Cfg::STAGES, NRT = Cfg::NRT;
+    constexpr int BN = Cfg::BN, STAGES = Cfg::STAGES;
     constexpr int A_BYTES = Cfg::A_BYTES, B_BYTES = Cfg::B_BYTES, SFA_BYTES = Cfg::SFA_BYTES;
     constexpr int STAGE_BYTES = Cfg::STAGE_BYTES, KCH = Cfg::KCH, NATOM = Cfg::NATOM;
     extern __shared__ uint8_t smem_raw[];

@@ -224,6 +224,152 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const QuantParams p) {
 }
 
 // ---------------------------------------------------------------------------
+// Dual output: 1D-row blocks (no RHT) and 1D-column blocks (optional RHT along
+// rows) of the same tensor from one read.  The recipe quantizes activations
+// and gradients both ways (row blocks for fprop/dgrad, blocks along tokens for
+// wgrad).  A persistent CTA streams 128 x 128 bf16 tiles through a
+// double-buffered shared-memory ring (cp.async, 272-byte row pitch: both the
+// per-row 64-byte reads and the per-column 32-bit reads are conflict-free):
+//   column blocks: thread (column pair p, row block b) reads two columns of
+//     32 rows, quantizes them, and stages 2 x 16 bytes of codes so that the
+//     128 transposed output rows leave as 64-byte contiguous stores;
+//   row blocks: thread (row r, column blocks 2h, 2h+1) reads 2 x 64 bytes of
+//     its row and stores 32 contiguous bytes of codes.
+// Either output may be disabled (DO_ROW / DO_COL).
+// ---------------------------------------------------------------------------
+constexpr int DT = 128;                    // tile rows = tile cols
+constexpr int DPITCH = DT + 8;             // bf16 per smem row (272 bytes)
+constexpr int DUAL_SMEM = 2 * DT * DPITCH * 2 + DT * 64;
+
+struct DualParams {
+    const uint16_t *x;
+    int64_t rows, cols, ld_x;
+    uint8_t *rcodes, *rscales;             // row output: [rows, cols/2], scales for (rows x cols)
+    int64_t ld_rcodes, ld_rscales, r_katoms;
+    uint8_t *ccodes, *cscales;             // column output: [cols, rows/2], scales for (cols x rows)
+    int64_t ld_ccodes, ld_cscales, c_katoms;
+    uint32_t seed_lo, seed_hi;
+    uint64_t r_offset, c_offset;           // SR stream index of each output's first element
+    uint32_t sgn_dup[32];
+};
+
+template <int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
+__global__ void __launch_bounds__(256) quant_dual_kernel(const DualParams p) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    uint16_t *tin = reinterpret_cast<uint16_t *>(dsm);                  // [2][DT][DPITCH]
+    uint8_t *tcol = dsm + 2 * DT * DPITCH * 2;                         // [DT out rows][64 bytes]
+    const int tid = threadIdx.x;
+    const int64_t tiles_r = (p.rows + DT - 1) / DT, tiles_c = (p.cols + DT - 1) / DT;
+    const int64_t ntiles = tiles_r * tiles_c;
+
+    auto load = [&](int64_t t, int buf) {
+        const int64_t r0 = (t / tiles_c) * DT, c0 = (t % tiles_c) * DT;
+        uint16_t *dst = tin + buf * DT * DPITCH;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int row = (tid >> 4) + 16 * i, ch = tid & 15;
+            const int64_t gr = r0 + row, gc = c0 + 8 * ch;
+            if (gr < p.rows && gc < p.cols) cp_async16(dst + row * DPITCH + 8 * ch, p.x + gr * p.ld_x + gc);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    int64_t t = blockIdx.x;
+    if (t < ntiles) load(t, 0);
+    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const int64_t tn = t + gridDim.x;
+        if (tn < ntiles) {
+            load(tn, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
+        const uint16_t *src = tin + buf * DT * DPITCH;
+        const int64_t r0 = (t / tiles_c) * DT, c0 = (t % tiles_c) * DT;
+
+        if constexpr (DO_COL) {
+            const int cp = tid & 63, rb = tid >> 6;              // column pair, 32-row block
+            const int64_t oc = c0 + 2 * cp, rbg = r0 + 32 * rb;
+            if (oc < p.cols && rbg < p.rows) {
+                const uint32_t *s32 = reinterpret_cast<const uint32_t *>(src);
+                float v0[32], v1[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    uint32_t u = s32[(32 * rb + i) * (DPITCH / 2) + cp];
+                    if constexpr (CRHT) u ^= p.sgn_dup[i % CRHT];
+                    v0[i] = bf16lo(u);
+                    v1[i] = bf16hi(u);
+                }
+                if constexpr (CRHT) {
+                    const float c = rht_norm<CRHT>();
+#pragma unroll
+                    for (int s = 0; s < 32; s += CRHT) { fwht<CRHT>(v0 + s); fwht<CRHT>(v1 + s); }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) { v0[i] = __fmul_rn(v0[i], c); v1[i] = __fmul_rn(v1[i], c); }
+                }
+                const uint64_t g0 = (uint64_t)(oc * p.rows + rbg) + p.c_offset;
+                uint4 q0, q1;
+                const uint32_t s0 = quantize32<SR>(v0, q0, g0, p.seed_lo, p.seed_hi);
+                const uint32_t s1 = quantize32<SR>(v1, q1, g0 + (uint64_t)p.rows, p.seed_lo, p.seed_hi);
+                *reinterpret_cast<uint4 *>(tcol + (2 * cp) * 64 + 16 * rb) = q0;
+                *reinterpret_cast<uint4 *>(tcol + (2 * cp + 1) * 64 + 16 * rb) = q1;
+                const int64_t kb = rbg >> 5;
+                if constexpr (MMA) {
+                    p.cscales[mma_scale_off(oc, kb, p.c_katoms)] = (uint8_t)s0;
+                    p.cscales[mma_scale_off(oc + 1, kb, p.c_katoms)] = (uint8_t)s1;
+                } else {
+                    p.cscales[oc * p.ld_cscales + kb] = (uint8_t)s0;
+                    p.cscales[(oc + 1) * p.ld_cscales + kb] = (uint8_t)s1;
+                }
+            }
+        }
+        if constexpr (DO_ROW) {
+            const int r = tid & 127, h = tid >> 7;               // row, pair of 32-column blocks
+            const int64_t gr = r0 + r;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int cb = 2 * h + j;
+                const int64_t gc = c0 + 32 * cb;
+                if (gr < p.rows && gc < p.cols) {
+                    const uint4 *s4 = reinterpret_cast<const uint4 *>(src + r * DPITCH + 32 * cb);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 u = s4[q];
+                        w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
+                    }
+                    float v[32];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) { v[2 * k] = bf16lo(w[k]); v[2 * k + 1] = bf16hi(w[k]); }
+                    uint4 q;
+                    const uint64_t g0 = (uint64_t)(gr * p.cols + gc) + p.r_offset;
+                    const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi);
+                    stg_v4(p.rcodes + gr * p.ld_rcodes + (gc >> 1), q);
+                    const int64_t kb = gc >> 5;
+                    if constexpr (MMA) p.rscales[mma_scale_off(gr, kb, p.r_katoms)] = (uint8_t)sc;
+                    else p.rscales[gr * p.ld_rscales + kb] = (uint8_t)sc;
+                }
+            }
+        }
+        __syncthreads();
+        if constexpr (DO_COL) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int o = (tid >> 2) + 64 * i, ch = tid & 3;   // output row, 16-byte chunk
+                const int64_t orow = c0 + o, rin = r0 + 32 * ch;
+                if (orow < p.cols && rin < p.rows)
+                    stg_v4(p.ccodes + orow * p.ld_ccodes + (rin >> 1),
+                           *reinterpret_cast<const uint4 *>(tcol + o * 64 + 16 * ch));
+            }
+        }
+        // the next iteration overwrites the other buffer and, for columns, tcol
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
 // 2D 32x32 blocks.  A CTA covers 32 rows x 256 columns: warp w owns the tile
 // of columns 32w..32w+31, lane l its row l.  amax is a warp max.  The
 // optional transposed copy is built through a byte-transposed 512-byte
@@ -563,6 +709,61 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, int64_t l
         case 0: return launch_quant_s<0>(layout, trans, mma, sr, p, s);
         case 16: return launch_quant_s<16>(layout, trans, mma, sr, p, s);
         default: return launch_quant_s<32>(layout, trans, mma, sr, p, s);
+    }
+}
+
+template <int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
+static cudaError_t launch_dual_t(const DualParams &p, cudaStream_t s) {
+    auto kern = quant_dual_kernel<CRHT, SR, MMA, DO_ROW, DO_COL>;
+    static int attr_done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DUAL_SMEM);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
+    }
+    const int64_t tiles = ((p.rows + DT - 1) / DT) * ((p.cols + DT - 1) / DT);
+    const int64_t cap = (int64_t)num_sms() * 2;
+    kern<<<(unsigned)(tiles < cap ? tiles : cap), 256, DUAL_SMEM, s>>>(p);
+    return cudaGetLastError();
+}
+
+template <int CRHT, bool SR, bool MMA>
+static cudaError_t launch_dual_o(bool do_row, bool do_col, const DualParams &p, cudaStream_t s) {
+    if (do_row && do_col) return launch_dual_t<CRHT, SR, MMA, true, true>(p, s);
+    if (do_col) return launch_dual_t<CRHT, SR, MMA, false, true>(p, s);
+    return launch_dual_t<CRHT, SR, MMA, true, false>(p, s);
+}
+
+template <int CRHT>
+static cudaError_t launch_dual_r(bool sr, bool mma, bool do_row, bool do_col, const DualParams &p, cudaStream_t s) {
+    if (sr) return mma ? launch_dual_o<CRHT, true, true>(do_row, do_col, p, s) : launch_dual_o<CRHT, true, false>(do_row, do_col, p, s);
+    return mma ? launch_dual_o<CRHT, false, true>(do_row, do_col, p, s) : launch_dual_o<CRHT, false, false>(do_row, do_col, p, s);
+}
+
+cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int col_rht, int rounding,
+                                 uint64_t seed, uint64_t row_offset, uint64_t col_offset, uint8_t *rcodes,
+                                 int64_t ld_rcodes, uint8_t *rscales, int64_t ld_rscales, uint8_t *ccodes,
+                                 int64_t ld_ccodes, uint8_t *cscales, int64_t ld_cscales, int scale_layout,
+                                 cudaStream_t s) {
+    DualParams p{};
+    p.x = static_cast<const uint16_t *>(x);
+    p.rows = rows; p.cols = cols; p.ld_x = ld_x;
+    p.rcodes = rcodes; p.rscales = rscales; p.ld_rcodes = ld_rcodes; p.ld_rscales = ld_rscales;
+    p.r_katoms = mma_katoms(cols);
+    p.ccodes = ccodes; p.cscales = cscales; p.ld_ccodes = ld_ccodes; p.ld_cscales = ld_cscales;
+    p.c_katoms = mma_katoms(rows);
+    p.seed_lo = (uint32_t)seed; p.seed_hi = (uint32_t)(seed >> 32);
+    p.r_offset = row_offset; p.c_offset = col_offset;
+    uint32_t pair_unused[16];
+    fill_signs(col_rht ? rht_sign_mask_hd(seed) : 0u, col_rht, pair_unused, p.sgn_dup);
+    const bool sr = rounding == MXFP4_ROUND_SR, mma = scale_layout == MXFP4_SCALES_MMA;
+    const bool do_row = rcodes != nullptr, do_col = ccodes != nullptr;
+    switch (col_rht) {
+        case 0: return launch_dual_r<0>(sr, mma, do_row, do_col, p, s);
+        case 16: return launch_dual_r<16>(sr, mma, do_row, do_col, p, s);
+        default: return launch_dual_r<32>(sr, mma, do_row, do_col, p, s);
     }
 }
 

@@ -157,3 +157,32 @@ def test_invalid_arguments_are_rejected():
     with pytest.raises(mx.MXFP4Error) as e:
         mx.mxfp4_quantize(x, mx.LAYOUT_1D_ROW, elem_offset=2)
     assert e.value.status == mx.MXFP4_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("scale_layout", [mx.SCALES_ROWMAJOR, mx.SCALES_MMA])
+@pytest.mark.parametrize("rnd", [mx.ROUND_RNE, mx.ROUND_SR])
+@pytest.mark.parametrize("rht", [0, 16, 32])
+@pytest.mark.parametrize("shape", [(96, 160), (256, 384), (320, 2880)])
+def test_dual_row_and_col_bit_exact(shape, rht, rnd, scale_layout):
+    rows, cols = shape
+    x = synth.student_t_bf16(shape, seed=400 + rows)
+    qr, qc = mx.mxfp4_quantize_dual(dev_bf16(x), rht, rnd, 42, scale_layout=scale_layout)
+    cr, sr_ = oracle.quantize(x, oracle.LAYOUT_1D_ROW, 0, rnd, 42)
+    cc, sc = oracle.quantize(x, oracle.LAYOUT_1D_COL, rht, rnd, 42)
+    assert np.array_equal(host(qr.codes), cr) and np.array_equal(host(qc.codes), cc)
+    if scale_layout == mx.SCALES_MMA:
+        assert np.array_equal(from_mma(host(qr.scales), rows, cols), sr_)
+        assert np.array_equal(from_mma(host(qc.scales), cols, rows), sc)
+    else:
+        assert np.array_equal(host(qr.scales), sr_) and np.array_equal(host(qc.scales), sc)
+
+
+def test_dual_single_outputs_and_offsets():
+    x = synth.student_t_bf16((128, 256), seed=9)
+    qr, qc = mx.mxfp4_quantize_dual(dev_bf16(x), 32, mx.ROUND_SR, 5, row_elem_offset=4096, col_elem_offset=8,
+                                    col=False)
+    assert qc is None
+    assert np.array_equal(host(qr.codes), oracle.quantize(x, oracle.LAYOUT_1D_ROW, 0, oracle.ROUND_SR, 5, 4096)[0])
+    qr, qc = mx.mxfp4_quantize_dual(dev_bf16(x), 32, mx.ROUND_SR, 5, col_elem_offset=8, row=False)
+    assert qr is None
+    assert np.array_equal(host(qc.codes), oracle.quantize(x, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_SR, 5, 8)[0])
