@@ -127,27 +127,84 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float *v) {
     return r;
 }
 
+// Shifts with the PTX rule for large amounts: a count of 32 or more (a
+// negative int passed as unsigned included) gives 0.
+__device__ __forceinline__ uint32_t shl_sat(uint32_t a, uint32_t n) {
+    uint32_t d;
+    asm("shl.b32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(n));
+    return d;
+}
+__device__ __forceinline__ uint32_t shr_sat(uint32_t a, uint32_t n) {
+    uint32_t d;
+    asm("shr.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(n));
+    return d;
+}
+
 // Stochastic rounding of one scaled value with random word r: lo <= |v| < hi
 // neighbouring grid values, up iff r < ceil(f * 2^32) with
-// f = (|v| - lo) / (hi - lo).  On [1, 6] the grid has one mantissa bit, so the
-// lower 22 mantissa bits are f * 2^22; on [0.5, 1) f is the 23-bit mantissa;
-// below 0.5, f * 2^32 = |v| * 2^33 (exact), rounded up to an integer.
-__device__ __forceinline__ uint32_t e2m1_sr(float v, uint32_t r) {
-    const uint32_t sign = (__float_as_uint(v) >> 28) & 8u;
+// f = (|v| - lo) / (hi - lo).  With m the 24-bit significand and e the biased
+// exponent of |v|, f * 2^32 = m << min(e - 117, 10) (mod 2^32) for every
+// |v| >= 2^-10: on [1, 6] the grid keeps one mantissa bit and the lower 22 are
+// f * 2^22; on [0.5, 1) f is the 23-bit mantissa; below 0.5 the grid step is
+// 0.5, so f * 2^32 = |v| * 2^33.  Below 2^-10 that product has a fractional
+// part and is rounded up (a rare branch; zero takes the main path, where the
+// shift count is negative and the threshold 0).
+// Stochastic rounding of one scaled value with random word r: lo <= |v| < hi
+// neighbouring grid values, up iff r < ceil(f * 2^32) with
+// f = (|v| - lo) / (hi - lo).  Returns the magnitude code.  With m the 24-bit
+// significand and e the biased exponent of |v|, f * 2^32 = m << min(e - 117, 10)
+// (mod 2^32) for every |v| >= 2^-10: on [1, 6] the grid keeps one mantissa bit
+// and the lower 22 are f * 2^22; on [0.5, 1) f is the 23-bit mantissa; below
+// 0.5 the grid step is 0.5, so f * 2^32 = |v| * 2^33.  Below 2^-10 that product
+// has a fractional part and is rounded up (a rare branch; zero takes the main
+// path, where the shift count is negative and the threshold 0).
+__device__ __forceinline__ uint32_t e2m1_sr_mag(float v, uint32_t r) {
     const uint32_t ab = __float_as_uint(fminf(fabsf(v), 6.0f));
-    uint32_t t, lo;
-    if (ab >= 0x3F000000u) {                 // |v| >= 0.5: one mantissa bit on the grid
-        const uint32_t big = ab >= 0x3F800000u ? 1u : 0u;
-        t = ab << (9u + big);                // 22 (or 23) fraction bits, scaled to 2^32
-        lo = big ? (ab >> 22) - 252u : 1u;   // 1 -> 2, 1.5 -> 3, 2 -> 4, 3 -> 5, 4 -> 6, 6 -> 7
-    } else if (ab >= 0x3A800000u) {          // 2^-10 <= |v| < 0.5: |v| * 2^33 is an integer
-        t = ((ab & 0x007FFFFFu) | 0x00800000u) << ((ab >> 23) - 117u);
-        lo = 0u;
-    } else {                                 // tiny or zero: ceil(|v| * 2^33), exact in fp32
-        t = __float2uint_ru(__uint_as_float(ab) * 8589934592.0f);
-        lo = 0u;
+    const int e = (int)(ab >> 23);
+    const uint32_t m = (ab & 0x007FFFFFu) | 0x00800000u;
+    uint32_t t = shl_sat(m, (uint32_t)min(e - 117, 10));
+    // grid index below |v|: 0 under 0.5, 1 on [0.5, 1), (bits >> 22) - 252 above
+    const int lo = max((int)(ab >> 22) - 252, ab >= 0x3F000000u ? 1 : 0);
+    uint32_t code = (uint32_t)lo + (r < t ? 1u : 0u);
+    if (ab - 1u < 0x3A7FFFFFu) {            // 0 < |v| < 2^-10: t = ceil(m * 2^(e - 117)) < 2^23
+        t = shr_sat(m - 1u, (uint32_t)(117 - e)) + 1u;
+        code = r < t ? 1u : 0u;
     }
-    return sign | (lo + (r < t ? 1u : 0u));
+    return code;
+}
+
+// Sign bits of 8 values as the sign bits (bit 3) of 8 packed E2M1 nibbles:
+// byte permutes with sign replication gather the even and the odd elements,
+// a select interleaves them.
+__device__ __forceinline__ uint32_t prmt_sign2(float a, float b) {
+    uint32_t d;    // byte 0 = sign(a) replicated, byte 1 = sign(b) replicated
+    asm("prmt.b32 %0, %1, %2, 0x00FB;" : "=r"(d) : "r"(__float_as_uint(a)), "r"(__float_as_uint(b)));
+    return d;
+}
+__device__ __forceinline__ uint32_t prmt_lo2(uint32_t a, uint32_t b) {
+    uint32_t d;    // bytes 0, 1 of a, then bytes 0, 1 of b
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t sign_nibbles8(const float *w) {
+    const uint32_t ev = prmt_lo2(prmt_sign2(w[0], w[2]), prmt_sign2(w[4], w[6]));
+    const uint32_t od = prmt_lo2(prmt_sign2(w[1], w[3]), prmt_sign2(w[5], w[7]));
+    return ((ev & 0x0F0F0F0Fu) | (od & 0xF0F0F0F0u)) & 0x88888888u;
+}
+
+// Eight scaled values to eight packed E2M1 codes by stochastic rounding with
+// the random words r0 (elements 0-3) and r1 (elements 4-7): magnitudes as a
+// multiply-add chain (the nibbles do not overlap), signs in one go.
+__device__ __forceinline__ uint32_t e2m1x8_sr(const float *w, const U4 &r0, const U4 &r1) {
+    uint32_t mag = e2m1_sr_mag(w[7], r1.w);
+    mag = mag * 16u + e2m1_sr_mag(w[6], r1.z);
+    mag = mag * 16u + e2m1_sr_mag(w[5], r1.y);
+    mag = mag * 16u + e2m1_sr_mag(w[4], r1.x);
+    mag = mag * 16u + e2m1_sr_mag(w[3], r0.w);
+    mag = mag * 16u + e2m1_sr_mag(w[2], r0.z);
+    mag = mag * 16u + e2m1_sr_mag(w[1], r0.y);
+    mag = mag * 16u + e2m1_sr_mag(w[0], r0.x);
+    return mag | sign_nibbles8(w);
 }
 
 // ---------------------------------------------------------------------------

@@ -65,9 +65,7 @@ __device__ __forceinline__ uint32_t quantize32(float *v, uint4 &out, uint64_t g0
             const U4 r0 = philox4x32_10((uint32_t)b0, (uint32_t)(b0 >> 32), 0u, 0u, k0, k1);
             const U4 r1 = philox4x32_10((uint32_t)b1, (uint32_t)(b1 >> 32), 0u, 0u, k0, k1);
             const float *w = v + 8 * q;
-            p[q] = e2m1_sr(w[0], r0.x) | (e2m1_sr(w[1], r0.y) << 4) | (e2m1_sr(w[2], r0.z) << 8) |
-                   (e2m1_sr(w[3], r0.w) << 12) | (e2m1_sr(w[4], r1.x) << 16) | (e2m1_sr(w[5], r1.y) << 20) |
-                   (e2m1_sr(w[6], r1.z) << 24) | (e2m1_sr(w[7], r1.w) << 28);
+            p[q] = e2m1x8_sr(w, r0, r1);
         }
     }
     out = make_uint4(p[0], p[1], p[2], p[3]);
@@ -227,19 +225,18 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const QuantParams p) {
 // Dual output: 1D-row blocks (no RHT) and 1D-column blocks (optional RHT along
 // rows) of the same tensor from one read.  The recipe quantizes activations
 // and gradients both ways (row blocks for fprop/dgrad, blocks along tokens for
-// wgrad).  A persistent CTA streams 128 x 128 bf16 tiles through a
-// double-buffered shared-memory ring (cp.async, 272-byte row pitch: both the
-// per-row 64-byte reads and the per-column 32-bit reads are conflict-free):
-//   column blocks: thread (column pair p, row block b) reads two columns of
-//     32 rows, quantizes them, and stages 2 x 16 bytes of codes so that the
-//     128 transposed output rows leave as 64-byte contiguous stores;
-//   row blocks: thread (row r, column blocks 2h, 2h+1) reads 2 x 64 bytes of
-//     its row and stores 32 contiguous bytes of codes.
+// wgrad).  One CTA per 64 x 128 bf16 tile (cp.async into shared memory, 272-byte
+// row pitch so that both access patterns below are conflict-free); many small
+// CTAs per SM hide the load latency and balance the tail.  Each thread does one
+// column job and one row job, through one inlined quantizer body:
+//   column job: thread (column c, row block b) reads 32 rows of column c,
+//     applies the RHT and stores 16 bytes of transposed codes;
+//   row job: thread (row r, column block b) reads 64 bytes of its row and
+//     stores 16 bytes of codes.
 // Either output may be disabled (DO_ROW / DO_COL).
 // ---------------------------------------------------------------------------
-constexpr int DT = 128;                    // tile rows = tile cols
-constexpr int DPITCH = DT + 8;             // bf16 per smem row (272 bytes)
-constexpr int DUAL_SMEM = 2 * DT * DPITCH * 2 + DT * 64;
+constexpr int DTR = 64, DTC = 128;         // tile rows, tile columns
+constexpr int DPITCH = DTC + 8;            // bf16 per smem row (272 bytes)
 
 struct DualParams {
     const uint16_t *x;
@@ -250,122 +247,81 @@ struct DualParams {
     int64_t ld_ccodes, ld_cscales, c_katoms;
     uint32_t seed_lo, seed_hi;
     uint64_t r_offset, c_offset;           // SR stream index of each output's first element
+    uint32_t tiles_c;                      // column tiles
     uint32_t sgn_dup[32];
 };
 
 template <int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(256) quant_dual_kernel(const DualParams p) {
-    extern __shared__ __align__(16) uint8_t dsm[];
-    uint16_t *tin = reinterpret_cast<uint16_t *>(dsm);                  // [2][DT][DPITCH]
-    uint8_t *tcol = dsm + 2 * DT * DPITCH * 2;                         // [DT out rows][64 bytes]
+__global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, const uint32_t ntiles) {
+    __shared__ __align__(16) uint16_t tin[DTR * DPITCH];
     const int tid = threadIdx.x;
-    const int64_t tiles_r = (p.rows + DT - 1) / DT, tiles_c = (p.cols + DT - 1) / DT;
-    const int64_t ntiles = tiles_r * tiles_c;
-
-    auto load = [&](int64_t t, int buf) {
-        const int64_t r0 = (t / tiles_c) * DT, c0 = (t % tiles_c) * DT;
-        uint16_t *dst = tin + buf * DT * DPITCH;
+    for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+        const int64_t r0 = (int64_t)(t / p.tiles_c) * DTR, c0 = (int64_t)(t % p.tiles_c) * DTC;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
             const int row = (tid >> 4) + 16 * i, ch = tid & 15;
             const int64_t gr = r0 + row, gc = c0 + 8 * ch;
-            if (gr < p.rows && gc < p.cols) cp_async16(dst + row * DPITCH + 8 * ch, p.x + gr * p.ld_x + gc);
+            if (gr < p.rows && gc < p.cols) cp_async16(tin + row * DPITCH + 8 * ch, p.x + gr * p.ld_x + gc);
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-
-    int64_t t = blockIdx.x;
-    if (t < ntiles) load(t, 0);
-    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
-        const int buf = it & 1;
-        const int64_t tn = t + gridDim.x;
-        if (tn < ntiles) {
-            load(tn, buf ^ 1);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        } else {
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        }
+        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
         __syncthreads();
-        const uint16_t *src = tin + buf * DT * DPITCH;
-        const int64_t r0 = (t / tiles_c) * DT, c0 = (t % tiles_c) * DT;
 
-        if constexpr (DO_COL) {
-            const int cp = tid & 63, rb = tid >> 6;              // column pair, 32-row block
-            const int64_t oc = c0 + 2 * cp, rbg = r0 + 32 * rb;
-            if (oc < p.cols && rbg < p.rows) {
-                const uint32_t *s32 = reinterpret_cast<const uint32_t *>(src);
-                float v0[32], v1[32];
+#pragma unroll 1
+        for (int job = DO_COL ? 0 : 1; job < (DO_ROW ? 2 : 1); ++job) {
+            float v[32];
+            bool ok;
+            uint64_t g0;
+            int64_t orow, kb;
+            if (job == 0) {                                  // column c, rows 32b .. 32b+31
+                const int c = tid & 127, b = tid >> 7;
+                orow = c0 + c;
+                const int64_t rin = r0 + 32 * b;
+                ok = orow < p.cols && rin < p.rows;
+                const uint16_t *col = tin + 32 * b * DPITCH + c;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    uint32_t u = s32[(32 * rb + i) * (DPITCH / 2) + cp];
-                    if constexpr (CRHT) u ^= p.sgn_dup[i % CRHT];
-                    v0[i] = bf16lo(u);
-                    v1[i] = bf16hi(u);
+                    uint32_t u = (uint32_t)col[i * DPITCH] << 16;
+                    if constexpr (CRHT) u ^= p.sgn_dup[i % CRHT] & 0x80000000u;
+                    v[i] = __uint_as_float(u);
                 }
                 if constexpr (CRHT) {
-                    const float c = rht_norm<CRHT>();
+                    const float cn = rht_norm<CRHT>();
 #pragma unroll
-                    for (int s = 0; s < 32; s += CRHT) { fwht<CRHT>(v0 + s); fwht<CRHT>(v1 + s); }
+                    for (int s = 0; s < 32; s += CRHT) fwht<CRHT>(v + s);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) { v0[i] = __fmul_rn(v0[i], c); v1[i] = __fmul_rn(v1[i], c); }
+                    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], cn);
                 }
-                const uint64_t g0 = (uint64_t)(oc * p.rows + rbg) + p.c_offset;
-                uint4 q0, q1;
-                const uint32_t s0 = quantize32<SR>(v0, q0, g0, p.seed_lo, p.seed_hi);
-                const uint32_t s1 = quantize32<SR>(v1, q1, g0 + (uint64_t)p.rows, p.seed_lo, p.seed_hi);
-                *reinterpret_cast<uint4 *>(tcol + (2 * cp) * 64 + 16 * rb) = q0;
-                *reinterpret_cast<uint4 *>(tcol + (2 * cp + 1) * 64 + 16 * rb) = q1;
-                const int64_t kb = rbg >> 5;
-                if constexpr (MMA) {
-                    p.cscales[mma_scale_off(oc, kb, p.c_katoms)] = (uint8_t)s0;
-                    p.cscales[mma_scale_off(oc + 1, kb, p.c_katoms)] = (uint8_t)s1;
-                } else {
-                    p.cscales[oc * p.ld_cscales + kb] = (uint8_t)s0;
-                    p.cscales[(oc + 1) * p.ld_cscales + kb] = (uint8_t)s1;
+                g0 = (uint64_t)(orow * p.rows + rin) + p.c_offset;
+                kb = rin >> 5;
+            } else {                                         // row r, columns 32b .. 32b+31
+                const int r = tid & 63, b = tid >> 6;
+                orow = r0 + r;
+                const int64_t gc = c0 + 32 * b;
+                ok = orow < p.rows && gc < p.cols;
+                const uint4 *s4 = reinterpret_cast<const uint4 *>(tin + r * DPITCH + 32 * b);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 u = s4[q];
+                    v[8 * q + 0] = bf16lo(u.x); v[8 * q + 1] = bf16hi(u.x);
+                    v[8 * q + 2] = bf16lo(u.y); v[8 * q + 3] = bf16hi(u.y);
+                    v[8 * q + 4] = bf16lo(u.z); v[8 * q + 5] = bf16hi(u.z);
+                    v[8 * q + 6] = bf16lo(u.w); v[8 * q + 7] = bf16hi(u.w);
                 }
+                g0 = (uint64_t)(orow * p.cols + gc) + p.r_offset;
+                kb = gc >> 5;
+            }
+            if (ok) {
+                uint4 q;
+                const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi);
+                uint8_t *codes = job == 0 ? p.ccodes : p.rcodes;
+                uint8_t *scales = job == 0 ? p.cscales : p.rscales;
+                const int64_t ldc = job == 0 ? p.ld_ccodes : p.ld_rcodes;
+                stg_v4(codes + orow * ldc + kb * 16, q);
+                if constexpr (MMA) scales[mma_scale_off(orow, kb, job == 0 ? p.c_katoms : p.r_katoms)] = (uint8_t)sc;
+                else scales[orow * (job == 0 ? p.ld_cscales : p.ld_rscales) + kb] = (uint8_t)sc;
             }
         }
-        if constexpr (DO_ROW) {
-            const int r = tid & 127, h = tid >> 7;               // row, pair of 32-column blocks
-            const int64_t gr = r0 + r;
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int cb = 2 * h + j;
-                const int64_t gc = c0 + 32 * cb;
-                if (gr < p.rows && gc < p.cols) {
-                    const uint4 *s4 = reinterpret_cast<const uint4 *>(src + r * DPITCH + 32 * cb);
-                    uint32_t w[16];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 u = s4[q];
-                        w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
-                    }
-                    float v[32];
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) { v[2 * k] = bf16lo(w[k]); v[2 * k + 1] = bf16hi(w[k]); }
-                    uint4 q;
-                    const uint64_t g0 = (uint64_t)(gr * p.cols + gc) + p.r_offset;
-                    const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi);
-                    stg_v4(p.rcodes + gr * p.ld_rcodes + (gc >> 1), q);
-                    const int64_t kb = gc >> 5;
-                    if constexpr (MMA) p.rscales[mma_scale_off(gr, kb, p.r_katoms)] = (uint8_t)sc;
-                    else p.rscales[gr * p.ld_rscales + kb] = (uint8_t)sc;
-                }
-            }
-        }
-        __syncthreads();
-        if constexpr (DO_COL) {
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int o = (tid >> 2) + 64 * i, ch = tid & 3;   // output row, 16-byte chunk
-                const int64_t orow = c0 + o, rin = r0 + 32 * ch;
-                if (orow < p.cols && rin < p.rows)
-                    stg_v4(p.ccodes + orow * p.ld_ccodes + (rin >> 1),
-                           *reinterpret_cast<const uint4 *>(tcol + o * 64 + 16 * ch));
-            }
-        }
-        // the next iteration overwrites the other buffer and, for columns, tcol
-        __syncthreads();
+        __syncthreads();                                     // the next tile overwrites tin
     }
 }
 
@@ -422,10 +378,7 @@ __global__ void __launch_bounds__(256) quant_2d_kernel(const QuantParams p) {
                         const U4 r0 = philox4x32_10((uint32_t)b0, (uint32_t)(b0 >> 32), 0u, 0u, p.seed_lo, p.seed_hi);
                         const U4 r1 = philox4x32_10((uint32_t)b1, (uint32_t)(b1 >> 32), 0u, 0u, p.seed_lo, p.seed_hi);
                         const float *x8 = v + 8 * q;
-                        pk[q] = e2m1_sr(x8[0], r0.x) | (e2m1_sr(x8[1], r0.y) << 4) | (e2m1_sr(x8[2], r0.z) << 8) |
-                                (e2m1_sr(x8[3], r0.w) << 12) | (e2m1_sr(x8[4], r1.x) << 16) |
-                                (e2m1_sr(x8[5], r1.y) << 20) | (e2m1_sr(x8[6], r1.z) << 24) |
-                                (e2m1_sr(x8[7], r1.w) << 28);
+                        pk[q] = e2m1x8_sr(x8, r0, r1);
                     }
                 }
                 packed = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -714,18 +667,11 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, int64_t l
 
 template <int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
 static cudaError_t launch_dual_t(const DualParams &p, cudaStream_t s) {
-    auto kern = quant_dual_kernel<CRHT, SR, MMA, DO_ROW, DO_COL>;
-    static int attr_done[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64 || !attr_done[dev]) {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, DUAL_SMEM);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) attr_done[dev] = 1;
-    }
-    const int64_t tiles = ((p.rows + DT - 1) / DT) * ((p.cols + DT - 1) / DT);
-    const int64_t cap = (int64_t)num_sms() * 2;
-    kern<<<(unsigned)(tiles < cap ? tiles : cap), 256, DUAL_SMEM, s>>>(p);
+    const uint64_t tiles = (uint64_t)((p.rows + DTR - 1) / DTR) * p.tiles_c;
+    if (tiles > 0xFFFFFFFFull - 0x7FFFFFFFull) return cudaErrorInvalidValue;   // tile index fits 32 bits
+    const uint64_t cap = 0x7FFFFFFFull;
+    quant_dual_kernel<CRHT, SR, MMA, DO_ROW, DO_COL>
+        <<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, s>>>(p, (uint32_t)tiles);
     return cudaGetLastError();
 }
 
@@ -756,6 +702,7 @@ cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int6
     p.c_katoms = mma_katoms(rows);
     p.seed_lo = (uint32_t)seed; p.seed_hi = (uint32_t)(seed >> 32);
     p.r_offset = row_offset; p.c_offset = col_offset;
+    p.tiles_c = (uint32_t)((cols + DTC - 1) / DTC);
     uint32_t pair_unused[16];
     fill_signs(col_rht ? rht_sign_mask_hd(seed) : 0u, col_rht, pair_unused, p.sgn_dup);
     const bool sr = rounding == MXFP4_ROUND_SR, mma = scale_layout == MXFP4_SCALES_MMA;
