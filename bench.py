@@ -57,6 +57,31 @@ QUANT_OPS = {"quant_x_dual": TOKENS * HIDDEN * QDUAL_BYTES, "quant_w_2d": INTER 
 KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
+# the ncu --set full capture of one bench step summarised in
+# profiles/expert_step_kernels_ncu_full.md.  The figures hold only for the
+# kernel sources they were taken from: a changed source gives traffic null.
+NCU_TRAFFIC = {
+    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "6ea2ff6b6680eb56",
+             "bytes": {"fprop": 51.57e6, "dgrad": 23.42e6, "wgrad": 29.79e6}},
+    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "8cb10ec7085a0bb0",
+              "bytes": {"quant_x_dual": 23.63e6, "quant_w_2d": 33.30e6, "quant_dy_dual_sr": 48.09e6}},
+}
+
+
+def ncu_traffic(kind: str, names):
+    """Mean DRAM bytes per launch over `names`, or None if the kernel changed."""
+    import hashlib
+    t = NCU_TRAFFIC[kind]
+    m = hashlib.sha1()
+    for f in t["sources"]:
+        with open(os.path.join(ROOT, "quantize_block_scaled_rht_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    if m.hexdigest()[:16] != t["sha1"]:
+        return None
+    return float(np.mean([t["bytes"][n] for n in names]))
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -350,12 +375,15 @@ def main():
     fp4_peak = 4 * peaks["bf16"]
     roofline = {"bound": "tensor", "kernel": "mxfp4_gemm_kernel (fprop+dgrad+wgrad launches)",
                 "achieved": gemm_tf, "peak": fp4_peak, "unit": "TFLOP/s", "frac": gemm_tf / fp4_peak,
-                "traffic": None,
+                "traffic": ncu_traffic("gemm", list(GEMMS)),
+                "traffic_note": "mean DRAM bytes per GEMM launch from ncu (cold caches); output lines still in "
+                                "L2 when the kernel ends are not counted as writes",
                 "peak_note": f"dense FP4 = 4 x {peaks['src']} bf16 burst ({peaks['bf16']} TFLOP/s), "
                              "the nominal 9 : 2.25 PFLOP/s ratio"}
     quant_gbs = quant_bytes / (quant_ms / 1e3) / 1e9
     roofline_q = {"bound": "hbm", "kernel": "mxfp4 quantize kernels (3 launches per step)", "achieved": quant_gbs,
-                  "peak": peaks["hbm"], "unit": "GB/s", "frac": quant_gbs / peaks["hbm"], "traffic": None,
+                  "peak": peaks["hbm"], "unit": "GB/s", "frac": quant_gbs / peaks["hbm"],
+                  "traffic": ncu_traffic("quant", list(QUANT_OPS)),
                   "peak_note": f"{peaks['src']} copy bandwidth"}
 
     # end to end through the public API with host buffers
