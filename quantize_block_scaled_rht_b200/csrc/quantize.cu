@@ -10,6 +10,8 @@
 // written per element): 128-bit loads/stores, in-register Hadamard butterflies,
 // and shared-memory staging only where a transpose is needed.
 #include <cstdint>
+#include <map>
+#include <mutex>
 #include <cstdio>
 
 #include "common.cuh"
@@ -253,18 +255,33 @@ struct DualParams {
 
 template <int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
 __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, const uint32_t ntiles) {
-    __shared__ __align__(16) uint16_t tin[DTR * DPITCH];
+    __shared__ __align__(16) uint16_t tin[2][DTR * DPITCH];
     const int tid = threadIdx.x;
-    for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    auto load = [&](uint32_t t, int buf) {
         const int64_t r0 = (int64_t)(t / p.tiles_c) * DTR, c0 = (int64_t)(t % p.tiles_c) * DTC;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int row = (tid >> 4) + 16 * i, ch = tid & 15;
             const int64_t gr = r0 + row, gc = c0 + 8 * ch;
-            if (gr < p.rows && gc < p.cols) cp_async16(tin + row * DPITCH + 8 * ch, p.x + gr * p.ld_x + gc);
+            if (gr < p.rows && gc < p.cols) cp_async16(tin[buf] + row * DPITCH + 8 * ch, p.x + gr * p.ld_x + gc);
         }
-        asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    uint32_t t = blockIdx.x;
+    if (t < ntiles) load(t, 0);
+    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+        // the next tile's load is in flight while this one is quantized
+        const int buf = it & 1;
+        const uint32_t tn = t + gridDim.x;
+        if (tn < ntiles) {
+            load(tn, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
         __syncthreads();
+        const uint16_t *tile = tin[buf];
+        const int64_t r0 = (int64_t)(t / p.tiles_c) * DTR, c0 = (int64_t)(t % p.tiles_c) * DTC;
 
 #pragma unroll 1
         for (int job = DO_COL ? 0 : 1; job < (DO_ROW ? 2 : 1); ++job) {
@@ -277,7 +294,7 @@ __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, 
                 orow = c0 + c;
                 const int64_t rin = r0 + 32 * b;
                 ok = orow < p.cols && rin < p.rows;
-                const uint16_t *col = tin + 32 * b * DPITCH + c;
+                const uint16_t *col = tile + 32 * b * DPITCH + c;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     uint32_t u = (uint32_t)col[i * DPITCH] << 16;
@@ -298,7 +315,7 @@ __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, 
                 orow = r0 + r;
                 const int64_t gc = c0 + 32 * b;
                 ok = orow < p.rows && gc < p.cols;
-                const uint4 *s4 = reinterpret_cast<const uint4 *>(tin + r * DPITCH + 32 * b);
+                const uint4 *s4 = reinterpret_cast<const uint4 *>(tile + r * DPITCH + 32 * b);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const uint4 u = s4[q];
@@ -321,33 +338,71 @@ __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, 
                 else scales[orow * (job == 0 ? p.ld_cscales : p.ld_rscales) + kb] = (uint8_t)sc;
             }
         }
-        __syncthreads();                                     // the next tile overwrites tin
+        __syncthreads();                                     // the load after next overwrites this buffer
     }
 }
 
 // ---------------------------------------------------------------------------
-// 2D 32x32 blocks.  A CTA covers 32 rows x 256 columns: warp w owns the tile
-// of columns 32w..32w+31, lane l its row l.  amax is a warp max.  The
-// optional transposed copy is built through a byte-transposed 512-byte
+// 2D 32x32 blocks.  A CTA streams tiles of 8 blocks through a double-buffered
+// shared-memory ring (cp.async of whole tile rows, so the global reads are
+// coalesced): 32 x 256 (one block row) without the transposed copy, 128 x 64
+// (four block rows, two block columns) with it, so that each row of the
+// transposed operand receives 64 contiguous bytes from one CTA.  Warp w owns
+// one block, lane l its row l (64 bytes from shared memory; the row pitch is
+// padded by 16 bytes, which keeps these reads conflict-free); amax is a warp
+// max.  The transposed copy is built through a byte-transposed 512-byte
 // shared-memory tile per warp.
 // ---------------------------------------------------------------------------
+template <bool TRANS>
+struct Q2Tile {
+    static constexpr int BR = TRANS ? 4 : 1;          // block rows per tile
+    static constexpr int BC = 8 / BR;                 // block columns per tile
+    static constexpr int ROWS = 32 * BR, COLS = 32 * BC;
+    static constexpr int PITCH = COLS + 8;            // bf16 per smem row
+    static constexpr int CHUNKS = COLS / 8;           // 16-byte chunks per row
+};
+
 template <int RHT, bool SR, bool MMA, bool TRANS>
-__global__ void __launch_bounds__(256) quant_2d_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(256, 3) quant_2d_kernel(const QuantParams p) {
+    using T = Q2Tile<TRANS>;
+    __shared__ __align__(16) uint16_t tin[2][T::ROWS * T::PITCH];
     __shared__ __align__(16) uint8_t tb[8][16][32];   // per warp: byte j of row r at [j][r]
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t nbr = p.rows >> 5, nbc = p.cols >> 5;
-    const int64_t groups_c = (nbc + 7) >> 3;
-    const int64_t ngroups = nbr * groups_c;
-    for (int64_t t = blockIdx.x; t < ngroups; t += gridDim.x) {
-        const int64_t br = t / groups_c;
-        const int64_t bc = (t - br * groups_c) * 8 + warp;
-        if (bc < nbc) {
+    const int64_t tiles_c = (nbc + T::BC - 1) / T::BC;
+    const int64_t ntiles = ((nbr + T::BR - 1) / T::BR) * tiles_c;
+    auto load = [&](int64_t t, int buf) {
+        const int64_t r0 = (t / tiles_c) * T::ROWS, c0 = (t % tiles_c) * T::COLS;
+#pragma unroll
+        for (int i = 0; i < T::ROWS * T::CHUNKS / 256; ++i) {
+            const int idx = tid + 256 * i, row = idx / T::CHUNKS, ch = idx % T::CHUNKS;
+            const int64_t gr = r0 + row, gc = c0 + 8 * ch;
+            if (gr < p.rows && gc < p.cols) cp_async16(tin[buf] + row * T::PITCH + 8 * ch, p.x + gr * p.ld_x + gc);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    int64_t t = blockIdx.x;
+    if (t < ntiles) load(t, 0);
+    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const int64_t tn = t + gridDim.x;
+        if (tn < ntiles) {
+            load(tn, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
+        const int wr = warp / T::BC, wc = warp % T::BC;   // this warp's block within the tile
+        const int64_t br = (t / tiles_c) * T::BR + wr;
+        const int64_t bc = (t % tiles_c) * T::BC + wc;
+        if (br < nbr && bc < nbc) {
             const int64_t r = (br << 5) + lane, c0 = bc << 5;
-            const uint16_t *src = p.x + r * p.ld_x + c0;
+            const uint4 *s4 = reinterpret_cast<const uint4 *>(tin[buf] + (32 * wr + lane) * T::PITCH + 32 * wc);
             uint32_t w[16];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint4 u = ldg_nc_v4(src + 8 * q);
+                const uint4 u = s4[q];
                 w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
             }
             float v[32];
@@ -423,6 +478,7 @@ __global__ void __launch_bounds__(256) quant_2d_kernel(const QuantParams p) {
                 }
             }
         }
+        __syncthreads();                     // the load after next overwrites this buffer
     }
 }
 
@@ -590,6 +646,20 @@ static int num_sms() {
     return g_num_sms;
 }
 
+// Resident CTAs per SM of a kernel (persistent grids are SMs x this).
+// Cached per kernel; the value depends only on the kernel and block size.
+static int resident_ctas(const void *kern, int threads) {
+    static std::mutex mu;
+    static std::map<const void *, int> cache;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(kern);
+    if (it != cache.end()) return it->second;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, 0) != cudaSuccess || occ <= 0) occ = 1;
+    cache[kern] = occ;
+    return occ;
+}
+
 static void fill_signs(uint32_t mask, int rht, uint32_t *pair, uint32_t *dup) {
     for (int j = 0; j < 16; ++j) {
         const uint32_t e0 = (uint32_t)(2 * j) % (uint32_t)(rht ? rht : 32);
@@ -619,11 +689,13 @@ static cudaError_t launch_quant_t(int layout, bool trans, const QuantParams &p, 
         const int64_t cap = (int64_t)num_sms() * 8;
         quant_col_kernel<RHT, SR, MMA><<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, s>>>(p);
     } else {
-        const int64_t groups = (p.rows / 32) * ((p.cols / 32 + 7) / 8);
-        const int64_t cap = (int64_t)num_sms() * 16;
-        const unsigned g = (unsigned)(groups < cap ? groups : cap);
-        if (trans) quant_2d_kernel<RHT, SR, MMA, true><<<g, 256, 0, s>>>(p);
-        else quant_2d_kernel<RHT, SR, MMA, false><<<g, 256, 0, s>>>(p);
+        const int br = trans ? Q2Tile<true>::BR : Q2Tile<false>::BR;
+        const int64_t tiles = ((p.rows / 32 + br - 1) / br) * ((p.cols / 32 + 8 / br - 1) / (8 / br));
+        auto kern = trans ? quant_2d_kernel<RHT, SR, MMA, true> : quant_2d_kernel<RHT, SR, MMA, false>;
+        // persistent for RNE (memory-bound), one CTA per tile for SR (ALU-bound)
+        const int64_t cap = SR ? 0x7FFFFFFFll
+                               : (int64_t)num_sms() * resident_ctas(reinterpret_cast<const void *>(kern), 256);
+        kern<<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, s>>>(p);
     }
     return cudaGetLastError();
 }
@@ -669,9 +741,13 @@ template <int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
 static cudaError_t launch_dual_t(const DualParams &p, cudaStream_t s) {
     const uint64_t tiles = (uint64_t)((p.rows + DTR - 1) / DTR) * p.tiles_c;
     if (tiles > 0xFFFFFFFFull - 0x7FFFFFFFull) return cudaErrorInvalidValue;   // tile index fits 32 bits
-    const uint64_t cap = 0x7FFFFFFFull;
-    quant_dual_kernel<CRHT, SR, MMA, DO_ROW, DO_COL>
-        <<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, s>>>(p, (uint32_t)tiles);
+    auto kern = quant_dual_kernel<CRHT, SR, MMA, DO_ROW, DO_COL>;
+    // RNE is memory-bound: a persistent grid at full occupancy keeps the next
+    // tile's load in flight.  SR is ALU-bound: one CTA per tile lets the
+    // hardware scheduler balance the tail.
+    const uint64_t cap = SR ? 0x7FFFFFFFull
+                            : (uint64_t)num_sms() * (uint64_t)resident_ctas(reinterpret_cast<const void *>(kern), 256);
+    kern<<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, s>>>(p, (uint32_t)tiles);
     return cudaGetLastError();
 }
 
