@@ -26,7 +26,9 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        # MXFP4_ORACLE_LIB points the mutation tests at an oracle built with a
+        # planted mistake; otherwise the regular build is used.
+        path = os.environ.get("MXFP4_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         u8p = ctypes.POINTER(ctypes.c_uint8)
         i64 = ctypes.c_int64

@@ -15,13 +15,16 @@ LIB = os.path.join(HERE, "libmxfp4_oracle.so")
 CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math", "-fopenmp"]
 
 
-def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
-        return LIB
-    cmd = ["gcc", *CFLAGS, SRC, "-o", LIB + ".tmp", "-lm"]
+def build(force: bool = False, mutant: int = 0, out: str | None = None) -> str:
+    """Build the oracle (or, for the mutation tests, the oracle with planted
+    mistake number `mutant` into `out`) and return the library path."""
+    lib = out or LIB
+    if not force and not mutant and os.path.exists(lib) and os.path.getmtime(lib) >= os.path.getmtime(SRC):
+        return lib
+    cmd = ["gcc", *CFLAGS, *([f"-DORC_MUTANT={mutant}"] if mutant else []), SRC, "-o", lib + ".tmp", "-lm"]
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -67,11 +67,22 @@
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fopenmp.  No FMA
  * contraction and no fast-math, so every float operation rounds as written.
+ *
+ * Mutation testing: building with -DORC_MUTANT=k (k >= 1) plants the k-th of
+ * the numbered plausible mistakes marked MUT(k) below (a wrong tie rule, an
+ * off-by-one exponent, swapped nibbles, ...).  tests/test_oracle_mutants.py
+ * builds each one and checks that the pins fail on it.  Normal builds leave
+ * ORC_MUTANT at 0, where every MUT(k) is the constant 0.
  */
 #include <math.h>
 #include <stdint.h>
 #include <stddef.h>
 #include <string.h>
+
+#ifndef ORC_MUTANT
+#define ORC_MUTANT 0
+#endif
+#define MUT(k) (ORC_MUTANT == (k))
 
 #define ORC_LAYOUT_1D_ROW 0
 #define ORC_LAYOUT_1D_COL 1
@@ -94,7 +105,7 @@ void orc_philox4x32_10(const uint32_t ctr_in[4], const uint32_t key_in[2], uint3
 {
     uint32_t c0 = ctr_in[0], c1 = ctr_in[1], c2 = ctr_in[2], c3 = ctr_in[3];
     uint32_t k0 = key_in[0], k1 = key_in[1];
-    for (int round = 0; round < 10; ++round) {
+    for (int round = 0; round < (MUT(10) ? 9 : 10); ++round) {
         uint64_t p0 = (uint64_t)PHILOX_M0 * (uint64_t)c0;
         uint64_t p1 = (uint64_t)PHILOX_M1 * (uint64_t)c2;
         uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
@@ -130,7 +141,7 @@ void orc_sr_words(uint64_t seed, uint64_t g0, int64_t n, uint32_t *out)
 /* R2: the sign mask of the RHT diagonal. */
 uint32_t orc_rht_sign_mask(uint64_t seed)
 {
-    uint32_t ctr[4] = {0u, 0u, 0u, 0x52485400u};
+    uint32_t ctr[4] = {MUT(5) ? 0x52485400u : 0u, 0u, 0u, MUT(5) ? 0u : 0x52485400u};
     uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
     uint32_t w[4];
     orc_philox4x32_10(ctr, key, w);
@@ -156,7 +167,7 @@ double orc_e2m1_decode(uint32_t code)
 double orc_e8m0_decode(uint32_t code)
 {
     if ((code & 0xFFu) == 0xFFu) return NAN;
-    return ldexp(1.0, (int)(code & 0xFFu) - 127);
+    return ldexp(1.0, (int)(code & 0xFFu) - (MUT(15) ? 128 : 127));
 }
 
 /* R1: bf16 bit pattern -> fp32 (exact). */
@@ -191,7 +202,7 @@ uint32_t orc_scale_code(float amax)
     /* amax = m * 2^ex with m in [0.5, 1): floor(log2 amax) = ex - 1, exact
      * also for subnormal amax. */
     (void)frexpf(amax, &ex);
-    int e = (ex - 1) - 2;                           /* [MX-CLIP] */
+    int e = (ex - 1) - (MUT(2) ? 1 : 2);            /* [MX-CLIP] */
     int code = e + 127;
     if (code < 0) code = 0;                         /* R5 */
     if (code > 254) code = 254;
@@ -206,14 +217,14 @@ uint32_t orc_scale_code(float amax)
  * nearest of the eight magnitudes; on an exact tie the even code wins. */
 uint32_t orc_e2m1_rne(float v)
 {
-    uint32_t sign = signbit(v) ? 8u : 0u;           /* R7 */
+    uint32_t sign = (MUT(6) ? v < 0.0f : signbit(v)) ? 8u : 0u;   /* R7 */
     double a = fabs((double)v);
     if (a > 6.0) return sign | 7u;                  /* saturation */
     int best = 0;
     double best_d = fabs(a - E2M1_MAG[0]);
     for (int i = 1; i < 8; ++i) {
         double d = fabs(a - E2M1_MAG[i]);
-        if (d < best_d || (d == best_d && (i & 1) == 0 && (best & 1) == 1)) {
+        if (d < best_d || (d == best_d && (MUT(1) || ((i & 1) == 0 && (best & 1) == 1)))) {
             best = i;
             best_d = d;
         }
@@ -232,7 +243,7 @@ uint32_t orc_e2m1_sr(float v, uint32_t r)
         if (E2M1_MAG[i] <= a) lo = i;
     if (lo == 7 || E2M1_MAG[lo] == a) return sign | (uint32_t)lo;
     double f = (a - E2M1_MAG[lo]) / (E2M1_MAG[lo + 1] - E2M1_MAG[lo]);
-    int up = (double)r < f * 4294967296.0;
+    int up = (double)r < f * (MUT(3) ? 2147483648.0 : 4294967296.0);
     return sign | (uint32_t)(lo + up);
 }
 
@@ -243,6 +254,7 @@ uint32_t orc_e2m1_sr(float v, uint32_t r)
 static float rht_norm(int d)
 {
     /* c_16 = 1/4 exactly; c_32 = 1/sqrt(32) rounded to fp32. */
+    if (MUT(11)) return 1.0f;
     return d == 16 ? 0.25f : (float)(1.0 / sqrt(32.0));
 }
 
@@ -254,7 +266,7 @@ void orc_fwht_f32(float *v, int d)
             if (i & h) continue;
             float a = v[i], b = v[i + h];
             v[i] = a + b;
-            v[i + h] = a - b;
+            v[i + h] = MUT(16) ? b - a : a - b;
         }
     }
 }
@@ -292,10 +304,10 @@ static uint32_t quantize_block(const float *y, int n, int rnd, uint64_t seed,
     int has_nan = 0;
     for (int i = 0; i < n; ++i) {
         if (isnan(y[i])) has_nan = 1;
-        float a = fabsf(y[i]);
+        float a = MUT(13) ? y[i] : fabsf(y[i]);
         if (a > amax) amax = a;
     }
-    uint32_t sc = has_nan ? 0xFFu : orc_scale_code(amax);
+    uint32_t sc = (has_nan && !MUT(9)) ? 0xFFu : orc_scale_code(amax);
     if (sc == 0xFFu) {                               /* R3 */
         for (int i = 0; i < n; ++i) codes4[i] = 0;
         return sc;
@@ -312,7 +324,7 @@ static uint32_t quantize_block(const float *y, int n, int rnd, uint64_t seed,
 static void put_nibble(uint8_t *row, int64_t pos, uint32_t code)
 {
     uint8_t *b = row + (pos >> 1);
-    if (pos & 1) *b = (uint8_t)((*b & 0x0Fu) | (code << 4));   /* R9 */
+    if ((pos & 1) ^ MUT(4)) *b = (uint8_t)((*b & 0x0Fu) | (code << 4));   /* R9 */
     else *b = (uint8_t)((*b & 0xF0u) | (code & 0x0Fu));
 }
 
@@ -362,7 +374,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
                     int64_t r = transposed ? ocol : orow;
                     int64_t c = transposed ? orow : ocol;
                     y[i] = orc_bf16_to_f32(x[r * ld_x + c]);
-                    g[i] = (uint64_t)(orow * ocols + ocol) + elem_offset;
+                    g[i] = (uint64_t)(MUT(17) ? r * cols + c : orow * ocols + ocol) + (MUT(12) ? 0 : elem_offset);
                 }
                 if (rht)
                     for (int s = 0; s < 32; s += rht) orc_rht_forward(y + s, rht, smask);
@@ -399,7 +411,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
                     for (int j = 0; j < 32; ++j) {
                         int64_t c = bc * 32 + j;
                         put_nibble(codes + r * ld_codes, c, c4[i * 32 + j]);
-                        if (codes_t) put_nibble(codes_t + c * ld_codes_t, r, c4[i * 32 + j]);
+                        if (codes_t) put_nibble(codes_t + c * ld_codes_t, MUT(8) ? r ^ 1 : r, c4[i * 32 + j]);
                     }
                 }
             }
@@ -437,9 +449,9 @@ int orc_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales
             double X = orc_e8m0_decode(sc);
             for (int i = 0; i < 32; ++i) {
                 double v = orc_e2m1_decode(orc_get_nibble(codes + orow * ld_codes, b * 32 + i));
-                y[i] = (float)(v * X);   /* exact unless it overflows fp32 */
+                y[i] = (float)(v * (MUT(14) ? 1.0 : X));   /* exact unless it overflows fp32 */
             }
-            if (rht)
+            if (rht && !MUT(20))
                 for (int s = 0; s < 32; s += rht) orc_rht_inverse(y + s, rht, smask);
             for (int i = 0; i < 32; ++i) {
                 int64_t ocol = b * 32 + i;
@@ -485,11 +497,11 @@ void orc_gemm_entry(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales
         for (int i = 0; i < 32; ++i) {
             int64_t k = kb * 32 + i;
             double a = orc_e2m1_decode(orc_get_nibble(a_codes + m * lda, k));
-            double b = orc_e2m1_decode(orc_get_nibble(b_codes + n * ldb, k));
+            double b = orc_e2m1_decode(orc_get_nibble(b_codes + n * ldb, MUT(19) ? k ^ 1 : k));
             dot += a * b;
             dabs += fabs(a * b);
         }
-        acc += xa * xb * dot;
+        acc += (MUT(7) ? xa / xb : xa * xb) * dot;
         sabs += xa * xb * dabs;
     }
     *c_out = acc;

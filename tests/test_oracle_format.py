@@ -113,14 +113,17 @@ def test_worked_clipping_example_from_page():
         amax, scale, stored = float(amax), float(scale), float(stored)
         code = oracle.scale_code(amax)
         assert oracle.e8m0_decode(code) == scale
-        # whole block through the quantizer: the amax element is stored as 6
-        vals = np.full(32, 0.5, np.float32)
-        vals[5] = amax
-        x = (vals.view(np.uint32) >> 16).astype(np.uint16)[None, :]
-        codes, scales = oracle.quantize(x, oracle.LAYOUT_1D_ROW)
-        assert oracle.e8m0_decode(int(scales[0, 0])) == scale
-        nib = (int(codes[0, 5 // 2]) >> (4 * (5 % 2))) & 0xF
-        assert oracle.e2m1_decode(nib) * scale == stored
+        # whole block through the quantizer: the amax element is stored as 6.
+        # The scale follows max |Vi| ("Conversion rules"), so the same holds
+        # with the sign flipped: -7.5 is stored as -6 under the same scale.
+        for sign in (1.0, -1.0):
+            vals = np.full(32, 0.5, np.float32)
+            vals[5] = sign * amax
+            x = (vals.view(np.uint32) >> 16).astype(np.uint16)[None, :]
+            codes, scales = oracle.quantize(x, oracle.LAYOUT_1D_ROW)
+            assert oracle.e8m0_decode(int(scales[0, 0])) == scale
+            nib = (int(codes[0, 5 // 2]) >> (4 * (5 % 2))) & 0xF
+            assert oracle.e2m1_decode(nib) * scale == sign * stored
 
 
 # ---- element rounding -------------------------------------------------------------------

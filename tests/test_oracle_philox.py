@@ -17,13 +17,20 @@ import oracle
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 
-@pytest.fixture(scope="module")
-def torch_philox():
+def build_torch_philox(out_dir: str) -> str:
+    """Compile the helper that prints PyTorch's Philox4x32-10 blocks."""
     import torch
     inc = os.path.join(os.path.dirname(torch.__file__), "include")
     src = os.path.join(HERE, "helpers", "torch_philox.cpp")
-    exe = os.path.join(tempfile.mkdtemp(), "torch_philox")
+    exe = os.path.join(out_dir, "torch_philox")
     subprocess.run(["g++", "-std=c++17", "-O1", "-I", inc, src, "-o", exe], check=True)
+    return exe
+
+
+@pytest.fixture(scope="module")
+def torch_philox():
+    # the mutation tests compile the helper once and pass it in
+    exe = os.environ.get("MXFP4_TORCH_PHILOX") or build_torch_philox(tempfile.mkdtemp())
 
     def run(triples):
         inp = "".join(f"{s} {q} {o}\n" for s, q, o in triples)
