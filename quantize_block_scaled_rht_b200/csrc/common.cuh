@@ -231,4 +231,33 @@ __device__ __forceinline__ float rht_norm() {
     return D == 16 ? 0.25f : __uint_as_float(0x3E3504F3u);  // fp32(1/sqrt(32))
 }
 
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of this library is launched
+// with the programmatic-stream-serialization attribute, so its CTAs may start
+// while the previous kernel on the stream is still draining.  Each kernel
+// therefore executes pdl_wait() (griddepcontrol.wait: the previous grid has
+// completed and its writes are visible) before its first global-memory read
+// or write, and pdl_trigger() once its own CTAs are running, which lets the
+// next kernel's launch and prologue overlap this one's tail.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 }  // namespace mxfp4
+

@@ -271,6 +271,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         tmem_alloc_pair(&sh->tmem_base, TMEM_COLS);
         tmem_relinquish_pair();
     }
+    // the prologue above touches no global memory; from here on the previous
+    // kernel's outputs are read (operands, group offsets) and C is written
+    pdl_wait();
+    pdl_trigger();
     if constexpr (GROUPED) {
         if (threadIdx.x == 32 * 2) {
             int acc = 0;
@@ -598,8 +602,9 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
         const int64_t tiles = ((g.M + 255) / 256) * ((g.N + BN - 1) / BN);
         pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
     }
-    mxfp4_gemm_kernel<Cfg, GROUPED><<<(unsigned)(2 * pairs), NUM_THREADS, Cfg::SMEM_BYTES, s>>>(ta, tb, tc, tsa, tsb, p);
-    return cudaGetLastError() == cudaSuccess ? 0 : MXFP4_ERR_CUDA;
+    const cudaError_t e = launch_pdl(mxfp4_gemm_kernel<Cfg, GROUPED>, dim3((unsigned)(2 * pairs)), dim3(NUM_THREADS),
+                                     (size_t)Cfg::SMEM_BYTES, s, ta, tb, tc, tsa, tsb, p);
+    return e == cudaSuccess ? 0 : MXFP4_ERR_CUDA;
 }
 
 int launch_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes, int64_t ldb,

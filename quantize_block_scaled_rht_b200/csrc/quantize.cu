@@ -111,6 +111,8 @@ __device__ __forceinline__ void stg_v4(void *p, uint4 v) {
 // ---------------------------------------------------------------------------
 template <int RHT, bool SR, bool MMA>
 __global__ void __launch_bounds__(256) quant_row_kernel(const QuantParams p) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t nb = p.cols >> 5;
     const int64_t total = p.rows * nb;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -157,6 +159,8 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 template <int RHT, bool SR, bool MMA>
 __global__ void __launch_bounds__(256) quant_col_kernel(const QuantParams p) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ __align__(16) uint32_t tin[COL_TR][COL_TC / 2];   // 32 KB: bf16 pairs
     __shared__ __align__(16) uint4 tout[COL_TC][COL_TR / 32];    // 8 KB: 64 rows x 128 B
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -255,6 +259,8 @@ struct DualParams {
 
 template <int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
 __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, const uint32_t ntiles) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ __align__(16) uint16_t tin[2][DTR * DPITCH];
     const int tid = threadIdx.x;
     auto load = [&](uint32_t t, int buf) {
@@ -364,6 +370,8 @@ struct Q2Tile {
 
 template <int RHT, bool SR, bool MMA, bool TRANS>
 __global__ void __launch_bounds__(256, 3) quant_2d_kernel(const QuantParams p) {
+    pdl_wait();
+    pdl_trigger();
     using T = Q2Tile<TRANS>;
     __shared__ __align__(16) uint16_t tin[2][T::ROWS * T::PITCH];
     __shared__ __align__(16) uint8_t tb[8][16][32];   // per warp: byte j of row r at [j][r]
@@ -538,6 +546,8 @@ __device__ __forceinline__ void inverse_rht32(float *v, const uint32_t *sgn_pair
 // [rows/32, cols/32], 2 = MMA layout per row.
 template <int RHT, bool F32, int SMODE>
 __global__ void __launch_bounds__(256) dequant_row_kernel(const DequantParams p) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t nb = p.cols >> 5;
     const int64_t total = p.rows * nb;
     for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < total;
@@ -574,6 +584,8 @@ __global__ void __launch_bounds__(256) dequant_row_kernel(const DequantParams p)
 // 128-byte (bf16) or 256-byte (fp32) warp store.
 template <int RHT, bool F32, bool MMA>
 __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p) {
+    pdl_wait();
+    pdl_trigger();
     __shared__ __align__(16) uint4 tin[COL_TC][8];                 // 8 KB of codes
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t tiles_r = (p.rows + COL_TR - 1) / COL_TR;
@@ -683,11 +695,11 @@ static int64_t grid_for(int64_t items, int threads) {
 template <int RHT, bool SR, bool MMA>
 static cudaError_t launch_quant_t(int layout, bool trans, const QuantParams &p, cudaStream_t s) {
     if (layout == MXFP4_LAYOUT_1D_ROW) {
-        quant_row_kernel<RHT, SR, MMA><<<(unsigned)grid_for(p.rows * (p.cols / 32), 256), 256, 0, s>>>(p);
+        return launch_pdl(quant_row_kernel<RHT, SR, MMA>, dim3((unsigned)grid_for(p.rows * (p.cols / 32), 256)), dim3(256), 0, s, p);
     } else if (layout == MXFP4_LAYOUT_1D_COL) {
         const int64_t tiles = ((p.rows + COL_TR - 1) / COL_TR) * ((p.cols + COL_TC - 1) / COL_TC);
         const int64_t cap = (int64_t)num_sms() * 8;
-        quant_col_kernel<RHT, SR, MMA><<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, s>>>(p);
+        return launch_pdl(quant_col_kernel<RHT, SR, MMA>, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(256), 0, s, p);
     } else {
         const int br = trans ? Q2Tile<true>::BR : Q2Tile<false>::BR;
         const int64_t tiles = ((p.rows / 32 + br - 1) / br) * ((p.cols / 32 + 8 / br - 1) / (8 / br));
@@ -695,7 +707,7 @@ static cudaError_t launch_quant_t(int layout, bool trans, const QuantParams &p, 
         // persistent for RNE (memory-bound), one CTA per tile for SR (ALU-bound)
         const int64_t cap = SR ? 0x7FFFFFFFll
                                : (int64_t)num_sms() * resident_ctas(reinterpret_cast<const void *>(kern), 256);
-        kern<<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, s>>>(p);
+        return launch_pdl(kern, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(256), 0, s, p);
     }
     return cudaGetLastError();
 }
@@ -747,8 +759,7 @@ static cudaError_t launch_dual_t(const DualParams &p, cudaStream_t s) {
     // hardware scheduler balance the tail.
     const uint64_t cap = SR ? 0x7FFFFFFFull
                             : (uint64_t)num_sms() * (uint64_t)resident_ctas(reinterpret_cast<const void *>(kern), 256);
-    kern<<<(unsigned)(tiles < cap ? tiles : cap), 256, 0, s>>>(p, (uint32_t)tiles);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(256), 0, s, p, (uint32_t)tiles);
 }
 
 template <int CRHT, bool SR, bool MMA>
@@ -796,13 +807,13 @@ static cudaError_t launch_dequant_t(int layout, int smode, const DequantParams &
         const int64_t tiles = ((p.rows + COL_TR - 1) / COL_TR) * ((p.cols + COL_TC - 1) / COL_TC);
         const int64_t cap = (int64_t)num_sms() * 8;
         const unsigned g = (unsigned)(tiles < cap ? tiles : cap);
-        if (smode == 2) dequant_col_kernel<RHT, F32, true><<<g, 256, 0, s>>>(p);
-        else dequant_col_kernel<RHT, F32, false><<<g, 256, 0, s>>>(p);
+        if (smode == 2) return launch_pdl(dequant_col_kernel<RHT, F32, true>, dim3(g), dim3(256), 0, s, p);
+        else return launch_pdl(dequant_col_kernel<RHT, F32, false>, dim3(g), dim3(256), 0, s, p);
     } else {
         const unsigned g = (unsigned)grid_for(p.rows * (p.cols / 32), 256);
-        if (smode == 0) dequant_row_kernel<RHT, F32, 0><<<g, 256, 0, s>>>(p);
-        else if (smode == 1) dequant_row_kernel<RHT, F32, 1><<<g, 256, 0, s>>>(p);
-        else dequant_row_kernel<RHT, F32, 2><<<g, 256, 0, s>>>(p);
+        if (smode == 0) return launch_pdl(dequant_row_kernel<RHT, F32, 0>, dim3(g), dim3(256), 0, s, p);
+        else if (smode == 1) return launch_pdl(dequant_row_kernel<RHT, F32, 1>, dim3(g), dim3(256), 0, s, p);
+        else return launch_pdl(dequant_row_kernel<RHT, F32, 2>, dim3(g), dim3(256), 0, s, p);
     }
     return cudaGetLastError();
 }
