@@ -317,21 +317,33 @@ def main():
 
     K = args.steps
     n_ops = len(ops)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ops + 1)] for _ in range(K)]
     sampler = ClockSampler(local)
+
+    def run_steps(n, per_op):
+        """n steps, L2 flushed before each; events at the step boundaries, or
+        also between kernels (the breakdown pass: an event between two launches
+        keeps the second from starting early, so the step time is taken
+        without them)."""
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ops + 1 if per_op else 2)] for _ in range(n)]
+        for i in range(n):
+            flush.zero_()                               # L2 flush between timed steps (outside the step)
+            e = evs[i]
+            e[0].record(stream)
+            for j, (_, fn) in enumerate(ops):
+                fn()
+                if per_op:
+                    e[j + 1].record(stream)
+            if not per_op:
+                e[1].record(stream)
+        return evs
+
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)   # let the sampler start before the load
     t_wall = time.perf_counter()
-    for i in range(K):
-        flush.zero_()                                   # L2 flush between timed steps (outside the step)
-        e = evs[i]
-        e[0].record(stream)
-        for j, (_, fn) in enumerate(ops):
-            fn()
-            e[j + 1].record(stream)
+    evs = run_steps(K, per_op=False)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
     if world > 1:
@@ -340,12 +352,7 @@ def main():
     err = mx.mxfp4_get_error()
     if err != mx.MXFP4_OK:
         raise RuntimeError(f"device-side error in the timed region: {mx.status_string(err)}")
-
-    per_op = np.zeros((K, n_ops))
-    for i in range(K):
-        for j in range(n_ops):
-            per_op[i, j] = evs[i][j].elapsed_time(evs[i][j + 1])     # ms
-    step_ms = per_op.sum(axis=1)
+    step_ms = np.array([e[0].elapsed_time(e[1]) for e in evs])
     total_ms = float(step_ms.sum())
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=device)
@@ -354,7 +361,16 @@ def main():
     ms_per_step = total_ms / K
     value = STEP_FLOPS * world / (total_ms / K / 1e3) / 1e12
 
-    # per-kernel figures (averaged over the timed launches)
+    # breakdown pass: the same steps with an event after every kernel
+    KB = min(K, 300)
+    evs_b = run_steps(KB, per_op=True)
+    torch.cuda.synchronize()
+    per_op = np.zeros((KB, n_ops))
+    for i in range(KB):
+        for j in range(n_ops):
+            per_op[i, j] = evs_b[i][j].elapsed_time(evs_b[i][j + 1])     # ms
+
+    # per-kernel figures (averaged over the breakdown pass)
     names = [n for n, _ in ops]
     avg_ms = per_op.mean(axis=0)
     kernels = {}
@@ -441,7 +457,8 @@ def main():
                            "l2": f"flushed between timed steps ({args.flush_mib} MiB write, outside step events)"},
                 "roofline": roofline, "roofline_quantize": roofline_q, "kernels": kernels,
                 "quantize_GBps": quant_gbs, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": KERNELS_PER_STEP * K, "clocks": clocks, "wall_s_timed_region": t_wall}
+                "gpu_launches": KERNELS_PER_STEP * K, "clocks": clocks, "wall_s_timed_region": t_wall,
+                "breakdown": f"per-kernel figures from {KB} further steps with an event after every kernel"}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
