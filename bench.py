@@ -62,10 +62,10 @@ KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 # profiles/expert_step_kernels_ncu_full.md.  The figures hold only for the
 # kernel sources they were taken from: a changed source gives traffic null.
 NCU_TRAFFIC = {
-    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "6ea2ff6b6680eb56",
-             "bytes": {"fprop": 51.57e6, "dgrad": 23.42e6, "wgrad": 29.79e6}},
-    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "8cb10ec7085a0bb0",
-              "bytes": {"quant_x_dual": 23.63e6, "quant_w_2d": 33.30e6, "quant_dy_dual_sr": 48.09e6}},
+    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "67fdbfcaf842e5d6",
+             "bytes": {"fprop": 51.87e6, "dgrad": 23.17e6, "wgrad": 29.66e6}},
+    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "fd74e2780ea8c56b",
+              "bytes": {"quant_x_dual": 23.65e6, "quant_w_2d": 33.27e6, "quant_dy_dual_sr": 47.90e6}},
 }
 
 
@@ -268,6 +268,100 @@ def run_reference(args, rank):
 
 
 # ---------------------------------------------------------------------------
+# rows the step does not exercise: the grouped MoE GEMM and the quantizer sweep
+# ---------------------------------------------------------------------------
+def _timed(torch, fn, reps):
+    """Median time of `reps` launches (ms), events on the current stream."""
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in ts]))
+
+
+def grouped_bench(mx, torch, device, peaks, reps=10):
+    """Grouped MoE GEMMs on 16384 tokens routed top-4 of 32 experts (Zipf 1.2,
+    rows sorted by expert, groups padded to 128 rows): gate_up 2880 -> 5760 and
+    down 2880 -> 2880.  Activations N(0,1) and weights N(0, 0.02^2) are drawn on
+    the device with seeded generators (the recipe of synth.grouped_inputs) and
+    quantized by the library (1D RNE rows, 2D RNE weights).  The operands
+    (A 94 MB, B up to 265 MB) and outputs (up to 1.5 GB) exceed L2, so no flush
+    is needed between launches."""
+    E, H, I = synth.EXPERTS, synth.HIDDEN, synth.INTERMEDIATE
+    choice = synth.route_tokens(synth.MOE_TOKENS, E, seed=6)
+    _, offsets, sizes, total = synth.grouped_layout(choice, E)
+    g = torch.Generator(device=device)
+    g.manual_seed(5)
+    a = torch.randn((total, H), generator=g, device=device).to(torch.bfloat16)
+    qa = mx.mxfp4_quantize(a, mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    del a
+    off_d = torch.from_numpy(offsets).to(device)
+    size_d = torch.from_numpy(sizes).to(device)
+    routed = int(sizes.sum())
+    out = {}
+    for name, n_out, seed in (("gate_up", I, 8), ("down", H, 9)):
+        g.manual_seed(seed)
+        codes, scales = [], []
+        for _ in range(E):
+            w = (torch.randn((n_out, H), generator=g, device=device) * 0.02).to(torch.bfloat16)
+            q = mx.mxfp4_quantize(w, mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA)
+            codes.append(q.codes)
+            scales.append(q.scales)
+        b_codes, b_scales = torch.stack(codes), torch.cat(scales)
+        del codes, scales
+        c = torch.empty((qa.codes.shape[0], n_out), dtype=torch.float32, device=device)
+        ms = _timed(torch, lambda: mx.mxfp4_grouped_gemm(qa.codes, qa.scales, off_d, size_d, b_codes, b_scales,
+                                                          n_out, H, out=c), reps)
+        if mx.mxfp4_get_error() != mx.MXFP4_OK:
+            raise RuntimeError("device-side error in the grouped GEMM")
+        tf = 2.0 * routed * n_out * H / (ms / 1e3) / 1e12
+        out[name] = {"us": ms * 1e3, "TFLOP/s": tf, "frac_fp4_peak": tf / (4 * peaks["bf16"]),
+                     "shape": f"{routed} routed rows ({qa.codes.shape[0]} padded) x {n_out} x {H}"}
+        del b_codes, b_scales, c
+    torch.cuda.empty_cache()
+    return out
+
+
+def sweep_bench(mx, torch, device, peaks, nbytes=1 << 30, reps=5):
+    """Quantize and dequantize (bf16 out) of a 1 GiB bf16 tensor [186368 x 2880]
+    of Student-t(3) values with 0.1% outliers x100 (drawn on the device), every
+    layout x RHT size x rounding.  Algorithmic bytes per element: 2 read + 0.5
+    + 1/32 written (1D; 2D: + 1/1024), and the reverse for dequantize.  The
+    tensor exceeds L2, so no flush is needed between launches."""
+    rows, cols = synth.sweep_shape(nbytes, 2880)
+    x = synth.student_t_bf16_device(rows, cols, seed=7, device=device)
+    n = rows * cols
+    res = {}
+    out = torch.empty_like(x)
+    for layout, lname in ((mx.LAYOUT_1D_ROW, "row"), (mx.LAYOUT_1D_COL, "col"), (mx.LAYOUT_2D, "2d")):
+        sbytes = 1 / 1024 if layout == mx.LAYOUT_2D else 1 / 32
+        for rht in (0, 16, 32):
+            for rnd, rname in ((mx.ROUND_RNE, "rne"), (mx.ROUND_SR, "sr")):
+                q = mx.mxfp4_quantize(x, layout, rht, rnd, 42)
+                tq = _timed(torch, lambda: mx.mxfp4_quantize(x, layout, rht, rnd, 42, out=q), reps)
+                td = _timed(torch, lambda: mx.mxfp4_dequantize(q.codes, q.scales, rows, cols, layout, rht, 42,
+                                                               out=out), reps)
+                gq = n * (2 + 0.5 + sbytes) / (tq / 1e3) / 1e9
+                gd = n * (2 + 0.5 + sbytes) / (td / 1e3) / 1e9
+                res[f"{lname}_rht{rht}_{rname}"] = {"quant_GBps": round(gq), "quant_frac_hbm": round(gq / peaks["hbm"], 3),
+                                                    "dequant_GBps": round(gd),
+                                                    "dequant_frac_hbm": round(gd / peaks["hbm"], 3)}
+                del q
+    if mx.mxfp4_get_error() != mx.MXFP4_OK:
+        raise RuntimeError("device-side error in the sweep")
+    del x, out
+    torch.cuda.empty_cache()
+    return {"tensor": f"{rows} x {cols} bf16 ({nbytes >> 20} MiB)", "modes": res,
+            "note": "SR modes are bound by the integer work of Philox4x32-10 and the exact SR decision, not HBM"}
+
+
+# ---------------------------------------------------------------------------
 # main
 # ---------------------------------------------------------------------------
 def main():
@@ -279,6 +373,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-mib", type=int, default=256)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the grouped-MoE GEMM and quantizer-sweep measurements (1-GPU runs only)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -444,6 +540,11 @@ def main():
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / args.e2e_steps}
 
+    extras = {}
+    if world == 1 and not args.no_extras:
+        extras["grouped_moe"] = grouped_bench(mx, torch, device, peaks)
+        extras["quantizer_sweep"] = sweep_bench(mx, torch, device, peaks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(x, w, dy)
@@ -458,7 +559,8 @@ def main():
                 "roofline": roofline, "roofline_quantize": roofline_q, "kernels": kernels,
                 "quantize_GBps": quant_gbs, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": KERNELS_PER_STEP * K, "clocks": clocks, "wall_s_timed_region": t_wall,
-                "breakdown": f"per-kernel figures from {KB} further steps with an event after every kernel"}
+                "breakdown": f"per-kernel figures from {KB} further steps with an event after every kernel",
+                **extras}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
