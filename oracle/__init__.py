@@ -19,6 +19,7 @@ from . import build as _build
 
 LAYOUT_1D_ROW, LAYOUT_1D_COL, LAYOUT_2D = 0, 1, 2
 ROUND_RNE, ROUND_SR = 0, 1
+SCALE_FLOOR, SCALE_ROUNDUP, SCALE_PRESCALE_34 = 0, 1, 2
 
 _lib = None
 
@@ -55,7 +56,9 @@ def lib():
         L.orc_rht_inverse.argtypes = [fp, ctypes.c_int, ctypes.c_uint32]
         L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
         L.orc_f32_to_bf16.restype = ctypes.c_uint16
-        L.orc_quantize.argtypes = [ctypes.c_void_p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        L.orc_scale_code_rule.argtypes = [ctypes.c_float, ctypes.c_int]
+        L.orc_scale_code_rule.restype = ctypes.c_uint32
+        L.orc_quantize.argtypes = [ctypes.c_void_p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_uint64, ctypes.c_uint64, u8p, i64, u8p, i64, ctypes.c_void_p, i64]
         L.orc_quantize.restype = ctypes.c_int
         L.orc_dequantize.argtypes = [u8p, i64, u8p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
@@ -149,8 +152,13 @@ def rht_inverse(v: np.ndarray, sign_mask: int) -> np.ndarray:
 
 # ---- tensor level ------------------------------------------------------------
 
+def scale_code_rule(amax: float, rule: int) -> int:
+    """E8M0 code of a block with the given amax under scale rule `rule`."""
+    return int(lib().orc_scale_code_rule(amax, rule))
+
+
 def quantize(x_bf16: np.ndarray, layout: int, rht: int = 0, rnd: int = ROUND_RNE, seed: int = 0,
-             elem_offset: int = 0, transposed_copy: bool = False):
+             elem_offset: int = 0, transposed_copy: bool = False, scale_rule: int = SCALE_FLOOR):
     """Quantize a bf16 tensor given as uint16 bit patterns [rows, cols].
 
     Returns (codes, scales) or (codes, scales, codes_t) in the canonical
@@ -168,7 +176,7 @@ def quantize(x_bf16: np.ndarray, layout: int, rht: int = 0, rnd: int = ROUND_RNE
         codes = np.zeros((rows, cols // 2), np.uint8)
         scales = np.zeros((rows, cols // 32), np.uint8)
     codes_t = np.zeros((cols, rows // 2), np.uint8) if (layout == LAYOUT_2D and transposed_copy) else None
-    rc = lib().orc_quantize(x.ctypes.data, rows, cols, cols, layout, rht, rnd, seed, elem_offset,
+    rc = lib().orc_quantize(x.ctypes.data, rows, cols, cols, layout, rht, rnd, scale_rule, seed, elem_offset,
                             _ptr(codes, ctypes.c_uint8), codes.shape[1], _ptr(scales, ctypes.c_uint8),
                             scales.shape[1], codes_t.ctypes.data if codes_t is not None else None,
                             codes_t.shape[1] if codes_t is not None else 0)

@@ -64,6 +64,13 @@
  *      and element 2j+1 in bits 7:4.
  *  R10 2D blocks are 32x32 tiles of the [rows, cols] tensor; the optional
  *      transposed copy stores element (r, c) at row c, position r.
+ *  R14 Scale rules besides R5 ([MX-CLIP] and the [MX-TRAIN] table):
+ *      round-up: the decode scale amax / 6 rounded up to a power of two, that
+ *        is the smallest e with 6 * 2^e >= amax, so no element saturates;
+ *      3/4 pre-scale: the block exponent comes from the unscaled amax as in
+ *        R5, and each element is multiplied by 3/4 in fp32 before the
+ *        division by X, so no element reaches the clipping range.  The codes
+ *        hold 3/4 of the values; the consumer undoes the factor.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fopenmp.  No FMA
  * contraction and no fast-math, so every float operation rounds as written.
@@ -89,6 +96,9 @@
 #define ORC_LAYOUT_2D 2
 #define ORC_ROUND_RNE 0
 #define ORC_ROUND_SR 1
+#define ORC_SCALE_FLOOR 0
+#define ORC_SCALE_ROUNDUP 1
+#define ORC_SCALE_PRESCALE_34 2
 
 /* ------------------------------------------------------------------------ */
 /* Philox4x32-10 [PHILOX].  Round function: two 32x32->64 products of the    */
@@ -209,6 +219,23 @@ uint32_t orc_scale_code(float amax)
     return (uint32_t)code;
 }
 
+/* R14: the scale code under one of the three rules. */
+uint32_t orc_scale_code_rule(float amax, int rule)
+{
+    if (rule != ORC_SCALE_ROUNDUP) return orc_scale_code(amax);
+    if (isnan(amax) || isinf(amax)) return 0xFFu;
+    if (amax == 0.0f) return 0u;
+    int ex;
+    (void)frexpf(amax, &ex);
+    int e = (ex - 1) - 2;                           /* amax / 2^e in [4, 8) */
+    /* the smallest e with 6 * 2^e >= amax: one more when amax / 2^e > 6 */
+    if ((double)amax > (MUT(21) ? 5.0 : 6.0) * ldexp(1.0, e)) e += 1;
+    int code = e + 127;
+    if (code < 0) code = 0;
+    if (code > 254) code = 254;
+    return (uint32_t)code;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Element conversion [MX-CONV]; readings R6, R7, R8.                        */
 /* ------------------------------------------------------------------------ */
@@ -297,7 +324,7 @@ void orc_rht_inverse(float *v, int d, uint32_t sign_mask)
 /* fp32 values.  n = 32 (1D) or 1024 (2D).  g[i] is the stream index of      */
 /* element i (used by SR only).                                              */
 /* ------------------------------------------------------------------------ */
-static uint32_t quantize_block(const float *y, int n, int rnd, uint64_t seed,
+static uint32_t quantize_block(const float *y, int n, int rnd, int rule, uint64_t seed,
                                const uint64_t *g, uint8_t *codes4)
 {
     float amax = 0.0f;
@@ -305,16 +332,19 @@ static uint32_t quantize_block(const float *y, int n, int rnd, uint64_t seed,
     for (int i = 0; i < n; ++i) {
         if (isnan(y[i])) has_nan = 1;
         float a = MUT(13) ? y[i] : fabsf(y[i]);
+        if (MUT(22) && rule == ORC_SCALE_PRESCALE_34) a = 0.75f * a;
         if (a > amax) amax = a;
     }
-    uint32_t sc = (has_nan && !MUT(9)) ? 0xFFu : orc_scale_code(amax);
+    uint32_t sc = (has_nan && !MUT(9)) ? 0xFFu : orc_scale_code_rule(amax, rule);
     if (sc == 0xFFu) {                               /* R3 */
         for (int i = 0; i < n; ++i) codes4[i] = 0;
         return sc;
     }
     int e = (int)sc - 127;
     for (int i = 0; i < n; ++i) {
-        float v = ldexpf(y[i], -e);                  /* Vi / X, exact or gradual underflow */
+        /* R14: the 3/4 pre-scale is one fp32 multiply before the division by X */
+        float vi = rule == ORC_SCALE_PRESCALE_34 ? 0.75f * y[i] : y[i];
+        float v = ldexpf(vi, -e);                    /* Vi / X, exact or gradual underflow */
         codes4[i] = (uint8_t)(rnd == ORC_ROUND_SR ? orc_e2m1_sr(v, orc_sr_word(seed, g[i]))
                                                   : orc_e2m1_rne(v));
     }
@@ -345,16 +375,18 @@ uint32_t orc_get_nibble(const uint8_t *row, int64_t pos)
  *                 cols/32]; if codes_t is given, also the transposed copy
  *                 codes_t [cols, rows/2] (ld_codes_t bytes).
  *
- * rht in {0, 16, 32}; rnd in {RNE, SR}; the SR index of an element is its
+ * rht in {0, 16, 32}; rnd in {RNE, SR}; rule in {FLOOR, ROUNDUP,
+ * PRESCALE_34} (R5, R14); the SR index of an element is its
  * linear index in the output view plus elem_offset.  Returns 0, or -1 on a
  * shape the format does not define.
  */
 int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
-                 int layout, int rht, int rnd, uint64_t seed, uint64_t elem_offset,
+                 int layout, int rht, int rnd, int rule, uint64_t seed, uint64_t elem_offset,
                  uint8_t *codes, int64_t ld_codes, uint8_t *scales, int64_t ld_scales,
                  uint8_t *codes_t, int64_t ld_codes_t)
 {
     if (rht != 0 && rht != 16 && rht != 32) return -1;
+    if (rule < ORC_SCALE_FLOOR || rule > ORC_SCALE_PRESCALE_34) return -1;
     uint32_t smask = rht ? orc_rht_sign_mask(seed) : 0u;
 
     if (layout == ORC_LAYOUT_1D_ROW || layout == ORC_LAYOUT_1D_COL) {
@@ -378,7 +410,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
                 }
                 if (rht)
                     for (int s = 0; s < 32; s += rht) orc_rht_forward(y + s, rht, smask);
-                uint32_t sc = quantize_block(y, 32, rnd, seed, g, c4);
+                uint32_t sc = quantize_block(y, 32, rnd, rule, seed, g, c4);
                 scales[orow * ld_scales + b] = (uint8_t)sc;
                 for (int i = 0; i < 32; ++i)
                     put_nibble(codes + orow * ld_codes, b * 32 + i, c4[i]);
@@ -404,7 +436,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
                     if (rht)
                         for (int s = 0; s < 32; s += rht) orc_rht_forward(y + i * 32 + s, rht, smask);
                 }
-                uint32_t sc = quantize_block(y, 1024, rnd, seed, g, c4);
+                uint32_t sc = quantize_block(y, 1024, rnd, rule, seed, g, c4);
                 scales[br * ld_scales + bc] = (uint8_t)sc;
                 for (int i = 0; i < 32; ++i) {
                     int64_t r = br * 32 + i;

@@ -39,10 +39,12 @@ MUTANTS = {
     17: "column layout draws SR words by input index instead of output index",
     19: "GEMM pairs element k of A with element k^1 of B",
     20: "dequantize skips the inverse RHT",
+    21: "round-up scale compares against 5 * 2^e instead of 6 * 2^e",
+    22: "3/4 pre-scale also applied to the amax that sets the exponent",
 }
 
 PIN_FILES = ["test_oracle_format.py", "test_oracle_gemm.py", "test_oracle_quantize.py", "test_oracle_rht.py",
-             "test_oracle_sr.py", "test_oracle_philox.py"]
+             "test_oracle_sr.py", "test_oracle_scale_rules.py", "test_oracle_philox.py"]
 
 
 @pytest.fixture(scope="module")
