@@ -62,9 +62,23 @@ extern "C" {
 #define MXFP4_LAYOUT_1D_COL 1   /* 32 consecutive elements of a column; stored transposed */
 #define MXFP4_LAYOUT_2D 2       /* 32 x 32 tiles */
 
-/* Element rounding. */
+/* Element rounding (bits 3:0 of the `rounding` argument). */
 #define MXFP4_ROUND_RNE 0
 #define MXFP4_ROUND_SR 1
+/* Scale rule (bits 5:4 of the `rounding` argument, OR-ed with the rounding).
+ * "MXFP4" (aiwiki.ai), "Clipping in the reference algorithm" and the
+ * "Training with MXFP4" table:
+ *   FLOOR       the reference rule, code = floor(log2 amax) - 2 + 127;
+ *   ROUNDUP     the decode scale amax / 6 rounded up to a power of two: the
+ *               smallest e with 6 * 2^e >= amax, so no element saturates;
+ *   PRESCALE_34 the FLOOR exponent (from the unscaled amax), and each element
+ *               multiplied by 3/4 in fp32 before the division by the scale, so
+ *               none reaches the clipping range.  The codes then hold 3/4 of
+ *               the values: dequantize returns those, and a GEMM of two such
+ *               operands returns 9/16 of the product; the caller undoes it. */
+#define MXFP4_SCALE_FLOOR 0x00
+#define MXFP4_SCALE_ROUNDUP 0x10
+#define MXFP4_SCALE_PRESCALE_34 0x20
 
 /* Scale storage. */
 #define MXFP4_SCALES_ROWMAJOR 0 /* canonical: one byte per block, row-major */
@@ -105,7 +119,8 @@ MXFP4_API int64_t mxfp4_mma_scale_offset(int64_t row, int64_t kb, int64_t k);
  * Sylvester Hadamard matrix as an fp32 butterfly with stages h = 1, 2, .., d/2;
  * c_16 = 1/4, c_32 = fp32(1/sqrt(32)); s_j = -1 when bit j of word 0 of
  * Philox4x32-10(key = seed, counter = (0, 0, 0, 0x52485400)) is set); amax
- * over the block; scale code clamp(floor(log2 amax) - 2 + 127, 0, 254) (0xFF
+ * over the block; scale code clamp(floor(log2 amax) - 2 + 127, 0, 254), or the
+ * rule selected in bits 5:4 of `rounding` (MXFP4_SCALE_*) (0xFF
  * and all-zero element codes if the block holds a NaN or amax is Inf; code 0
  * if amax is 0); elements y * 2^-(code-127) rounded to E2M1 with saturation
  * at +-6, by nearest-even or, for MXFP4_ROUND_SR, up with probability

@@ -33,6 +33,8 @@ MXFP4_ERR_CUDA = 4
 MXFP4_ERR_TIMEOUT = 5
 LAYOUT_1D_ROW, LAYOUT_1D_COL, LAYOUT_2D = 0, 1, 2
 ROUND_RNE, ROUND_SR = 0, 1
+# scale rules, OR-ed into the rounding argument (MXFP4_SCALE_* in include/mxfp4.h)
+SCALE_FLOOR, SCALE_ROUNDUP, SCALE_PRESCALE_34 = 0x00, 0x10, 0x20
 SCALES_ROWMAJOR, SCALES_MMA = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 
@@ -146,7 +148,8 @@ def _scale_tensor(rows, k, scale_layout, device, two_d=False):
 
 def mxfp4_quantize(x: torch.Tensor, layout: int = LAYOUT_1D_ROW, rht_size: int = 0, rounding: int = ROUND_RNE,
                    seed: int = 0, elem_offset: int = 0, scale_layout: int = SCALES_ROWMAJOR,
-                   transposed_copy: bool = False, stream=None, out: Optional[Quantized] = None) -> Quantized:
+                   transposed_copy: bool = False, stream=None, out: Optional[Quantized] = None,
+                   scale_rule: int = SCALE_FLOOR) -> Quantized:
     """Quantize a 2-D bf16 CUDA tensor to MXFP4 (see mxfp4_quantize in include/mxfp4.h)."""
     if x.dtype != torch.bfloat16 or x.dim() != 2:
         raise ValueError("x must be a 2-D bfloat16 tensor")
@@ -167,7 +170,7 @@ def mxfp4_quantize(x: torch.Tensor, layout: int = LAYOUT_1D_ROW, rht_size: int =
     ld_sc = out.scales.shape[1] if out.scales.dim() == 2 else 0
     ld_sct = out.scales_t.shape[1] if (out.scales_t is not None and out.scales_t.dim() == 2) else 0
     rc = lib().mxfp4_quantize(
-        _ptr(x), rows, cols, x.stride(0), layout, rht_size, rounding, seed & 0xFFFFFFFFFFFFFFFF, elem_offset,
+        _ptr(x), rows, cols, x.stride(0), layout, rht_size, rounding | scale_rule, seed & 0xFFFFFFFFFFFFFFFF, elem_offset,
         _ptr(out.codes), out.codes.stride(0), _ptr(out.scales), ld_sc, scale_layout,
         _ptr(out.codes_t), out.codes_t.stride(0) if out.codes_t is not None else 0,
         _ptr(out.scales_t), ld_sct, _stream(stream))
@@ -178,7 +181,7 @@ def mxfp4_quantize(x: torch.Tensor, layout: int = LAYOUT_1D_ROW, rht_size: int =
 def mxfp4_quantize_dual(x: torch.Tensor, col_rht_size: int = 0, rounding: int = ROUND_RNE, seed: int = 0,
                         row_elem_offset: int = 0, col_elem_offset: int = 0, scale_layout: int = SCALES_ROWMAJOR,
                         row: bool = True, col: bool = True, stream=None, out_row: Optional[Quantized] = None,
-                        out_col: Optional[Quantized] = None):
+                        out_col: Optional[Quantized] = None, scale_rule: int = SCALE_FLOOR):
     """Row blocks and column blocks (RHT along rows) of one bf16 tensor from a
     single read (see mxfp4_quantize_dual in include/mxfp4.h).  Returns
     (row Quantized or None, column Quantized or None)."""
@@ -196,7 +199,7 @@ def mxfp4_quantize_dual(x: torch.Tensor, col_rht_size: int = 0, rounding: int = 
     c = out_col if col else None
     ld = lambda q: (q.scales.shape[1] if q.scales.dim() == 2 else 0) if q is not None else 0
     rc = lib().mxfp4_quantize_dual(
-        _ptr(x), rows, cols, x.stride(0), col_rht_size, rounding, seed & 0xFFFFFFFFFFFFFFFF, row_elem_offset,
+        _ptr(x), rows, cols, x.stride(0), col_rht_size, rounding | scale_rule, seed & 0xFFFFFFFFFFFFFFFF, row_elem_offset,
         col_elem_offset, _ptr(r.codes) if r else None, r.codes.stride(0) if r else 0, _ptr(r.scales) if r else None,
         ld(r), _ptr(c.codes) if c else None, c.codes.stride(0) if c else 0, _ptr(c.scales) if c else None, ld(c),
         scale_layout, _stream(stream))

@@ -59,6 +59,14 @@ int64_t mxfp4_mma_scale_offset(int64_t row, int64_t kb, int64_t k) {
     return mxfp4::mma_scale_off(row, kb, mxfp4::mma_katoms(k));
 }
 
+// `rounding` = element rounding (bits 3:0) | scale rule (bits 5:4); no other bits.
+static bool valid_rounding(int rounding) {
+    const int rnd = rounding & 0x0F, rule = rounding & 0x30;
+    if ((rounding & ~0x3F) != 0) return false;
+    if (rnd != MXFP4_ROUND_RNE && rnd != MXFP4_ROUND_SR) return false;
+    return rule == MXFP4_SCALE_FLOOR || rule == MXFP4_SCALE_ROUNDUP || rule == MXFP4_SCALE_PRESCALE_34;
+}
+
 int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rht_size, int rounding,
                    uint64_t seed, uint64_t elem_offset, uint8_t *codes, int64_t ld_codes, uint8_t *scales,
                    int64_t ld_scales, int scale_layout, uint8_t *codes_t, int64_t ld_codes_t, uint8_t *scales_t,
@@ -68,7 +76,7 @@ int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int 
     if (layout != MXFP4_LAYOUT_1D_ROW && layout != MXFP4_LAYOUT_1D_COL && layout != MXFP4_LAYOUT_2D)
         return MXFP4_ERR_INVALID_ARG;
     if (rht_size != 0 && rht_size != 16 && rht_size != 32) return MXFP4_ERR_INVALID_ARG;
-    if (rounding != MXFP4_ROUND_RNE && rounding != MXFP4_ROUND_SR) return MXFP4_ERR_INVALID_ARG;
+    if (!valid_rounding(rounding)) return MXFP4_ERR_INVALID_ARG;
     if (scale_layout != MXFP4_SCALES_ROWMAJOR && scale_layout != MXFP4_SCALES_MMA) return MXFP4_ERR_INVALID_ARG;
     if ((elem_offset & 3u) != 0) return MXFP4_ERR_INVALID_ARG;
     if (layout == MXFP4_LAYOUT_1D_ROW && (cols % 32)) return MXFP4_ERR_INVALID_ARG;
@@ -105,7 +113,7 @@ int mxfp4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
     if ((row_codes && !row_scales) || (col_codes && !col_scales)) return MXFP4_ERR_INVALID_ARG;
     if (rows <= 0 || cols <= 0 || (rows % 32) || (cols % 32)) return MXFP4_ERR_INVALID_ARG;
     if (col_rht_size != 0 && col_rht_size != 16 && col_rht_size != 32) return MXFP4_ERR_INVALID_ARG;
-    if (rounding != MXFP4_ROUND_RNE && rounding != MXFP4_ROUND_SR) return MXFP4_ERR_INVALID_ARG;
+    if (!valid_rounding(rounding)) return MXFP4_ERR_INVALID_ARG;
     if (scale_layout != MXFP4_SCALES_ROWMAJOR && scale_layout != MXFP4_SCALES_MMA) return MXFP4_ERR_INVALID_ARG;
     if ((row_elem_offset & 3u) || (col_elem_offset & 3u)) return MXFP4_ERR_INVALID_ARG;
     if (ld_x < cols) return MXFP4_ERR_INVALID_ARG;

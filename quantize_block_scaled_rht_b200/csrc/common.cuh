@@ -97,6 +97,29 @@ __device__ __forceinline__ uint32_t scale_code_from_amax(float amax) {
     return e > 0 ? (uint32_t)e : 0u;
 }
 
+// Scale code under the round-up rule: the smallest e with 6 * 2^e >= amax.
+// With amax = 1.m * 2^(E - 127), amax / 2^(E - 129) = 4 * 1.m, which exceeds 6
+// exactly when the mantissa field is above 0x400000 (1.m > 1.5).
+__device__ __forceinline__ uint32_t scale_code_roundup(float amax) {
+    const uint32_t b = __float_as_uint(amax);
+    if (b >= 0x7F800000u) return 0xFFu;
+    const int e = (int)(b >> 23) - 2 + ((b & 0x007FFFFFu) > 0x00400000u ? 1 : 0);
+    return e > 0 ? (uint32_t)min(e, 254) : 0u;
+}
+
+// Scale code of a block under a scale rule (MXFP4_SCALE_* >> 4): 0 the
+// reference floor rule, 1 round-up, 2 the 3/4 pre-scale (floor exponent).
+__device__ __forceinline__ uint32_t scale_code_rule(float amax, int rule) {
+    return rule == 1 ? scale_code_roundup(amax) : scale_code_from_amax(amax);
+}
+
+// Element scaling: y / X, or (3/4 y) / X under the pre-scale rule, each
+// product rounded in fp32 (the division by the power of two X is exact
+// unless the result is subnormal).
+__device__ __forceinline__ float scale_element(float y, float inv, int rule) {
+    return __fmul_rn(rule == 2 ? __fmul_rn(y, 0.75f) : y, inv);
+}
+
 // 2^-(code - 127) as fp32 for code in [0, 252]: biased exponent 254 - code.
 __device__ __forceinline__ float inv_scale_from_code(uint32_t code) {
     return __uint_as_float((254u - code) << 23);

@@ -30,6 +30,7 @@ struct QuantParams {
     uint8_t *scales_t;
     int64_t ld_scales_t, katoms_t;
     uint32_t seed_lo, seed_hi;
+    int scale_rule;                        // MXFP4_SCALE_* >> 4
     uint64_t elem_offset;
     // RHT signs as xor words: pair[j] flips the bf16 halves of word j of a
     // 32-element row segment (elements 2j, 2j+1); dup[i] flips both halves of
@@ -43,18 +44,19 @@ struct QuantParams {
 // code and 16 bytes of codes.  `g0` is the stream index of element 0.
 // ---------------------------------------------------------------------------
 template <bool SR>
-__device__ __forceinline__ uint32_t quantize32(float *v, uint4 &out, uint64_t g0, uint32_t k0, uint32_t k1) {
+__device__ __forceinline__ uint32_t quantize32(float *v, uint4 &out, uint64_t g0, uint32_t k0, uint32_t k1,
+                                           int rule) {
     float amax = 0.0f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = amax_nan(amax, v[i]);
-    const uint32_t code = scale_code_from_amax(amax);
+    const uint32_t code = scale_code_rule(amax, rule);
     if (code == 0xFFu) {
         out = make_uint4(0, 0, 0, 0);
         return code;
     }
     const float inv = inv_scale_from_code(code);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], inv);
+    for (int i = 0; i < 32; ++i) v[i] = scale_element(v[i], inv, rule);
     uint32_t p[4];
     if constexpr (!SR) {
 #pragma unroll
@@ -132,7 +134,7 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const QuantParams p) {
         unpack_row32<RHT>(w, v, p);
         uint4 packed;
         const uint64_t g0 = (uint64_t)(r * p.cols + (kb << 5)) + p.elem_offset;
-        const uint32_t code = quantize32<SR>(v, packed, g0, p.seed_lo, p.seed_hi);
+        const uint32_t code = quantize32<SR>(v, packed, g0, p.seed_lo, p.seed_hi, p.scale_rule);
         stg_v4(p.codes + r * p.ld_codes + (kb << 4), packed);
         if constexpr (MMA) p.scales[mma_scale_off(r, kb, p.katoms)] = (uint8_t)code;
         else p.scales[r * p.ld_scales + kb] = (uint8_t)code;
@@ -201,8 +203,8 @@ __global__ void __launch_bounds__(256) quant_col_kernel(const QuantParams p) {
             const int64_t kb = rb >> 5;           // output K-block
             uint4 q0, q1;
             const uint64_t g0 = (uint64_t)(oc * p.rows + rb) + p.elem_offset;
-            const uint32_t s0 = quantize32<SR>(v0, q0, g0, p.seed_lo, p.seed_hi);
-            const uint32_t s1 = quantize32<SR>(v1, q1, g0 + (uint64_t)p.rows, p.seed_lo, p.seed_hi);
+            const uint32_t s0 = quantize32<SR>(v0, q0, g0, p.seed_lo, p.seed_hi, p.scale_rule);
+            const uint32_t s1 = quantize32<SR>(v1, q1, g0 + (uint64_t)p.rows, p.seed_lo, p.seed_hi, p.scale_rule);
             const int sw = lane & 7;
             tout[2 * lane][warp ^ sw] = q0;
             tout[2 * lane + 1][warp ^ sw] = q1;
@@ -252,6 +254,7 @@ struct DualParams {
     uint8_t *ccodes, *cscales;             // column output: [cols, rows/2], scales for (cols x rows)
     int64_t ld_ccodes, ld_cscales, c_katoms;
     uint32_t seed_lo, seed_hi;
+    int scale_rule;                        // MXFP4_SCALE_* >> 4
     uint64_t r_offset, c_offset;           // SR stream index of each output's first element
     uint32_t tiles_c;                      // column tiles
     uint32_t sgn_dup[32];
@@ -335,7 +338,7 @@ __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, 
             }
             if (ok) {
                 uint4 q;
-                const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi);
+                const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
                 uint8_t *codes = job == 0 ? p.ccodes : p.rcodes;
                 uint8_t *scales = job == 0 ? p.cscales : p.rscales;
                 const int64_t ldc = job == 0 ? p.ld_ccodes : p.ld_rcodes;
@@ -423,12 +426,12 @@ __global__ void __launch_bounds__(256, 3) quant_2d_kernel(const QuantParams p) {
                 const float other = __shfl_xor_sync(0xFFFFFFFFu, amax, o);
                 asm("max.NaN.f32 %0, %0, %1;" : "+f"(amax) : "f"(other));
             }
-            const uint32_t code = scale_code_from_amax(amax);
+            const uint32_t code = scale_code_rule(amax, p.scale_rule);
             uint4 packed = make_uint4(0, 0, 0, 0);
             if (code != 0xFFu) {
                 const float inv = inv_scale_from_code(code);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], inv);
+                for (int i = 0; i < 32; ++i) v[i] = scale_element(v[i], inv, p.scale_rule);
                 uint32_t pk[4];
                 if constexpr (!SR) {
 #pragma unroll
@@ -740,7 +743,8 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, int64_t l
     p.elem_offset = elem_offset;
     fill_signs(rht ? rht_sign_mask_hd(seed) : 0u, rht, p.sgn_pair, p.sgn_dup);
     const bool mma = scale_layout == MXFP4_SCALES_MMA;
-    const bool sr = rounding == MXFP4_ROUND_SR;
+    const bool sr = (rounding & 0x0F) == MXFP4_ROUND_SR;
+    p.scale_rule = (rounding >> 4) & 3;
     const bool trans = codes_t != nullptr;
     switch (rht) {
         case 0: return launch_quant_s<0>(layout, trans, mma, sr, p, s);
@@ -792,7 +796,8 @@ cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int6
     p.tiles_c = (uint32_t)((cols + DTC - 1) / DTC);
     uint32_t pair_unused[16];
     fill_signs(col_rht ? rht_sign_mask_hd(seed) : 0u, col_rht, pair_unused, p.sgn_dup);
-    const bool sr = rounding == MXFP4_ROUND_SR, mma = scale_layout == MXFP4_SCALES_MMA;
+    const bool sr = (rounding & 0x0F) == MXFP4_ROUND_SR, mma = scale_layout == MXFP4_SCALES_MMA;
+    p.scale_rule = (rounding >> 4) & 3;
     const bool do_row = rcodes != nullptr, do_col = ccodes != nullptr;
     switch (col_rht) {
         case 0: return launch_dual_r<0>(sr, mma, do_row, do_col, p, s);

@@ -54,6 +54,10 @@ def test_invalid_arguments_rejected_without_gpu():
     assert L.mxfp4_quantize(fake, 32, 64, 64, 0, 0, 0, 0, 0, fake, 32, fake, 2, 0, fake, 16, None, 0, None) == 1
     # misaligned leading dimension
     assert L.mxfp4_quantize(fake, 32, 64, 68, 0, 0, 0, 0, 0, fake, 32, fake, 2, 0, None, 0, None, 0, None) == 2
+    # rounding: unknown rounding mode, unknown scale rule, stray bits
+    for bad in (2, 0x30, 0x40, 0x101):
+        assert L.mxfp4_quantize(fake, 32, 64, 64, 0, 0, bad, 0, 0, fake, 32, fake, 2, 0, None, 0, None, 0,
+                                None) == 1
     # GEMM: K not a multiple of 64 -> unsupported; not of 32 -> invalid
     assert L.mxfp4_gemm(fake, 16, fake, fake, 16, fake, 128, 128, 96, fake, 128, None) == 3
     assert L.mxfp4_gemm(fake, 16, fake, fake, 16, fake, 128, 128, 80, fake, 128, None) == 1

@@ -186,3 +186,55 @@ def test_dual_single_outputs_and_offsets():
     qr, qc = mx.mxfp4_quantize_dual(dev_bf16(x), 32, mx.ROUND_SR, 5, col_elem_offset=8, row=False)
     assert qr is None
     assert np.array_equal(host(qc.codes), oracle.quantize(x, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_SR, 5, 8)[0])
+
+
+RULES = [(mx.SCALE_ROUNDUP, oracle.SCALE_ROUNDUP), (mx.SCALE_PRESCALE_34, oracle.SCALE_PRESCALE_34)]
+
+
+@pytest.mark.parametrize("rule", RULES)
+@pytest.mark.parametrize("rnd", [mx.ROUND_RNE, mx.ROUND_SR])
+@pytest.mark.parametrize("rht", [0, 32])
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_scale_rules_bit_exact(layout, rht, rnd, rule):
+    rows, cols = SHAPES[layout]
+    x = synth.student_t_bf16((rows, cols), seed=500 + layout + rht)
+    trans = layout == mx.LAYOUT_2D
+    q = mx.mxfp4_quantize(dev_bf16(x), layout, rht, rnd, 42, transposed_copy=trans, scale_rule=rule[0])
+    ref = oracle.quantize(x, layout, rht, rnd, 42, transposed_copy=trans, scale_rule=rule[1])
+    assert np.array_equal(host(q.codes), ref[0])
+    assert np.array_equal(host(q.scales), ref[1])
+    if trans:
+        assert np.array_equal(host(q.codes_t), ref[2])
+
+
+@pytest.mark.parametrize("rule", RULES)
+def test_scale_rules_every_bf16_pattern(rule):
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    a = np.random.default_rng(6).permutation(allbits).reshape(256, 256)
+    b = a.copy()
+    b[:, ::32] = 0x40C0                                   # 6.0: the round-up boundary
+    x = np.concatenate([a, b], axis=0)
+    for layout in LAYOUTS:
+        for rnd in (mx.ROUND_RNE, mx.ROUND_SR):
+            q = mx.mxfp4_quantize(dev_bf16(x), layout, 0, rnd, 9, scale_rule=rule[0])
+            ref = oracle.quantize(x, layout, 0, rnd, 9, scale_rule=rule[1])
+            assert np.array_equal(host(q.codes), ref[0]), (layout, rnd)
+            assert np.array_equal(host(q.scales), ref[1]), (layout, rnd)
+
+
+@pytest.mark.parametrize("rule", RULES)
+def test_scale_rules_dual(rule):
+    x = synth.student_t_bf16((256, 384), seed=510)
+    qr, qc = mx.mxfp4_quantize_dual(dev_bf16(x), 32, mx.ROUND_SR, 42, scale_rule=rule[0])
+    cr, sr_ = oracle.quantize(x, oracle.LAYOUT_1D_ROW, 0, oracle.ROUND_SR, 42, scale_rule=rule[1])
+    cc, sc = oracle.quantize(x, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_SR, 42, scale_rule=rule[1])
+    assert np.array_equal(host(qr.codes), cr) and np.array_equal(host(qr.scales), sr_)
+    assert np.array_equal(host(qc.codes), cc) and np.array_equal(host(qc.scales), sc)
+
+
+def test_bad_rounding_bits_rejected():
+    x = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    for bad in (2, 0x30, 0x40, 0x100):
+        with pytest.raises(mx.MXFP4Error) as e:
+            mx.mxfp4_quantize(x, mx.LAYOUT_1D_ROW, rounding=bad)
+        assert e.value.status == mx.MXFP4_ERR_INVALID_ARG
