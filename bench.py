@@ -353,6 +353,15 @@ def sweep_bench(mx, torch, device, peaks, nbytes=1 << 30, reps=5):
                                                     "dequant_GBps": round(gd),
                                                     "dequant_frac_hbm": round(gd / peaks["hbm"], 3)}
                 del q
+    # the scale-rule variants cost no extra traffic; measured on the 1D-row and 2D RNE paths
+    for layout, lname in ((mx.LAYOUT_1D_ROW, "row"), (mx.LAYOUT_2D, "2d")):
+        sbytes = 1 / 1024 if layout == mx.LAYOUT_2D else 1 / 32
+        for rule, rname in ((mx.SCALE_ROUNDUP, "roundup"), (mx.SCALE_PRESCALE_34, "prescale34")):
+            q = mx.mxfp4_quantize(x, layout, 0, mx.ROUND_RNE, 42, scale_rule=rule)
+            tq = _timed(torch, lambda: mx.mxfp4_quantize(x, layout, 0, mx.ROUND_RNE, 42, out=q, scale_rule=rule), reps)
+            gq = n * (2 + 0.5 + sbytes) / (tq / 1e3) / 1e9
+            res[f"{lname}_rht0_rne_{rname}"] = {"quant_GBps": round(gq), "quant_frac_hbm": round(gq / peaks["hbm"], 3)}
+            del q
     if mx.mxfp4_get_error() != mx.MXFP4_OK:
         raise RuntimeError("device-side error in the sweep")
     del x, out

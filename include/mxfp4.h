@@ -242,6 +242,35 @@ MXFP4_API int mxfp4_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint
                        int64_t N, int64_t K, float *c, int64_t ldc, void *stream);
 
 /*
+ * mxfp4_grouped_gemm_wgrad -- per group (expert) g:
+ *     C_g[M, N] = sum over k in [group_offsets[g], group_offsets[g+1]) of
+ *                 A[:, k] B[:, k]^T
+ * the weight gradient of an MoE layer, dW_g = dY_g^T X_g, whose reduction
+ * runs over the tokens routed to expert g.  ("Conversion rules": block dot
+ * products summed in FP32; ALTO abstract: hybrid 1D/2D quantization, here the
+ * 1D blocks along tokens of both operands.)  A and B are the 1D-column
+ * quantizations of the expert-sorted routed tensors (dY [K, M] and X [K, N]),
+ * so their blocks of 32 tokens never straddle two experts when every group
+ * offset is a multiple of 128.
+ *
+ * a_codes [M, K/2] (lda bytes), a_scales MMA layout for (M x K); b_codes
+ * [N, K/2] (ldb), b_scales MMA layout for (N x K); group_offsets: DEVICE int32
+ * [num_groups + 1], multiples of 128, non-decreasing, group_offsets[num_groups]
+ * <= K (token rows between a group's routed rows and the next offset are
+ * padding and must be zero in A or B); c [num_groups * M, N] FP32 (ldc),
+ * group g's output in rows [g * M, (g + 1) * M), fully overwritten (zero for
+ * an empty group).  A bad offset is reported through mxfp4_get_error() as
+ * MXFP4_ERR_INVALID_ARG and empties its group.
+ *
+ * Requirements: M, N >= 1; 1 <= num_groups <= 1024; K % 128 == 0; alignment
+ * as for mxfp4_gemm.
+ */
+MXFP4_API int mxfp4_grouped_gemm_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales,
+                                       const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
+                                       const int32_t *group_offsets, int num_groups, int64_t M, int64_t N,
+                                       int64_t K, float *c, int64_t ldc, void *stream);
+
+/*
  * mxfp4_get_error -- synchronize `stream`, then return and clear the first
  * error any kernel of this library recorded on the current device since the
  * last call (MXFP4_OK if none): MXFP4_ERR_TIMEOUT for a bounded wait that

@@ -40,7 +40,8 @@ OUT_BF16, OUT_F32 = 0, 1
 
 ABI_FUNCTIONS = (
     "mxfp4_status_string", "mxfp4_version", "mxfp4_mma_scales_bytes", "mxfp4_mma_scale_offset",
-    "mxfp4_quantize", "mxfp4_quantize_dual", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_grouped_gemm", "mxfp4_get_error",
+    "mxfp4_quantize", "mxfp4_quantize_dual", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_grouped_gemm",
+    "mxfp4_grouped_gemm_wgrad", "mxfp4_get_error",
     "mxfp4_set_wait_limit_ns", "mxfp4_wait_probe",
 )
 
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.mxfp4_gemm.restype = i32
         L.mxfp4_grouped_gemm.argtypes = [vp, i64, vp, i64, vp, vp, i32, vp, i64, vp, i64, i64, vp, i64, vp]
         L.mxfp4_grouped_gemm.restype = i32
+        L.mxfp4_grouped_gemm_wgrad.argtypes = [vp, i64, vp, vp, i64, vp, vp, i32, i64, i64, i64, vp, i64, vp]
+        L.mxfp4_grouped_gemm_wgrad.restype = i32
         L.mxfp4_get_error.argtypes = [vp]
         L.mxfp4_get_error.restype = i32
         L.mxfp4_set_wait_limit_ns.argtypes = [u64]
@@ -247,6 +250,23 @@ def mxfp4_grouped_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, group_offs
                                   _ptr(group_sizes), G, _ptr(b_codes), b_codes.stride(-2), _ptr(b_scales), N, K,
                                   _ptr(out), out.stride(0), _stream(stream))
     _check(rc, "mxfp4_grouped_gemm")
+    return out
+
+
+def mxfp4_grouped_gemm_wgrad(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor,
+                             b_scales: torch.Tensor, group_offsets: torch.Tensor, K: int,
+                             out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per group g: C_g = A[:, K range g] B[:, K range g]^T (the MoE weight
+    gradient).  a_codes [M, K/2], b_codes [N, K/2]; group_offsets is a device
+    int32 tensor of G + 1 offsets along K; returns [G * M, N] FP32."""
+    M, N = a_codes.shape[0], b_codes.shape[0]
+    G = group_offsets.numel() - 1
+    if out is None:
+        out = torch.empty((G * M, N), dtype=torch.float32, device=a_codes.device)
+    rc = lib().mxfp4_grouped_gemm_wgrad(_ptr(a_codes), a_codes.stride(0), _ptr(a_scales), _ptr(b_codes),
+                                        b_codes.stride(0), _ptr(b_scales), _ptr(group_offsets), G, M, N, K,
+                                        _ptr(out), out.stride(0), _stream(stream))
+    _check(rc, "mxfp4_grouped_gemm_wgrad")
     return out
 
 

@@ -25,6 +25,9 @@ int launch_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, co
 int launch_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
                         const int32_t *offsets, const int32_t *sizes, int G, const uint8_t *b_codes, int64_t ldb,
                         const uint8_t *b_scales, int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s);
+int launch_grouped_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                         int64_t ldb, const uint8_t *b_scales, const int32_t *offsets, int G, int64_t M, int64_t N,
+                         int64_t K, float *c, int64_t ldc, cudaStream_t s);
 int get_error(cudaStream_t s);
 int launch_wait_probe(int arrive, cudaStream_t s);
 uint64_t set_wait_limit(uint64_t ns);
@@ -197,6 +200,19 @@ int mxfp4_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_sca
     if (a_rows > (int64_t)1 << 31 || (int64_t)num_groups * N > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
     return mxfp4::launch_grouped_gemm(a_codes, lda, a_scales, a_rows, group_offsets, group_sizes, num_groups,
                                       b_codes, ldb, b_scales, N, K, c, ldc, static_cast<cudaStream_t>(stream));
+}
+
+int mxfp4_grouped_gemm_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                             int64_t ldb, const uint8_t *b_scales, const int32_t *group_offsets, int num_groups,
+                             int64_t M, int64_t N, int64_t K, float *c, int64_t ldc, void *stream) {
+    if (!group_offsets || num_groups <= 0 || M <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (num_groups > 1024) return MXFP4_ERR_UNSUPPORTED;
+    const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc);
+    if (rc != MXFP4_OK) return rc;
+    if (K % 128) return MXFP4_ERR_INVALID_ARG;
+    if (M > (int64_t)1 << 31 || (int64_t)num_groups * M > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    return mxfp4::launch_grouped_wgrad(a_codes, lda, a_scales, b_codes, ldb, b_scales, group_offsets, num_groups, M,
+                                       N, K, c, ldc, static_cast<cudaStream_t>(stream));
 }
 
 int mxfp4_get_error(void *stream) { return mxfp4::get_error(static_cast<cudaStream_t>(stream)); }

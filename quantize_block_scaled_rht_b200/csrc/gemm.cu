@@ -143,20 +143,44 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
 }
 
 struct TileInfo {
-    int64_t row0;       // first A/C row of this CTA's half
+    int64_t row0;       // first A row of this CTA's half
+    int64_t c_row0;     // first C row of this CTA's half
     int rows_valid;     // rows of this CTA's half that belong to the problem (grouped: to the group)
     int64_t n0;         // first C column
     int64_t b_row;      // TMA row coordinate of the first B row of the pair tile
     int64_t sfb_rt_base;  // first 128-row scale tile of this B operand (expert)
+    int64_t k0;         // first K element of the tile's reduction (grouped K: the group's offset)
+    int64_t kg;         // K elements of the reduction
 };
 
+// Kernel modes: dense; grouped rows (per-expert row ranges of A, one B per
+// expert); grouped K (per-expert K ranges of both operands, one C per expert).
+constexpr int MODE_DENSE = 0, MODE_GROUPED_M = 1, MODE_GROUPED_K = 2;
+
 // Pair tile t -> coordinates.  Dense: M in steps of 256 (fastest), then N.
-// Grouped: group g owns cum[g+1] - cum[g] pair tiles.
-template <int BN, bool GROUPED>
+// Grouped rows: group g owns cum[g+1] - cum[g] pair tiles.  Grouped K: group
+// g owns tiles_m x tiles_n tiles of its [M, N] output over K range
+// [cum[g], cum[g+1]) (cum holds the validated K offsets).
+template <int BN, int MODE>
 __device__ __forceinline__ TileInfo get_tile(int t, uint32_t rank, const GemmParams &p, const int *cum,
                                              int tiles_n) {
     TileInfo ti;
-    if constexpr (!GROUPED) {
+    ti.k0 = 0;
+    ti.kg = p.K;
+    if constexpr (MODE == MODE_GROUPED_K) {
+        const int tiles_m = (int)((p.M + 255) / 256);
+        const int g = t / (tiles_m * tiles_n), local = t - g * (tiles_m * tiles_n);
+        const int tm = local % tiles_m, tn = local / tiles_m;
+        ti.row0 = (int64_t)tm * 256 + 128 * rank;
+        ti.c_row0 = (int64_t)g * p.M + ti.row0;
+        const int64_t left = p.M - ti.row0;
+        ti.rows_valid = left <= 0 ? 0 : (left < BM ? (int)left : BM);
+        ti.n0 = (int64_t)tn * BN;
+        ti.b_row = ti.n0;
+        ti.sfb_rt_base = 0;
+        ti.k0 = cum[g];
+        ti.kg = (int64_t)cum[g + 1] - cum[g];
+    } else if constexpr (MODE == MODE_DENSE) {
         const int tiles_m = (int)((p.M + 255) / 256);
         const int tm = t % tiles_m, tn = t / tiles_m;
         ti.row0 = (int64_t)tm * 256 + 128 * rank;
@@ -165,6 +189,7 @@ __device__ __forceinline__ TileInfo get_tile(int t, uint32_t rank, const GemmPar
         ti.n0 = (int64_t)tn * BN;
         ti.b_row = ti.n0;
         ti.sfb_rt_base = 0;
+        ti.c_row0 = ti.row0;
     } else {
         int g = 0;
         while (g + 1 < p.num_groups && cum[g + 1] <= t) ++g;
@@ -179,6 +204,7 @@ __device__ __forceinline__ TileInfo get_tile(int t, uint32_t rank, const GemmPar
         ti.n0 = (int64_t)tn * BN;
         ti.b_row = (int64_t)g * p.N + ti.n0;
         ti.sfb_rt_base = (int64_t)g * p.b_rowtiles;
+        ti.c_row0 = ti.row0;
     }
     return ti;
 }
@@ -232,7 +258,7 @@ __device__ __noinline__ void issue_stage_tail(uint32_t d_tmem, uint32_t st, uint
     }
 }
 
-template <class Cfg, bool GROUPED>
+template <class Cfg, int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     mxfp4_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                       const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ CUtensorMap tma_sfa,
@@ -245,13 +271,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     uint8_t *stage_base = smem;
     uint8_t *epi_base = smem + STAGES * STAGE_BYTES;
     Shared *sh = reinterpret_cast<Shared *>(epi_base + EPI_BYTES);
-    __shared__ int cum[GROUPED ? MAX_GROUPS + 1 : 1];
+    constexpr bool GROUPED = MODE == MODE_GROUPED_M;
+    __shared__ int cum[MODE != MODE_DENSE ? MAX_GROUPS + 1 : 1];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();               // 0 = MMA issuer of the pair
     const int pair = (int)cluster_id_x(), npairs = (int)nclusters_x();
     const int tiles_n = (int)((p.N + BN - 1) / BN);
-    const int ktiles = (int)((p.K + Cfg::KSTEP - 1) / Cfg::KSTEP);
+    auto ktiles_of = [](const TileInfo &ti) { return (int)((ti.kg + Cfg::KSTEP - 1) / Cfg::KSTEP); };
     const uint64_t limit = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
@@ -293,6 +320,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             cum[p.num_groups] = acc;
             sh->ntiles = acc;
         }
+    } else if constexpr (MODE == MODE_GROUPED_K) {
+        if (threadIdx.x == 32 * 2) {
+            // K offsets: multiples of 128, non-decreasing, within K; a bad
+            // entry records INVALID_ARG and empties the group
+            int prev = 0;
+            bool bad = false;
+            for (int g = 0; g <= p.num_groups; ++g) {
+                int o = p.group_offsets[g];
+                if (o % 128 != 0 || o < prev || o > p.K) { bad = true; o = prev; }
+                cum[g] = o;
+                prev = o;
+            }
+            if (bad && rank == 0) record_error(MXFP4_ERR_INVALID_ARG);
+            sh->ntiles = p.num_groups * (int)((p.M + 255) / 256) * tiles_n;
+        }
     } else {
         if (threadIdx.x == 0) sh->ntiles = (int)((p.M + 255) / 256) * tiles_n;
     }
@@ -313,9 +355,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             int s = 0;
             uint32_t ph = 0;
             for (int t = pair; t < ntiles && !sh->abort; t += npairs) {
-                const TileInfo ti = get_tile<BN, GROUPED>(t, rank, p, cum, tiles_n);
+                const TileInfo ti = get_tile<BN, MODE>(t, rank, p, cum, tiles_n);
                 const int32_t sfa_rt = (int32_t)(ti.row0 / 128);
                 const int32_t sfb_rt = (int32_t)(ti.sfb_rt_base + ti.n0 / 128);
+                const int ktiles = ktiles_of(ti);
+                const int32_t katom0 = (int32_t)(ti.k0 / 128);       // grouped K: the group's first scale atom
                 bool ok = true;
                 for (int kt = 0; kt < ktiles; ++kt) {
                     if (!wait_phase(&sh->empty[s], ph ^ 1u, sh, limit)) { ok = false; break; }
@@ -329,15 +373,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                         if (rank == 0) mbar_arrive_expect_tx(&sh->full[s], Cfg::STAGE_TX);
 #pragma unroll
                         for (int c = 0; c < KCH; ++c) {
-                            const int32_t kx = (kt * KCH + c) * CHUNK;
+                            const int32_t kx = (int32_t)(ti.k0 / 2) + (kt * KCH + c) * CHUNK;
                             tma_load_2d_pair(st + c * Cfg::A_CHUNK, &tma_a, kx, (int32_t)ti.row0, full_leader);
                             tma_load_2d_pair(st + A_BYTES + c * Cfg::B_CHUNK, &tma_b, kx,
                                              (int32_t)(ti.b_row + rank * (BN / 2)), full_leader);
                         }
                         // scale atoms: NATOM consecutive K atoms of one (A) or NRT (B) 128-row tiles
-                        tma_load_3d_pair(st + A_BYTES + B_BYTES, &tma_sfa, 0, kt * NATOM, sfa_rt, full_leader);
-                        tma_load_3d_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &tma_sfb, 0, kt * NATOM, sfb_rt,
+                        tma_load_3d_pair(st + A_BYTES + B_BYTES, &tma_sfa, 0, katom0 + kt * NATOM, sfa_rt,
                                          full_leader);
+                        tma_load_3d_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &tma_sfb, 0, katom0 + kt * NATOM,
+                                         sfb_rt, full_leader);
                     }
                     __syncwarp();
                     if (++s == STAGES) { s = 0; ph ^= 1u; }
@@ -362,17 +407,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             int acc = 0;
             uint32_t acc_ph = 0;
             for (int t = pair; t < ntiles && !sh->abort; t += npairs) {
-                const TileInfo ti = get_tile<BN, GROUPED>(t, 0, p, cum, tiles_n);
+                const TileInfo ti = get_tile<BN, MODE>(t, 0, p, cum, tiles_n);
                 const int64_t rt0 = ti.n0 / 128;
                 const uint32_t b_shift = (uint32_t)((ti.n0 - rt0 * 128) / 32);
                 if (!wait_phase(&sh->tmem_empty[acc], acc_ph ^ 1u, sh, limit)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (acc ? Cfg::ACC1_COL : 0u);
+                const int ktiles = ktiles_of(ti);
                 bool ok = true;
                 for (int kt = 0; kt < ktiles; ++kt) {
                     if (!wait_phase(&sh->full[s], ph, sh, limit)) { ok = false; break; }
                     tc_fence_after();
-                    const int64_t kleft = p.K - (int64_t)kt * Cfg::KSTEP;
+                    const int64_t kleft = ti.kg - (int64_t)kt * Cfg::KSTEP;
                     const uint32_t sfa_col = tmem + Cfg::SF_COL + Cfg::SF_STAGE_COLS * (kglobal & 1u);
                     const uint32_t st = smem_u32(stage_base + s * STAGE_BYTES);
                     if (kleft >= Cfg::KSTEP)
@@ -405,16 +451,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         uint32_t acc_ph = 0;
         uint32_t buf_i = 0;
         for (int t = pair; t < ntiles; t += npairs) {
-            const TileInfo ti = get_tile<BN, GROUPED>(t, rank, p, cum, tiles_n);
+            const TileInfo ti = get_tile<BN, MODE>(t, rank, p, cum, tiles_n);
             if (!wait_phase(&sh->tmem_full[acc], acc_ph, sh, limit)) break;
             tc_fence_after();
             const int row_lo = 32 * q;
-            const bool full_box = !GROUPED || (row_lo + 32 <= ti.rows_valid);
+            const bool full_box = MODE == MODE_DENSE || (row_lo + 32 <= ti.rows_valid);
             const bool any_row = row_lo < ti.rows_valid;
+            const bool empty_k = ti.kg <= 0;              // grouped K: an empty group's output is zero
             for (int j = 0; j < BN / 32; ++j) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (acc ? Cfg::ACC1_COL : 0u) + 32u * j, v);
                 tmem_ld_wait();
+                if (empty_k) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0u;
+                }
                 if (j == BN / 32 - 1) {
                     tc_fence_before();
                     __syncwarp();
@@ -437,12 +488,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        tma_store_2d(&tma_c, (int32_t)col0, (int32_t)(ti.row0 + row_lo), buf);
+                        tma_store_2d(&tma_c, (int32_t)col0, (int32_t)(ti.c_row0 + row_lo), buf);
                         bulk_commit_group();
                     }
                     ++buf_i;
                 } else if (row_lo + lane < ti.rows_valid) {
-                    float *dst = p.c + (ti.row0 + row_lo + lane) * p.ldc + col0;
+                    float *dst = p.c + (ti.c_row0 + row_lo + lane) * p.ldc + col0;
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         const int64_t cc = col0 + 4 * c;
@@ -548,14 +599,14 @@ static int sm_count() {
     return n > 0 ? n : 148;
 }
 
-template <class Cfg, bool GROUPED>
+template <class Cfg, int MODE>
 static cudaError_t set_smem_attr() {
     // once per device and instantiation: keep cudaFuncSetAttribute off the hot path
     static int done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<Cfg, GROUPED>,
+    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<Cfg, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
     return e;
@@ -570,10 +621,13 @@ struct GemmArgs {
 };
 
 // Returns 0 on success, MXFP4_ERR_CUDA when a map or launch fails.
-template <class Cfg, bool GROUPED>
+// Grouped K: a and b are [M, K/2] and [N, K/2] over all groups' K ranges, c is
+// [G * M, N]; the B operand and C map cover G groups only in grouped-rows mode.
+template <class Cfg, int MODE>
 static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
     constexpr int BN = Cfg::BN;
-    const int G = GROUPED ? g.G : 1;
+    const int G = MODE == MODE_GROUPED_M ? g.G : 1;
+    const int64_t c_rows = MODE == MODE_GROUPED_K ? (int64_t)g.G * g.M : g.M;
     const int64_t katoms = mma_katoms(g.K);
     const int64_t a_tiles = (g.M + 127) / 128, b_tiles = (g.N + 127) / 128;
     CUtensorMap ta, tb, tc, tsa, tsb;
@@ -581,14 +635,14 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
                   (uint64_t)g.lda, CHUNK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b_codes, (uint64_t)(g.K / 2), (uint64_t)G * g.N,
                   (uint64_t)g.ldb, CHUNK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.c, (uint64_t)g.N, (uint64_t)g.M, (uint64_t)g.ldc * 4, 32,
-                  32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.c, (uint64_t)g.N, (uint64_t)c_rows, (uint64_t)g.ldc * 4,
+                  32, 32, CU_TENSOR_MAP_SWIZZLE_128B) ||
         // scale atoms as a 3D tensor [128-row tile][K atom][512 bytes = 128 x 32-bit]:
         // one box holds NATOM consecutive atoms of one (A) or NRT (B) row tiles
         !make_map_3d(&tsa, g.a_scales, (uint64_t)katoms, (uint64_t)a_tiles, Cfg::NATOM, 1) ||
         !make_map_3d(&tsb, g.b_scales, (uint64_t)katoms, (uint64_t)(G * b_tiles), Cfg::NATOM, Cfg::NRT))
         return MXFP4_ERR_CUDA;
-    if (set_smem_attr<Cfg, GROUPED>() != cudaSuccess) return MXFP4_ERR_CUDA;
+    if (set_smem_attr<Cfg, MODE>() != cudaSuccess) return MXFP4_ERR_CUDA;
     GemmParams p{};
     p.M = g.M; p.N = g.N; p.K = g.K;
     p.katoms = katoms;
@@ -598,11 +652,11 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
     p.wait_limit_ns = g_wait_limit_ns;
     const int pairs_max = sm_count() / 2;
     int pairs = pairs_max;
-    if (!GROUPED) {
-        const int64_t tiles = ((g.M + 255) / 256) * ((g.N + BN - 1) / BN);
+    if (MODE != MODE_GROUPED_M) {
+        const int64_t tiles = (MODE == MODE_GROUPED_K ? g.G : 1) * ((g.M + 255) / 256) * ((g.N + BN - 1) / BN);
         pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
     }
-    const cudaError_t e = launch_pdl(mxfp4_gemm_kernel<Cfg, GROUPED>, dim3((unsigned)(2 * pairs)), dim3(NUM_THREADS),
+    const cudaError_t e = launch_pdl(mxfp4_gemm_kernel<Cfg, MODE>, dim3((unsigned)(2 * pairs)), dim3(NUM_THREADS),
                                      (size_t)Cfg::SMEM_BYTES, s, ta, tb, tc, tsa, tsb, p);
     return e == cudaSuccess ? 0 : MXFP4_ERR_CUDA;
 }
@@ -610,14 +664,21 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
 int launch_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes, int64_t ldb,
                 const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s) {
     GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, M, N, K, ldc, c, nullptr, nullptr, 1};
-    return launch_cfg<DefaultCfg, false>(g, s);
+    return launch_cfg<DefaultCfg, MODE_DENSE>(g, s);
 }
 
 int launch_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
                         const int32_t *offsets, const int32_t *sizes, int G, const uint8_t *b_codes, int64_t ldb,
                         const uint8_t *b_scales, int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s) {
     GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, a_rows, N, K, ldc, c, offsets, sizes, G};
-    return launch_cfg<DefaultCfg, true>(g, s);
+    return launch_cfg<DefaultCfg, MODE_GROUPED_M>(g, s);
+}
+
+int launch_grouped_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                         int64_t ldb, const uint8_t *b_scales, const int32_t *offsets, int G, int64_t M, int64_t N,
+                         int64_t K, float *c, int64_t ldc, cudaStream_t s) {
+    GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, M, N, K, ldc, c, offsets, nullptr, G};
+    return launch_cfg<DefaultCfg, MODE_GROUPED_K>(g, s);
 }
 
 int get_error(cudaStream_t s) {

@@ -179,3 +179,84 @@ def test_bounded_wait_reports_timeout_and_context_survives():
         mx.mxfp4_set_wait_limit_ns(old)
     # the context is still usable
     test_gemm_shapes(128, 192, 64)
+
+
+def _routed_wgrad_case(sizes, M, N, seed):
+    """Expert-sorted routed tensors dY [K, M] and X [K, N] with groups padded
+    to 128 rows (padding rows zero), and the offsets along K."""
+    g = np.random.default_rng(seed)
+    padded = [((s + 127) // 128) * 128 for s in sizes]
+    offsets = np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+    K = int(offsets[-1])
+    dy = np.zeros((K, M), np.float32)
+    x = np.zeros((K, N), np.float32)
+    for e, s in enumerate(sizes):
+        o = offsets[e]
+        dy[o:o + s] = g.standard_normal((s, M)) * 1e-3
+        x[o:o + s] = g.standard_normal((s, N))
+    return synth.bf16_bits(dy), synth.bf16_bits(x), offsets, K
+
+
+@pytest.mark.parametrize("sizes", [[200, 0, 513, 128], [1024], [0, 0, 300]])
+def test_grouped_wgrad_matches_oracle(sizes):
+    M, N = 320, 224
+    dy, x, offsets, K = _routed_wgrad_case(sizes, M, N, seed=len(sizes) + sum(sizes))
+    qa = mx.mxfp4_quantize(dev_bf16(dy), mx.LAYOUT_1D_COL, 32, mx.ROUND_SR, 42, scale_layout=mx.SCALES_MMA)
+    qb = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_COL, 32, mx.ROUND_RNE, 42, scale_layout=mx.SCALES_MMA)
+    c = mx.mxfp4_grouped_gemm_wgrad(qa.codes, qa.scales, qb.codes, qb.scales,
+                                    torch.from_numpy(offsets).cuda(), K)
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    c = host(c)
+    ca, sa = oracle.quantize(dy, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_SR, 42)
+    cb, sb = oracle.quantize(x, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_RNE, 42)
+    for e in range(len(sizes)):
+        o0, o1 = int(offsets[e]), int(offsets[e + 1])
+        ce = c[e * M:(e + 1) * M]
+        if o1 == o0:
+            assert np.all(ce == 0.0)
+            continue
+        ref, s = oracle.gemm(ca[:, o0 // 2:o1 // 2], sa[:, o0 // 32:o1 // 32], cb[:, o0 // 2:o1 // 2],
+                             sb[:, o0 // 32:o1 // 32], o1 - o0)
+        assert_gemm_close(ce.astype(np.float64), ref, s)
+
+
+def test_grouped_wgrad_bad_offset_reported():
+    M, N = 128, 128
+    dy, x, offsets, K = _routed_wgrad_case([128, 128], M, N, seed=3)
+    qa = mx.mxfp4_quantize(dev_bf16(dy), mx.LAYOUT_1D_COL, scale_layout=mx.SCALES_MMA)
+    qb = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_COL, scale_layout=mx.SCALES_MMA)
+    bad = torch.tensor([0, 64, 256], dtype=torch.int32, device="cuda")
+    mx.mxfp4_grouped_gemm_wgrad(qa.codes, qa.scales, qb.codes, qb.scales, bad, K)
+    assert mx.mxfp4_get_error() == mx.MXFP4_ERR_INVALID_ARG
+
+
+def test_grouped_dgrad_with_transposed_weight_copies():
+    """MoE dgrad: dX_e = dY_e W_e, with B_e the 2D transposed copy of expert
+    e's weight (W and W^T share one quantization)."""
+    sizes, I, H = [100, 0, 260], 256, 192
+    g = np.random.default_rng(11)
+    padded = [((s + 127) // 128) * 128 for s in sizes]
+    offsets = np.concatenate([[0], np.cumsum(padded)]).astype(np.int32)
+    rows = int(offsets[-1])
+    dy = np.zeros((rows, I), np.float32)
+    for e, s in enumerate(sizes):
+        dy[offsets[e]:offsets[e] + s] = g.standard_normal((s, I)) * 1e-3
+    dy = synth.bf16_bits(dy)
+    ws = [synth.normal_bf16((I, H), 30 + e, 0.02) for e in range(len(sizes))]
+    qa = mx.mxfp4_quantize(dev_bf16(dy), mx.LAYOUT_1D_ROW, 0, mx.ROUND_SR, 42, scale_layout=mx.SCALES_MMA)
+    qw = [mx.mxfp4_quantize(dev_bf16(w), mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA, transposed_copy=True) for w in ws]
+    c = mx.mxfp4_grouped_gemm(qa.codes, qa.scales, torch.from_numpy(offsets).cuda(),
+                              torch.tensor(sizes, dtype=torch.int32, device="cuda"),
+                              torch.stack([q.codes_t for q in qw]), torch.cat([q.scales_t for q in qw]), H, I)
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    c = host(c)
+    ca, sa = oracle.quantize(dy, oracle.LAYOUT_1D_ROW, 0, oracle.ROUND_SR, 42)
+    for e, s in enumerate(sizes):
+        if s == 0:
+            continue
+        cw, sw, cwt = oracle.quantize(ws[e], oracle.LAYOUT_2D, transposed_copy=True)
+        o = int(offsets[e])
+        pairs = [(o + r, n) for r in range(0, s, 7) for n in range(0, H, 5)] + [(o + s - 1, H - 1)]
+        ref, sabs = oracle.gemm_entries(ca, sa, cwt, sw, I, pairs, 0, 2)
+        got = np.array([c[m, n] for m, n in pairs], np.float64)
+        assert_gemm_close(got, ref, sabs)
