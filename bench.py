@@ -287,43 +287,79 @@ def _timed(torch, fn, reps):
 
 def grouped_bench(mx, torch, device, peaks, reps=10):
     """Grouped MoE GEMMs on 16384 tokens routed top-4 of 32 experts (Zipf 1.2,
-    rows sorted by expert, groups padded to 128 rows): gate_up 2880 -> 5760 and
-    down 2880 -> 2880.  Activations N(0,1) and weights N(0, 0.02^2) are drawn on
-    the device with seeded generators (the recipe of synth.grouped_inputs) and
-    quantized by the library (1D RNE rows, 2D RNE weights).  The operands
-    (A 94 MB, B up to 265 MB) and outputs (up to 1.5 GB) exceed L2, so no flush
-    is needed between launches."""
+    rows sorted by expert, groups padded to 128 rows), forward and backward of
+    the expert layers: gate_up 2880 -> 5760 and down 2880 -> 2880 (fprop), and
+    for gate_up the dgrad (dY W_e through the 2D transposed weight copies) and
+    the wgrad (dW_e = dY_e^T X_e over each expert's tokens, both operands
+    quantized along tokens with RHT-32).  Activations N(0,1), gradients
+    N(0, 1e-3^2) and weights N(0, 0.02^2) are drawn on the device with seeded
+    generators (the recipe of synth.grouped_inputs), padding rows zero, and
+    quantized by the library.  Operands (A 94-190 MB, B up to 265 MB) and
+    outputs (0.75-2.1 GB) exceed L2, so no flush is needed between launches.
+    TFLOP/s count the routed rows, not the padding."""
     E, H, I = synth.EXPERTS, synth.HIDDEN, synth.INTERMEDIATE
     choice = synth.route_tokens(synth.MOE_TOKENS, E, seed=6)
     _, offsets, sizes, total = synth.grouped_layout(choice, E)
+    valid = np.zeros(total, bool)
+    for e in range(E):
+        valid[offsets[e]:offsets[e] + sizes[e]] = True
+    pad = torch.from_numpy(~valid).to(device)
     g = torch.Generator(device=device)
     g.manual_seed(5)
     a = torch.randn((total, H), generator=g, device=device).to(torch.bfloat16)
+    a[pad] = 0
     qa = mx.mxfp4_quantize(a, mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
-    del a
     off_d = torch.from_numpy(offsets).to(device)
     size_d = torch.from_numpy(sizes).to(device)
     routed = int(sizes.sum())
     out = {}
+
+    def record(name, ms, flops, shape):
+        tf = flops / (ms / 1e3) / 1e12
+        out[name] = {"us": ms * 1e3, "TFLOP/s": tf, "frac_fp4_peak": tf / (4 * peaks["bf16"]), "shape": shape}
+
+    wt_codes = wt_scales = None
     for name, n_out, seed in (("gate_up", I, 8), ("down", H, 9)):
         g.manual_seed(seed)
-        codes, scales = [], []
+        codes, scales, codes_t, scales_t = [], [], [], []
         for _ in range(E):
             w = (torch.randn((n_out, H), generator=g, device=device) * 0.02).to(torch.bfloat16)
-            q = mx.mxfp4_quantize(w, mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA)
+            q = mx.mxfp4_quantize(w, mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA, transposed_copy=name == "gate_up")
             codes.append(q.codes)
             scales.append(q.scales)
+            if name == "gate_up":
+                codes_t.append(q.codes_t)
+                scales_t.append(q.scales_t)
         b_codes, b_scales = torch.stack(codes), torch.cat(scales)
-        del codes, scales
+        if name == "gate_up":
+            wt_codes, wt_scales = torch.stack(codes_t), torch.cat(scales_t)
+        del codes, scales, codes_t, scales_t
         c = torch.empty((qa.codes.shape[0], n_out), dtype=torch.float32, device=device)
         ms = _timed(torch, lambda: mx.mxfp4_grouped_gemm(qa.codes, qa.scales, off_d, size_d, b_codes, b_scales,
                                                           n_out, H, out=c), reps)
-        if mx.mxfp4_get_error() != mx.MXFP4_OK:
-            raise RuntimeError("device-side error in the grouped GEMM")
-        tf = 2.0 * routed * n_out * H / (ms / 1e3) / 1e12
-        out[name] = {"us": ms * 1e3, "TFLOP/s": tf, "frac_fp4_peak": tf / (4 * peaks["bf16"]),
-                     "shape": f"{routed} routed rows ({qa.codes.shape[0]} padded) x {n_out} x {H}"}
+        record(name, ms, 2.0 * routed * n_out * H, f"{routed} routed rows ({total} padded) x {n_out} x {H}")
         del b_codes, b_scales, c
+
+    # backward of gate_up: dgrad through W^T copies, wgrad over each expert's tokens
+    g.manual_seed(4)
+    dy = (torch.randn((total, I), generator=g, device=device) * 1e-3).to(torch.bfloat16)
+    dy[pad] = 0
+    qdy = mx.mxfp4_quantize(dy, mx.LAYOUT_1D_ROW, 0, mx.ROUND_SR, synth.SR_SEED, scale_layout=mx.SCALES_MMA)
+    c = torch.empty((total, H), dtype=torch.float32, device=device)
+    ms = _timed(torch, lambda: mx.mxfp4_grouped_gemm(qdy.codes, qdy.scales, off_d, size_d, wt_codes, wt_scales,
+                                                      H, I, out=c), reps)
+    record("gate_up_dgrad", ms, 2.0 * routed * H * I, f"{routed} routed rows ({total} padded) x {H} x {I}")
+    del c, qdy, wt_codes, wt_scales
+    qdyt = mx.mxfp4_quantize(dy, mx.LAYOUT_1D_COL, 32, mx.ROUND_SR, synth.SR_SEED, scale_layout=mx.SCALES_MMA)
+    qxt = mx.mxfp4_quantize(a, mx.LAYOUT_1D_COL, 32, mx.ROUND_RNE, synth.SR_SEED, scale_layout=mx.SCALES_MMA)
+    del dy, a
+    c = torch.empty((E * I, H), dtype=torch.float32, device=device)
+    ms = _timed(torch, lambda: mx.mxfp4_grouped_gemm_wgrad(qdyt.codes, qdyt.scales, qxt.codes, qxt.scales, off_d,
+                                                            total, out=c), reps)
+    record("gate_up_wgrad", ms, 2.0 * routed * I * H, f"{E} experts x {I} x {H}, K = {routed} routed rows")
+    if mx.mxfp4_get_error() != mx.MXFP4_OK:
+        raise RuntimeError("device-side error in the grouped GEMMs")
+    del c, qdyt, qxt, qa
     torch.cuda.empty_cache()
     return out
 

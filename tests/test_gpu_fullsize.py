@@ -79,9 +79,14 @@ def test_expert_gemms_sampled(expert_step):
     _check_sampled(host(st.dw), cdyt, sdyt, cxt, sxt, T, _sample_pairs(I, H, 2000, 3))
 
 
-def test_grouped_moe_gate_up_sampled():
+@pytest.fixture(scope="module")
+def moe():
+    return synth.grouped_inputs()
+
+
+def test_grouped_moe_gate_up_sampled(moe):
     """16384 tokens x 2880, top-4 of 32 experts (Zipf 1.2), gate_up 2880 -> 5760."""
-    d = synth.grouped_inputs()
+    d = moe
     E, N, K = synth.EXPERTS, synth.INTERMEDIATE, synth.HIDDEN
     rows = d["a"].shape[0]
     qa = mx.mxfp4_quantize(dev_bf16(d["a"]), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
@@ -107,6 +112,66 @@ def test_grouped_moe_gate_up_sampled():
         ref, s = oracle.gemm_entries(ca, sa, cw, sw, K, pairs, 0, 1)
         got = np.array([c[m, nn] for m, nn in pairs], np.float64)
         assert_gemm_close(got, ref, s)
+
+
+def test_grouped_moe_backward_sampled(moe):
+    """Backward of the gate_up expert layer on the same routing: dgrad
+    dX_e = dY_e W_e through the 2D transposed weight copies, and wgrad
+    dW_e = dY_e^T X_e over each expert's tokens (operands quantized along
+    tokens with RHT-32; SR for dY).  Sampled entries against the oracle, which
+    quantizes only the sampled rows / columns (with their stream offsets)."""
+    d = moe
+    E, I, H = synth.EXPERTS, synth.INTERMEDIATE, synth.HIDDEN
+    offsets, sizes = d["offsets"], d["sizes"]
+    total = d["a"].shape[0]
+    valid = d["row_token"] >= 0
+    dy = np.zeros((total, I), np.uint16)
+    dy[valid] = synth.normal_bf16((int(valid.sum()), I), 12, 1e-3)
+    seed = synth.SR_SEED
+    qdy = mx.mxfp4_quantize(dev_bf16(dy), mx.LAYOUT_1D_ROW, 0, mx.ROUND_SR, seed, scale_layout=mx.SCALES_MMA)
+    experts = [0, 1, 17, 31]
+    codes_t, scales_t = [], []
+    for e in range(E):
+        q = mx.mxfp4_quantize(dev_bf16(d["w_gate_up"][e]), mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA,
+                              transposed_copy=True)
+        codes_t.append(q.codes_t)
+        scales_t.append(q.scales_t)
+    off_d, size_d = torch.from_numpy(offsets).cuda(), torch.from_numpy(sizes).cuda()
+    dx = host(mx.mxfp4_grouped_gemm(qdy.codes, qdy.scales, off_d, size_d, torch.stack(codes_t),
+                                    torch.cat(scales_t), H, I))
+    del codes_t, scales_t, qdy
+    qdyt = mx.mxfp4_quantize(dev_bf16(dy), mx.LAYOUT_1D_COL, 32, mx.ROUND_SR, seed, scale_layout=mx.SCALES_MMA)
+    qxt = mx.mxfp4_quantize(dev_bf16(d["a"]), mx.LAYOUT_1D_COL, 32, mx.ROUND_RNE, seed, scale_layout=mx.SCALES_MMA)
+    dw = mx.mxfp4_grouped_gemm_wgrad(qdyt.codes, qdyt.scales, qxt.codes, qxt.scales, off_d, total)
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    g = np.random.default_rng(13)
+    for e in experts:
+        o, n = int(offsets[e]), int(sizes[e])
+        if n == 0:
+            continue
+        _, sw, cwt = oracle.quantize(d["w_gate_up"][e], oracle.LAYOUT_2D, transposed_copy=True)
+        # dgrad: sampled rows of the expert, quantized with their stream offsets
+        for r in np.unique(np.concatenate([g.integers(0, n, 4), [n - 1]])):
+            row = o + int(r)
+            ca, sa = oracle.quantize(dy[row:row + 1], oracle.LAYOUT_1D_ROW, 0, oracle.ROUND_SR, seed,
+                                     elem_offset=row * I)
+            cols = [int(c) for c in g.integers(0, H, 6)] + [H - 1]
+            ref, s = oracle.gemm_entries(ca, sa, cwt, sw, I, [(0, c) for c in cols], 0, 2)
+            assert_gemm_close(dx[row, cols].astype(np.float64), ref, s)
+        # wgrad: sampled (m, n) of dW_e from single columns of dY and X over the expert's tokens
+        k0, k1 = o, int(offsets[e + 1])
+        for m, col in zip(g.integers(0, I, 4), g.integers(0, H, 4)):
+            m, col = int(m), int(col)
+            ca, sa = oracle.quantize(np.ascontiguousarray(dy[:, m:m + 1]), oracle.LAYOUT_1D_COL, 32,
+                                     oracle.ROUND_SR, seed, elem_offset=m * total)
+            cb, sb = oracle.quantize(np.ascontiguousarray(d["a"][:, col:col + 1]), oracle.LAYOUT_1D_COL, 32,
+                                     oracle.ROUND_RNE, seed, elem_offset=col * total)
+            ref, s = oracle.gemm_entries(ca[:, k0 // 2:k1 // 2], sa[:, k0 // 32:k1 // 32], cb[:, k0 // 2:k1 // 2],
+                                         sb[:, k0 // 32:k1 // 32], k1 - k0, [(0, 0)])
+            got = float(dw[e * I + m, col].item())
+            assert_gemm_close(np.array([got]), ref, s)
+    del qdyt, qxt, dw
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("layout", [mx.LAYOUT_1D_ROW, mx.LAYOUT_1D_COL, mx.LAYOUT_2D])
