@@ -144,107 +144,42 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const QuantParams p) {
     }
 }
 
-// ---------------------------------------------------------------------------
-// 1D column blocks (output = transposed view).  A CTA stages a 256 x 64 bf16
-// tile in shared memory with coalesced 16-byte copies; warp w quantizes the
-// 32-row block w of the tile, lane l the two columns 2l and 2l+1; the codes of
-// the 64 output rows x 128 bytes go back through shared memory so that the
-// global stores are full 128-byte lines.
-// ---------------------------------------------------------------------------
+// Tile of the column dequantizer: 256 rows x 64 columns of the output.
 constexpr int COL_TR = 256, COL_TC = 64;
 
+// 16-byte global -> shared copy that bypasses L1 (cp.async.cg).
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-template <int RHT, bool SR, bool MMA>
-__global__ void __launch_bounds__(256) quant_col_kernel(const QuantParams p) {
-    pdl_wait();
-    pdl_trigger();
-    __shared__ __align__(16) uint32_t tin[COL_TR][COL_TC / 2];   // 32 KB: bf16 pairs
-    __shared__ __align__(16) uint4 tout[COL_TC][COL_TR / 32];    // 8 KB: 64 rows x 128 B
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t tiles_r = (p.rows + COL_TR - 1) / COL_TR;
-    const int64_t tiles_c = (p.cols + COL_TC - 1) / COL_TC;
-    const int64_t ntiles = tiles_r * tiles_c;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
-        const int64_t r0 = tr * COL_TR, c0 = tc * COL_TC;
-        // load: 256 rows x 8 chunks of 16 B
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int row = (tid >> 3) + 32 * i, ch = tid & 7;
-            const int64_t gr = r0 + row, gc = c0 + 8 * ch;
-            if (gr < p.rows && gc < p.cols) cp_async16(&tin[row][4 * ch], p.x + gr * p.ld_x + gc);
-        }
-        cp_async_wait_all();
-        __syncthreads();
-        const int64_t rb = r0 + 32 * warp;        // first input row of this warp's block
-        const int64_t oc = c0 + 2 * lane;         // first of the two output rows of this lane
-        const bool blk_ok = rb < p.rows;
-        if (blk_ok && oc < p.cols) {
-            float v0[32], v1[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                uint32_t u = tin[32 * warp + i][lane];
-                if constexpr (RHT) u ^= p.sgn_dup[i % RHT];
-                v0[i] = bf16lo(u);
-                v1[i] = bf16hi(u);
-            }
-            if constexpr (RHT) {
-                const float c = rht_norm<RHT>();
-#pragma unroll
-                for (int s = 0; s < 32; s += RHT) { fwht<RHT>(v0 + s); fwht<RHT>(v1 + s); }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) { v0[i] = __fmul_rn(v0[i], c); v1[i] = __fmul_rn(v1[i], c); }
-            }
-            const int64_t kb = rb >> 5;           // output K-block
-            uint4 q0, q1;
-            const uint64_t g0 = (uint64_t)(oc * p.rows + rb) + p.elem_offset;
-            const uint32_t s0 = quantize32<SR>(v0, q0, g0, p.seed_lo, p.seed_hi, p.scale_rule);
-            const uint32_t s1 = quantize32<SR>(v1, q1, g0 + (uint64_t)p.rows, p.seed_lo, p.seed_hi, p.scale_rule);
-            const int sw = lane & 7;
-            tout[2 * lane][warp ^ sw] = q0;
-            tout[2 * lane + 1][warp ^ sw] = q1;
-            if constexpr (MMA) {
-                p.scales[mma_scale_off(oc, kb, p.katoms)] = (uint8_t)s0;
-                p.scales[mma_scale_off(oc + 1, kb, p.katoms)] = (uint8_t)s1;
-            } else {
-                p.scales[oc * p.ld_scales + kb] = (uint8_t)s0;
-                p.scales[(oc + 1) * p.ld_scales + kb] = (uint8_t)s1;
-            }
-        }
-        __syncthreads();
-        // store: 64 output rows x 8 chunks of 16 B
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const int row = (tid >> 3) + 32 * i, ch = tid & 7;
-            const int64_t orow = c0 + row, rin = r0 + 32 * ch;
-            if (orow < p.cols && rin < p.rows)
-                stg_v4(p.codes + orow * p.ld_codes + (rin >> 1), tout[row][ch ^ ((row >> 1) & 7)]);
-        }
-        __syncthreads();
-    }
-}
 
 // ---------------------------------------------------------------------------
 // Dual output: 1D-row blocks (no RHT) and 1D-column blocks (optional RHT along
 // rows) of the same tensor from one read.  The recipe quantizes activations
 // and gradients both ways (row blocks for fprop/dgrad, blocks along tokens for
-// wgrad).  One CTA per 64 x 128 bf16 tile (cp.async into shared memory, 272-byte
-// row pitch so that both access patterns below are conflict-free); many small
-// CTAs per SM hide the load latency and balance the tail.  Each thread does one
-// column job and one row job, through one inlined quantizer body:
-//   column job: thread (column c, row block b) reads 32 rows of column c,
-//     applies the RHT and stores 16 bytes of transposed codes;
+// wgrad).  A CTA streams TR x TC bf16 tiles through a double-buffered
+// shared-memory ring (cp.async; the row pitch is padded by 16 bytes, which
+// keeps both access patterns below conflict-free).  Each thread does one
+// column job and one row job through one inlined quantizer body:
+//   column job: thread (column c, row block b) reads 32 rows of column c and
+//     applies the RHT; the 16 bytes of transposed codes are staged in shared
+//     memory so that each output row leaves as TR/2 contiguous bytes;
 //   row job: thread (row r, column block b) reads 64 bytes of its row and
 //     stores 16 bytes of codes.
-// Either output may be disabled (DO_ROW / DO_COL).
+// Either output may be disabled (DO_ROW / DO_COL); the column-only form with
+// tall 128 x 64 tiles is the 1D-column quantizer.
 // ---------------------------------------------------------------------------
-constexpr int DTR = 64, DTC = 128;         // tile rows, tile columns
-constexpr int DPITCH = DTC + 8;            // bf16 per smem row (272 bytes)
+template <int TR_, int TC_>
+struct DualTile {
+    static constexpr int TR = TR_, TC = TC_;          // tile rows, tile columns (TR * TC = 8192)
+    static constexpr int PITCH = TC + 8;              // bf16 per smem row
+    static constexpr int OCH = TR / 32;               // 16-byte code chunks per column output row
+    static constexpr int OSH = OCH == 4 ? 1 : 2;      // swizzle of those chunks (conflict-free staging)
+    static_assert(TR * TC == 8192 && (OCH == 2 || OCH == 4), "tile shape");
+};
+using DualBoth = DualTile<64, 128>;                  // row + column outputs
+using DualCol = DualTile<128, 64>;                   // column output only
 
 struct DualParams {
     const uint16_t *x;
@@ -260,19 +195,21 @@ struct DualParams {
     uint32_t sgn_dup[32];
 };
 
-template <int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
+template <class T, int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
 __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, const uint32_t ntiles) {
     pdl_wait();
     pdl_trigger();
-    __shared__ __align__(16) uint16_t tin[2][DTR * DPITCH];
+    constexpr int TR = T::TR, TC = T::TC, PITCH = T::PITCH, OCH = T::OCH;
+    __shared__ __align__(16) uint16_t tin[2][TR * PITCH];
+    __shared__ __align__(16) uint4 tout[DO_COL ? TC * OCH : 1];   // column codes: TC rows x TR/2 bytes
     const int tid = threadIdx.x;
     auto load = [&](uint32_t t, int buf) {
-        const int64_t r0 = (int64_t)(t / p.tiles_c) * DTR, c0 = (int64_t)(t % p.tiles_c) * DTC;
+        const int64_t r0 = (int64_t)(t / p.tiles_c) * TR, c0 = (int64_t)(t % p.tiles_c) * TC;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const int row = (tid >> 4) + 16 * i, ch = tid & 15;
+            const int idx = tid + 256 * i, row = idx / (TC / 8), ch = idx % (TC / 8);
             const int64_t gr = r0 + row, gc = c0 + 8 * ch;
-            if (gr < p.rows && gc < p.cols) cp_async16(tin[buf] + row * DPITCH + 8 * ch, p.x + gr * p.ld_x + gc);
+            if (gr < p.rows && gc < p.cols) cp_async16(tin[buf] + row * PITCH + 8 * ch, p.x + gr * p.ld_x + gc);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
@@ -290,7 +227,7 @@ __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, 
         }
         __syncthreads();
         const uint16_t *tile = tin[buf];
-        const int64_t r0 = (int64_t)(t / p.tiles_c) * DTR, c0 = (int64_t)(t % p.tiles_c) * DTC;
+        const int64_t r0 = (int64_t)(t / p.tiles_c) * TR, c0 = (int64_t)(t % p.tiles_c) * TC;
 
 #pragma unroll 1
         for (int job = DO_COL ? 0 : 1; job < (DO_ROW ? 2 : 1); ++job) {
@@ -298,15 +235,17 @@ __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, 
             bool ok;
             uint64_t g0;
             int64_t orow, kb;
+            int c = 0, b = 0;
             if (job == 0) {                                  // column c, rows 32b .. 32b+31
-                const int c = tid & 127, b = tid >> 7;
+                c = tid % TC;
+                b = tid / TC;
                 orow = c0 + c;
                 const int64_t rin = r0 + 32 * b;
                 ok = orow < p.cols && rin < p.rows;
-                const uint16_t *col = tile + 32 * b * DPITCH + c;
+                const uint16_t *col = tile + 32 * b * PITCH + c;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    uint32_t u = (uint32_t)col[i * DPITCH] << 16;
+                    uint32_t u = (uint32_t)col[i * PITCH] << 16;
                     if constexpr (CRHT) u ^= p.sgn_dup[i % CRHT] & 0x80000000u;
                     v[i] = __uint_as_float(u);
                 }
@@ -320,11 +259,12 @@ __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, 
                 g0 = (uint64_t)(orow * p.rows + rin) + p.c_offset;
                 kb = rin >> 5;
             } else {                                         // row r, columns 32b .. 32b+31
-                const int r = tid & 63, b = tid >> 6;
+                const int r = tid % TR;
+                b = tid / TR;
                 orow = r0 + r;
                 const int64_t gc = c0 + 32 * b;
                 ok = orow < p.rows && gc < p.cols;
-                const uint4 *s4 = reinterpret_cast<const uint4 *>(tile + r * DPITCH + 32 * b);
+                const uint4 *s4 = reinterpret_cast<const uint4 *>(tile + r * PITCH + 32 * b);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const uint4 u = s4[q];
@@ -339,13 +279,24 @@ __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, 
             if (ok) {
                 uint4 q;
                 const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
-                uint8_t *codes = job == 0 ? p.ccodes : p.rcodes;
-                uint8_t *scales = job == 0 ? p.cscales : p.rscales;
-                const int64_t ldc = job == 0 ? p.ld_ccodes : p.ld_rcodes;
-                stg_v4(codes + orow * ldc + kb * 16, q);
-                if constexpr (MMA) scales[mma_scale_off(orow, kb, job == 0 ? p.c_katoms : p.r_katoms)] = (uint8_t)sc;
-                else scales[orow * (job == 0 ? p.ld_cscales : p.ld_rscales) + kb] = (uint8_t)sc;
+                if (job == 0) {
+                    tout[c * OCH + (b ^ ((c >> T::OSH) & (OCH - 1)))] = q;
+                    if constexpr (MMA) p.cscales[mma_scale_off(orow, kb, p.c_katoms)] = (uint8_t)sc;
+                    else p.cscales[orow * p.ld_cscales + kb] = (uint8_t)sc;
+                } else {
+                    stg_v4(p.rcodes + orow * p.ld_rcodes + kb * 16, q);
+                    if constexpr (MMA) p.rscales[mma_scale_off(orow, kb, p.r_katoms)] = (uint8_t)sc;
+                    else p.rscales[orow * p.ld_rscales + kb] = (uint8_t)sc;
+                }
             }
+        }
+        if constexpr (DO_COL) {
+            __syncthreads();
+            // column codes: TC output rows x OCH chunks of 16 bytes, one chunk per thread
+            const int row = tid / OCH, ch = tid % OCH;
+            const int64_t orow = c0 + row, rin = r0 + 32 * ch;
+            if (orow < p.cols && rin < p.rows)
+                stg_v4(p.ccodes + orow * p.ld_ccodes + (rin >> 1), tout[row * OCH + (ch ^ ((row >> T::OSH) & (OCH - 1)))]);
         }
         __syncthreads();                                     // the load after next overwrites this buffer
     }
@@ -696,13 +647,14 @@ static int64_t grid_for(int64_t items, int threads) {
 }
 
 template <int RHT, bool SR, bool MMA>
+static cudaError_t launch_col_dual(const QuantParams &q, cudaStream_t s);
+
+template <int RHT, bool SR, bool MMA>
 static cudaError_t launch_quant_t(int layout, bool trans, const QuantParams &p, cudaStream_t s) {
     if (layout == MXFP4_LAYOUT_1D_ROW) {
         return launch_pdl(quant_row_kernel<RHT, SR, MMA>, dim3((unsigned)grid_for(p.rows * (p.cols / 32), 256)), dim3(256), 0, s, p);
     } else if (layout == MXFP4_LAYOUT_1D_COL) {
-        const int64_t tiles = ((p.rows + COL_TR - 1) / COL_TR) * ((p.cols + COL_TC - 1) / COL_TC);
-        const int64_t cap = (int64_t)num_sms() * 8;
-        return launch_pdl(quant_col_kernel<RHT, SR, MMA>, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(256), 0, s, p);
+        return launch_col_dual<RHT, SR, MMA>(p, s);      // the dual kernel, column output only
     } else {
         const int br = trans ? Q2Tile<true>::BR : Q2Tile<false>::BR;
         const int64_t tiles = ((p.rows / 32 + br - 1) / br) * ((p.cols / 32 + 8 / br - 1) / (8 / br));
@@ -753,11 +705,12 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, int64_t l
     }
 }
 
-template <int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
-static cudaError_t launch_dual_t(const DualParams &p, cudaStream_t s) {
-    const uint64_t tiles = (uint64_t)((p.rows + DTR - 1) / DTR) * p.tiles_c;
+template <class T, int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
+static cudaError_t launch_dual_t(DualParams p, cudaStream_t s) {
+    p.tiles_c = (uint32_t)((p.cols + T::TC - 1) / T::TC);
+    const uint64_t tiles = (uint64_t)((p.rows + T::TR - 1) / T::TR) * p.tiles_c;
     if (tiles > 0xFFFFFFFFull - 0x7FFFFFFFull) return cudaErrorInvalidValue;   // tile index fits 32 bits
-    auto kern = quant_dual_kernel<CRHT, SR, MMA, DO_ROW, DO_COL>;
+    auto kern = quant_dual_kernel<T, CRHT, SR, MMA, DO_ROW, DO_COL>;
     // RNE is memory-bound: a persistent grid at full occupancy keeps the next
     // tile's load in flight.  SR is ALU-bound: one CTA per tile lets the
     // hardware scheduler balance the tail.
@@ -766,11 +719,26 @@ static cudaError_t launch_dual_t(const DualParams &p, cudaStream_t s) {
     return launch_pdl(kern, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(256), 0, s, p, (uint32_t)tiles);
 }
 
+// 1D-column quantization: the column-only dual kernel on 128 x 64 tiles.
+template <int RHT, bool SR, bool MMA>
+static cudaError_t launch_col_dual(const QuantParams &q, cudaStream_t s) {
+    DualParams p{};
+    p.x = q.x;
+    p.rows = q.rows; p.cols = q.cols; p.ld_x = q.ld_x;
+    p.ccodes = q.codes; p.ld_ccodes = q.ld_codes;
+    p.cscales = q.scales; p.ld_cscales = q.ld_scales; p.c_katoms = q.katoms;
+    p.seed_lo = q.seed_lo; p.seed_hi = q.seed_hi;
+    p.scale_rule = q.scale_rule;
+    p.c_offset = q.elem_offset;
+    for (int i = 0; i < 32; ++i) p.sgn_dup[i] = q.sgn_dup[i];
+    return launch_dual_t<DualCol, RHT, SR, MMA, false, true>(p, s);
+}
+
 template <int CRHT, bool SR, bool MMA>
 static cudaError_t launch_dual_o(bool do_row, bool do_col, const DualParams &p, cudaStream_t s) {
-    if (do_row && do_col) return launch_dual_t<CRHT, SR, MMA, true, true>(p, s);
-    if (do_col) return launch_dual_t<CRHT, SR, MMA, false, true>(p, s);
-    return launch_dual_t<CRHT, SR, MMA, true, false>(p, s);
+    if (do_row && do_col) return launch_dual_t<DualBoth, CRHT, SR, MMA, true, true>(p, s);
+    if (do_col) return launch_dual_t<DualCol, CRHT, SR, MMA, false, true>(p, s);
+    return launch_dual_t<DualBoth, CRHT, SR, MMA, true, false>(p, s);
 }
 
 template <int CRHT>
@@ -793,7 +761,6 @@ cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int6
     p.c_katoms = mma_katoms(rows);
     p.seed_lo = (uint32_t)seed; p.seed_hi = (uint32_t)(seed >> 32);
     p.r_offset = row_offset; p.c_offset = col_offset;
-    p.tiles_c = (uint32_t)((cols + DTC - 1) / DTC);
     uint32_t pair_unused[16];
     fill_signs(col_rht ? rht_sign_mask_hd(seed) : 0u, col_rht, pair_unused, p.sgn_dup);
     const bool sr = (rounding & 0x0F) == MXFP4_ROUND_SR, mma = scale_layout == MXFP4_SCALES_MMA;
