@@ -56,6 +56,21 @@ def lib():
         L.orc_rht_inverse.argtypes = [fp, ctypes.c_int, ctypes.c_uint32]
         L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
         L.orc_f32_to_bf16.restype = ctypes.c_uint16
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint32]
+        L.orc_e4m3_decode.restype = ctypes.c_double
+        L.orc_e4m3_rne.argtypes = [ctypes.c_double]
+        L.orc_e4m3_rne.restype = ctypes.c_uint32
+        L.orc_nvfp4_tensor_scale.argtypes = [ctypes.c_float]
+        L.orc_nvfp4_tensor_scale.restype = ctypes.c_float
+        L.orc_nvfp4_quantize.argtypes = [ctypes.c_void_p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
+                                         ctypes.c_uint64, u8p, i64, u8p, i64, ctypes.POINTER(ctypes.c_float)]
+        L.orc_nvfp4_quantize.restype = ctypes.c_int
+        L.orc_nvfp4_dequantize.argtypes = [u8p, i64, u8p, i64, i64, i64, ctypes.c_int, ctypes.c_float,
+                                           ctypes.POINTER(ctypes.c_float), i64]
+        L.orc_nvfp4_dequantize.restype = ctypes.c_int
+        L.orc_nvfp4_gemm_entry.argtypes = [u8p, i64, u8p, i64, ctypes.c_float, u8p, i64, u8p, i64, ctypes.c_float,
+                                           i64, i64, i64, ctypes.POINTER(ctypes.c_double),
+                                           ctypes.POINTER(ctypes.c_double)]
         L.orc_scale_code_rule.argtypes = [ctypes.c_float, ctypes.c_int]
         L.orc_scale_code_rule.restype = ctypes.c_uint32
         L.orc_quantize.argtypes = [ctypes.c_void_p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -232,5 +247,68 @@ def gemm_entries(a_codes, a_scales, b_codes, b_scales, K: int, pairs, a_mode: in
     for i, (m, n) in enumerate(pairs):
         L.orc_gemm_entry(pa, a_codes.shape[1], pas, a_scales.shape[1], a_mode, pb, b_codes.shape[1], pbs,
                          b_scales.shape[1], b_mode, K, int(m), int(n), ctypes.byref(c), ctypes.byref(s))
+        out_c[i], out_s[i] = c.value, s.value
+    return out_c, out_s
+
+
+# ---- NVFP4 (reading R16 of the C file) ------------------------------------------------
+
+def e4m3_decode(code: int) -> float:
+    return float(lib().orc_e4m3_decode(code))
+
+
+def e4m3_rne(a: float) -> int:
+    """Nearest non-negative E4M3 code (ties to even), saturating at 448."""
+    return int(lib().orc_e4m3_rne(a))
+
+
+def nvfp4_tensor_scale(amax: float) -> float:
+    return float(lib().orc_nvfp4_tensor_scale(amax))
+
+
+def nvfp4_quantize(x_bf16: np.ndarray, layout: int, rnd: int = ROUND_RNE, seed: int = 0, elem_offset: int = 0):
+    """NVFP4 of a bf16 tensor [rows, cols] (uint16 bit patterns): returns
+    (codes, scales (E4M3 bytes, row-major), tensor_amax)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    orows, k = (cols, rows) if layout == LAYOUT_1D_COL else (rows, cols)
+    codes = np.zeros((orows, k // 2), np.uint8)
+    scales = np.zeros((orows, k // 16), np.uint8)
+    amax = ctypes.c_float()
+    rc = lib().orc_nvfp4_quantize(x.ctypes.data, rows, cols, cols, layout, rnd, seed, elem_offset,
+                                  _ptr(codes, ctypes.c_uint8), codes.shape[1], _ptr(scales, ctypes.c_uint8),
+                                  scales.shape[1], ctypes.byref(amax))
+    if rc != 0:
+        raise ValueError("oracle: shape not defined for NVFP4")
+    return codes, scales, float(amax.value)
+
+
+def nvfp4_dequantize(codes, scales, rows: int, cols: int, layout: int, tensor_amax: float) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    out = np.zeros((rows, cols), np.float32)
+    rc = lib().orc_nvfp4_dequantize(_ptr(codes, ctypes.c_uint8), codes.shape[1], _ptr(scales, ctypes.c_uint8),
+                                    scales.shape[1], rows, cols, layout, tensor_amax,
+                                    _ptr(out, ctypes.c_float), cols)
+    if rc != 0:
+        raise ValueError("oracle: shape not defined for NVFP4")
+    return out
+
+
+def nvfp4_gemm_entries(a_codes, a_scales, a_amax: float, b_codes, b_scales, b_amax: float, K: int, pairs):
+    """NVFP4 C[m, n] = A[m, :] B[n, :]^T and sum |terms| for the listed pairs."""
+    a_codes = np.ascontiguousarray(a_codes, np.uint8)
+    b_codes = np.ascontiguousarray(b_codes, np.uint8)
+    a_scales = np.ascontiguousarray(a_scales, np.uint8)
+    b_scales = np.ascontiguousarray(b_scales, np.uint8)
+    out_c = np.zeros(len(pairs), np.float64)
+    out_s = np.zeros(len(pairs), np.float64)
+    c, s = ctypes.c_double(), ctypes.c_double()
+    L = lib()
+    for i, (m, n) in enumerate(pairs):
+        L.orc_nvfp4_gemm_entry(_ptr(a_codes, ctypes.c_uint8), a_codes.shape[1], _ptr(a_scales, ctypes.c_uint8),
+                               a_scales.shape[1], a_amax, _ptr(b_codes, ctypes.c_uint8), b_codes.shape[1],
+                               _ptr(b_scales, ctypes.c_uint8), b_scales.shape[1], b_amax, K, int(m), int(n),
+                               ctypes.byref(c), ctypes.byref(s))
         out_c[i], out_s[i] = c.value, s.value
     return out_c, out_s

@@ -31,6 +31,9 @@
  *             (thesingularityreport.com), abstract: hybrid 1D/2D block
  *             quantization, randomized Hadamard transforms and stochastic
  *             rounding on GPT-OSS-20B.
+ *  [MX-NV]    same page, "Comparison with NVFP4": E2M1 elements in blocks of
+ *             16, an FP8 E4M3 block scale (fractional, fitted to each block),
+ *             a second-level FP32 scale per tensor, 4.5 bits per value.
  *  [PHILOX]   Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as
  *             1, 2, 3", SC'11: the Philox4x32-10 counter-based generator.
  *
@@ -64,6 +67,17 @@
  *      and element 2j+1 in bits 7:4.
  *  R10 2D blocks are 32x32 tiles of the [rows, cols] tensor; the optional
  *      transposed copy stores element (r, c) at row c, position r.
+ *  R16 NVFP4 [MX-NV] (the page gives the format, not the scale rule): tensor
+ *      scale S = fp32(amax_tensor / 2688), 2688 = 6 * 448 so the largest
+ *      block scale is E4M3's maximum; block scale code = E4M3 nearest-even of
+ *      fp32(amax_block / fp32(6 S)), saturating at 448; element divisor
+ *      X = fp32(decode(code) * S); elements fp32(x / X) rounded to E2M1 (RNE
+ *      or SR as R8).  A block whose scale rounds to 0 stores +-0; a tensor
+ *      with amax 0 stores zeros; a NaN or Inf in the tensor makes every
+ *      block scale NaN (0x7F) with codes 0.  E4M3 is the OCP FP8 format:
+ *      bias 7, 3 mantissa bits, subnormals m * 2^-9, no Inf, 0x7F = NaN.
+ *      Blocks run along the last dimension (1D row) or dimension 0 (1D
+ *      column, transposed output), as for MXFP4; no RHT.
  *  R14 Scale rules besides R5 ([MX-CLIP] and the [MX-TRAIN] table):
  *      round-up: the decode scale amax / 6 rounded up to a power of two, that
  *        is the smallest e with 6 * 2^e >= amax, so no element saturates;
@@ -549,6 +563,172 @@ void orc_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int6
         for (int64_t n = 0; n < N; ++n)
             orc_gemm_entry(a_codes, lda, a_scales, ld_as, a_mode, b_codes, ldb, b_scales, ld_bs, b_mode,
                            K, m, n, &c[m * ldc + n], s ? &s[m * lds + n] : NULL);
+}
+
+/* ======================================================================== */
+/* NVFP4 [MX-NV], reading R16.                                                */
+/* ======================================================================== */
+
+/* E4M3 decode: (-1)^s (1 + m/8) 2^(e-7), subnormal m 2^-9, 0x7F/0xFF NaN. */
+double orc_e4m3_decode(uint32_t code)
+{
+    code &= 0xFFu;
+    int sgn = (int)(code >> 7), e = (int)((code >> 3) & 15u), m = (int)(code & 7u);
+    if (e == 15 && m == 7) return NAN;
+    double v = e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+    return sgn ? -v : v;
+}
+
+/* Nearest non-negative E4M3 code to a >= 0 (ties to the even code), by search
+ * over the 127 non-negative finite values; saturates at 448 (code 0x7E). */
+uint32_t orc_e4m3_rne(double a)
+{
+    if (a >= 448.0) return 0x7Eu;
+    int best = 0;
+    double bd = fabs(a);
+    for (int c = 1; c < 0x7F; ++c) {
+        double d = fabs(a - orc_e4m3_decode((uint32_t)c));
+        if (d < bd || (d == bd && (MUT(24) ? (c & 1) == 1 : ((c & 1) == 0 && (best & 1) == 1)))) {
+            best = c;
+            bd = d;
+        }
+    }
+    return (uint32_t)best;
+}
+
+/* Tensor scale S = amax / (6 * 448) in fp32. */
+float orc_nvfp4_tensor_scale(float amax)
+{
+    return amax / (MUT(23) ? 1536.0f : 2688.0f);
+}
+
+/* One NVFP4 block of 16 values with tensor scale S: the scale code and the
+ * element codes (g[i]: SR stream index of element i). */
+static uint32_t nv_block(const float *y, float S, int rnd, uint64_t seed, const uint64_t *g, uint8_t *c4)
+{
+    if (!isfinite(S)) {                                   /* NaN or Inf in the tensor */
+        for (int i = 0; i < 16; ++i) c4[i] = 0;
+        return 0x7Fu;
+    }
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float a = fabsf(y[i]);
+        if (a > amax) amax = a;
+    }
+    uint32_t code = 0;
+    if (S > 0.0f) {
+        float six_s = 6.0f * S;
+        float q = amax / six_s;
+        code = orc_e4m3_rne((double)q);
+    }
+    float X = MUT(26) ? (float)orc_e4m3_decode(code) : (float)orc_e4m3_decode(code) * S;
+    for (int i = 0; i < 16; ++i) {
+        if (X == 0.0f) {                                  /* scale rounded to 0: +-0 */
+            c4[i] = (uint8_t)orc_e2m1_rne(copysignf(0.0f, y[i]));
+            continue;
+        }
+        float v = y[i] / X;
+        c4[i] = (uint8_t)(rnd == ORC_ROUND_SR ? orc_e2m1_sr(v, orc_sr_word(seed, g[i])) : orc_e2m1_rne(v));
+    }
+    return code;
+}
+
+/* amax over a bf16 tensor, NaN if any element is NaN. */
+static float nv_tensor_amax(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x)
+{
+    float amax = 0.0f;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t c = 0; c < cols; ++c) {
+            float v = orc_bf16_to_f32(x[r * ld_x + c]);
+            if (isnan(v)) return NAN;
+            if (fabsf(v) > amax) amax = fabsf(v);
+        }
+    return amax;
+}
+
+/*
+ * NVFP4 quantize of x[rows, cols]: layout 1D_ROW (blocks of 16 along cols;
+ * codes [rows, cols/2], scales [rows, cols/16]) or 1D_COL (blocks along rows,
+ * transposed view: codes [cols, rows/2], scales [cols, rows/16]).  Writes the
+ * tensor amax (the second-level scale is amax / 2688) to *tensor_amax.
+ */
+int orc_nvfp4_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rnd,
+                       uint64_t seed, uint64_t elem_offset, uint8_t *codes, int64_t ld_codes, uint8_t *scales,
+                       int64_t ld_scales, float *tensor_amax)
+{
+    if (layout != ORC_LAYOUT_1D_ROW && layout != ORC_LAYOUT_1D_COL) return -1;
+    int transposed = layout == ORC_LAYOUT_1D_COL;
+    int64_t orows = transposed ? cols : rows;
+    int64_t ocols = transposed ? rows : cols;
+    if (ocols % 16) return -1;
+    float amax_t = nv_tensor_amax(x, rows, cols, ld_x);
+    *tensor_amax = amax_t;
+    float S = isnan(amax_t) ? NAN : orc_nvfp4_tensor_scale(amax_t);
+    #pragma omp parallel for schedule(static)
+    for (int64_t orow = 0; orow < orows; ++orow) {
+        float y[16];
+        uint64_t g[16];
+        uint8_t c4[16];
+        for (int64_t b = 0; b < ocols / 16; ++b) {
+            for (int i = 0; i < 16; ++i) {
+                int64_t ocol = b * 16 + i;
+                int64_t r = transposed ? ocol : orow;
+                int64_t c = transposed ? orow : ocol;
+                y[i] = orc_bf16_to_f32(x[r * ld_x + c]);
+                g[i] = (uint64_t)(orow * ocols + ocol) + elem_offset;
+            }
+            scales[orow * ld_scales + b] = (uint8_t)nv_block(y, S, rnd, seed, g, c4);
+            for (int i = 0; i < 16; ++i) put_nibble(codes + orow * ld_codes, b * 16 + i, c4[i]);
+        }
+    }
+    return 0;
+}
+
+/* NVFP4 dequantize: value = fp32(fp32(decode(code) * decode(scale)) * S). */
+int orc_nvfp4_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
+                         int64_t rows, int64_t cols, int layout, float tensor_amax, float *out, int64_t ld_out)
+{
+    int transposed = layout == ORC_LAYOUT_1D_COL;
+    int64_t orows = transposed ? cols : rows;
+    int64_t ocols = transposed ? rows : cols;
+    if (ocols % 16) return -1;
+    float S = orc_nvfp4_tensor_scale(tensor_amax);
+    for (int64_t orow = 0; orow < orows; ++orow)
+        for (int64_t ocol = 0; ocol < ocols; ++ocol) {
+            float sv = (float)orc_e4m3_decode(scales[orow * ld_scales + ocol / 16]);
+            float e = (float)orc_e2m1_decode(orc_get_nibble(codes + orow * ld_codes, ocol));
+            float v = (e * sv) * S;
+            int64_t r = transposed ? ocol : orow, c = transposed ? orow : ocol;
+            out[r * ld_out + c] = v;
+        }
+    return 0;
+}
+
+/* NVFP4 block dot products: C[m][n] = S_a S_b sum over 16-blocks of
+ * s_a s_b sum a_k b_k in fp64; S[m][n] the matching sum of |terms|. */
+void orc_nvfp4_gemm_entry(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t ld_as,
+                          float a_amax, const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
+                          int64_t ld_bs, float b_amax, int64_t K, int64_t m, int64_t n, double *c_out,
+                          double *s_out)
+{
+    double acc = 0.0, sabs = 0.0;
+    double ts = (double)orc_nvfp4_tensor_scale(a_amax) * (double)orc_nvfp4_tensor_scale(b_amax);
+    for (int64_t kb = 0; kb < K / 16; ++kb) {
+        double xa = orc_e4m3_decode(a_scales[m * ld_as + kb]);
+        double xb = orc_e4m3_decode(b_scales[n * ld_bs + kb]);
+        double dot = 0.0, dabs = 0.0;
+        for (int i = 0; i < 16; ++i) {
+            int64_t k = kb * 16 + i;
+            double a = orc_e2m1_decode(orc_get_nibble(a_codes + m * lda, k));
+            double b = orc_e2m1_decode(orc_get_nibble(b_codes + n * ldb, k));
+            dot += a * b;
+            dabs += fabs(a * b);
+        }
+        acc += xa * xb * dot;
+        sabs += fabs(xa * xb) * dabs;
+    }
+    *c_out = MUT(25) ? acc : acc * ts;
+    if (s_out) *s_out = sabs * fabs(ts);
 }
 
 /* Number of OpenMP threads the oracle runs with (1 without OpenMP). */

@@ -41,10 +41,14 @@ MUTANTS = {
     20: "dequantize skips the inverse RHT",
     21: "round-up scale compares against 5 * 2^e instead of 6 * 2^e",
     22: "3/4 pre-scale also applied to the amax that sets the exponent",
+    23: "NVFP4 tensor scale amax / (6 * 256) instead of / (6 * 448)",
+    24: "E4M3 rounding ties to the odd code",
+    25: "NVFP4 GEMM drops the per-tensor scales",
+    26: "NVFP4 element divisor without the tensor scale",
 }
 
 PIN_FILES = ["test_oracle_format.py", "test_oracle_gemm.py", "test_oracle_quantize.py", "test_oracle_rht.py",
-             "test_oracle_sr.py", "test_oracle_scale_rules.py", "test_oracle_philox.py"]
+             "test_oracle_sr.py", "test_oracle_scale_rules.py", "test_oracle_nvfp4.py", "test_oracle_philox.py"]
 
 
 @pytest.fixture(scope="module")
