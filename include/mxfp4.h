@@ -271,6 +271,51 @@ MXFP4_API int mxfp4_grouped_gemm_wgrad(const uint8_t *a_codes, int64_t lda, cons
                                        int64_t K, float *c, int64_t ldc, void *stream);
 
 /*
+ * NVFP4 ("MXFP4" (aiwiki.ai), "Comparison with NVFP4"): E2M1 elements in
+ * blocks of 16, an FP8 E4M3 block scale, a second-level FP32 scale per
+ * tensor; 4.5 bits per value.  The page gives the format, not the scale
+ * rule; this library's rule: S = amax_tensor / 2688 (2688 = 6 * 448, so the
+ * largest block scale is E4M3's maximum); block scale = E4M3 nearest-even of
+ * amax_block / (6 S), saturating at 448; X = fp32(scale * S); elements
+ * fp32(x / X) rounded to E2M1 (nearest-even, or MXFP4_ROUND_SR with the
+ * Philox stream of mxfp4_quantize).  A block whose scale rounds to 0 stores
+ * +-0; a NaN or Inf in the tensor gives every block the NaN scale 0x7F.
+ *
+ * mxfp4_nvfp4_quantize: computes the tensor amax into *tensor_amax (a DEVICE
+ * float owned by the caller, overwritten; keep it for dequantize and the
+ * GEMM), then quantizes.  layout 1D_ROW: blocks of 16 along cols, codes
+ * [rows, cols/2], scales [rows, cols/16] bytes (ROWMAJOR) or the MMA layout
+ * for a (rows x cols) NVFP4 operand (atoms of 4 blocks of 16); 1D_COL: blocks
+ * along rows, transposed output (codes [cols, rows/2]).  No RHT.
+ * Requirements: rows, cols multiples of 16; x, codes 16-byte aligned; ld_x %
+ * 8 == 0; ld_codes % 16 == 0; elem_offset % 4 == 0; rounding RNE or SR.
+ */
+MXFP4_API int mxfp4_nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout,
+                                   int rounding, uint64_t seed, uint64_t elem_offset, float *tensor_amax,
+                                   uint8_t *codes, int64_t ld_codes, uint8_t *scales, int64_t ld_scales,
+                                   int scale_layout, void *stream);
+
+/*
+ * mxfp4_nvfp4_dequantize: out = fp32(fp32(code * scale) * S), S from the
+ * DEVICE float *tensor_amax; out FP32 [rows, cols] (ld_out elements, 16-byte
+ * aligned, ld_out % 4 == 0); layout and scale layout as for quantize.
+ */
+MXFP4_API int mxfp4_nvfp4_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales,
+                                     int64_t ld_scales, int scale_layout, const float *tensor_amax, int64_t rows,
+                                     int64_t cols, int layout, float *out, int64_t ld_out, void *stream);
+
+/*
+ * mxfp4_nvfp4_gemm: C[M, N] = S_a S_b * sum over 16-blocks of s_a s_b sum a b,
+ * FP32 accumulation (tcgen05.mma kind::mxf4nvf4, UE4M3 scales per 16), the
+ * second-level scales applied in the epilogue from the DEVICE floats a_amax,
+ * b_amax written by mxfp4_nvfp4_quantize.  Scales in the MMA layout;
+ * otherwise as mxfp4_gemm.
+ */
+MXFP4_API int mxfp4_nvfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const float *a_amax,
+                               const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, const float *b_amax,
+                               int64_t M, int64_t N, int64_t K, float *c, int64_t ldc, void *stream);
+
+/*
  * mxfp4_get_error -- synchronize `stream`, then return and clear the first
  * error any kernel of this library recorded on the current device since the
  * last call (MXFP4_OK if none): MXFP4_ERR_TIMEOUT for a bounded wait that

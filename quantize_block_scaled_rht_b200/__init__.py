@@ -41,7 +41,8 @@ OUT_BF16, OUT_F32 = 0, 1
 ABI_FUNCTIONS = (
     "mxfp4_status_string", "mxfp4_version", "mxfp4_mma_scales_bytes", "mxfp4_mma_scale_offset",
     "mxfp4_quantize", "mxfp4_quantize_dual", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_grouped_gemm",
-    "mxfp4_grouped_gemm_wgrad", "mxfp4_get_error",
+    "mxfp4_grouped_gemm_wgrad", "mxfp4_nvfp4_quantize", "mxfp4_nvfp4_dequantize", "mxfp4_nvfp4_gemm",
+    "mxfp4_get_error",
     "mxfp4_set_wait_limit_ns", "mxfp4_wait_probe",
 )
 
@@ -84,6 +85,12 @@ def lib() -> ctypes.CDLL:
         L.mxfp4_grouped_gemm.restype = i32
         L.mxfp4_grouped_gemm_wgrad.argtypes = [vp, i64, vp, vp, i64, vp, vp, i32, i64, i64, i64, vp, i64, vp]
         L.mxfp4_grouped_gemm_wgrad.restype = i32
+        L.mxfp4_nvfp4_quantize.argtypes = [vp, i64, i64, i64, i32, i32, u64, u64, vp, vp, i64, vp, i64, i32, vp]
+        L.mxfp4_nvfp4_quantize.restype = i32
+        L.mxfp4_nvfp4_dequantize.argtypes = [vp, i64, vp, i64, i32, vp, i64, i64, i32, vp, i64, vp]
+        L.mxfp4_nvfp4_dequantize.restype = i32
+        L.mxfp4_nvfp4_gemm.argtypes = [vp, i64, vp, vp, vp, i64, vp, vp, i64, i64, i64, vp, i64, vp]
+        L.mxfp4_nvfp4_gemm.restype = i32
         L.mxfp4_get_error.argtypes = [vp]
         L.mxfp4_get_error.restype = i32
         L.mxfp4_set_wait_limit_ns.argtypes = [u64]
@@ -267,6 +274,73 @@ def mxfp4_grouped_gemm_wgrad(a_codes: torch.Tensor, a_scales: torch.Tensor, b_co
                                         b_codes.stride(0), _ptr(b_scales), _ptr(group_offsets), G, M, N, K,
                                         _ptr(out), out.stride(0), _stream(stream))
     _check(rc, "mxfp4_grouped_gemm_wgrad")
+    return out
+
+
+@dataclass
+class NvQuantized:
+    """NVFP4 codes, E4M3 block scales and the device tensor amax (a 1-element
+    float32 tensor) of one tensor."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    amax: torch.Tensor
+    rows: int
+    k: int
+    layout: int
+    scale_layout: int
+
+
+def nv_mma_scales_bytes(rows: int, k: int) -> int:
+    """Bytes of NVFP4 scales in the MMA layout: 512-byte atoms of 128 rows x 4 blocks of 16."""
+    return ((rows + 127) // 128) * ((k // 16 + 3) // 4) * 512
+
+
+def mxfp4_nvfp4_quantize(x: torch.Tensor, layout: int = LAYOUT_1D_ROW, rounding: int = ROUND_RNE, seed: int = 0,
+                         elem_offset: int = 0, scale_layout: int = SCALES_ROWMAJOR, stream=None,
+                         out: Optional[NvQuantized] = None) -> NvQuantized:
+    """NVFP4 quantization (see mxfp4_nvfp4_quantize in include/mxfp4.h)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    orows, k = (cols, rows) if layout == LAYOUT_1D_COL else (rows, cols)
+    if out is None:
+        dev = x.device
+        codes = torch.empty((orows, k // 2), dtype=torch.uint8, device=dev)
+        if scale_layout == SCALES_MMA:
+            scales = torch.zeros((nv_mma_scales_bytes(orows, k),), dtype=torch.uint8, device=dev)
+        else:
+            scales = torch.empty((orows, k // 16), dtype=torch.uint8, device=dev)
+        out = NvQuantized(codes, scales, torch.empty(1, dtype=torch.float32, device=dev), orows, k, layout,
+                          scale_layout)
+    ld_sc = out.scales.shape[1] if out.scales.dim() == 2 else 0
+    rc = lib().mxfp4_nvfp4_quantize(_ptr(x), rows, cols, x.stride(0), layout, rounding, seed & 0xFFFFFFFFFFFFFFFF,
+                                    elem_offset, _ptr(out.amax), _ptr(out.codes), out.codes.stride(0),
+                                    _ptr(out.scales), ld_sc, scale_layout, _stream(stream))
+    _check(rc, "mxfp4_nvfp4_quantize")
+    return out
+
+
+def mxfp4_nvfp4_dequantize(q: NvQuantized, rows: int, cols: int, out: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.float32, device=q.codes.device)
+    ld_sc = q.scales.shape[1] if q.scales.dim() == 2 else 0
+    rc = lib().mxfp4_nvfp4_dequantize(_ptr(q.codes), q.codes.stride(0), _ptr(q.scales), ld_sc, q.scale_layout,
+                                      _ptr(q.amax), rows, cols, q.layout, _ptr(out), out.stride(0), _stream(stream))
+    _check(rc, "mxfp4_nvfp4_dequantize")
+    return out
+
+
+def mxfp4_nvfp4_gemm(a: NvQuantized, b: NvQuantized, out: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """C = A B^T for NVFP4 operands quantized with SCALES_MMA."""
+    M, N, K = a.rows, b.rows, a.k
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32, device=a.codes.device)
+    rc = lib().mxfp4_nvfp4_gemm(_ptr(a.codes), a.codes.stride(0), _ptr(a.scales), _ptr(a.amax), _ptr(b.codes),
+                                b.codes.stride(0), _ptr(b.scales), _ptr(b.amax), M, N, K, _ptr(out), out.stride(0),
+                                _stream(stream))
+    _check(rc, "mxfp4_nvfp4_gemm")
     return out
 
 

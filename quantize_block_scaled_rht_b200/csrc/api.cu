@@ -28,6 +28,16 @@ int launch_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_sc
 int launch_grouped_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
                          int64_t ldb, const uint8_t *b_scales, const int32_t *offsets, int G, int64_t M, int64_t N,
                          int64_t K, float *c, int64_t ldc, cudaStream_t s);
+cudaError_t launch_nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rounding,
+                                  uint64_t seed, uint64_t elem_offset, float *tensor_amax, uint8_t *codes,
+                                  int64_t ld_codes, uint8_t *scales, int64_t ld_scales, int scale_layout,
+                                  cudaStream_t s);
+cudaError_t launch_nvfp4_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
+                                    int scale_layout, const float *tensor_amax, int64_t rows, int64_t cols,
+                                    int layout, float *out, int64_t ld_out, cudaStream_t s);
+int launch_nvfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const float *a_amax,
+                      const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, const float *b_amax, int64_t M,
+                      int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s);
 int get_error(cudaStream_t s);
 int launch_wait_probe(int arrive, cudaStream_t s);
 uint64_t set_wait_limit(uint64_t ns);
@@ -213,6 +223,59 @@ int mxfp4_grouped_gemm_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t 
     if (M > (int64_t)1 << 31 || (int64_t)num_groups * M > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
     return mxfp4::launch_grouped_wgrad(a_codes, lda, a_scales, b_codes, ldb, b_scales, group_offsets, num_groups, M,
                                        N, K, c, ldc, static_cast<cudaStream_t>(stream));
+}
+
+int mxfp4_nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rounding,
+                         uint64_t seed, uint64_t elem_offset, float *tensor_amax, uint8_t *codes, int64_t ld_codes,
+                         uint8_t *scales, int64_t ld_scales, int scale_layout, void *stream) {
+    if (!x || !codes || !scales || !tensor_amax) return MXFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (layout != MXFP4_LAYOUT_1D_ROW && layout != MXFP4_LAYOUT_1D_COL) return MXFP4_ERR_INVALID_ARG;
+    if (rounding != MXFP4_ROUND_RNE && rounding != MXFP4_ROUND_SR) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout != MXFP4_SCALES_ROWMAJOR && scale_layout != MXFP4_SCALES_MMA) return MXFP4_ERR_INVALID_ARG;
+    const bool col = layout == MXFP4_LAYOUT_1D_COL;
+    const int64_t orows = col ? cols : rows, k = col ? rows : cols;
+    if (rows % 16 || cols % 16 || (elem_offset % 4)) return MXFP4_ERR_INVALID_ARG;
+    if (ld_x < cols || ld_codes < k / 2) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout == MXFP4_SCALES_ROWMAJOR && ld_scales < k / 16) return MXFP4_ERR_INVALID_ARG;
+    if (!aligned16(x) || (ld_x % 8) || !aligned16(codes) || (ld_codes % 16) ||
+        (reinterpret_cast<uintptr_t>(tensor_amax) & 3u))
+        return MXFP4_ERR_ALIGNMENT;
+    if (orows > (int64_t)1 << 31 || k > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    const cudaError_t e = mxfp4::launch_nvfp4_quantize(x, rows, cols, ld_x, layout, rounding, seed, elem_offset,
+                                                       tensor_amax, codes, ld_codes, scales, ld_scales, scale_layout,
+                                                       static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
+}
+
+int mxfp4_nvfp4_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
+                           int scale_layout, const float *tensor_amax, int64_t rows, int64_t cols, int layout,
+                           float *out, int64_t ld_out, void *stream) {
+    if (!codes || !scales || !tensor_amax || !out) return MXFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16) return MXFP4_ERR_INVALID_ARG;
+    if (layout != MXFP4_LAYOUT_1D_ROW && layout != MXFP4_LAYOUT_1D_COL) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout != MXFP4_SCALES_ROWMAJOR && scale_layout != MXFP4_SCALES_MMA) return MXFP4_ERR_INVALID_ARG;
+    const bool col = layout == MXFP4_LAYOUT_1D_COL;
+    const int64_t k = col ? rows : cols;
+    if (ld_codes < k / 2 || ld_out < cols) return MXFP4_ERR_INVALID_ARG;
+    if (scale_layout == MXFP4_SCALES_ROWMAJOR && ld_scales < k / 16) return MXFP4_ERR_INVALID_ARG;
+    if ((ld_codes % 8) || (reinterpret_cast<uintptr_t>(codes) & 7u) || !aligned16(out) || (ld_out % 4))
+        return MXFP4_ERR_ALIGNMENT;
+    const cudaError_t e = mxfp4::launch_nvfp4_dequantize(codes, ld_codes, scales, ld_scales, scale_layout,
+                                                         tensor_amax, rows, cols, layout, out, ld_out,
+                                                         static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
+}
+
+int mxfp4_nvfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const float *a_amax,
+                     const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, const float *b_amax, int64_t M,
+                     int64_t N, int64_t K, float *c, int64_t ldc, void *stream) {
+    if (M <= 0 || !a_amax || !b_amax) return MXFP4_ERR_INVALID_ARG;
+    const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc);
+    if (rc != MXFP4_OK) return rc;
+    if (M > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    return mxfp4::launch_nvfp4_gemm(a_codes, lda, a_scales, a_amax, b_codes, ldb, b_scales, b_amax, M, N, K, c, ldc,
+                                    static_cast<cudaStream_t>(stream));
 }
 
 int mxfp4_get_error(void *stream) { return mxfp4::get_error(static_cast<cudaStream_t>(stream)); }

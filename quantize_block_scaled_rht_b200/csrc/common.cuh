@@ -163,6 +163,15 @@ __device__ __forceinline__ uint32_t shr_sat(uint32_t a, uint32_t n) {
     return d;
 }
 
+// E2M1 code (bit 3 the sign) -> fp32, exact.  Bit pattern of an E2M1 magnitude code m (0..7): m >= 2 -> (252 + m) << 22
+// (1.0 .. 6.0), m == 1 -> 0.5, m == 0 -> 0.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+    const uint32_t m = c & 7u;
+    uint32_t b = m >= 2u ? (252u + m) << 22 : (m ? 0x3F000000u : 0u);
+    b |= (c & 8u) << 28;
+    return __uint_as_float(b);
+}
+
 // Stochastic rounding of one scaled value with random word r: lo <= |v| < hi
 // neighbouring grid values, up iff r < ceil(f * 2^32) with
 // f = (|v| - lo) / (hi - lo).  With m the 24-bit significand and e the biased

@@ -50,13 +50,18 @@ constexpr int MAX_STAGES = 8;
 
 // Tile configuration: a pair tile is 256 x BN; each stage of the STAGES-deep
 // smem ring holds KCH chunks of K (KCH * 256 E2M1 elements, 4 * KCH MMAs).
-template <int BN_, int STAGES_, int KCH_>
+// NV: NVFP4 operands (UE4M3 scales per 16 elements, kind::mxf4nvf4) instead of
+// MXFP4 (UE8M0 per 32, kind::mxf4).  A scale atom holds 4 blocks of every row
+// of a 128-row tile: 128 K-elements for MXFP4, 64 for NVFP4.
+template <int BN_, int STAGES_, int KCH_, bool NV_ = false>
 struct TileCfg {
     static constexpr int BN = BN_;
     static constexpr int STAGES = STAGES_;
     static constexpr int KCH = KCH_;
+    static constexpr bool NV = NV_;
     static constexpr int KSTEP = 256 * KCH;           // E2M1 elements of K per stage
-    static constexpr int NATOM = 2 * KCH;             // 4-block scale atoms per row tile per stage
+    static constexpr int KATOM = NV ? 64 : 128;       // K-elements per scale atom
+    static constexpr int NATOM = KSTEP / KATOM;       // scale atoms per row tile per stage
     // B scale atoms span one 128-row tile when BN = 128, two when BN = 192
     // (a 192-column tile starts at 0 or 64 within a 128-row scale tile).
     static constexpr int NRT = BN == 128 ? 1 : 2;
@@ -77,8 +82,8 @@ struct TileCfg {
     // Instruction descriptor, kind::mxf4 block-scaled: A/B E2M1 (1), K-major,
     // N >> 3 at bit 17, UE8M0 scales (bit 23), M >> 4 at bit 24 (M = 256 for
     // the pair), scale-factor byte selectors at bits 4 (B) and 29 (A).
-    static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
-                                      ((uint32_t)(256 >> 4) << 24);
+    static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                      ((NV ? 0u : 1u) << 23) | ((uint32_t)(256 >> 4) << 24);
     static_assert(BN == 128 || BN == 192, "tile width");
     static_assert(KCH == 1 || KCH == 2, "chunks per stage");
     static_assert(STAGES <= MAX_STAGES, "stages");
@@ -88,6 +93,7 @@ struct TileCfg {
 };
 
 using DefaultCfg = TileCfg<192, 3, 2>;
+using NvCfg = TileCfg<192, 5, 1, true>;
 
 __device__ unsigned int g_error_code;
 
@@ -101,6 +107,7 @@ struct GemmParams {
     int64_t ldc;
     const int32_t *group_offsets;
     const int32_t *group_sizes;
+    const float *a_amax, *b_amax;   // NVFP4 tensor amaxes (second-level scales amax / 2688)
     int num_groups;
     uint64_t wait_limit_ns;
 };
@@ -233,11 +240,17 @@ __device__ __forceinline__ void issue_stage(uint32_t d_tmem, uint32_t st, uint32
     const uint64_t bdesc = smem_desc(st + Cfg::A_BYTES, 16, 1024, 2);
 #pragma unroll
     for (int k = 0; k < NK; ++k) {
-        const uint32_t idesc = (k & 1) ? (Cfg::IDESC | (2u << 29) | (2u << 4)) : Cfg::IDESC;
         const uint64_t a_off = (uint64_t)(((k >> 2) * Cfg::A_CHUNK + (k & 3) * 32) >> 4);
         const uint64_t b_off = (uint64_t)(((k >> 2) * Cfg::B_CHUNK + (k & 3) * 32) >> 4);
-        mma_mxf4_pair_elect(d_tmem, adesc + a_off, bdesc + b_off, idesc, sfa_col + 4u * (uint32_t)(k >> 1),
-                            sfb_col + 4u * NRT * (uint32_t)(k >> 1) + b_shift, (k == 0 && first) ? 0u : 1u);
+        if constexpr (Cfg::NV) {
+            // one atom (4 scales of 16) per K = 64 instruction
+            mma_nvf4_pair_elect(d_tmem, adesc + a_off, bdesc + b_off, Cfg::IDESC, sfa_col + 4u * (uint32_t)k,
+                                sfb_col + 4u * NRT * (uint32_t)k + b_shift, (k == 0 && first) ? 0u : 1u);
+        } else {
+            const uint32_t idesc = (k & 1) ? (Cfg::IDESC | (2u << 29) | (2u << 4)) : Cfg::IDESC;
+            mma_mxf4_pair_elect(d_tmem, adesc + a_off, bdesc + b_off, idesc, sfa_col + 4u * (uint32_t)(k >> 1),
+                                sfb_col + 4u * NRT * (uint32_t)(k >> 1) + b_shift, (k == 0 && first) ? 0u : 1u);
+        }
     }
 }
 
@@ -246,6 +259,15 @@ __device__ __forceinline__ void issue_stage(uint32_t d_tmem, uint32_t st, uint32
 template <class Cfg>
 __device__ __noinline__ void issue_stage_tail(uint32_t d_tmem, uint32_t st, uint32_t sfa_col, uint32_t b_shift,
                                               bool first, int nk) {
+    if constexpr (Cfg::NV) {                  // one atom per MMA; a stage holds 4 * KCH MMAs
+        switch (nk) {
+            case 1: issue_stage<Cfg, 1, 1>(d_tmem, st, sfa_col, b_shift, first); break;
+            case 2: issue_stage<Cfg, 2, 2>(d_tmem, st, sfa_col, b_shift, first); break;
+            case 3: issue_stage<Cfg, 3, 3>(d_tmem, st, sfa_col, b_shift, first); break;
+            default: break;
+        }
+        return;
+    }
     switch (nk) {
         case 1: issue_stage<Cfg, 1, 1>(d_tmem, st, sfa_col, b_shift, first); break;
         case 2: issue_stage<Cfg, 1, 2>(d_tmem, st, sfa_col, b_shift, first); break;
@@ -359,7 +381,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 const int32_t sfa_rt = (int32_t)(ti.row0 / 128);
                 const int32_t sfb_rt = (int32_t)(ti.sfb_rt_base + ti.n0 / 128);
                 const int ktiles = ktiles_of(ti);
-                const int32_t katom0 = (int32_t)(ti.k0 / 128);       // grouped K: the group's first scale atom
+                const int32_t katom0 = (int32_t)(ti.k0 / Cfg::KATOM);   // grouped K: the group's first scale atom
                 bool ok = true;
                 for (int kt = 0; kt < ktiles; ++kt) {
                     if (!wait_phase(&sh->empty[s], ph ^ 1u, sh, limit)) { ok = false; break; }
@@ -450,6 +472,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         int acc = 0;
         uint32_t acc_ph = 0;
         uint32_t buf_i = 0;
+        // NVFP4: the product of the two second-level scales (amax / 2688 each)
+        float nv_scale = 1.0f;
+        if constexpr (Cfg::NV) nv_scale = __fmul_rn(__fdiv_rn(*p.a_amax, 2688.0f), __fdiv_rn(*p.b_amax, 2688.0f));
         for (int t = pair; t < ntiles; t += npairs) {
             const TileInfo ti = get_tile<BN, MODE>(t, rank, p, cum, tiles_n);
             if (!wait_phase(&sh->tmem_full[acc], acc_ph, sh, limit)) break;
@@ -465,6 +490,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 if (empty_k) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = 0u;
+                }
+                if constexpr (Cfg::NV) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), nv_scale));
                 }
                 if (j == BN / 32 - 1) {
                     tc_fence_before();
@@ -618,6 +647,7 @@ struct GemmArgs {
     float *c;
     const int32_t *offsets, *sizes;
     int G;
+    const float *a_amax = nullptr, *b_amax = nullptr;
 };
 
 // Returns 0 on success, MXFP4_ERR_CUDA when a map or launch fails.
@@ -628,7 +658,7 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
     constexpr int BN = Cfg::BN;
     const int G = MODE == MODE_GROUPED_M ? g.G : 1;
     const int64_t c_rows = MODE == MODE_GROUPED_K ? (int64_t)g.G * g.M : g.M;
-    const int64_t katoms = mma_katoms(g.K);
+    const int64_t katoms = (g.K + Cfg::KATOM - 1) / Cfg::KATOM;
     const int64_t a_tiles = (g.M + 127) / 128, b_tiles = (g.N + 127) / 128;
     CUtensorMap ta, tb, tc, tsa, tsb;
     if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.a_codes, (uint64_t)(g.K / 2), (uint64_t)g.M,
@@ -649,6 +679,7 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
     p.b_rowtiles = b_tiles;
     p.c = g.c; p.ldc = g.ldc;
     p.group_offsets = g.offsets; p.group_sizes = g.sizes; p.num_groups = g.G;
+    p.a_amax = g.a_amax; p.b_amax = g.b_amax;
     p.wait_limit_ns = g_wait_limit_ns;
     const int pairs_max = sm_count() / 2;
     int pairs = pairs_max;
@@ -679,6 +710,13 @@ int launch_grouped_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_s
                          int64_t K, float *c, int64_t ldc, cudaStream_t s) {
     GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, M, N, K, ldc, c, offsets, nullptr, G};
     return launch_cfg<DefaultCfg, MODE_GROUPED_K>(g, s);
+}
+
+int launch_nvfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const float *a_amax,
+                      const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, const float *b_amax, int64_t M,
+                      int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s) {
+    GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, M, N, K, ldc, c, nullptr, nullptr, 1, a_amax, b_amax};
+    return launch_cfg<NvCfg, MODE_DENSE>(g, s);
 }
 
 int get_error(cudaStream_t s) {

@@ -246,6 +246,19 @@ __device__ __forceinline__ void mma_mxf4_pair_elect(uint32_t d_tmem, uint64_t a_
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
 }
+// NVFP4: E2M1 operands with one UE4M3 scale per 16 K-elements (four per
+// K = 64 instruction, all four bytes of the 32-bit scale word).
+__device__ __forceinline__ void mma_nvf4_pair_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                    uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                    uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
 __device__ __forceinline__ void tc_cp_32x128_warpx4_pair_elect(uint32_t taddr, uint64_t sdesc) {
     asm volatile(
         "{\n\t.reg .pred e;\n\t"

@@ -459,14 +459,6 @@ struct DequantParams {
     uint32_t sgn_dup[32];
 };
 
-// fp32 bit pattern of an E2M1 magnitude code m (0..7): m >= 2 -> (252 + m) << 22
-// (1.0 .. 6.0), m == 1 -> 0.5, m == 0 -> 0.
-__device__ __forceinline__ float e2m1_value(uint32_t c) {
-    const uint32_t m = c & 7u;
-    uint32_t b = m >= 2u ? (252u + m) << 22 : (m ? 0x3F000000u : 0u);
-    b |= (c & 8u) << 28;
-    return __uint_as_float(b);
-}
 
 __device__ __forceinline__ void decode32(const uint4 q, uint32_t scode, float *v) {
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};

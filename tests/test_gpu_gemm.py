@@ -260,3 +260,21 @@ def test_grouped_dgrad_with_transposed_weight_copies():
         ref, sabs = oracle.gemm_entries(ca, sa, cwt, sw, I, pairs, 0, 2)
         got = np.array([c[m, n] for m, n in pairs], np.float64)
         assert_gemm_close(got, ref, sabs)
+
+
+@pytest.mark.parametrize("shape", [(256, 192, 256), (304, 208, 576), (512, 384, 1024)])
+def test_nvfp4_gemm_matches_oracle(shape):
+    M, N, K = shape
+    a = synth.normal_bf16((M, K), 40)
+    b = synth.normal_bf16((N, K), 41, 0.02)
+    qa = mx.mxfp4_nvfp4_quantize(dev_bf16(a), scale_layout=mx.SCALES_MMA)
+    qb = mx.mxfp4_nvfp4_quantize(dev_bf16(b), scale_layout=mx.SCALES_MMA)
+    c = host(mx.mxfp4_nvfp4_gemm(qa, qb))
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    ca, sa, aa = oracle.nvfp4_quantize(a, oracle.LAYOUT_1D_ROW)
+    cb, sb, ab = oracle.nvfp4_quantize(b, oracle.LAYOUT_1D_ROW)
+    g = np.random.default_rng(M + N)
+    pairs = list(zip(g.integers(0, M, 400), g.integers(0, N, 400))) + [(0, 0), (M - 1, N - 1)]
+    ref, s = oracle.nvfp4_gemm_entries(ca, sa, aa, cb, sb, ab, K, pairs)
+    got = np.array([c[m, n] for m, n in pairs], np.float64)
+    assert_gemm_close(got, ref, s)

@@ -238,3 +238,53 @@ def test_bad_rounding_bits_rejected():
         with pytest.raises(mx.MXFP4Error) as e:
             mx.mxfp4_quantize(x, mx.LAYOUT_1D_ROW, rounding=bad)
         assert e.value.status == mx.MXFP4_ERR_INVALID_ARG
+
+
+# ---- NVFP4 ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("scale_layout", [mx.SCALES_ROWMAJOR, mx.SCALES_MMA])
+@pytest.mark.parametrize("rnd", [mx.ROUND_RNE, mx.ROUND_SR])
+@pytest.mark.parametrize("layout", [mx.LAYOUT_1D_ROW, mx.LAYOUT_1D_COL])
+def test_nvfp4_quantize_bit_exact(layout, rnd, scale_layout):
+    rows, cols = (80, 224) if layout == mx.LAYOUT_1D_ROW else (224, 80)
+    x = synth.student_t_bf16((rows, cols), seed=600 + layout)
+    q = mx.mxfp4_nvfp4_quantize(dev_bf16(x), layout, rnd, 42, scale_layout=scale_layout)
+    codes, scales, amax = oracle.nvfp4_quantize(x, layout, rnd, 42)
+    assert float(q.amax.item()) == amax
+    assert np.array_equal(host(q.codes), codes)
+    s = host(q.scales)
+    if scale_layout == mx.SCALES_MMA:
+        K = q.k
+        s = np.array([[s[((r // 128) * ((K // 16 + 3) // 4) + kb // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4
+                         + kb % 4] for kb in range(scales.shape[1])] for r in range(scales.shape[0])], np.uint8)
+    assert np.array_equal(s, scales)
+
+
+def test_nvfp4_every_bf16_pattern_and_specials():
+    allbits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    finite = allbits[(allbits & 0x7F80) != 0x7F80]                     # no NaN / Inf
+    g = np.random.default_rng(8)
+    x = g.permutation(np.resize(finite, 256 * 256)).reshape(256, 256)
+    for rnd in (mx.ROUND_RNE, mx.ROUND_SR):
+        q = mx.mxfp4_nvfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_ROW, rnd, 9)
+        codes, scales, amax = oracle.nvfp4_quantize(x, oracle.LAYOUT_1D_ROW, rnd, 9)
+        assert np.array_equal(host(q.codes), codes) and np.array_equal(host(q.scales), scales)
+    for bad in (0x7FC0, 0xFF80):                                      # NaN, -Inf
+        y = x.copy()
+        y[5, 9] = bad
+        q = mx.mxfp4_nvfp4_quantize(dev_bf16(y), mx.LAYOUT_1D_ROW)
+        codes, scales, _ = oracle.nvfp4_quantize(y, oracle.LAYOUT_1D_ROW)
+        assert np.array_equal(host(q.codes), codes) and np.array_equal(host(q.scales), scales)
+    z = mx.mxfp4_nvfp4_quantize(torch.zeros((32, 64), dtype=torch.bfloat16, device="cuda"))
+    assert float(z.amax.item()) == 0.0 and not host(z.codes).any() and not host(z.scales).any()
+
+
+@pytest.mark.parametrize("layout", [mx.LAYOUT_1D_ROW, mx.LAYOUT_1D_COL])
+def test_nvfp4_dequantize_matches_oracle(layout):
+    rows, cols = 96, 160
+    x = synth.student_t_bf16((rows, cols), seed=610)
+    q = mx.mxfp4_nvfp4_quantize(dev_bf16(x), layout, mx.ROUND_SR, 3)
+    out = host(mx.mxfp4_nvfp4_dequantize(q, rows, cols))
+    codes, scales, amax = oracle.nvfp4_quantize(x, layout, oracle.ROUND_SR, 3)
+    ref = oracle.nvfp4_dequantize(codes, scales, rows, cols, layout, amax)
+    assert np.array_equal(out.view(np.uint32), ref.view(np.uint32))
