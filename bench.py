@@ -406,6 +406,52 @@ def sweep_bench(mx, torch, device, peaks, nbytes=1 << 30, reps=5):
             "note": "SR modes are bound by the integer work of Philox4x32-10 and the exact SR decision, not HBM"}
 
 
+def nvfp4_bench(mx, torch, device, peaks, reps=10):
+    """NVFP4 ("Comparison with NVFP4": blocks of 16, E4M3 block scale, FP32
+    tensor scale): quantize (tensor amax + blocks) of the 1 GiB sweep tensor,
+    and the GEMM at the expert fprop shape 4096 x 5760 x 2880 (activations
+    N(0,1), weights N(0, 0.02^2), L2 flushed before each launch)."""
+    rows, cols = synth.sweep_shape(1 << 30, 2880)
+    x = synth.student_t_bf16_device(rows, cols, seed=7, device=device)
+    n = rows * cols
+    q = mx.mxfp4_nvfp4_quantize(x)
+    tq = _timed(torch, lambda: mx.mxfp4_nvfp4_quantize(x, out=q), 5)
+    # bytes: the amax pass reads x once more; 2 + 2 read, 0.5 + 1/16 written
+    gq = n * (2 + 0.5 + 1 / 16) / (tq / 1e3) / 1e9
+    del q, x
+    g = torch.Generator(device=device)
+    g.manual_seed(2)
+    a = torch.randn((TOKENS, HIDDEN), generator=g, device=device).to(torch.bfloat16)
+    w = (torch.randn((INTER, HIDDEN), generator=g, device=device) * 0.02).to(torch.bfloat16)
+    qa = mx.mxfp4_nvfp4_quantize(a, scale_layout=mx.SCALES_MMA)
+    qw = mx.mxfp4_nvfp4_quantize(w, scale_layout=mx.SCALES_MMA)
+    c = torch.empty((TOKENS, INTER), dtype=torch.float32, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    # time the GEMM alone: events around the launch, the flush before them
+    mx.mxfp4_nvfp4_gemm(qa, qw, out=c)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mx.mxfp4_nvfp4_gemm(qa, qw, out=c)
+        e1.record()
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = float(np.median([e0.elapsed_time(e1) for e0, e1 in ts]))
+    if mx.mxfp4_get_error() != mx.MXFP4_OK:
+        raise RuntimeError("device-side error in the NVFP4 measurements")
+    tf = 2.0 * TOKENS * INTER * HIDDEN / (ms / 1e3) / 1e12
+    del qa, qw, c, a, w, flush
+    torch.cuda.empty_cache()
+    return {"quantize_1GiB": {"us": tq * 1e3, "GB/s": gq, "frac_hbm": gq / peaks["hbm"],
+                              "note": "algorithmic bytes 2.5625 per element; the amax pass reads the tensor again"},
+            "gemm_fprop": {"us": ms * 1e3, "TFLOP/s": tf, "frac_fp4_peak": tf / (4 * peaks["bf16"]),
+                           "shape": f"{TOKENS} x {INTER} x {HIDDEN}"}}
+
+
 # ---------------------------------------------------------------------------
 # main
 # ---------------------------------------------------------------------------
@@ -589,6 +635,7 @@ def main():
     if world == 1 and not args.no_extras:
         extras["grouped_moe"] = grouped_bench(mx, torch, device, peaks)
         extras["quantizer_sweep"] = sweep_bench(mx, torch, device, peaks)
+        extras["nvfp4"] = nvfp4_bench(mx, torch, device, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

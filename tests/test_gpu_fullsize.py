@@ -214,3 +214,21 @@ def test_sweep_2gib_sampled_rows():
         assert np.array_equal(host(qc.scales[c0:c0 + 8]), scales)
     del qc, x
     torch.cuda.empty_cache()
+
+
+def test_nvfp4_expert_fprop_sampled():
+    """NVFP4 at the expert fprop shape: X 4096 x 2880 (with the outlier
+    columns), W 5760 x 2880; quantizers bit-exact, GEMM on sampled entries."""
+    x, w = synth.fprop_inputs()
+    qx = mx.mxfp4_nvfp4_quantize(dev_bf16(x), scale_layout=mx.SCALES_MMA)
+    qw = mx.mxfp4_nvfp4_quantize(dev_bf16(w), scale_layout=mx.SCALES_MMA)
+    c = host(mx.mxfp4_nvfp4_gemm(qx, qw))
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    cx, sx, ax = oracle.nvfp4_quantize(x, oracle.LAYOUT_1D_ROW)
+    cw, sw, aw = oracle.nvfp4_quantize(w, oracle.LAYOUT_1D_ROW)
+    assert np.array_equal(host(qx.codes), cx) and np.array_equal(host(qw.codes), cw)
+    assert float(qx.amax.item()) == ax and float(qw.amax.item()) == aw
+    pairs = _sample_pairs(4096, 5760, 1500, 21)
+    ref, s = oracle.nvfp4_gemm_entries(cx, sx, ax, cw, sw, aw, 2880, pairs)
+    got = np.array([c[m, n] for m, n in pairs], np.float64)
+    assert_gemm_close(got, ref, s)
