@@ -38,11 +38,11 @@ __device__ __forceinline__ U4 philox4x32_10(uint32_t c0, uint32_t c1, uint32_t c
     constexpr uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
 #pragma unroll
     for (int r = 0; r < 10; ++r) {
-        const uint32_t lo0 = M0 * c0, hi0 = __umulhi(M0, c0);
-        const uint32_t lo1 = M1 * c2, hi1 = __umulhi(M1, c2);
-        const uint32_t n0 = hi1 ^ c1 ^ k0;
-        const uint32_t n2 = hi0 ^ c3 ^ k1;
-        c0 = n0; c1 = lo1; c2 = n2; c3 = lo0;
+        const uint64_t p0 = (uint64_t)M0 * c0;   // one widening multiply each
+        const uint64_t p1 = (uint64_t)M1 * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        c0 = n0; c1 = (uint32_t)p1; c2 = n2; c3 = (uint32_t)p0;
         k0 += W0; k1 += W1;
     }
     return U4{c0, c1, c2, c3};
@@ -74,6 +74,33 @@ __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w &
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
+}
+
+// Eight bf16 values (a uint4, element 0 in the low half of .x) to fp32.
+__device__ __forceinline__ void unpack_bf16x8(const uint4 &u, float *w) {
+    w[0] = bf16lo(u.x); w[1] = bf16hi(u.x); w[2] = bf16lo(u.y); w[3] = bf16hi(u.y);
+    w[4] = bf16lo(u.z); w[5] = bf16hi(u.z); w[6] = bf16lo(u.w); w[7] = bf16hi(u.w);
+}
+
+// max(|a|, |b|) of two bf16 pairs, NaN if either operand is NaN; the sign
+// bits of the result are the operands' sign xor, not used here.
+__device__ __forceinline__ uint32_t bf16x2_absmax(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// amax of 32 bf16 values packed in four uint4, as fp32 (exact: a maximum of
+// bf16 magnitudes needs no rounding); NaN if any value is NaN.
+__device__ __forceinline__ float amax_bf16x32(const uint4 *u) {
+    const uint32_t a = bf16x2_absmax(bf16x2_absmax(u[0].x, u[0].y), bf16x2_absmax(u[0].z, u[0].w));
+    const uint32_t b = bf16x2_absmax(bf16x2_absmax(u[1].x, u[1].y), bf16x2_absmax(u[1].z, u[1].w));
+    const uint32_t c = bf16x2_absmax(bf16x2_absmax(u[2].x, u[2].y), bf16x2_absmax(u[2].z, u[2].w));
+    const uint32_t d = bf16x2_absmax(bf16x2_absmax(u[3].x, u[3].y), bf16x2_absmax(u[3].z, u[3].w));
+    const uint32_t m = bf16x2_absmax(bf16x2_absmax(a, b), bf16x2_absmax(c, d)) & 0x7FFF7FFFu;
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(bf16lo(m)), "f"(bf16hi(m)));
     return r;
 }
 
@@ -115,9 +142,19 @@ __device__ __forceinline__ uint32_t scale_code_rule(float amax, int rule) {
 
 // Element scaling: y / X, or (3/4 y) / X under the pre-scale rule, each
 // product rounded in fp32 (the division by the power of two X is exact
-// unless the result is subnormal).
-__device__ __forceinline__ float scale_element(float y, float inv, int rule) {
-    return __fmul_rn(rule == 2 ? __fmul_rn(y, 0.75f) : y, inv);
+// unless the result is subnormal).  The rule is tested once per group.
+__device__ __forceinline__ void scale8(float *w, float inv, int rule) {
+    if (rule == 2) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = __fmul_rn(__fmul_rn(w[i], 0.75f), inv);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = __fmul_rn(w[i], inv);
+    }
+}
+__device__ __forceinline__ void scale_block32(float *v, float inv, int rule) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) scale8(v + 8 * q, inv, rule);
 }
 
 // 2^-(code - 127) as fp32 for code in [0, 252]: biased exponent 254 - code.
@@ -224,19 +261,75 @@ __device__ __forceinline__ uint32_t sign_nibbles8(const float *w) {
     return ((ev & 0x0F0F0F0Fu) | (od & 0xF0F0F0F0u)) & 0x88888888u;
 }
 
-// Eight scaled values to eight packed E2M1 codes by stochastic rounding with
-// the random words r0 (elements 0-3) and r1 (elements 4-7): magnitudes as a
-// multiply-add chain (the nibbles do not overlap), signs in one go.
-__device__ __forceinline__ uint32_t e2m1x8_sr(const float *w, const U4 &r0, const U4 &r1) {
-    uint32_t mag = e2m1_sr_mag(w[7], r1.w);
-    mag = mag * 16u + e2m1_sr_mag(w[6], r1.z);
-    mag = mag * 16u + e2m1_sr_mag(w[5], r1.y);
-    mag = mag * 16u + e2m1_sr_mag(w[4], r1.x);
-    mag = mag * 16u + e2m1_sr_mag(w[3], r0.w);
-    mag = mag * 16u + e2m1_sr_mag(w[2], r0.z);
-    mag = mag * 16u + e2m1_sr_mag(w[1], r0.y);
-    mag = mag * 16u + e2m1_sr_mag(w[0], r0.x);
-    return mag | sign_nibbles8(w);
+// Stochastic rounding of one clamped magnitude (bits ab, 0 <= |v| <= 6) as a
+// fixed-point add.  With s = min(e - 117, 10) >= 0 (|v| >= 2^-10), the 64-bit
+// number W * 2^s has the index of the grid point below |v| in its high word
+// and f * 2^32 (f the position between the two neighbours, the SR threshold)
+// in its low word; W is the 24-bit significand m below 1 and
+// ab - (126 << 23) = ((e - 126) << 23) | mantissa from 1 up (grid steps 1 and
+// 2 above 2 shift the index by 2 per binade), i.e. max(ab - 0x3F000000, m).
+// Adding ~r carries into the high word exactly when r < f * 2^32, so the high
+// word of W * 2^s + ~r is the rounded code.  Integer work: two add-min/max,
+// one shift, one mask; the multiply-add runs on the FMA pipe.
+__device__ __forceinline__ int32_t sr_shift(uint32_t ab) {
+    return __viaddmin_s32((int32_t)(ab >> 23), -117, 10);
+}
+__device__ __forceinline__ uint32_t e2m1_sr_fixed(uint32_t ab, int32_t s, uint32_t nr) {
+    const uint32_t m = (ab & 0x007FFFFFu) | 0x00800000u;
+    const uint32_t w = (uint32_t)__viaddmax_s32((int32_t)ab, -0x3F000000, (int32_t)m);
+    uint32_t p;    // 2^s; shl clamps a shift past 32 (s < 0 is never used)
+    asm("shl.b32 %0, %1, %2;" : "=r"(p) : "r"(1u), "r"(s));
+    return (uint32_t)(((uint64_t)w * p + nr) >> 32);
+}
+
+// Eight scaled values to eight packed E2M1 codes by stochastic rounding.  The
+// random words are those of the Philox blocks b0 (elements 0-3) and b0 + 1
+// (elements 4-7) under the key (k0, k1).  Magnitudes take the fixed-point add
+// and are packed by a multiply-add chain (the nibbles do not overlap); signs
+// go in at once.  A group holding a magnitude under 2^-10 (or a zero) adds
+// the round-up bits of those magnitudes afterwards.
+// Round-up bits of the magnitudes under 2^-10 in a group of eight.  The
+// fixed-point add gives them code 0; the exact rule rounds such a value up to
+// 0.5 when r < ceil(m * 2^(e - 117)) (m its 24-bit significand, e its biased
+// exponent).  The random words are regenerated one Philox block at a time.
+__device__ __forceinline__ uint32_t e2m1x8_sr_tiny(const float *w, uint64_t b0, uint32_t k0, uint32_t k1) {
+    uint32_t up = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint64_t b = b0 + h;
+        const U4 r = philox4x32_10((uint32_t)b, (uint32_t)(b >> 32), 0u, 0u, k0, k1);
+        const uint32_t rr[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t ab = __float_as_uint(fminf(fabsf(w[4 * h + j]), 6.0f));
+            const uint32_t e = ab >> 23;
+            const uint32_t m = (ab & 0x007FFFFFu) | 0x00800000u;
+            const uint32_t t = shr_sat(m - 1u, 117u - e) + 1u;
+            if (ab - 1u < 0x3A7FFFFFu && rr[j] < t) up |= 1u << (4 * (4 * h + j));
+        }
+    }
+    return up;
+}
+
+__device__ __forceinline__ uint32_t e2m1x8_sr(const float *w, uint64_t b0, uint32_t k0, uint32_t k1) {
+    const uint64_t b1 = b0 + 1;
+    const uint32_t sgn = sign_nibbles8(w);
+    uint32_t mag = 0;
+    int32_t any = 0;
+    {
+        const U4 r0 = philox4x32_10((uint32_t)b0, (uint32_t)(b0 >> 32), 0u, 0u, k0, k1);
+        const U4 r1 = philox4x32_10((uint32_t)b1, (uint32_t)(b1 >> 32), 0u, 0u, k0, k1);
+        const uint32_t rr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+        for (int i = 7; i >= 0; --i) {
+            const uint32_t ab = __float_as_uint(fminf(fabsf(w[i]), 6.0f));
+            const int32_t sh = sr_shift(ab);
+            any |= sh;
+            mag = mag * 16u + e2m1_sr_fixed(ab, sh, ~rr[i]);
+        }
+    }
+    if (__builtin_expect(any < 0, 0)) mag |= e2m1x8_sr_tiny(w, b0, k0, k1);
+    return mag | sgn;
 }
 
 // ---------------------------------------------------------------------------

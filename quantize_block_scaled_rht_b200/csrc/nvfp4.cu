@@ -117,10 +117,7 @@ __device__ __forceinline__ uint32_t nv_block(float *v, const NvTensor &t, uint64
         uint32_t p[2];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-            const uint64_t b0 = blk + 2 * q, b1 = b0 + 1;
-            const U4 r0 = philox4x32_10((uint32_t)b0, (uint32_t)(b0 >> 32), 0u, 0u, k0, k1);
-            const U4 r1 = philox4x32_10((uint32_t)b1, (uint32_t)(b1 >> 32), 0u, 0u, k0, k1);
-            p[q] = e2m1x8_sr(v + 8 * q, r0, r1);
+            p[q] = e2m1x8_sr(v + 8 * q, blk + 2 * q, k0, k1);
         }
         out = make_uint2(p[0], p[1]);
     }

@@ -36,44 +36,62 @@ struct QuantParams {
     // 32-element row segment (elements 2j, 2j+1); dup[i] flips both halves of
     // a word for element i of a column segment.
     uint32_t sgn_pair[16];
-    uint32_t sgn_dup[32];
+    uint32_t sgn_bit[32];                  // RHT sign of element i (mod the RHT size) as bit 31
 };
 
 // ---------------------------------------------------------------------------
-// Per-block quantization core: 32 fp32 values (already transformed) -> scale
-// code and 16 bytes of codes.  `g0` is the stream index of element 0.
+// Per-block quantization core: the scale code from the block's amax, then the
+// four groups of 8 values (unscaled, from get8(q, w)) scaled and encoded into
+// 16 bytes of codes.  `g0` is the stream index of element 0.
 // ---------------------------------------------------------------------------
-template <bool SR>
-__device__ __forceinline__ uint32_t quantize32(float *v, uint4 &out, uint64_t g0, uint32_t k0, uint32_t k1,
-                                           int rule) {
-    float amax = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) amax = amax_nan(amax, v[i]);
+template <bool SR, class Get8>
+__device__ __forceinline__ uint32_t quantize_groups(float amax, Get8 &&get8, uint4 &out, uint64_t g0, uint32_t k0,
+                                                    uint32_t k1, int rule) {
     const uint32_t code = scale_code_rule(amax, rule);
     if (code == 0xFFu) {
         out = make_uint4(0, 0, 0, 0);
         return code;
     }
     const float inv = inv_scale_from_code(code);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = scale_element(v[i], inv, rule);
+    const uint64_t blk = g0 >> 2;  // g0 % 4 == 0
     uint32_t p[4];
-    if constexpr (!SR) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) p[q] = e2m1x8_rn(v + 8 * q);
-    } else {
-        const uint64_t blk = g0 >> 2;  // g0 % 4 == 0
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const uint64_t b0 = blk + 2 * q, b1 = b0 + 1;
-            const U4 r0 = philox4x32_10((uint32_t)b0, (uint32_t)(b0 >> 32), 0u, 0u, k0, k1);
-            const U4 r1 = philox4x32_10((uint32_t)b1, (uint32_t)(b1 >> 32), 0u, 0u, k0, k1);
-            const float *w = v + 8 * q;
-            p[q] = e2m1x8_sr(w, r0, r1);
-        }
+    for (int q = 0; q < 4; ++q) {
+        float w[8];
+        get8(q, w);
+        scale8(w, inv, rule);
+        if constexpr (SR) p[q] = e2m1x8_sr(w, blk + 2 * q, k0, k1);
+        else p[q] = e2m1x8_rn(w);
     }
     out = make_uint4(p[0], p[1], p[2], p[3]);
     return code;
+}
+
+// The same for 32 fp32 values already in registers (transformed if the RHT
+// applies).
+template <bool SR>
+__device__ __forceinline__ uint32_t quantize32(const float *v, uint4 &out, uint64_t g0, uint32_t k0, uint32_t k1,
+                                           int rule) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = amax_nan(amax, v[i]);
+    return quantize_groups<SR>(
+        amax,
+        [&](int q, float *w) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) w[j] = v[8 * q + j];
+        },
+        out, g0, k0, k1, rule);
+}
+
+// The same for 32 bf16 values packed in four uint4 (no transform): amax on
+// the packed pairs, each group unpacked when it is encoded, so that the block
+// occupies 16 registers rather than 32.
+template <bool SR>
+__device__ __forceinline__ uint32_t quantize32_bf16(const uint4 *u, uint4 &out, uint64_t g0, uint32_t k0, uint32_t k1,
+                                                int rule) {
+    return quantize_groups<SR>(
+        amax_bf16x32(u), [&](int q, float *w) { unpack_bf16x8(u[q], w); }, out, g0, k0, k1, rule);
 }
 
 // Unpack 16 bf16x2 words to 32 fp32 values, with RHT sign flips and butterfly.
@@ -192,11 +210,13 @@ struct DualParams {
     int scale_rule;                        // MXFP4_SCALE_* >> 4
     uint64_t r_offset, c_offset;           // SR stream index of each output's first element
     uint32_t tiles_c;                      // column tiles
-    uint32_t sgn_dup[32];
+    uint32_t sgn_bit[32];                  // RHT sign of element i (mod the RHT size) as bit 31
 };
 
+// SR instantiations get up to 80 registers (3 CTAs per SM): the column block
+// (32 transformed values) and the Philox state together do not fit in 64.
 template <class T, int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, const uint32_t ntiles) {
+__global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualParams p, const uint32_t ntiles) {
     pdl_wait();
     pdl_trigger();
     constexpr int TR = T::TR, TC = T::TC, PITCH = T::PITCH, OCH = T::OCH;
@@ -229,61 +249,45 @@ __global__ void __launch_bounds__(256, 4) quant_dual_kernel(const DualParams p, 
         const uint16_t *tile = tin[buf];
         const int64_t r0 = (int64_t)(t / p.tiles_c) * TR, c0 = (int64_t)(t % p.tiles_c) * TC;
 
-#pragma unroll 1
-        for (int job = DO_COL ? 0 : 1; job < (DO_ROW ? 2 : 1); ++job) {
-            float v[32];
-            bool ok;
-            uint64_t g0;
-            int64_t orow, kb;
-            int c = 0, b = 0;
-            if (job == 0) {                                  // column c, rows 32b .. 32b+31
-                c = tid % TC;
-                b = tid / TC;
-                orow = c0 + c;
-                const int64_t rin = r0 + 32 * b;
-                ok = orow < p.cols && rin < p.rows;
-                const uint16_t *col = tile + 32 * b * PITCH + c;
+        {
+            if constexpr (DO_COL) {                          // column c, rows 32b .. 32b+31
+                const int c = tid % TC, b = tid / TC;
+                const int64_t orow = c0 + c, rin = r0 + 32 * b;
+                if (orow < p.cols && rin < p.rows) {
+                    const uint16_t *col = tile + 32 * b * PITCH + c;
+                    float v[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    uint32_t u = (uint32_t)col[i * PITCH] << 16;
-                    if constexpr (CRHT) u ^= p.sgn_dup[i % CRHT] & 0x80000000u;
-                    v[i] = __uint_as_float(u);
-                }
-                if constexpr (CRHT) {
-                    const float cn = rht_norm<CRHT>();
+                    for (int i = 0; i < 32; ++i) {
+                        // bf16 -> fp32 with the RHT sign: adding 2^31 flips bit 31
+                        const uint32_t u = (uint32_t)col[i * PITCH] * 65536u + (CRHT ? p.sgn_bit[i % 32] : 0u);
+                        v[i] = __uint_as_float(u);
+                    }
+                    if constexpr (CRHT) {
+                        const float cn = rht_norm<CRHT>();
 #pragma unroll
-                    for (int s = 0; s < 32; s += CRHT) fwht<CRHT>(v + s);
+                        for (int s = 0; s < 32; s += CRHT) fwht<CRHT>(v + s);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], cn);
-                }
-                g0 = (uint64_t)(orow * p.rows + rin) + p.c_offset;
-                kb = rin >> 5;
-            } else {                                         // row r, columns 32b .. 32b+31
-                const int r = tid % TR;
-                b = tid / TR;
-                orow = r0 + r;
-                const int64_t gc = c0 + 32 * b;
-                ok = orow < p.rows && gc < p.cols;
-                const uint4 *s4 = reinterpret_cast<const uint4 *>(tile + r * PITCH + 32 * b);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint4 u = s4[q];
-                    v[8 * q + 0] = bf16lo(u.x); v[8 * q + 1] = bf16hi(u.x);
-                    v[8 * q + 2] = bf16lo(u.y); v[8 * q + 3] = bf16hi(u.y);
-                    v[8 * q + 4] = bf16lo(u.z); v[8 * q + 5] = bf16hi(u.z);
-                    v[8 * q + 6] = bf16lo(u.w); v[8 * q + 7] = bf16hi(u.w);
-                }
-                g0 = (uint64_t)(orow * p.cols + gc) + p.r_offset;
-                kb = gc >> 5;
-            }
-            if (ok) {
-                uint4 q;
-                const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
-                if (job == 0) {
+                        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], cn);
+                    }
+                    uint4 q;
+                    const uint64_t g0 = (uint64_t)(orow * p.rows + rin) + p.c_offset;
+                    const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
                     tout[c * OCH + (b ^ ((c >> T::OSH) & (OCH - 1)))] = q;
+                    const int64_t kb = rin >> 5;
                     if constexpr (MMA) p.cscales[mma_scale_off(orow, kb, p.c_katoms)] = (uint8_t)sc;
                     else p.cscales[orow * p.ld_cscales + kb] = (uint8_t)sc;
-                } else {
+                }
+            }
+            if constexpr (DO_ROW) {                          // row r, columns 32b .. 32b+31
+                const int r = tid % TR, b = tid / TR;
+                const int64_t orow = r0 + r, gc = c0 + 32 * b;
+                if (orow < p.rows && gc < p.cols) {
+                    const uint4 *s4 = reinterpret_cast<const uint4 *>(tile + r * PITCH + 32 * b);
+                    const uint4 u[4] = {s4[0], s4[1], s4[2], s4[3]};
+                    uint4 q;
+                    const uint64_t g0 = (uint64_t)(orow * p.cols + gc) + p.r_offset;
+                    const uint32_t sc = quantize32_bf16<SR>(u, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
+                    const int64_t kb = gc >> 5;
                     stg_v4(p.rcodes + orow * p.ld_rcodes + kb * 16, q);
                     if constexpr (MMA) p.rscales[mma_scale_off(orow, kb, p.r_katoms)] = (uint8_t)sc;
                     else p.rscales[orow * p.ld_rscales + kb] = (uint8_t)sc;
@@ -381,8 +385,7 @@ __global__ void __launch_bounds__(256, 3) quant_2d_kernel(const QuantParams p) {
             uint4 packed = make_uint4(0, 0, 0, 0);
             if (code != 0xFFu) {
                 const float inv = inv_scale_from_code(code);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = scale_element(v[i], inv, p.scale_rule);
+                scale_block32(v, inv, p.scale_rule);
                 uint32_t pk[4];
                 if constexpr (!SR) {
 #pragma unroll
@@ -391,11 +394,7 @@ __global__ void __launch_bounds__(256, 3) quant_2d_kernel(const QuantParams p) {
                     const uint64_t blk = ((uint64_t)(r * p.cols + c0) + p.elem_offset) >> 2;
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint64_t b0 = blk + 2 * q, b1 = b0 + 1;
-                        const U4 r0 = philox4x32_10((uint32_t)b0, (uint32_t)(b0 >> 32), 0u, 0u, p.seed_lo, p.seed_hi);
-                        const U4 r1 = philox4x32_10((uint32_t)b1, (uint32_t)(b1 >> 32), 0u, 0u, p.seed_lo, p.seed_hi);
-                        const float *x8 = v + 8 * q;
-                        pk[q] = e2m1x8_sr(x8, r0, r1);
+                        pk[q] = e2m1x8_sr(v + 8 * q, blk + 2 * q, p.seed_lo, p.seed_hi);
                     }
                 }
                 packed = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -456,7 +455,7 @@ struct DequantParams {
     void *out;
     int64_t ld_out;
     uint32_t sgn_pair[16];
-    uint32_t sgn_dup[32];
+    uint32_t sgn_bit[32];                  // RHT sign of element i (mod the RHT size) as bit 31
 };
 
 
@@ -568,7 +567,7 @@ __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p)
                 for (int s = 0; s < 32; s += RHT) { fwht<RHT>(v0 + s); fwht<RHT>(v1 + s); }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const uint32_t fl = p.sgn_dup[i % RHT] & 0x80000000u;
+                    const uint32_t fl = p.sgn_bit[i % RHT];
                     v0[i] = __uint_as_float(__float_as_uint(__fmul_rn(v0[i], c)) ^ fl);
                     v1[i] = __uint_as_float(__float_as_uint(__fmul_rn(v1[i], c)) ^ fl);
                 }
@@ -618,7 +617,7 @@ static int resident_ctas(const void *kern, int threads) {
     return occ;
 }
 
-static void fill_signs(uint32_t mask, int rht, uint32_t *pair, uint32_t *dup) {
+static void fill_signs(uint32_t mask, int rht, uint32_t *pair, uint32_t *bit) {
     for (int j = 0; j < 16; ++j) {
         const uint32_t e0 = (uint32_t)(2 * j) % (uint32_t)(rht ? rht : 32);
         const uint32_t e1 = (uint32_t)(2 * j + 1) % (uint32_t)(rht ? rht : 32);
@@ -628,7 +627,7 @@ static void fill_signs(uint32_t mask, int rht, uint32_t *pair, uint32_t *dup) {
     }
     for (int i = 0; i < 32; ++i) {
         const uint32_t s = rht ? (mask >> (i % rht)) & 1u : 0u;
-        dup[i] = s ? 0x80008000u : 0u;
+        bit[i] = s ? 0x80000000u : 0u;
     }
 }
 
@@ -685,7 +684,7 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, int64_t l
     p.katoms_t = mma_katoms(rows);
     p.seed_lo = (uint32_t)seed; p.seed_hi = (uint32_t)(seed >> 32);
     p.elem_offset = elem_offset;
-    fill_signs(rht ? rht_sign_mask_hd(seed) : 0u, rht, p.sgn_pair, p.sgn_dup);
+    fill_signs(rht ? rht_sign_mask_hd(seed) : 0u, rht, p.sgn_pair, p.sgn_bit);
     const bool mma = scale_layout == MXFP4_SCALES_MMA;
     const bool sr = (rounding & 0x0F) == MXFP4_ROUND_SR;
     p.scale_rule = (rounding >> 4) & 3;
@@ -722,7 +721,7 @@ static cudaError_t launch_col_dual(const QuantParams &q, cudaStream_t s) {
     p.seed_lo = q.seed_lo; p.seed_hi = q.seed_hi;
     p.scale_rule = q.scale_rule;
     p.c_offset = q.elem_offset;
-    for (int i = 0; i < 32; ++i) p.sgn_dup[i] = q.sgn_dup[i];
+    for (int i = 0; i < 32; ++i) p.sgn_bit[i] = q.sgn_bit[i];
     return launch_dual_t<DualCol, RHT, SR, MMA, false, true>(p, s);
 }
 
@@ -754,7 +753,7 @@ cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int6
     p.seed_lo = (uint32_t)seed; p.seed_hi = (uint32_t)(seed >> 32);
     p.r_offset = row_offset; p.c_offset = col_offset;
     uint32_t pair_unused[16];
-    fill_signs(col_rht ? rht_sign_mask_hd(seed) : 0u, col_rht, pair_unused, p.sgn_dup);
+    fill_signs(col_rht ? rht_sign_mask_hd(seed) : 0u, col_rht, pair_unused, p.sgn_bit);
     const bool sr = (rounding & 0x0F) == MXFP4_ROUND_SR, mma = scale_layout == MXFP4_SCALES_MMA;
     p.scale_rule = (rounding >> 4) & 3;
     const bool do_row = rcodes != nullptr, do_col = ccodes != nullptr;
@@ -795,7 +794,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, int64_t ld_codes, const uint
     p.scales = scales; p.ld_scales = ld_scales;
     p.rows = rows; p.cols = cols; p.out = out; p.ld_out = ld_out;
     p.katoms = mma_katoms(layout == MXFP4_LAYOUT_1D_COL ? rows : cols);
-    fill_signs(rht ? rht_sign_mask_hd(seed) : 0u, rht, p.sgn_pair, p.sgn_dup);
+    fill_signs(rht ? rht_sign_mask_hd(seed) : 0u, rht, p.sgn_pair, p.sgn_bit);
     const int smode = scale_layout == MXFP4_SCALES_MMA ? 2 : (layout == MXFP4_LAYOUT_2D ? 1 : 0);
     const bool f32 = out_dtype == MXFP4_OUT_F32;
     switch (rht) {
