@@ -62,10 +62,10 @@ KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 # profiles/expert_step_kernels_ncu_full.md.  The figures hold only for the
 # kernel sources they were taken from: a changed source gives traffic null.
 NCU_TRAFFIC = {
-    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "67fdbfcaf842e5d6",
-             "bytes": {"fprop": 51.87e6, "dgrad": 23.17e6, "wgrad": 29.66e6}},
-    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "fd74e2780ea8c56b",
-              "bytes": {"quant_x_dual": 23.65e6, "quant_w_2d": 33.27e6, "quant_dy_dual_sr": 47.90e6}},
+    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "749f84de0bbb3a8f",
+             "bytes": {"fprop": 51.79e6, "dgrad": 23.32e6, "wgrad": 29.59e6}},
+    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "5b7f4ae361de04d1",
+              "bytes": {"quant_x_dual": 23.61e6, "quant_w_2d": 33.29e6, "quant_dy_dual_sr": 49.18e6}},
 }
 
 
