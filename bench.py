@@ -338,7 +338,16 @@ def grouped_bench(mx, torch, device, peaks, reps=10):
         ms = _timed(torch, lambda: mx.mxfp4_grouped_gemm(qa.codes, qa.scales, off_d, size_d, b_codes, b_scales,
                                                           n_out, H, out=c), reps)
         record(name, ms, 2.0 * routed * n_out * H, f"{routed} routed rows ({total} padded) x {n_out} x {H}")
-        del b_codes, b_scales, c
+        del c
+        if name == "gate_up":
+            # the same product with the bf16 epilogue (half the output bytes)
+            c16 = torch.empty((qa.codes.shape[0], n_out), dtype=torch.bfloat16, device=device)
+            ms = _timed(torch, lambda: mx.mxfp4_grouped_gemm_bf16(qa.codes, qa.scales, off_d, size_d, b_codes,
+                                                                   b_scales, n_out, H, out=c16), reps)
+            record("gate_up_bf16_out", ms, 2.0 * routed * n_out * H,
+                   f"{routed} routed rows ({total} padded) x {n_out} x {H}, bf16 output")
+            del c16
+        del b_codes, b_scales
 
     # backward of gate_up: dgrad through W^T copies, wgrad over each expert's tokens
     g.manual_seed(4)
@@ -404,6 +413,45 @@ def sweep_bench(mx, torch, device, peaks, nbytes=1 << 30, reps=5):
     torch.cuda.empty_cache()
     return {"tensor": f"{rows} x {cols} bf16 ({nbytes >> 20} MiB)", "modes": res,
             "note": "SR modes are bound by the integer work of Philox4x32-10 and the exact SR decision, not HBM"}
+
+
+def bf16_out_bench(mx, torch, device, peaks, reps=20):
+    """The expert fprop GEMM (4096 x 5760 x 2880, activations N(0,1), weights
+    N(0, 0.02^2) drawn on the device) with its FP32 and its bf16 output; L2
+    flushed before each launch."""
+    g = torch.Generator(device=device)
+    g.manual_seed(2)
+    a = torch.randn((TOKENS, HIDDEN), generator=g, device=device).to(torch.bfloat16)
+    w = (torch.randn((INTER, HIDDEN), generator=g, device=device) * 0.02).to(torch.bfloat16)
+    qa = mx.mxfp4_quantize(a, mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    qw = mx.mxfp4_quantize(w, mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA)
+    c32 = torch.empty((TOKENS, INTER), dtype=torch.float32, device=device)
+    c16 = torch.empty((TOKENS, INTER), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    res = {}
+    for name, fn in (("fp32_out", lambda: mx.mxfp4_gemm(qa.codes, qa.scales, qw.codes, qw.scales, HIDDEN, out=c32)),
+                     ("bf16_out", lambda: mx.mxfp4_gemm_bf16(qa.codes, qa.scales, qw.codes, qw.scales, HIDDEN,
+                                                             out=c16))):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            ts.append((e0, e1))
+        torch.cuda.synchronize()
+        ms = float(np.median([e0.elapsed_time(e1) for e0, e1 in ts]))
+        tf = 2.0 * TOKENS * INTER * HIDDEN / (ms / 1e3) / 1e12
+        res[name] = {"us": ms * 1e3, "TFLOP/s": tf, "frac_fp4_peak": tf / (4 * peaks["bf16"])}
+    if mx.mxfp4_get_error() != mx.MXFP4_OK:
+        raise RuntimeError("device-side error in the bf16-output measurements")
+    del qa, qw, c32, c16, a, w, flush
+    torch.cuda.empty_cache()
+    res["shape"] = f"{TOKENS} x {INTER} x {HIDDEN}"
+    return res
 
 
 def nvfp4_bench(mx, torch, device, peaks, reps=10):
@@ -636,6 +684,7 @@ def main():
         extras["grouped_moe"] = grouped_bench(mx, torch, device, peaks)
         extras["quantizer_sweep"] = sweep_bench(mx, torch, device, peaks)
         extras["nvfp4"] = nvfp4_bench(mx, torch, device, peaks)
+        extras["gemm_bf16_out"] = bf16_out_bench(mx, torch, device, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

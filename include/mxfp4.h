@@ -242,6 +242,28 @@ MXFP4_API int mxfp4_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint
                        int64_t N, int64_t K, float *c, int64_t ldc, void *stream);
 
 /*
+ * mxfp4_gemm_bf16, mxfp4_grouped_gemm_bf16 -- the same products as
+ * mxfp4_gemm and mxfp4_grouped_gemm with a bf16 output: each FP32 accumulator
+ * is rounded to the nearest bf16 (ties to even) in the epilogue, so C costs
+ * 2 bytes per element of HBM writes instead of 4.  c holds bf16 bit patterns
+ * [M or a_rows, N] (row stride ldc elements), fully overwritten (grouped:
+ * padding rows untouched).  The FP32 value rounded is the one mxfp4_gemm
+ * would store.
+ *
+ * Requirements and errors as for the FP32 forms, except ldc % 8 == 0 (16-byte
+ * rows for the tensor-memory-access stores).  This output form is one of the
+ * fused GEMM epilogues the recipe's next step calls for (the pages quantize
+ * and multiply but fix no output precision beyond FP32 accumulation).
+ */
+MXFP4_API int mxfp4_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales,
+                              const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
+                              int64_t M, int64_t N, int64_t K, uint16_t *c, int64_t ldc, void *stream);
+MXFP4_API int mxfp4_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
+                                      const int32_t *group_offsets, const int32_t *group_sizes, int num_groups,
+                                      const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
+                                      int64_t N, int64_t K, uint16_t *c, int64_t ldc, void *stream);
+
+/*
  * mxfp4_grouped_gemm_wgrad -- per group (expert) g:
  *     C_g[M, N] = sum over k in [group_offsets[g], group_offsets[g+1]) of
  *                 A[:, k] B[:, k]^T

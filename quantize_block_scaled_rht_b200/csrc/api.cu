@@ -28,6 +28,13 @@ int launch_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_sc
 int launch_grouped_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
                          int64_t ldb, const uint8_t *b_scales, const int32_t *offsets, int G, int64_t M, int64_t N,
                          int64_t K, float *c, int64_t ldc, cudaStream_t s);
+int launch_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                     int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
+                     cudaStream_t s);
+int launch_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
+                             const int32_t *offsets, const int32_t *sizes, int G, const uint8_t *b_codes,
+                             int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
+                             cudaStream_t s);
 cudaError_t launch_nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rounding,
                                   uint64_t seed, uint64_t elem_offset, float *tensor_amax, uint8_t *codes,
                                   int64_t ld_codes, uint8_t *scales, int64_t ld_scales, int scale_layout,
@@ -173,16 +180,17 @@ int mxfp4_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scal
     return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
 }
 
+// c_elem: bytes per output element (4 FP32, 2 bf16); TMA stores need 16-byte rows.
 static int check_gemm_common(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
-                             int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, const float *c,
-                             int64_t ldc) {
+                             int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, const void *c,
+                             int64_t ldc, int c_elem = 4) {
     if (!a_codes || !a_scales || !b_codes || !b_scales || !c) return MXFP4_ERR_INVALID_ARG;
     if (N <= 0 || K <= 0) return MXFP4_ERR_INVALID_ARG;
     if (K % 32) return MXFP4_ERR_INVALID_ARG;
     if (K % 64) return MXFP4_ERR_UNSUPPORTED;
     if (lda < K / 2 || ldb < K / 2 || ldc < N) return MXFP4_ERR_INVALID_ARG;
     if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
-        !aligned16(c) || (lda % 16) || (ldb % 16) || (ldc % 4))
+        !aligned16(c) || (lda % 16) || (ldb % 16) || ((ldc * c_elem) % 16))
         return MXFP4_ERR_ALIGNMENT;
     if (N > (int64_t)1 << 31 || K > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
     return MXFP4_OK;
@@ -210,6 +218,31 @@ int mxfp4_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_sca
     if (a_rows > (int64_t)1 << 31 || (int64_t)num_groups * N > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
     return mxfp4::launch_grouped_gemm(a_codes, lda, a_scales, a_rows, group_offsets, group_sizes, num_groups,
                                       b_codes, ldb, b_scales, N, K, c, ldc, static_cast<cudaStream_t>(stream));
+}
+
+int mxfp4_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                    int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
+                    void *stream) {
+    if (M <= 0) return MXFP4_ERR_INVALID_ARG;
+    const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc, 2);
+    if (rc != MXFP4_OK) return rc;
+    if (M > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    return mxfp4::launch_gemm_bf16(a_codes, lda, a_scales, b_codes, ldb, b_scales, M, N, K, c, ldc,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+int mxfp4_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
+                            const int32_t *group_offsets, const int32_t *group_sizes, int num_groups,
+                            const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K,
+                            uint16_t *c, int64_t ldc, void *stream) {
+    if (!group_offsets || !group_sizes) return MXFP4_ERR_INVALID_ARG;
+    if (num_groups <= 0 || a_rows <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (num_groups > 1024) return MXFP4_ERR_UNSUPPORTED;
+    const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc, 2);
+    if (rc != MXFP4_OK) return rc;
+    if (a_rows > (int64_t)1 << 31 || (int64_t)num_groups * N > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    return mxfp4::launch_grouped_gemm_bf16(a_codes, lda, a_scales, a_rows, group_offsets, group_sizes, num_groups,
+                                           b_codes, ldb, b_scales, N, K, c, ldc, static_cast<cudaStream_t>(stream));
 }
 
 int mxfp4_grouped_gemm_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,

@@ -103,7 +103,7 @@ struct GemmParams {
     int64_t M, N, K;
     int64_t katoms;            // ceil(K / 128): scale atoms per 128-row tile
     int64_t b_rowtiles;        // ceil(N / 128): 128-row scale tiles of one B operand
-    float *c;
+    void *c;                   // FP32 or, with the bf16 epilogue, bf16 [.., ldc]
     int64_t ldc;
     const int32_t *group_offsets;
     const int32_t *group_sizes;
@@ -280,7 +280,7 @@ __device__ __noinline__ void issue_stage_tail(uint32_t d_tmem, uint32_t st, uint
     }
 }
 
-template <class Cfg, int MODE>
+template <class Cfg, int MODE, bool OBF16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     mxfp4_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                       const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ CUtensorMap tma_sfa,
@@ -483,56 +483,124 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const bool full_box = MODE == MODE_DENSE || (row_lo + 32 <= ti.rows_valid);
             const bool any_row = row_lo < ti.rows_valid;
             const bool empty_k = ti.kg <= 0;              // grouped K: an empty group's output is zero
-            for (int j = 0; j < BN / 32; ++j) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (acc ? Cfg::ACC1_COL : 0u) + 32u * j, v);
-                tmem_ld_wait();
-                if (empty_k) {
+            if constexpr (OBF16) {
+                // 64 columns per step: two 32-column TMEM loads rounded to
+                // bf16 pairs (RNE), one 128-byte row segment per lane
+                const uint32_t tm = tmem + ((uint32_t)(32 * q) << 16) + (acc ? Cfg::ACC1_COL : 0u);
+                for (int j = 0; j < BN / 64; ++j) {
+                    uint32_t w[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = 0u;
-                }
-                if constexpr (Cfg::NV) {
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(tm + 64u * j + 32u * h, v);
+                        tmem_ld_wait();
+                        if (empty_k) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), nv_scale));
-                }
-                if (j == BN / 32 - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(acc ? empty_leader1 : empty_leader0);
-                }
-                if (!any_row) continue;
-                const int64_t col0 = ti.n0 + 32 * j;
-                if (col0 >= p.N) continue;
-                if (full_box) {
-                    uint8_t *buf = epi_base + (ew * 2 + (buf_i & 1u)) * EPI_BUF;
-                    if (lane == 0) bulk_wait_group_read<1>();
-                    __syncwarp();
+                            for (int i = 0; i < 32; ++i) v[i] = 0u;
+                        }
+                        if constexpr (Cfg::NV) {
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint32_t off = (uint32_t)lane * 128u + (((uint32_t)c ^ (uint32_t)(lane & 7)) << 4);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(buf) + off),
-                                     "r"(v[4 * c]), "r"(v[4 * c + 1]), "r"(v[4 * c + 2]), "r"(v[4 * c + 3])
-                                     : "memory");
+                            for (int i = 0; i < 32; ++i)
+                                v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), nv_scale));
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            w[16 * h + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
                     }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tma_c, (int32_t)col0, (int32_t)(ti.c_row0 + row_lo), buf);
-                        bulk_commit_group();
+                    if (j == BN / 64 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(acc ? empty_leader1 : empty_leader0);
                     }
-                    ++buf_i;
-                } else if (row_lo + lane < ti.rows_valid) {
-                    float *dst = p.c + (ti.c_row0 + row_lo + lane) * p.ldc + col0;
+                    if (!any_row) continue;
+                    const int64_t col0 = ti.n0 + 64 * j;
+                    if (col0 >= p.N) continue;
+                    if (full_box) {
+                        uint8_t *buf = epi_base + (ew * 2 + (buf_i & 1u)) * EPI_BUF;
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const int64_t cc = col0 + 4 * c;
-                        if (cc + 4 <= p.N) {
-                            asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * c), "r"(v[4 * c]),
-                                         "r"(v[4 * c + 1]), "r"(v[4 * c + 2]), "r"(v[4 * c + 3])
+                        for (int c = 0; c < 8; ++c) {
+                            const uint32_t off = (uint32_t)lane * 128u + (((uint32_t)c ^ (uint32_t)(lane & 7)) << 4);
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(buf) + off),
+                                         "r"(w[4 * c]), "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
                                          : "memory");
-                        } else {
-                            for (int e = 0; e < 4; ++e)
-                                if (cc + e < p.N) dst[4 * c + e] = __uint_as_float(v[4 * c + e]);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tma_c, (int32_t)col0, (int32_t)(ti.c_row0 + row_lo), buf);
+                            bulk_commit_group();
+                        }
+                        ++buf_i;
+                    } else if (row_lo + lane < ti.rows_valid) {
+                        uint16_t *dst = static_cast<uint16_t *>(p.c) + (ti.c_row0 + row_lo + lane) * p.ldc + col0;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int64_t cc = col0 + 8 * c;
+                            if (cc + 8 <= p.N) {
+                                asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 8 * c),
+                                             "r"(w[4 * c]), "r"(w[4 * c + 1]), "r"(w[4 * c + 2]), "r"(w[4 * c + 3])
+                                             : "memory");
+                            } else {
+                                for (int e = 0; e < 8; ++e)
+                                    if (cc + e < p.N) dst[8 * c + e] = (uint16_t)(w[4 * c + e / 2] >> (16 * (e & 1)));
+                            }
+                        }
+                    }
+                }
+            } else {
+                for (int j = 0; j < BN / 32; ++j) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + (acc ? Cfg::ACC1_COL : 0u) + 32u * j, v);
+                    tmem_ld_wait();
+                    if (empty_k) {
+    #pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = 0u;
+                    }
+                    if constexpr (Cfg::NV) {
+    #pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__fmul_rn(__uint_as_float(v[i]), nv_scale));
+                    }
+                    if (j == BN / 32 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(acc ? empty_leader1 : empty_leader0);
+                    }
+                    if (!any_row) continue;
+                    const int64_t col0 = ti.n0 + 32 * j;
+                    if (col0 >= p.N) continue;
+                    if (full_box) {
+                        uint8_t *buf = epi_base + (ew * 2 + (buf_i & 1u)) * EPI_BUF;
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+    #pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const uint32_t off = (uint32_t)lane * 128u + (((uint32_t)c ^ (uint32_t)(lane & 7)) << 4);
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(buf) + off),
+                                         "r"(v[4 * c]), "r"(v[4 * c + 1]), "r"(v[4 * c + 2]), "r"(v[4 * c + 3])
+                                         : "memory");
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tma_c, (int32_t)col0, (int32_t)(ti.c_row0 + row_lo), buf);
+                            bulk_commit_group();
+                        }
+                        ++buf_i;
+                    } else if (row_lo + lane < ti.rows_valid) {
+                        float *dst = static_cast<float *>(p.c) + (ti.c_row0 + row_lo + lane) * p.ldc + col0;
+    #pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int64_t cc = col0 + 4 * c;
+                            if (cc + 4 <= p.N) {
+                                asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(dst + 4 * c), "r"(v[4 * c]),
+                                             "r"(v[4 * c + 1]), "r"(v[4 * c + 2]), "r"(v[4 * c + 3])
+                                             : "memory");
+                            } else {
+                                for (int e = 0; e < 4; ++e)
+                                    if (cc + e < p.N) dst[4 * c + e] = __uint_as_float(v[4 * c + e]);
+                            }
                         }
                     }
                 }
@@ -628,14 +696,14 @@ static int sm_count() {
     return n > 0 ? n : 148;
 }
 
-template <class Cfg, int MODE>
+template <class Cfg, int MODE, bool OBF16>
 static cudaError_t set_smem_attr() {
     // once per device and instantiation: keep cudaFuncSetAttribute off the hot path
     static int done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<Cfg, MODE>,
+    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<Cfg, MODE, OBF16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
     return e;
@@ -644,7 +712,7 @@ static cudaError_t set_smem_attr() {
 struct GemmArgs {
     const uint8_t *a_codes, *a_scales, *b_codes, *b_scales;
     int64_t lda, ldb, M, N, K, ldc;
-    float *c;
+    void *c;
     const int32_t *offsets, *sizes;
     int G;
     const float *a_amax = nullptr, *b_amax = nullptr;
@@ -653,7 +721,8 @@ struct GemmArgs {
 // Returns 0 on success, MXFP4_ERR_CUDA when a map or launch fails.
 // Grouped K: a and b are [M, K/2] and [N, K/2] over all groups' K ranges, c is
 // [G * M, N]; the B operand and C map cover G groups only in grouped-rows mode.
-template <class Cfg, int MODE>
+// OBF16: C is bf16 (RNE of the FP32 accumulators), stored in 64-column boxes.
+template <class Cfg, int MODE, bool OBF16 = false>
 static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
     constexpr int BN = Cfg::BN;
     const int G = MODE == MODE_GROUPED_M ? g.G : 1;
@@ -665,14 +734,15 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
                   (uint64_t)g.lda, CHUNK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b_codes, (uint64_t)(g.K / 2), (uint64_t)G * g.N,
                   (uint64_t)g.ldb, CHUNK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.c, (uint64_t)g.N, (uint64_t)c_rows, (uint64_t)g.ldc * 4,
-                  32, 32, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tc, OBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.c,
+                  (uint64_t)g.N, (uint64_t)c_rows, (uint64_t)g.ldc * (OBF16 ? 2 : 4), OBF16 ? 64 : 32, 32,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
         // scale atoms as a 3D tensor [128-row tile][K atom][512 bytes = 128 x 32-bit]:
         // one box holds NATOM consecutive atoms of one (A) or NRT (B) row tiles
         !make_map_3d(&tsa, g.a_scales, (uint64_t)katoms, (uint64_t)a_tiles, Cfg::NATOM, 1) ||
         !make_map_3d(&tsb, g.b_scales, (uint64_t)katoms, (uint64_t)(G * b_tiles), Cfg::NATOM, Cfg::NRT))
         return MXFP4_ERR_CUDA;
-    if (set_smem_attr<Cfg, MODE>() != cudaSuccess) return MXFP4_ERR_CUDA;
+    if (set_smem_attr<Cfg, MODE, OBF16>() != cudaSuccess) return MXFP4_ERR_CUDA;
     GemmParams p{};
     p.M = g.M; p.N = g.N; p.K = g.K;
     p.katoms = katoms;
@@ -687,7 +757,7 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
         const int64_t tiles = (MODE == MODE_GROUPED_K ? g.G : 1) * ((g.M + 255) / 256) * ((g.N + BN - 1) / BN);
         pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
     }
-    const cudaError_t e = launch_pdl(mxfp4_gemm_kernel<Cfg, MODE>, dim3((unsigned)(2 * pairs)), dim3(NUM_THREADS),
+    const cudaError_t e = launch_pdl(mxfp4_gemm_kernel<Cfg, MODE, OBF16>, dim3((unsigned)(2 * pairs)), dim3(NUM_THREADS),
                                      (size_t)Cfg::SMEM_BYTES, s, ta, tb, tc, tsa, tsb, p);
     return e == cudaSuccess ? 0 : MXFP4_ERR_CUDA;
 }
@@ -703,6 +773,21 @@ int launch_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_sc
                         const uint8_t *b_scales, int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s) {
     GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, a_rows, N, K, ldc, c, offsets, sizes, G};
     return launch_cfg<DefaultCfg, MODE_GROUPED_M>(g, s);
+}
+
+int launch_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                     int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
+                     cudaStream_t s) {
+    GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, M, N, K, ldc, c, nullptr, nullptr, 1};
+    return launch_cfg<DefaultCfg, MODE_DENSE, true>(g, s);
+}
+
+int launch_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
+                             const int32_t *offsets, const int32_t *sizes, int G, const uint8_t *b_codes,
+                             int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
+                             cudaStream_t s) {
+    GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, a_rows, N, K, ldc, c, offsets, sizes, G};
+    return launch_cfg<DefaultCfg, MODE_GROUPED_M, true>(g, s);
 }
 
 int launch_grouped_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,

@@ -62,6 +62,14 @@ def test_invalid_arguments_rejected_without_gpu():
     assert L.mxfp4_gemm(fake, 16, fake, fake, 16, fake, 128, 128, 96, fake, 128, None) == 3
     assert L.mxfp4_gemm(fake, 16, fake, fake, 16, fake, 128, 128, 80, fake, 128, None) == 1
     assert L.mxfp4_gemm(fake, 40, fake, fake, 32, fake, 128, 128, 64, fake, 128, None) == 2
+    # bf16-output GEMM: ldc must give 16-byte rows (8 bf16), K rules as for FP32
+    assert L.mxfp4_gemm_bf16(fake, 32, fake, fake, 32, fake, 128, 132, 64, fake, 132, None) == 2
+    assert L.mxfp4_gemm_bf16(fake, 16, fake, fake, 16, fake, 128, 128, 96, fake, 128, None) == 3
+    assert L.mxfp4_gemm_bf16(fake, 32, fake, fake, 32, fake, 0, 128, 64, fake, 128, None) == 1
+    assert L.mxfp4_grouped_gemm_bf16(fake, 32, fake, 128, fake, fake, 5000, fake, 32, fake, 128, 64, fake, 128,
+                                     None) == 3
+    assert L.mxfp4_grouped_gemm_bf16(fake, 32, fake, 128, fake, fake, 2, fake, 32, fake, 132, 64, fake, 132,
+                                     None) == 2
     # grouped wgrad: K not a multiple of 128, too many groups
     assert L.mxfp4_grouped_gemm_wgrad(fake, 32, fake, fake, 32, fake, fake, 2, 128, 128, 64, fake, 128, None) == 1
     assert L.mxfp4_grouped_gemm_wgrad(fake, 64, fake, fake, 64, fake, fake, 5000, 128, 128, 128, fake, 128,

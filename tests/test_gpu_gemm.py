@@ -278,3 +278,86 @@ def test_nvfp4_gemm_matches_oracle(shape):
     ref, s = oracle.nvfp4_gemm_entries(ca, sa, aa, cb, sb, ab, K, pairs)
     got = np.array([c[m, n] for m, n in pairs], np.float64)
     assert_gemm_close(got, ref, s)
+
+
+def _assert_bf16_close(c16: np.ndarray, ref: np.ndarray, s: np.ndarray):
+    """bf16 output: the FP32 bound of assert_gemm_close plus one bf16 rounding
+    of the FP32 value (8 significant bits, so round to nearest is within
+    2^-8 of the value)."""
+    nan_ref = np.isnan(ref)
+    assert np.array_equal(np.isnan(c16), nan_ref)
+    ok = ~nan_ref
+    err = np.abs(c16[ok].astype(np.float64) - ref[ok])
+    fp32_bound = 1e-5 * s[ok]
+    bound = fp32_bound + 2.0 ** -8 * (np.abs(ref[ok]) + fp32_bound)
+    assert not (err > bound).any(), f"{int((err > bound).sum())} entries outside the bf16 bound"
+
+
+def _bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).cpu().numpy()
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 192, 64), (300, 200, 320), (1, 8, 128), (257, 392, 576),
+                                   (512, 768, 1024), (130, 72, 2880)])
+def test_gemm_bf16_output(M, N, K):
+    """bf16 epilogue: within the oracle bound, and bit-equal to the RNE of the
+    FP32 path's output for the same operands (same accumulators)."""
+    a = synth.normal_bf16((M, K), 30 + M)
+    b = synth.normal_bf16((N, K), 40 + N, 0.02)
+    ca, sa = _oracle_operand(a)
+    cb, sb = _oracle_operand(b)
+    args = (dev_u8(ca), dev_u8(to_mma(sa, K)), dev_u8(cb), dev_u8(to_mma(sb, K)), K)
+    c16 = mx.mxfp4_gemm_bf16(*args)
+    c32 = mx.mxfp4_gemm(*args)
+    torch.cuda.synchronize()
+    assert np.array_equal(_bf16_bits(c16), _bf16_bits(c32.to(torch.bfloat16)))
+    ref, s = oracle.gemm(ca, sa, cb, sb, K)
+    _assert_bf16_close(c16.float().cpu().numpy(), ref, s)
+
+
+def test_gemm_bf16_nan_and_strided_output():
+    """NaN scales give NaN rows/columns; a wider output row stride leaves the
+    columns past N untouched."""
+    M, N, K = 256, 200, 256
+    a = synth.normal_bf16((M, K), 7)
+    b = synth.normal_bf16((N, K), 8, 0.02)
+    ca, sa = _oracle_operand(a)
+    cb, sb = _oracle_operand(b)
+    sa = sa.copy(); sa[3, 1] = 0xFF
+    big = torch.full((M, N + 24), 77.0, dtype=torch.bfloat16, device="cuda")
+    out = big[:, :N]
+    mx.mxfp4_gemm_bf16(dev_u8(ca), dev_u8(to_mma(sa, K)), dev_u8(cb), dev_u8(to_mma(sb, K)), K, out=out)
+    torch.cuda.synchronize()
+    c = out.float().cpu().numpy()
+    assert np.all(np.isnan(c[3]))
+    assert torch.all(big[:, N:] == 77.0)
+    ref, s = oracle.gemm(ca, sa, cb, sb, K)
+    _assert_bf16_close(c, ref, s)
+
+
+@pytest.mark.parametrize("sizes,N,K", [([1, 130, 0, 257, 128], 192, 256), ([300, 5, 64], 384, 576),
+                                       ([17], 224, 128)])
+def test_grouped_gemm_bf16(sizes, N, K):
+    sizes, offsets, rows, a, w = _grouped_case(sizes, N, K)
+    G = len(sizes)
+    qa = mx.mxfp4_quantize(dev_bf16(a), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    qw = [mx.mxfp4_quantize(dev_bf16(w[g]), mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA) for g in range(G)]
+    b_codes = torch.stack([q.codes for q in qw])
+    b_scales = torch.cat([q.scales for q in qw])
+    d_off, d_sz = torch.from_numpy(offsets).cuda(), torch.from_numpy(sizes).cuda()
+    out16 = torch.full((rows, N), 1280.0, dtype=torch.bfloat16, device="cuda")
+    mx.mxfp4_grouped_gemm_bf16(qa.codes, qa.scales, d_off, d_sz, b_codes, b_scales, N, K, out=out16)
+    out32 = torch.full((rows, N), 1280.0, dtype=torch.float32, device="cuda")
+    mx.mxfp4_grouped_gemm(qa.codes, qa.scales, d_off, d_sz, b_codes, b_scales, N, K, out=out32)
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    # the padding rows keep 1280 (exact in bf16) in both; every written entry is the RNE of the FP32 one
+    assert np.array_equal(_bf16_bits(out16), _bf16_bits(out32.to(torch.bfloat16)))
+    c = out16.float().cpu().numpy()
+    ca, sa = oracle.quantize(a, oracle.LAYOUT_1D_ROW)
+    for g in range(G):
+        o, n = int(offsets[g]), int(sizes[g])
+        if n:
+            cw, sw = oracle.quantize(w[g], oracle.LAYOUT_2D)
+            ref, s = oracle.gemm(ca[o:o + n], sa[o:o + n], cw, sw, K, 0, 1)
+            _assert_bf16_close(c[o:o + n], ref, s)
+        assert np.all(c[o + n:int(offsets[g + 1])] == 1280.0)
