@@ -62,8 +62,8 @@ KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 # profiles/expert_step_kernels_ncu_full.md.  The figures hold only for the
 # kernel sources they were taken from: a changed source gives traffic null.
 NCU_TRAFFIC = {
-    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "749f84de0bbb3a8f",
-             "bytes": {"fprop": 51.79e6, "dgrad": 23.32e6, "wgrad": 29.59e6}},
+    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "2d6ee8083374b6a6",
+             "bytes": {"fprop": 52.84e6, "dgrad": 24.32e6, "wgrad": 30.56e6}},
     "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "5b7f4ae361de04d1",
               "bytes": {"quant_x_dual": 23.61e6, "quant_w_2d": 33.29e6, "quant_dy_dual_sr": 49.18e6}},
 }
@@ -637,35 +637,64 @@ def main():
                   "traffic": ncu_traffic("quant", list(QUANT_OPS)),
                   "peak_note": f"{peaks['src']} copy bandwidth"}
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers.  Every step copies
+    # its inputs in from pinned host memory and its three results out, inside
+    # the timed region.  Two device buffer sets and three streams (upload,
+    # compute, download) let step i+1's upload and step i-1's download run
+    # while step i computes; the host link is full duplex.  Events order the
+    # reuse of each set: its inputs are overwritten only after the step that
+    # read them has finished, its outputs only after their download.
     e2e = None
     if args.e2e_steps > 0:
+        sets = [step, ExpertStep(mx, torch, x, w, dy, device)]
+        set_ops = [st.ops() for st in sets]
         hx = step.x.cpu().pin_memory()
         hw = step.w.cpu().pin_memory()
         hdy = step.dy.cpu().pin_memory()
-        hy = torch.empty(step.y.shape, dtype=torch.float32).pin_memory()
-        hdx = torch.empty(step.dx.shape, dtype=torch.float32).pin_memory()
-        hdw = torch.empty(step.dw.shape, dtype=torch.float32).pin_memory()
+        hout = [tuple(torch.empty(t.shape, dtype=torch.float32).pin_memory() for t in (st.y, st.dx, st.dw))
+                for st in sets]
+        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        used = [False, False]
 
-        def e2e_step():
-            step.x.copy_(hx, non_blocking=True)
-            step.w.copy_(hw, non_blocking=True)
-            step.dy.copy_(hdy, non_blocking=True)
-            for _, fn in ops:
+        def e2e_step(i):
+            b = i & 1
+            st = sets[b]
+            with torch.cuda.stream(s_in):
+                if used[b]:
+                    s_in.wait_event(ev_done[b])
+                st.x.copy_(hx, non_blocking=True)
+                st.w.copy_(hw, non_blocking=True)
+                st.dy.copy_(hdy, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if used[b]:
+                stream.wait_event(ev_out[b])
+            for _, fn in set_ops[b]:
                 fn()
-            hy.copy_(step.y, non_blocking=True)
-            hdx.copy_(step.dx, non_blocking=True)
-            hdw.copy_(step.dw, non_blocking=True)
+            ev_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[b])
+                for h, d in zip(hout[b], (st.y, st.dx, st.dw)):
+                    h.copy_(d, non_blocking=True)
+                ev_out[b].record(s_out)
+            used[b] = True
 
-        for _ in range(3):
-            e2e_step()
+        for i in range(4):
+            e2e_step(i)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(4, 4 + args.e2e_steps):
+            e2e_step(i)
+        stream.wait_event(ev_out[0])
+        stream.wait_event(ev_out[1])
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1)
@@ -673,6 +702,7 @@ def main():
             t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             e2e_ms = float(t.item())
+        hy, hdx, hdw = hout[0]
         h2d = (hx.numel() + hw.numel() + hdy.numel()) * 2
         d2h = (hy.numel() + hdx.numel() + hdw.numel()) * 4
         e2e = {"value": STEP_FLOPS * world / (e2e_ms / args.e2e_steps / 1e3) / 1e12, "unit": "TFLOP/s",
