@@ -13,14 +13,17 @@
 // rows of A and BN/2 rows of B, so every SM streams 128 + BN/2 operand rows per
 // K step instead of 128 + BN.  Per CTA, 6 warps:
 //   warp 0      TMA producer: its A rows, its half of B and the scale atoms
-//               (A: its own 128 rows; B: all BN rows) into a 6-stage ring;
-//               every load completes on the even CTA's stage barrier;
+//               (A: its own 128 rows; B: all BN rows) into a STAGES-deep ring
+//               (MXFP4: 3 stages of 512 K-elements); every load completes on
+//               the even CTA's stage barrier;
 //   warp 1      TMEM owner; in the even CTA also the MMA issuer: scale atoms
-//               to TMEM (tcgen05.cp, both CTAs), 4 pair MMAs per stage into one
-//               of two accumulators, stage release by a commit to both CTAs;
+//               to TMEM (tcgen05.cp, both CTAs), 4 * KCH pair MMAs of K = 64
+//               per stage into one of two accumulators, stage release by a
+//               commit to both CTAs;
 //   warps 2..5  epilogue: TMEM -> registers -> swizzled smem -> TMA store of
-//               this CTA's 128 rows, overlapping the next tile's MMAs, then an
-//               arrive on the even CTA's accumulator-empty barrier.
+//               this CTA's 128 rows (FP32, or bf16 rounded to nearest even),
+//               overlapping the next tile's MMAs, then an arrive on the even
+//               CTA's accumulator-empty barrier.
 // Every barrier wait is bounded by the GPU global timer; a wait that runs out
 // records MXFP4_ERR_TIMEOUT, raises the CTA's abort flag, and each role drains
 // what it has in flight before both CTAs meet at the final cluster barrier.
