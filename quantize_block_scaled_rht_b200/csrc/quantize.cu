@@ -522,31 +522,49 @@ __global__ void __launch_bounds__(256) dequant_row_kernel(const DequantParams p)
     }
 }
 
-// Transposed-view codes [cols, rows/2] back to out[rows, cols].  A CTA handles
+// Transposed-view codes [cols, rows/2] back to out[rows, cols].  A tile is
 // 64 code rows (= output columns) x 8 blocks (= 256 output rows): the codes
-// are staged with coalesced 16-byte loads; warp w decodes block w, lane l the
-// output columns 2l and 2l+1, so each output row is written as one contiguous
-// 128-byte (bf16) or 256-byte (fp32) warp store.
+// are staged with coalesced 16-byte cp.async loads into a two-tile ring, the
+// next tile's load in flight while this one is decoded (persistent grid);
+// warp w decodes block w, lane l the output columns 2l and 2l+1, so each
+// output row is written as one contiguous 128-byte (bf16) or 256-byte (fp32)
+// warp store.
 template <int RHT, bool F32, bool MMA>
 __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p) {
     pdl_wait();
     pdl_trigger();
-    __shared__ __align__(16) uint4 tin[COL_TC][8];                 // 8 KB of codes
+    __shared__ __align__(16) uint4 tin[2][COL_TC][8];              // 2 x 8 KB of codes
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t tiles_r = (p.rows + COL_TR - 1) / COL_TR;
     const int64_t tiles_c = (p.cols + COL_TC - 1) / COL_TC;
     const int64_t ntiles = tiles_r * tiles_c;
-    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x) {
+    auto load = [&](int64_t t, int buf) {
         const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
         const int64_t r0 = tr * COL_TR, c0 = tc * COL_TC;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int row = (tid >> 3) + 32 * i, ch = tid & 7;
             const int64_t crow = c0 + row, rin = r0 + 32 * ch;
-            if (crow < p.cols && rin < p.rows)
-                tin[row][ch] = ldg_nc_v4(p.codes + crow * p.ld_codes + (rin >> 1));
+            if (crow < p.cols && rin < p.rows) cp_async16(&tin[buf][row][ch], p.codes + crow * p.ld_codes + (rin >> 1));
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    int64_t t = blockIdx.x;
+    if (t < ntiles) load(t, 0);
+    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+        // the buffer refilled here was read in the previous iteration, which
+        // ended with a barrier
+        const int buf = it & 1;
+        const int64_t tn = t + gridDim.x;
+        if (tn < ntiles) {
+            load(tn, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
+        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
+        const int64_t r0 = tr * COL_TR, c0 = tc * COL_TC;
         const int64_t rb = r0 + 32 * warp, oc = c0 + 2 * lane;
         if (rb < p.rows && oc < p.cols) {
             const int64_t kb = rb >> 5;
@@ -558,29 +576,53 @@ __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p)
                 s0 = p.scales[oc * p.ld_scales + kb];
                 s1 = p.scales[(oc + 1) * p.ld_scales + kb];
             }
-            float v0[32], v1[32];
-            decode32(tin[2 * lane][warp], s0, v0);
-            decode32(tin[2 * lane + 1][warp], s1, v1);
-            if constexpr (RHT) {
-                const float c = rht_norm<RHT>();
-#pragma unroll
-                for (int s = 0; s < 32; s += RHT) { fwht<RHT>(v0 + s); fwht<RHT>(v1 + s); }
+            if constexpr (RHT == 0) {
+                // no transform: decode and store one row pair at a time, so
+                // that only the packed codes stay in registers
+                const uint4 q0 = tin[buf][2 * lane][warp], q1 = tin[buf][2 * lane + 1][warp];
+                const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
+                const float X0 = scale_from_code(s0), X1 = scale_from_code(s1);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const uint32_t fl = p.sgn_bit[i % RHT];
-                    v0[i] = __uint_as_float(__float_as_uint(__fmul_rn(v0[i], c)) ^ fl);
-                    v1[i] = __uint_as_float(__float_as_uint(__fmul_rn(v1[i], c)) ^ fl);
+                    const float a = s0 == 0xFFu ? __uint_as_float(0x7FFFFFFFu)
+                                                : __fmul_rn(e2m1_value((w0[i >> 3] >> (4 * (i & 7))) & 0xFu), X0);
+                    const float b = s1 == 0xFFu ? __uint_as_float(0x7FFFFFFFu)
+                                                : __fmul_rn(e2m1_value((w1[i >> 3] >> (4 * (i & 7))) & 0xFu), X1);
+                    const int64_t gr = rb + i;
+                    if constexpr (F32) {
+                        float2 *dst = reinterpret_cast<float2 *>(reinterpret_cast<float *>(p.out) + gr * p.ld_out + oc);
+                        *dst = make_float2(a, b);
+                    } else {
+                        uint32_t *dst =
+                            reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(p.out) + gr * p.ld_out + oc);
+                        *dst = pack_bf16x2(a, b);
+                    }
                 }
-            }
+            } else {
+                float v0[32], v1[32];
+                decode32(tin[buf][2 * lane][warp], s0, v0);
+                decode32(tin[buf][2 * lane + 1][warp], s1, v1);
+                if constexpr (RHT) {
+                    const float c = rht_norm<RHT>();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int64_t gr = rb + i;
-                if constexpr (F32) {
-                    float2 *dst = reinterpret_cast<float2 *>(reinterpret_cast<float *>(p.out) + gr * p.ld_out + oc);
-                    *dst = make_float2(v0[i], v1[i]);
-                } else {
-                    uint32_t *dst = reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(p.out) + gr * p.ld_out + oc);
-                    *dst = pack_bf16x2(v0[i], v1[i]);
+                    for (int s = 0; s < 32; s += RHT) { fwht<RHT>(v0 + s); fwht<RHT>(v1 + s); }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const uint32_t fl = p.sgn_bit[i % RHT];
+                        v0[i] = __uint_as_float(__float_as_uint(__fmul_rn(v0[i], c)) ^ fl);
+                        v1[i] = __uint_as_float(__float_as_uint(__fmul_rn(v1[i], c)) ^ fl);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int64_t gr = rb + i;
+                    if constexpr (F32) {
+                        float2 *dst = reinterpret_cast<float2 *>(reinterpret_cast<float *>(p.out) + gr * p.ld_out + oc);
+                        *dst = make_float2(v0[i], v1[i]);
+                    } else {
+                        uint32_t *dst = reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(p.out) + gr * p.ld_out + oc);
+                        *dst = pack_bf16x2(v0[i], v1[i]);
+                    }
                 }
             }
         }
@@ -767,11 +809,12 @@ cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int6
 template <int RHT, bool F32>
 static cudaError_t launch_dequant_t(int layout, int smode, const DequantParams &p, cudaStream_t s) {
     if (layout == MXFP4_LAYOUT_1D_COL) {
+        // persistent at full occupancy: each CTA keeps its next tile's load in flight
         const int64_t tiles = ((p.rows + COL_TR - 1) / COL_TR) * ((p.cols + COL_TC - 1) / COL_TC);
-        const int64_t cap = (int64_t)num_sms() * 8;
+        auto kern = smode == 2 ? dequant_col_kernel<RHT, F32, true> : dequant_col_kernel<RHT, F32, false>;
+        const int64_t cap = (int64_t)num_sms() * resident_ctas(reinterpret_cast<const void *>(kern), 256);
         const unsigned g = (unsigned)(tiles < cap ? tiles : cap);
-        if (smode == 2) return launch_pdl(dequant_col_kernel<RHT, F32, true>, dim3(g), dim3(256), 0, s, p);
-        else return launch_pdl(dequant_col_kernel<RHT, F32, false>, dim3(g), dim3(256), 0, s, p);
+        return launch_pdl(kern, dim3(g), dim3(256), 0, s, p);
     } else {
         const unsigned g = (unsigned)grid_for(p.rows * (p.cols / 32), 256);
         if (smode == 0) return launch_pdl(dequant_row_kernel<RHT, F32, 0>, dim3(g), dim3(256), 0, s, p);

@@ -146,6 +146,22 @@ def test_dequantize_mma_scales():
     assert np.array_equal(host(out), b16)
 
 
+@pytest.mark.parametrize("rht", [0, 32])
+@pytest.mark.parametrize("mma", [False, True])
+def test_dequantize_column_many_tiles(rht, mma):
+    """Column dequantize on more 256 x 64 tiles (720) than resident CTAs, so
+    that each CTA walks several tiles through its two-tile prefetch ring."""
+    rows, cols = 4096, 2880
+    x = synth.normal_bf16((rows, cols), 77)
+    sl = mx.SCALES_MMA if mma else mx.SCALES_ROWMAJOR
+    q = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_COL, rht, mx.ROUND_RNE, 5, 0, sl)
+    out = mx.mxfp4_dequantize(q.codes, q.scales, rows, cols, mx.LAYOUT_1D_COL, rht, 5, scale_layout=sl)
+    codes, scales = oracle.quantize(x, oracle.LAYOUT_1D_COL, rht, oracle.ROUND_RNE, 5)[:2]
+    assert np.array_equal(host(q.codes), codes)
+    _, b16 = oracle.dequantize(codes, scales, rows, cols, oracle.LAYOUT_1D_COL, rht, 5)
+    assert np.array_equal(host(out), b16)
+
+
 def test_invalid_arguments_are_rejected():
     x = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(mx.MXFP4Error) as e:
