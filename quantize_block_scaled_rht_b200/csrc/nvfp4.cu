@@ -63,12 +63,26 @@ __global__ void __launch_bounds__(256) nv_amax_kernel(const uint16_t *x, int64_t
     pdl_trigger();
     uint32_t m = 0;
     const int64_t chunks = cols / 8, n = rows * chunks;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / chunks, c = (i - r * chunks) * 8;
-        const uint4 u = nv_ldg_v4(x + r * ld_x + c);
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    // (row, chunk) of the flat index i, stepped by the grid stride without a
+    // division per iteration
+    const int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t dr = stride / chunks, dc = stride - dr * chunks;
+    int64_t r = i0 / chunks, ch = i0 - r * chunks;
+    auto step = [&]() {
+        r += dr;
+        ch += dc;
+        if (ch >= chunks) { ch -= chunks; ++r; }
+    };
+    // two loads in flight per thread
+    for (int64_t i = i0; i < n; i += 2 * stride) {
+        const uint4 u = nv_ldg_v4(x + r * ld_x + 8 * ch);
+        step();
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (i + stride < n) v = nv_ldg_v4(x + r * ld_x + 8 * ch);
+        step();
+        const uint32_t w[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
+        for (int j = 0; j < 8; ++j) m = max(m, max(w[j] & 0x7FFFu, (w[j] >> 16) & 0x7FFFu));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
@@ -136,8 +150,16 @@ __global__ void __launch_bounds__(256) nv_quant_row_kernel(const NvParams p) {
     pdl_trigger();
     const NvTensor t = nv_tensor(p.amax_bits);
     const int64_t nb = p.cols / 16, n = p.rows * nb;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / nb, kb = i - r * nb;
+    // (row, block) of the flat index i, stepped by the grid stride without a
+    // division per iteration
+    const int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t dr = stride / nb, dk = stride - dr * nb;
+    int64_t rr = i0 / nb, kk = i0 - rr * nb;
+    for (int64_t i = i0; i < n; i += stride) {
+        const int64_t r = rr, kb = kk;
+        rr += dr;
+        kk += dk;
+        if (kk >= nb) { kk -= nb; ++rr; }
         const uint16_t *src = p.x + r * p.ld_x + 16 * kb;
         const uint4 u0 = nv_ldg_v4(src), u1 = nv_ldg_v4(src + 8);
         const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
