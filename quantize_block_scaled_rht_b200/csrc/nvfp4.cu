@@ -244,8 +244,15 @@ __global__ void __launch_bounds__(256) nv_dequant_kernel(const NvDeqParams p) {
     const float S = __fdiv_rn(__uint_as_float(*p.amax_bits), 2688.0f);
     const int64_t orows = COL ? p.cols : p.rows, k = COL ? p.rows : p.cols;
     const int64_t nb = k / 16, n = orows * nb;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t orow = i / nb, kb = i - orow * nb;
+    // (output row, block) of the flat index i, stepped by the grid stride
+    const int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t dr = stride / nb, dk = stride - dr * nb;
+    int64_t rr = i0 / nb, kk = i0 - rr * nb;
+    for (int64_t i = i0; i < n; i += stride) {
+        const int64_t orow = rr, kb = kk;
+        rr += dr;
+        kk += dk;
+        if (kk >= nb) { kk -= nb; ++rr; }
         const uint32_t sc = MMA ? p.scales[mma_scale_off(orow, kb, p.katoms)] : p.scales[orow * p.ld_scales + kb];
         const bool nan = (sc & 0x7Fu) == 0x7Fu;
         const float s = nan ? __uint_as_float(0x7FC00000u) : e4m3_to_f32(sc);

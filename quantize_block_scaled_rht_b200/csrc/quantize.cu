@@ -495,9 +495,16 @@ __global__ void __launch_bounds__(256) dequant_row_kernel(const DequantParams p)
     pdl_trigger();
     const int64_t nb = p.cols >> 5;
     const int64_t total = p.rows * nb;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < total;
-         b += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = b / nb, kb = b - r * nb;
+    // (row, block) of the flat index b, stepped by the grid stride without a
+    // division per iteration
+    const int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t dr = stride / nb, dk = stride - dr * nb;
+    int64_t rr = b0 / nb, kk = b0 - rr * nb;
+    for (int64_t b = b0; b < total; b += stride) {
+        const int64_t r = rr, kb = kk;
+        rr += dr;
+        kk += dk;
+        if (kk >= nb) { kk -= nb; ++rr; }
         const uint4 q = ldg_nc_v4(p.codes + r * p.ld_codes + (kb << 4));
         uint32_t sc;
         if constexpr (SMODE == 0) sc = p.scales[r * p.ld_scales + kb];
