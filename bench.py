@@ -65,8 +65,24 @@ NCU_TRAFFIC = {
     "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "2d8f1d1fed03afc6",
              "bytes": {"fprop": 52.84e6, "dgrad": 24.32e6, "wgrad": 30.56e6}},
     "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "46d7edb1f1c1c306",
-              "bytes": {"quant_x_dual": 23.61e6, "quant_w_2d": 33.29e6, "quant_dy_dual_sr": 49.18e6}},
+              "bytes": {"quant_x_dual": 23.61e6, "quant_w_2d": 33.29e6, "quant_dy_dual_sr": 49.18e6},
+              # thread instructions per element (ncu smsp__inst_executed x 32 / elements)
+              "inst_per_elem": {"quant_dy_dual_sr": 80.0}},
 }
+
+
+def ncu_inst_per_elem(name: str):
+    """Thread instructions per element of a quantizer launch (ncu), or None if
+    the kernel source changed since they were counted."""
+    import hashlib
+    t = NCU_TRAFFIC["quant"]
+    m = hashlib.sha1()
+    for f in t["sources"]:
+        with open(os.path.join(ROOT, "quantize_block_scaled_rht_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    if m.hexdigest()[:16] != t["sha1"]:
+        return None
+    return t["inst_per_elem"].get(name)
 
 
 def ncu_traffic(kind: str, names):
@@ -637,6 +653,22 @@ def main():
                   "traffic": ncu_traffic("quant", list(QUANT_OPS)),
                   "peak_note": f"{peaks['src']} copy bandwidth"}
 
+    # The SR dual quantizer of dY is bound by integer issue, not by HBM: its
+    # thread instructions per second (ncu count per element x elements / the
+    # breakdown pass's time) against the issue rate of 4 schedulers x 32 lanes
+    # per SM per cycle at the SM clock sampled during the timed region.
+    roofline_sr = None
+    ipe = ncu_inst_per_elem("quant_dy_dual_sr")
+    if ipe is not None and clocks:
+        n_sms = torch.cuda.get_device_properties(device).multi_processor_count
+        ach = ipe * TOKENS * INTER / (kernels["quant_dy_dual_sr"]["us"] / 1e6) / 1e12
+        peak_i = n_sms * 4 * 32 * clocks["sm_mhz"] * 1e6 / 1e12
+        roofline_sr = {"bound": "alu", "kernel": "quant_dual_kernel (dY: row SR + column RHT-32 SR)",
+                       "achieved": ach, "peak": peak_i, "unit": "T thread-instructions/s", "frac": ach / peak_i,
+                       "traffic": ncu_traffic("quant", ["quant_dy_dual_sr"]),
+                       "peak_note": f"issue rate {n_sms} SMs x 4 schedulers x 32 lanes x {clocks['sm_mhz']:.0f} MHz "
+                                    f"(median sampled); {ipe} thread instructions per element from ncu"}
+
     # end to end through the public API with host buffers.  Every step copies
     # its inputs in from pinned host memory and its three results out, inside
     # the timed region.  Two device buffer sets and three streams (upload,
@@ -727,7 +759,8 @@ def main():
                 "config": {"workload": WORKLOAD, "tokens_per_gpu": TOKENS, "hidden": HIDDEN, "intermediate": INTER,
                            "parallelism": f"dp{world} (independent tokens per rank, no collective)",
                            "l2": f"flushed between timed steps ({args.flush_mib} MiB write, outside step events)"},
-                "roofline": roofline, "roofline_quantize": roofline_q, "kernels": kernels,
+                "roofline": roofline, "roofline_quantize": roofline_q, "roofline_sr_dual": roofline_sr,
+                "kernels": kernels,
                 "quantize_GBps": quant_gbs, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": KERNELS_PER_STEP * K, "clocks": clocks, "wall_s_timed_region": t_wall,
                 "breakdown": f"per-kernel figures from {KB} further steps with an event after every kernel",
