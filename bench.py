@@ -62,9 +62,9 @@ KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 # profiles/expert_step_kernels_ncu_full.md.  The figures hold only for the
 # kernel sources they were taken from: a changed source gives traffic null.
 NCU_TRAFFIC = {
-    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "2d8f1d1fed03afc6",
+    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "35558fb82fcc3c15",
              "bytes": {"fprop": 52.84e6, "dgrad": 24.32e6, "wgrad": 30.56e6}},
-    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "46d7edb1f1c1c306",
+    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "bff124f409a3937d",
               "bytes": {"quant_x_dual": 23.61e6, "quant_w_2d": 33.29e6, "quant_dy_dual_sr": 49.18e6},
               # thread instructions per element (ncu smsp__inst_executed x 32 / elements)
               "inst_per_elem": {"quant_dy_dual_sr": 80.0}},

@@ -187,13 +187,8 @@ __device__ __forceinline__ uint32_t e2m1x8_rn(const float *v) {
     return r;
 }
 
-// Shifts with the PTX rule for large amounts: a count of 32 or more (a
+// Right shift with the PTX rule for large amounts: a count of 32 or more (a
 // negative int passed as unsigned included) gives 0.
-__device__ __forceinline__ uint32_t shl_sat(uint32_t a, uint32_t n) {
-    uint32_t d;
-    asm("shl.b32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(n));
-    return d;
-}
 __device__ __forceinline__ uint32_t shr_sat(uint32_t a, uint32_t n) {
     uint32_t d;
     asm("shr.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(n));
@@ -207,39 +202,6 @@ __device__ __forceinline__ float e2m1_value(uint32_t c) {
     uint32_t b = m >= 2u ? (252u + m) << 22 : (m ? 0x3F000000u : 0u);
     b |= (c & 8u) << 28;
     return __uint_as_float(b);
-}
-
-// Stochastic rounding of one scaled value with random word r: lo <= |v| < hi
-// neighbouring grid values, up iff r < ceil(f * 2^32) with
-// f = (|v| - lo) / (hi - lo).  With m the 24-bit significand and e the biased
-// exponent of |v|, f * 2^32 = m << min(e - 117, 10) (mod 2^32) for every
-// |v| >= 2^-10: on [1, 6] the grid keeps one mantissa bit and the lower 22 are
-// f * 2^22; on [0.5, 1) f is the 23-bit mantissa; below 0.5 the grid step is
-// 0.5, so f * 2^32 = |v| * 2^33.  Below 2^-10 that product has a fractional
-// part and is rounded up (a rare branch; zero takes the main path, where the
-// shift count is negative and the threshold 0).
-// Stochastic rounding of one scaled value with random word r: lo <= |v| < hi
-// neighbouring grid values, up iff r < ceil(f * 2^32) with
-// f = (|v| - lo) / (hi - lo).  Returns the magnitude code.  With m the 24-bit
-// significand and e the biased exponent of |v|, f * 2^32 = m << min(e - 117, 10)
-// (mod 2^32) for every |v| >= 2^-10: on [1, 6] the grid keeps one mantissa bit
-// and the lower 22 are f * 2^22; on [0.5, 1) f is the 23-bit mantissa; below
-// 0.5 the grid step is 0.5, so f * 2^32 = |v| * 2^33.  Below 2^-10 that product
-// has a fractional part and is rounded up (a rare branch; zero takes the main
-// path, where the shift count is negative and the threshold 0).
-__device__ __forceinline__ uint32_t e2m1_sr_mag(float v, uint32_t r) {
-    const uint32_t ab = __float_as_uint(fminf(fabsf(v), 6.0f));
-    const int e = (int)(ab >> 23);
-    const uint32_t m = (ab & 0x007FFFFFu) | 0x00800000u;
-    uint32_t t = shl_sat(m, (uint32_t)min(e - 117, 10));
-    // grid index below |v|: 0 under 0.5, 1 on [0.5, 1), (bits >> 22) - 252 above
-    const int lo = max((int)(ab >> 22) - 252, ab >= 0x3F000000u ? 1 : 0);
-    uint32_t code = (uint32_t)lo + (r < t ? 1u : 0u);
-    if (ab - 1u < 0x3A7FFFFFu) {            // 0 < |v| < 2^-10: t = ceil(m * 2^(e - 117)) < 2^23
-        t = shr_sat(m - 1u, (uint32_t)(117 - e)) + 1u;
-        code = r < t ? 1u : 0u;
-    }
-    return code;
 }
 
 // Sign bits of 8 values as the sign bits (bit 3) of 8 packed E2M1 nibbles:
