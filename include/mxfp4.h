@@ -91,7 +91,8 @@ extern "C" {
 /* Human-readable name of a status code (static string, never NULL). */
 MXFP4_API const char *mxfp4_status_string(int status);
 
-/* ABI version (major * 100 + minor). */
+/* ABI version (major * 100 + minor).  1.01 added mxfp4_gemm_bf16 and
+ * mxfp4_grouped_gemm_bf16. */
 MXFP4_API int mxfp4_version(void);
 
 /*

@@ -68,7 +68,7 @@ const char *mxfp4_status_string(int status) {
     }
 }
 
-int mxfp4_version(void) { return 100; }
+int mxfp4_version(void) { return 101; }
 
 int64_t mxfp4_mma_scales_bytes(int64_t rows, int64_t k) {
     if (rows <= 0 || k <= 0) return 0;

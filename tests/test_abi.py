@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_layout_helpers():
     assert mx.status_string(mx.MXFP4_OK) == "MXFP4_OK"
     assert mx.status_string(mx.MXFP4_ERR_TIMEOUT) == "MXFP4_ERR_TIMEOUT"
-    assert mx.lib().mxfp4_version() == 100
+    assert mx.lib().mxfp4_version() == 101
     # 128 rows x 4 K-blocks per 512-byte atom
     assert mx.mma_scales_bytes(128, 128) == 512
     assert mx.mma_scales_bytes(129, 2880) == 2 * 23 * 512
