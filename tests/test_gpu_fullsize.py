@@ -79,6 +79,30 @@ def test_expert_gemms_sampled(expert_step):
     _check_sampled(host(st.dw), cdyt, sdyt, cxt, sxt, T, _sample_pairs(I, H, 2000, 3))
 
 
+def test_expert_gemms_bf16_output(expert_step):
+    """The three expert GEMMs with the bf16 epilogue, from the step's quantized
+    operands: every entry is the round-to-nearest-even of the FP32 product,
+    and sampled entries fall within the bf16 bound of the fp64 oracle."""
+    x, w, dy, st = expert_step
+    T, H, I = synth.TOKENS, synth.HIDDEN, synth.INTERMEDIATE
+    cases = [(st.qx, st.qw.codes, st.qw.scales, H, st.y), (st.qdy, st.qw.codes_t, st.qw.scales_t, I, st.dx),
+             (st.qdyt, st.qxt.codes, st.qxt.scales, T, st.dw)]
+    for qa, b_codes, b_scales, K, c32 in cases:
+        c16 = mx.mxfp4_gemm_bf16(qa.codes, qa.scales, b_codes, b_scales, K)
+        torch.cuda.synchronize()
+        assert torch.equal(c16.view(torch.int16), c32.to(torch.bfloat16).view(torch.int16))
+    cx, sx = oracle.quantize(x, oracle.LAYOUT_1D_ROW)
+    cw, sw = oracle.quantize(w, oracle.LAYOUT_2D)[:2]
+    pairs = _sample_pairs(T, I, 2000, 4)
+    ref, s = oracle.gemm_entries(cx, sx, cw, sw, H, pairs, 0, 1)
+    c16 = host(mx.mxfp4_gemm_bf16(st.qx.codes, st.qx.scales, st.qw.codes, st.qw.scales, H).float())
+    got = np.array([c16[m, n] for m, n in pairs], np.float64)
+    err = np.abs(got - ref)
+    bound = 1e-5 * s + 2.0 ** -8 * (np.abs(ref) + 1e-5 * s)   # FP32 bound + one bf16 rounding
+    assert np.all(err <= bound)
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+
+
 @pytest.fixture(scope="module")
 def moe():
     return synth.grouped_inputs()
