@@ -433,8 +433,9 @@ def sweep_bench(mx, torch, device, peaks, nbytes=1 << 30, reps=5):
 
 def bf16_out_bench(mx, torch, device, peaks, reps=20):
     """The expert fprop GEMM (4096 x 5760 x 2880, activations N(0,1), weights
-    N(0, 0.02^2) drawn on the device) with its FP32 and its bf16 output; L2
-    flushed before each launch."""
+    N(0, 0.02^2) drawn on the device) with its FP32 output and with the fused
+    epilogues (bf16 output; MXFP4 output, 1D row blocks RNE); L2 flushed
+    before each launch."""
     g = torch.Generator(device=device)
     g.manual_seed(2)
     a = torch.randn((TOKENS, HIDDEN), generator=g, device=device).to(torch.bfloat16)
@@ -443,11 +444,14 @@ def bf16_out_bench(mx, torch, device, peaks, reps=20):
     qw = mx.mxfp4_quantize(w, mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA)
     c32 = torch.empty((TOKENS, INTER), dtype=torch.float32, device=device)
     c16 = torch.empty((TOKENS, INTER), dtype=torch.bfloat16, device=device)
+    cq = mx.mxfp4_gemm_mxfp4(qa.codes, qa.scales, qw.codes, qw.scales, HIDDEN, scale_layout=mx.SCALES_MMA)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
     res = {}
     for name, fn in (("fp32_out", lambda: mx.mxfp4_gemm(qa.codes, qa.scales, qw.codes, qw.scales, HIDDEN, out=c32)),
                      ("bf16_out", lambda: mx.mxfp4_gemm_bf16(qa.codes, qa.scales, qw.codes, qw.scales, HIDDEN,
-                                                             out=c16))):
+                                                             out=c16)),
+                     ("mxfp4_out", lambda: mx.mxfp4_gemm_mxfp4(qa.codes, qa.scales, qw.codes, qw.scales, HIDDEN,
+                                                               scale_layout=mx.SCALES_MMA, out=cq))):
         fn()
         torch.cuda.synchronize()
         ts = []
@@ -464,7 +468,7 @@ def bf16_out_bench(mx, torch, device, peaks, reps=20):
         res[name] = {"us": ms * 1e3, "TFLOP/s": tf, "frac_fp4_peak": tf / (4 * peaks["bf16"])}
     if mx.mxfp4_get_error() != mx.MXFP4_OK:
         raise RuntimeError("device-side error in the bf16-output measurements")
-    del qa, qw, c32, c16, a, w, flush
+    del qa, qw, c32, c16, cq, a, w, flush
     torch.cuda.empty_cache()
     res["shape"] = f"{TOKENS} x {INTER} x {HIDDEN}"
     return res

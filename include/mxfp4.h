@@ -92,7 +92,7 @@ extern "C" {
 MXFP4_API const char *mxfp4_status_string(int status);
 
 /* ABI version (major * 100 + minor).  1.01 added mxfp4_gemm_bf16 and
- * mxfp4_grouped_gemm_bf16. */
+ * mxfp4_grouped_gemm_bf16; 1.02 mxfp4_gemm_mxfp4. */
 MXFP4_API int mxfp4_version(void);
 
 /*
@@ -263,6 +263,30 @@ MXFP4_API int mxfp4_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const
                                       const int32_t *group_offsets, const int32_t *group_sizes, int num_groups,
                                       const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
                                       int64_t N, int64_t K, uint16_t *c, int64_t ldc, void *stream);
+
+/*
+ * mxfp4_gemm_mxfp4 -- the product of mxfp4_gemm requantized to MXFP4 in the
+ * epilogue, for a next layer that takes C as a quantized operand: each run of
+ * 32 FP32 results along a row of C (a 1D row block) gets the reference scale
+ * rule and round-to-nearest-even E2M1 codes exactly as mxfp4_quantize would
+ * give them for those FP32 values ("Conversion rules": amax, scale
+ * X = 2^floor(log2 amax) / 4, saturating RNE; NaN or Inf in a block -> scale
+ * 0xFF and zero codes).  The FP32 results themselves are never stored: C
+ * costs 0.53 bytes per element of HBM writes instead of 4.
+ *
+ * c_codes [M, N/2] (row stride ld_c_codes bytes), c_scales row-major
+ * [M, N/32] (ld_c_scales) or the GEMM-ready layout for (M x N)
+ * (c_scale_layout MXFP4_SCALES_MMA, mxfp4_mma_scales_bytes(M, N) bytes), both
+ * fully overwritten.  Operands and requirements as for mxfp4_gemm, plus
+ * N % 32 == 0 and ld_c_codes % 16 == 0.  Because the FP32 accumulation order
+ * is the implementation's, a block whose amax, or an element whose scaled
+ * value, lies within the GEMM tolerance of a scale or rounding boundary may
+ * take either neighbouring code.
+ */
+MXFP4_API int mxfp4_gemm_mxfp4(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales,
+                               const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
+                               int64_t M, int64_t N, int64_t K, uint8_t *c_codes, int64_t ld_c_codes,
+                               uint8_t *c_scales, int64_t ld_c_scales, int c_scale_layout, void *stream);
 
 /*
  * mxfp4_grouped_gemm_wgrad -- per group (expert) g:

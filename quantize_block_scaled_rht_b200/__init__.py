@@ -41,7 +41,7 @@ OUT_BF16, OUT_F32 = 0, 1
 ABI_FUNCTIONS = (
     "mxfp4_status_string", "mxfp4_version", "mxfp4_mma_scales_bytes", "mxfp4_mma_scale_offset",
     "mxfp4_quantize", "mxfp4_quantize_dual", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_grouped_gemm",
-    "mxfp4_gemm_bf16", "mxfp4_grouped_gemm_bf16", "mxfp4_grouped_gemm_wgrad", "mxfp4_nvfp4_quantize", "mxfp4_nvfp4_dequantize", "mxfp4_nvfp4_gemm",
+    "mxfp4_gemm_bf16", "mxfp4_grouped_gemm_bf16", "mxfp4_gemm_mxfp4", "mxfp4_grouped_gemm_wgrad", "mxfp4_nvfp4_quantize", "mxfp4_nvfp4_dequantize", "mxfp4_nvfp4_gemm",
     "mxfp4_get_error",
     "mxfp4_set_wait_limit_ns", "mxfp4_wait_probe",
 )
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
         L.mxfp4_gemm_bf16.restype = i32
         L.mxfp4_grouped_gemm_bf16.argtypes = [vp, i64, vp, i64, vp, vp, i32, vp, i64, vp, i64, i64, vp, i64, vp]
         L.mxfp4_grouped_gemm_bf16.restype = i32
+        L.mxfp4_gemm_mxfp4.argtypes = [vp, i64, vp, vp, i64, vp, i64, i64, i64, vp, i64, vp, i64, i32, vp]
+        L.mxfp4_gemm_mxfp4.restype = i32
         L.mxfp4_grouped_gemm_wgrad.argtypes = [vp, i64, vp, vp, i64, vp, vp, i32, i64, i64, i64, vp, i64, vp]
         L.mxfp4_grouped_gemm_wgrad.restype = i32
         L.mxfp4_nvfp4_quantize.argtypes = [vp, i64, i64, i64, i32, i32, u64, u64, vp, vp, i64, vp, i64, i32, vp]
@@ -275,6 +277,24 @@ def mxfp4_gemm_bf16(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torc
     rc = lib().mxfp4_gemm_bf16(_ptr(a_codes), a_codes.stride(0), _ptr(a_scales), _ptr(b_codes), b_codes.stride(0),
                                _ptr(b_scales), M, N, K, _ptr(out), out.stride(0), _stream(stream))
     _check(rc, "mxfp4_gemm_bf16")
+    return out
+
+
+def mxfp4_gemm_mxfp4(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Tensor,
+                     K: int, scale_layout: int = SCALES_ROWMAJOR, out: Optional[Quantized] = None,
+                     stream=None) -> Quantized:
+    """mxfp4_gemm with C requantized to MXFP4 (1D row blocks, reference scale
+    rule, RNE) in the epilogue; returns C as a Quantized [M, N]."""
+    M, N = a_codes.shape[0], b_codes.shape[0]
+    dev = a_codes.device
+    if out is None:
+        out = Quantized(torch.empty((M, N // 2), dtype=torch.uint8, device=dev), _scale_tensor(M, N, scale_layout, dev),
+                        M, N, LAYOUT_1D_ROW, scale_layout)
+    ld_sc = out.scales.shape[1] if out.scales.dim() == 2 else 0
+    rc = lib().mxfp4_gemm_mxfp4(_ptr(a_codes), a_codes.stride(0), _ptr(a_scales), _ptr(b_codes), b_codes.stride(0),
+                                _ptr(b_scales), M, N, K, _ptr(out.codes), out.codes.stride(0), _ptr(out.scales), ld_sc,
+                                scale_layout, _stream(stream))
+    _check(rc, "mxfp4_gemm_mxfp4")
     return out
 
 

@@ -31,6 +31,9 @@ int launch_grouped_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_s
 int launch_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
                      int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
                      cudaStream_t s);
+int launch_gemm_mx(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                   int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint8_t *c_codes,
+                   int64_t ld_c_codes, uint8_t *c_scales, int64_t ld_c_scales, int c_scale_mma, cudaStream_t s);
 int launch_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
                              const int32_t *offsets, const int32_t *sizes, int G, const uint8_t *b_codes,
                              int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
@@ -68,7 +71,7 @@ const char *mxfp4_status_string(int status) {
     }
 }
 
-int mxfp4_version(void) { return 101; }
+int mxfp4_version(void) { return 102; }
 
 int64_t mxfp4_mma_scales_bytes(int64_t rows, int64_t k) {
     if (rows <= 0 || k <= 0) return 0;
@@ -229,6 +232,24 @@ int mxfp4_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales
     if (M > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
     return mxfp4::launch_gemm_bf16(a_codes, lda, a_scales, b_codes, ldb, b_scales, M, N, K, c, ldc,
                                    static_cast<cudaStream_t>(stream));
+}
+
+int mxfp4_gemm_mxfp4(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                     int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint8_t *c_codes,
+                     int64_t ld_c_codes, uint8_t *c_scales, int64_t ld_c_scales, int c_scale_layout, void *stream) {
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !c_codes || !c_scales) return MXFP4_ERR_INVALID_ARG;
+    if (M <= 0 || N <= 0 || K <= 0 || (N % 32) || (K % 32)) return MXFP4_ERR_INVALID_ARG;
+    if (c_scale_layout != MXFP4_SCALES_ROWMAJOR && c_scale_layout != MXFP4_SCALES_MMA) return MXFP4_ERR_INVALID_ARG;
+    if (K % 64) return MXFP4_ERR_UNSUPPORTED;
+    if (lda < K / 2 || ldb < K / 2 || ld_c_codes < N / 2) return MXFP4_ERR_INVALID_ARG;
+    if (c_scale_layout == MXFP4_SCALES_ROWMAJOR && ld_c_scales < N / 32) return MXFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(b_codes) || !aligned16(a_scales) || !aligned16(b_scales) ||
+        !aligned16(c_codes) || (lda % 16) || (ldb % 16) || (ld_c_codes % 16))
+        return MXFP4_ERR_ALIGNMENT;
+    if (M > (int64_t)1 << 31 || N > (int64_t)1 << 31 || K > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    return mxfp4::launch_gemm_mx(a_codes, lda, a_scales, b_codes, ldb, b_scales, M, N, K, c_codes, ld_c_codes,
+                                 c_scales, ld_c_scales, c_scale_layout == MXFP4_SCALES_MMA,
+                                 static_cast<cudaStream_t>(stream));
 }
 
 int mxfp4_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,

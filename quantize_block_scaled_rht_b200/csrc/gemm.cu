@@ -95,6 +95,10 @@ struct TileCfg {
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
+// Output of the epilogue: FP32, bf16 (nearest even), or MXFP4 (each 1D row
+// block of 32 FP32 results requantized: amax, E8M0 scale, E2M1 RNE codes).
+constexpr int OUT_F32 = 0, OUT_BF16 = 1, OUT_MX = 2;
+
 using DefaultCfg = TileCfg<192, 3, 2>;
 using NvCfg = TileCfg<192, 5, 1, true>;
 
@@ -106,8 +110,11 @@ struct GemmParams {
     int64_t M, N, K;
     int64_t katoms;            // ceil(K / 128): scale atoms per 128-row tile
     int64_t b_rowtiles;        // ceil(N / 128): 128-row scale tiles of one B operand
-    void *c;                   // FP32 or, with the bf16 epilogue, bf16 [.., ldc]
+    void *c;                   // FP32, bf16 [.., ldc elements] or MXFP4 codes [.., ldc bytes]
     int64_t ldc;
+    uint8_t *c_scales;         // MXFP4 output: scales, row-major [.., ld_c_scales] or GEMM-ready
+    int64_t ld_c_scales, c_katoms;
+    int c_scale_mma;
     const int32_t *group_offsets;
     const int32_t *group_sizes;
     const float *a_amax, *b_amax;   // NVFP4 tensor amaxes (second-level scales amax / 2688)
@@ -283,7 +290,7 @@ __device__ __noinline__ void issue_stage_tail(uint32_t d_tmem, uint32_t st, uint
     }
 }
 
-template <class Cfg, int MODE, bool OBF16>
+template <class Cfg, int MODE, int OUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     mxfp4_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
                       const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ CUtensorMap tma_sfa,
@@ -486,7 +493,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             const bool full_box = MODE == MODE_DENSE || (row_lo + 32 <= ti.rows_valid);
             const bool any_row = row_lo < ti.rows_valid;
             const bool empty_k = ti.kg <= 0;              // grouped K: an empty group's output is zero
-            if constexpr (OBF16) {
+            if constexpr (OUT == OUT_MX) {
+                // fused requantization: after each 32-column TMEM load a lane
+                // holds 32 consecutive results of one row, i.e. one 1D row
+                // block of C: amax, E8M0 scale and RNE E2M1 codes as in
+                // mxfp4_quantize, stored straight from registers
+                static_assert(MODE == MODE_DENSE, "MXFP4 output: dense GEMM only");
+                const uint32_t tm = tmem + ((uint32_t)(32 * q) << 16) + (acc ? Cfg::ACC1_COL : 0u);
+                const int64_t row = ti.c_row0 + row_lo + lane;
+                const bool row_ok = row < p.M;
+                for (int j = 0; j < BN / 32; ++j) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tm + 32u * j, v);
+                    tmem_ld_wait();
+                    if (j == BN / 32 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(acc ? empty_leader1 : empty_leader0);
+                    }
+                    const int64_t col0 = ti.n0 + 32 * j;
+                    if (!row_ok || col0 >= p.N) continue;
+                    float f[32];
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        f[i] = __uint_as_float(v[i]);
+                        if constexpr (Cfg::NV) f[i] = __fmul_rn(f[i], nv_scale);
+                        amax = amax_nan(amax, f[i]);
+                    }
+                    const uint32_t code = scale_code_from_amax(amax);
+                    uint4 qv = make_uint4(0, 0, 0, 0);
+                    if (code != 0xFFu) {
+                        const float inv = inv_scale_from_code(code);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) f[i] = __fmul_rn(f[i], inv);
+                        qv = make_uint4(e2m1x8_rn(f), e2m1x8_rn(f + 8), e2m1x8_rn(f + 16), e2m1x8_rn(f + 24));
+                    }
+                    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(static_cast<uint8_t *>(p.c) +
+                                                                                 row * p.ldc + (col0 >> 1)),
+                                 "r"(qv.x), "r"(qv.y), "r"(qv.z), "r"(qv.w)
+                                 : "memory");
+                    const int64_t kb = col0 >> 5;
+                    if (p.c_scale_mma) p.c_scales[mma_scale_off(row, kb, p.c_katoms)] = (uint8_t)code;
+                    else p.c_scales[row * p.ld_c_scales + kb] = (uint8_t)code;
+                }
+            } else if constexpr (OUT == OUT_BF16) {
                 // 64 columns per step: two 32-column TMEM loads rounded to
                 // bf16 pairs (RNE), one 128-byte row segment per lane
                 const uint32_t tm = tmem + ((uint32_t)(32 * q) << 16) + (acc ? Cfg::ACC1_COL : 0u);
@@ -699,14 +750,14 @@ static int sm_count() {
     return n > 0 ? n : 148;
 }
 
-template <class Cfg, int MODE, bool OBF16>
+template <class Cfg, int MODE, int OUT>
 static cudaError_t set_smem_attr() {
     // once per device and instantiation: keep cudaFuncSetAttribute off the hot path
     static int done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<Cfg, MODE, OBF16>,
+    cudaError_t e = cudaFuncSetAttribute(mxfp4_gemm_kernel<Cfg, MODE, OUT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
     if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = 1;
     return e;
@@ -719,13 +770,18 @@ struct GemmArgs {
     const int32_t *offsets, *sizes;
     int G;
     const float *a_amax = nullptr, *b_amax = nullptr;
+    uint8_t *c_scales = nullptr;
+    int64_t ld_c_scales = 0;
+    int c_scale_mma = 0;
 };
 
 // Returns 0 on success, MXFP4_ERR_CUDA when a map or launch fails.
 // Grouped K: a and b are [M, K/2] and [N, K/2] over all groups' K ranges, c is
 // [G * M, N]; the B operand and C map cover G groups only in grouped-rows mode.
-// OBF16: C is bf16 (RNE of the FP32 accumulators), stored in 64-column boxes.
-template <class Cfg, int MODE, bool OBF16 = false>
+// OUT_BF16: C is bf16 (RNE of the FP32 accumulators), stored in 64-column
+// boxes; OUT_MX: C is MXFP4 codes + scales written without the C tensor map
+// (a map over the codes is still passed, never used).
+template <class Cfg, int MODE, int OUT = OUT_F32>
 static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
     constexpr int BN = Cfg::BN;
     const int G = MODE == MODE_GROUPED_M ? g.G : 1;
@@ -737,20 +793,25 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
                   (uint64_t)g.lda, CHUNK, BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.b_codes, (uint64_t)(g.K / 2), (uint64_t)G * g.N,
                   (uint64_t)g.ldb, CHUNK, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tc, OBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.c,
-                  (uint64_t)g.N, (uint64_t)c_rows, (uint64_t)g.ldc * (OBF16 ? 2 : 4), OBF16 ? 64 : 32, 32,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !(OUT == OUT_MX
+              ? make_map(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, g.c, (uint64_t)(g.N / 2), (uint64_t)c_rows,
+                         (uint64_t)g.ldc, 16, 32, CU_TENSOR_MAP_SWIZZLE_NONE)
+              : make_map(&tc, OUT == OUT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                         g.c, (uint64_t)g.N, (uint64_t)c_rows, (uint64_t)g.ldc * (OUT == OUT_BF16 ? 2 : 4),
+                         OUT == OUT_BF16 ? 64 : 32, 32, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         // scale atoms as a 3D tensor [128-row tile][K atom][512 bytes = 128 x 32-bit]:
         // one box holds NATOM consecutive atoms of one (A) or NRT (B) row tiles
         !make_map_3d(&tsa, g.a_scales, (uint64_t)katoms, (uint64_t)a_tiles, Cfg::NATOM, 1) ||
         !make_map_3d(&tsb, g.b_scales, (uint64_t)katoms, (uint64_t)(G * b_tiles), Cfg::NATOM, Cfg::NRT))
         return MXFP4_ERR_CUDA;
-    if (set_smem_attr<Cfg, MODE, OBF16>() != cudaSuccess) return MXFP4_ERR_CUDA;
+    if (set_smem_attr<Cfg, MODE, OUT>() != cudaSuccess) return MXFP4_ERR_CUDA;
     GemmParams p{};
     p.M = g.M; p.N = g.N; p.K = g.K;
     p.katoms = katoms;
     p.b_rowtiles = b_tiles;
     p.c = g.c; p.ldc = g.ldc;
+    p.c_scales = g.c_scales; p.ld_c_scales = g.ld_c_scales; p.c_scale_mma = g.c_scale_mma;
+    p.c_katoms = (g.N / 32 + 3) / 4;
     p.group_offsets = g.offsets; p.group_sizes = g.sizes; p.num_groups = g.G;
     p.a_amax = g.a_amax; p.b_amax = g.b_amax;
     p.wait_limit_ns = g_wait_limit_ns;
@@ -760,7 +821,7 @@ static int launch_cfg(const GemmArgs &g, cudaStream_t s) {
         const int64_t tiles = (MODE == MODE_GROUPED_K ? g.G : 1) * ((g.M + 255) / 256) * ((g.N + BN - 1) / BN);
         pairs = (int)(tiles < pairs_max ? tiles : pairs_max);
     }
-    const cudaError_t e = launch_pdl(mxfp4_gemm_kernel<Cfg, MODE, OBF16>, dim3((unsigned)(2 * pairs)), dim3(NUM_THREADS),
+    const cudaError_t e = launch_pdl(mxfp4_gemm_kernel<Cfg, MODE, OUT>, dim3((unsigned)(2 * pairs)), dim3(NUM_THREADS),
                                      (size_t)Cfg::SMEM_BYTES, s, ta, tb, tc, tsa, tsb, p);
     return e == cudaSuccess ? 0 : MXFP4_ERR_CUDA;
 }
@@ -782,7 +843,7 @@ int launch_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scale
                      int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
                      cudaStream_t s) {
     GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, M, N, K, ldc, c, nullptr, nullptr, 1};
-    return launch_cfg<DefaultCfg, MODE_DENSE, true>(g, s);
+    return launch_cfg<DefaultCfg, MODE_DENSE, OUT_BF16>(g, s);
 }
 
 int launch_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
@@ -790,7 +851,17 @@ int launch_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t 
                              int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
                              cudaStream_t s) {
     GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, a_rows, N, K, ldc, c, offsets, sizes, G};
-    return launch_cfg<DefaultCfg, MODE_GROUPED_M, true>(g, s);
+    return launch_cfg<DefaultCfg, MODE_GROUPED_M, OUT_BF16>(g, s);
+}
+
+int launch_gemm_mx(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                   int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint8_t *c_codes,
+                   int64_t ld_c_codes, uint8_t *c_scales, int64_t ld_c_scales, int c_scale_mma, cudaStream_t s) {
+    GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, M, N, K, ld_c_codes, c_codes, nullptr, nullptr, 1};
+    g.c_scales = c_scales;
+    g.ld_c_scales = ld_c_scales;
+    g.c_scale_mma = c_scale_mma;
+    return launch_cfg<DefaultCfg, MODE_DENSE, OUT_MX>(g, s);
 }
 
 int launch_grouped_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,

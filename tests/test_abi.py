@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_layout_helpers():
     assert mx.status_string(mx.MXFP4_OK) == "MXFP4_OK"
     assert mx.status_string(mx.MXFP4_ERR_TIMEOUT) == "MXFP4_ERR_TIMEOUT"
-    assert mx.lib().mxfp4_version() == 101
+    assert mx.lib().mxfp4_version() == 102
     # 128 rows x 4 K-blocks per 512-byte atom
     assert mx.mma_scales_bytes(128, 128) == 512
     assert mx.mma_scales_bytes(129, 2880) == 2 * 23 * 512
@@ -70,6 +70,11 @@ def test_invalid_arguments_rejected_without_gpu():
                                      None) == 3
     assert L.mxfp4_grouped_gemm_bf16(fake, 32, fake, 128, fake, fake, 2, fake, 32, fake, 132, 64, fake, 132,
                                      None) == 2
+    # MXFP4-output GEMM: N a multiple of 32, 16-byte code rows, a known scale layout
+    assert L.mxfp4_gemm_mxfp4(fake, 32, fake, fake, 32, fake, 128, 200, 64, fake, 112, fake, 8, 0, None) == 1
+    assert L.mxfp4_gemm_mxfp4(fake, 32, fake, fake, 32, fake, 128, 192, 64, fake, 104, fake, 6, 0, None) == 2
+    assert L.mxfp4_gemm_mxfp4(fake, 32, fake, fake, 32, fake, 128, 192, 64, fake, 96, fake, 6, 7, None) == 1
+    assert L.mxfp4_gemm_mxfp4(fake, 16, fake, fake, 16, fake, 128, 192, 96, fake, 96, fake, 6, 0, None) == 3
     # grouped wgrad: K not a multiple of 128, too many groups
     assert L.mxfp4_grouped_gemm_wgrad(fake, 32, fake, fake, 32, fake, fake, 2, 128, 128, 64, fake, 128, None) == 1
     assert L.mxfp4_grouped_gemm_wgrad(fake, 64, fake, fake, 64, fake, fake, 5000, 128, 128, 128, fake, 128,

@@ -13,7 +13,7 @@ import torch
 import oracle
 import quantize_block_scaled_rht_b200 as mx
 import synth
-from mxfp4_testutil import assert_gemm_close, dev_bf16, dev_u8, expand_2d, host, to_mma
+from mxfp4_testutil import assert_gemm_close, dev_bf16, dev_u8, expand_2d, from_mma, host, to_mma
 
 pytestmark = pytest.mark.gpu
 
@@ -361,3 +361,88 @@ def test_grouped_gemm_bf16(sizes, N, K):
             ref, s = oracle.gemm(ca[o:o + n], sa[o:o + n], cw, sw, K, 0, 1)
             _assert_bf16_close(c[o:o + n], ref, s)
         assert np.all(c[o + n:int(offsets[g + 1])] == 1280.0)
+
+
+# --- MXFP4-output epilogue ------------------------------------------------------
+_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _scale_code(amax: np.ndarray) -> np.ndarray:
+    """E8M0 code of the reference rule for finite amax >= 0 (0 -> 0):
+    floor(log2 amax) - 2 + 127, the exponent taken exactly by frexp."""
+    _, e = np.frexp(np.where(amax > 0, amax, 1.0))
+    return np.where(amax > 0, np.clip(e.astype(np.int64) - 1 - 2 + 127, 0, 254), 0).astype(np.int64)
+
+
+def _rne_value(y: np.ndarray) -> np.ndarray:
+    """Signed E2M1 value nearest to y (ties to the even code), saturating at 6."""
+    a = np.minimum(np.abs(y), 6.0)
+    d = np.abs(a[..., None] - _GRID) + (np.arange(8) % 2) * 1e-9
+    return np.sign(y) * _GRID[np.argmin(d, axis=-1)]
+
+
+def _decode(codes: np.ndarray) -> np.ndarray:
+    nib = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(codes.shape[0], -1)
+    return np.where(nib & 8, -1.0, 1.0) * _GRID[nib & 7]
+
+
+def _requantize_f32(c32: np.ndarray):
+    """Test-side 1D-row requantization of FP32 values (reference scale rule,
+    RNE): the scaled values are formed in fp32 as the kernels form them."""
+    M, N = c32.shape
+    blk = c32.reshape(M, N // 32, 32)
+    amax = np.abs(blk).max(axis=-1).astype(np.float64)
+    sc = _scale_code(amax)
+    inv = np.ldexp(np.float32(1.0), (127 - sc).astype(np.int32)).astype(np.float32)
+    y = (blk * inv[..., None]).astype(np.float32)
+    return _rne_value(y.astype(np.float64)).reshape(M, N), sc
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 192, 512), (300, 224, 320), (130, 384, 2880)])
+@pytest.mark.parametrize("mma", [False, True])
+def test_gemm_mxfp4_output(M, N, K, mma):
+    """MXFP4-output epilogue: (1) bit-equal to the 1D-row RNE requantization
+    of the FP32 kernel's own product; (2) every scale and element code is one
+    that an FP32 product within 1e-5 * sum|ab| of the exact one can give."""
+    a = synth.normal_bf16((M, K), 50 + M)
+    b = synth.normal_bf16((N, K), 60 + N, 0.02)
+    ca, sa = _oracle_operand(a)
+    cb, sb = _oracle_operand(b)
+    args = (dev_u8(ca), dev_u8(to_mma(sa, K)), dev_u8(cb), dev_u8(to_mma(sb, K)), K)
+    sl = mx.SCALES_MMA if mma else mx.SCALES_ROWMAJOR
+    q = mx.mxfp4_gemm_mxfp4(*args, scale_layout=sl)
+    c32 = mx.mxfp4_gemm(*args)
+    torch.cuda.synchronize()
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    sc = host(q.scales)
+    sc = from_mma(sc, M, N) if mma else sc
+    got = _decode(host(q.codes)) * np.repeat(np.ldexp(1.0, sc.astype(np.int64) - 127), 32, axis=1)
+    # (1) the same accumulators, requantized on the host
+    want_v, want_sc = _requantize_f32(host(c32))
+    assert np.array_equal(sc, want_sc)
+    assert np.array_equal(_decode(host(q.codes)), want_v)
+    # (2) against the exact product, within the GEMM tolerance
+    ref, s = oracle.gemm(ca, sa, cb, sb, K)
+    tol = 1e-5 * s
+    blk = lambda x: x.reshape(M, N // 32, 32)
+    amax_lo = np.maximum(np.abs(blk(ref)) - blk(tol), 0).max(axis=-1)
+    amax_hi = (np.abs(blk(ref)) + blk(tol)).max(axis=-1)
+    assert np.all((_scale_code(amax_lo) <= sc) & (sc <= _scale_code(amax_hi)))
+    X = np.repeat(np.ldexp(1.0, sc.astype(np.int64) - 127), 32, axis=1)
+    lo, hi = _rne_value((ref - tol) / X) * X, _rne_value((ref + tol) / X) * X
+    assert np.all((lo <= got) & (got <= hi))
+    assert np.mean(lo == hi) > 0.99          # almost every code is fixed by the exact product
+
+
+def test_gemm_mxfp4_output_nan_rows():
+    M, N, K = 128, 192, 256
+    a = synth.normal_bf16((M, K), 3)
+    b = synth.normal_bf16((N, K), 4, 0.02)
+    ca, sa = _oracle_operand(a)
+    cb, sb = _oracle_operand(b)
+    sa = sa.copy(); sa[9, 2] = 0xFF
+    q = mx.mxfp4_gemm_mxfp4(dev_u8(ca), dev_u8(to_mma(sa, K)), dev_u8(cb), dev_u8(to_mma(sb, K)), K)
+    torch.cuda.synchronize()
+    sc, codes = host(q.scales), host(q.codes)
+    assert np.all(sc[9] == 0xFF) and np.all(codes[9] == 0)
+    assert np.all(np.delete(sc, 9, axis=0) != 0xFF)
