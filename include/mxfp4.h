@@ -92,7 +92,8 @@ extern "C" {
 MXFP4_API const char *mxfp4_status_string(int status);
 
 /* ABI version (major * 100 + minor).  1.01 added mxfp4_gemm_bf16 and
- * mxfp4_grouped_gemm_bf16; 1.02 mxfp4_gemm_mxfp4. */
+ * mxfp4_grouped_gemm_bf16; 1.02 mxfp4_gemm_mxfp4; 1.03
+ * mxfp4_grouped_gemm_wgrad_bf16. */
 MXFP4_API int mxfp4_version(void);
 
 /*
@@ -316,6 +317,18 @@ MXFP4_API int mxfp4_grouped_gemm_wgrad(const uint8_t *a_codes, int64_t lda, cons
                                        const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
                                        const int32_t *group_offsets, int num_groups, int64_t M, int64_t N,
                                        int64_t K, float *c, int64_t ldc, void *stream);
+
+/*
+ * mxfp4_grouped_gemm_wgrad_bf16 -- mxfp4_grouped_gemm_wgrad with a bf16
+ * output: each FP32 accumulator rounded to the nearest bf16 (ties to even) in
+ * the epilogue (an empty group's output is zero).  c holds bf16 bit patterns
+ * [num_groups * M, N]; requirements as for mxfp4_grouped_gemm_wgrad except
+ * ldc % 8 == 0.
+ */
+MXFP4_API int mxfp4_grouped_gemm_wgrad_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales,
+                                            const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
+                                            const int32_t *group_offsets, int num_groups, int64_t M, int64_t N,
+                                            int64_t K, uint16_t *c, int64_t ldc, void *stream);
 
 /*
  * NVFP4 ("MXFP4" (aiwiki.ai), "Comparison with NVFP4"): E2M1 elements in

@@ -41,7 +41,8 @@ OUT_BF16, OUT_F32 = 0, 1
 ABI_FUNCTIONS = (
     "mxfp4_status_string", "mxfp4_version", "mxfp4_mma_scales_bytes", "mxfp4_mma_scale_offset",
     "mxfp4_quantize", "mxfp4_quantize_dual", "mxfp4_dequantize", "mxfp4_gemm", "mxfp4_grouped_gemm",
-    "mxfp4_gemm_bf16", "mxfp4_grouped_gemm_bf16", "mxfp4_gemm_mxfp4", "mxfp4_grouped_gemm_wgrad", "mxfp4_nvfp4_quantize", "mxfp4_nvfp4_dequantize", "mxfp4_nvfp4_gemm",
+    "mxfp4_gemm_bf16", "mxfp4_grouped_gemm_bf16", "mxfp4_gemm_mxfp4", "mxfp4_grouped_gemm_wgrad",
+    "mxfp4_grouped_gemm_wgrad_bf16", "mxfp4_nvfp4_quantize", "mxfp4_nvfp4_dequantize", "mxfp4_nvfp4_gemm",
     "mxfp4_get_error",
     "mxfp4_set_wait_limit_ns", "mxfp4_wait_probe",
 )
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.mxfp4_gemm_mxfp4.restype = i32
         L.mxfp4_grouped_gemm_wgrad.argtypes = [vp, i64, vp, vp, i64, vp, vp, i32, i64, i64, i64, vp, i64, vp]
         L.mxfp4_grouped_gemm_wgrad.restype = i32
+        L.mxfp4_grouped_gemm_wgrad_bf16.argtypes = [vp, i64, vp, vp, i64, vp, vp, i32, i64, i64, i64, vp, i64, vp]
+        L.mxfp4_grouped_gemm_wgrad_bf16.restype = i32
         L.mxfp4_nvfp4_quantize.argtypes = [vp, i64, i64, i64, i32, i32, u64, u64, vp, vp, i64, vp, i64, i32, vp]
         L.mxfp4_nvfp4_quantize.restype = i32
         L.mxfp4_nvfp4_dequantize.argtypes = [vp, i64, vp, i64, i32, vp, i64, i64, i32, vp, i64, vp]
@@ -329,6 +332,23 @@ def mxfp4_grouped_gemm_wgrad(a_codes: torch.Tensor, a_scales: torch.Tensor, b_co
                                         b_codes.stride(0), _ptr(b_scales), _ptr(group_offsets), G, M, N, K,
                                         _ptr(out), out.stride(0), _stream(stream))
     _check(rc, "mxfp4_grouped_gemm_wgrad")
+    return out
+
+
+def mxfp4_grouped_gemm_wgrad_bf16(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor,
+                                  b_scales: torch.Tensor, group_offsets: torch.Tensor, K: int,
+                                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """mxfp4_grouped_gemm_wgrad with a bf16 output; returns [G * M, N] bf16."""
+    M, N = a_codes.shape[0], b_codes.shape[0]
+    G = group_offsets.numel() - 1
+    if out is None:
+        out = torch.empty((G * M, N), dtype=torch.bfloat16, device=a_codes.device)
+    if out.dtype != torch.bfloat16:
+        raise ValueError("out must be bfloat16")
+    rc = lib().mxfp4_grouped_gemm_wgrad_bf16(_ptr(a_codes), a_codes.stride(0), _ptr(a_scales), _ptr(b_codes),
+                                             b_codes.stride(0), _ptr(b_scales), _ptr(group_offsets), G, M, N, K,
+                                             _ptr(out), out.stride(0), _stream(stream))
+    _check(rc, "mxfp4_grouped_gemm_wgrad_bf16")
     return out
 
 

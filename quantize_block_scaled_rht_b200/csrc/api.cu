@@ -34,6 +34,9 @@ int launch_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scale
 int launch_gemm_mx(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
                    int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint8_t *c_codes,
                    int64_t ld_c_codes, uint8_t *c_scales, int64_t ld_c_scales, int c_scale_mma, cudaStream_t s);
+int launch_grouped_wgrad_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                              int64_t ldb, const uint8_t *b_scales, const int32_t *offsets, int G, int64_t M,
+                              int64_t N, int64_t K, uint16_t *c, int64_t ldc, cudaStream_t s);
 int launch_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, int64_t a_rows,
                              const int32_t *offsets, const int32_t *sizes, int G, const uint8_t *b_codes,
                              int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
@@ -71,7 +74,7 @@ const char *mxfp4_status_string(int status) {
     }
 }
 
-int mxfp4_version(void) { return 102; }
+int mxfp4_version(void) { return 103; }
 
 int64_t mxfp4_mma_scales_bytes(int64_t rows, int64_t k) {
     if (rows <= 0 || k <= 0) return 0;
@@ -277,6 +280,20 @@ int mxfp4_grouped_gemm_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t 
     if (M > (int64_t)1 << 31 || (int64_t)num_groups * M > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
     return mxfp4::launch_grouped_wgrad(a_codes, lda, a_scales, b_codes, ldb, b_scales, group_offsets, num_groups, M,
                                        N, K, c, ldc, static_cast<cudaStream_t>(stream));
+}
+
+int mxfp4_grouped_gemm_wgrad_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales,
+                                  const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
+                                  const int32_t *group_offsets, int num_groups, int64_t M, int64_t N, int64_t K,
+                                  uint16_t *c, int64_t ldc, void *stream) {
+    if (!group_offsets || num_groups <= 0 || M <= 0) return MXFP4_ERR_INVALID_ARG;
+    if (num_groups > 1024) return MXFP4_ERR_UNSUPPORTED;
+    const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc, 2);
+    if (rc != MXFP4_OK) return rc;
+    if (K % 128) return MXFP4_ERR_INVALID_ARG;
+    if (M > (int64_t)1 << 31 || (int64_t)num_groups * M > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
+    return mxfp4::launch_grouped_wgrad_bf16(a_codes, lda, a_scales, b_codes, ldb, b_scales, group_offsets,
+                                            num_groups, M, N, K, c, ldc, static_cast<cudaStream_t>(stream));
 }
 
 int mxfp4_nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rounding,

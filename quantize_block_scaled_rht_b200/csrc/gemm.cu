@@ -871,6 +871,13 @@ int launch_grouped_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_s
     return launch_cfg<DefaultCfg, MODE_GROUPED_K>(g, s);
 }
 
+int launch_grouped_wgrad_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
+                              int64_t ldb, const uint8_t *b_scales, const int32_t *offsets, int G, int64_t M,
+                              int64_t N, int64_t K, uint16_t *c, int64_t ldc, cudaStream_t s) {
+    GemmArgs g{a_codes, a_scales, b_codes, b_scales, lda, ldb, M, N, K, ldc, c, offsets, nullptr, G};
+    return launch_cfg<DefaultCfg, MODE_GROUPED_K, OUT_BF16>(g, s);
+}
+
 int launch_nvfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const float *a_amax,
                       const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, const float *b_amax, int64_t M,
                       int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s) {

@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_layout_helpers():
     assert mx.status_string(mx.MXFP4_OK) == "MXFP4_OK"
     assert mx.status_string(mx.MXFP4_ERR_TIMEOUT) == "MXFP4_ERR_TIMEOUT"
-    assert mx.lib().mxfp4_version() == 102
+    assert mx.lib().mxfp4_version() == 103
     # 128 rows x 4 K-blocks per 512-byte atom
     assert mx.mma_scales_bytes(128, 128) == 512
     assert mx.mma_scales_bytes(129, 2880) == 2 * 23 * 512
@@ -75,6 +75,9 @@ def test_invalid_arguments_rejected_without_gpu():
     assert L.mxfp4_gemm_mxfp4(fake, 32, fake, fake, 32, fake, 128, 192, 64, fake, 104, fake, 6, 0, None) == 2
     assert L.mxfp4_gemm_mxfp4(fake, 32, fake, fake, 32, fake, 128, 192, 64, fake, 96, fake, 6, 7, None) == 1
     assert L.mxfp4_gemm_mxfp4(fake, 16, fake, fake, 16, fake, 128, 192, 96, fake, 96, fake, 6, 0, None) == 3
+    # bf16 grouped wgrad: ldc must give 16-byte rows
+    assert L.mxfp4_grouped_gemm_wgrad_bf16(fake, 64, fake, fake, 64, fake, fake, 2, 128, 132, 128, fake, 132,
+                                           None) == 2
     # grouped wgrad: K not a multiple of 128, too many groups
     assert L.mxfp4_grouped_gemm_wgrad(fake, 32, fake, fake, 32, fake, fake, 2, 128, 128, 64, fake, 128, None) == 1
     assert L.mxfp4_grouped_gemm_wgrad(fake, 64, fake, fake, 64, fake, fake, 5000, 128, 128, 128, fake, 128,

@@ -446,3 +446,19 @@ def test_gemm_mxfp4_output_nan_rows():
     sc, codes = host(q.scales), host(q.codes)
     assert np.all(sc[9] == 0xFF) and np.all(codes[9] == 0)
     assert np.all(np.delete(sc, 9, axis=0) != 0xFF)
+
+
+@pytest.mark.parametrize("sizes", [[200, 0, 513, 128], [0, 0, 300]])
+def test_grouped_wgrad_bf16(sizes):
+    """bf16 grouped wgrad: bit-equal to the RNE of the FP32 grouped wgrad on
+    the same operands (empty groups zero)."""
+    M, N = 320, 224
+    dy, x, offsets, K = _routed_wgrad_case(sizes, M, N, seed=len(sizes) + sum(sizes))
+    qa = mx.mxfp4_quantize(dev_bf16(dy), mx.LAYOUT_1D_COL, 32, mx.ROUND_SR, 42, scale_layout=mx.SCALES_MMA)
+    qb = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_COL, 32, mx.ROUND_RNE, 42, scale_layout=mx.SCALES_MMA)
+    off = torch.from_numpy(offsets).cuda()
+    c32 = mx.mxfp4_grouped_gemm_wgrad(qa.codes, qa.scales, qb.codes, qb.scales, off, K)
+    c16 = mx.mxfp4_grouped_gemm_wgrad_bf16(qa.codes, qa.scales, qb.codes, qb.scales, off, K)
+    torch.cuda.synchronize()
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    assert torch.equal(c16.view(torch.int16), c32.to(torch.bfloat16).view(torch.int16))
