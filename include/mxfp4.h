@@ -30,7 +30,8 @@
  *     returns an error code and launches nothing.  Launch failures return
  *     MXFP4_ERR_CUDA.  Nothing crosses the ABI as an exception.
  *   - Leading dimensions: ld_x / ld_out in elements, ld_codes / ld_scales /
- *     lda / ldb in bytes, ldc in elements.
+ *     lda / ldb in bytes, ldc in elements (ld_c_codes / ld_c_scales of the
+ *     MXFP4-output GEMM in bytes).
  *   - Element codes: byte j of a 32-value block holds element 2j in bits 3:0
  *     and element 2j+1 in bits 7:4; bit 3 of a code is the sign.
  */
