@@ -187,6 +187,14 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 //     stores 16 bytes of codes.
 // Either output may be disabled (DO_ROW / DO_COL); the column-only form with
 // tall 128 x 64 tiles is the 1D-column quantizer.
+//
+// Tiles are visited in strips of `strip` vertically adjacent tiles (same
+// columns, consecutive row bands), a CTA taking whole strips.  The column-only
+// form keeps a strip's scale bytes in shared memory and writes them when the
+// strip ends: each output row then receives 4 * strip contiguous bytes from
+// one CTA instead of 4-byte pieces from `strip` CTAs at different times (the
+// scattered partial-sector writes cost about a quarter of the kernel's time
+// on a 1 GiB tensor).  The dual form runs strips of one tile.
 // ---------------------------------------------------------------------------
 template <int TR_, int TC_>
 struct DualTile {
@@ -209,22 +217,30 @@ struct DualParams {
     uint32_t seed_lo, seed_hi;
     int scale_rule;                        // MXFP4_SCALE_* >> 4
     uint64_t r_offset, c_offset;           // SR stream index of each output's first element
-    uint32_t tiles_c;                      // column tiles
+    uint32_t tiles_c, tiles_r;             // column tiles, row tiles
+    uint32_t strip;                        // tiles per strip (1 unless column-only; at most 8)
     uint32_t sgn_bit[32];                  // RHT sign of element i (mod the RHT size) as bit 31
 };
 
 // SR instantiations get up to 80 registers (3 CTAs per SM): the column block
 // (32 transformed values) and the Philox state together do not fit in 64.
 template <class T, int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualParams p, const uint32_t ntiles) {
+__global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualParams p, const uint32_t nstrips) {
     pdl_wait();
     pdl_trigger();
     constexpr int TR = T::TR, TC = T::TC, PITCH = T::PITCH, OCH = T::OCH;
+    constexpr bool STRIP = DO_COL && !DO_ROW;          // column scales staged per strip
+    constexpr int SPITCH = 9;                          // words per output row: 8 tiles x 4 bytes, +1 against bank conflicts
+    static_assert(!STRIP || OCH == 4, "one 4-byte scale word per output row and tile");
     __shared__ __align__(16) uint16_t tin[2][TR * PITCH];
     __shared__ __align__(16) uint4 tout[DO_COL ? TC * OCH : 1];   // column codes: TC rows x TR/2 bytes
+    __shared__ __align__(16) uint32_t ssc[STRIP ? TC * SPITCH : 1];
+    constexpr bool MULTI = STRIP && !SR;                // strips of several tiles (SR and dual: one tile)
     const int tid = threadIdx.x;
-    auto load = [&](uint32_t t, int buf) {
-        const int64_t r0 = (int64_t)(t / p.tiles_c) * TR, c0 = (int64_t)(t % p.tiles_c) * TC;
+    const uint32_t strip = MULTI ? p.strip : 1u;
+    // tile k of strip S: row band (S / tiles_c) * strip + k, column band S % tiles_c
+    auto load = [&](uint32_t S, uint32_t k, int buf) {
+        const int64_t r0 = ((int64_t)(S / p.tiles_c) * strip + (MULTI ? k : 0u)) * TR, c0 = (int64_t)(S % p.tiles_c) * TC;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int idx = tid + 256 * i, row = idx / (TC / 8), ch = idx % (TC / 8);
@@ -233,21 +249,23 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualP
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    uint32_t t = blockIdx.x;
-    if (t < ntiles) load(t, 0);
-    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+    uint32_t S = blockIdx.x, k = 0;
+    if (S < nstrips) load(S, 0, 0);
+    for (int it = 0; S < nstrips; ++it) {
         // the next tile's load is in flight while this one is quantized
         const int buf = it & 1;
-        const uint32_t tn = t + gridDim.x;
-        if (tn < ntiles) {
-            load(tn, buf ^ 1);
+        const uint32_t band = S / p.tiles_c, tr = MULTI ? band * strip + k : band;
+        const bool last = !MULTI || k + 1 == strip || tr + 1 >= p.tiles_r;   // last tile of this strip
+        const uint32_t Sn = last ? S + gridDim.x : S, kn = (MULTI && !last) ? k + 1 : 0u;
+        if (Sn < nstrips) {
+            load(Sn, kn, buf ^ 1);
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
         const uint16_t *tile = tin[buf];
-        const int64_t r0 = (int64_t)(t / p.tiles_c) * TR, c0 = (int64_t)(t % p.tiles_c) * TC;
+        const int64_t r0 = (int64_t)tr * TR, c0 = (int64_t)(S - band * p.tiles_c) * TC;
 
         {
             if constexpr (DO_COL) {                          // column c, rows 32b .. 32b+31
@@ -274,7 +292,8 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualP
                     const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
                     tout[c * OCH + (b ^ ((c >> T::OSH) & (OCH - 1)))] = q;
                     const int64_t kb = rin >> 5;
-                    if constexpr (MMA) p.cscales[mma_scale_off(orow, kb, p.c_katoms)] = (uint8_t)sc;
+                    if constexpr (STRIP) reinterpret_cast<uint8_t *>(ssc)[4 * (c * SPITCH + (MULTI ? k : 0u)) + b] = (uint8_t)sc;
+                    else if constexpr (MMA) p.cscales[mma_scale_off(orow, kb, p.c_katoms)] = (uint8_t)sc;
                     else p.cscales[orow * p.ld_cscales + kb] = (uint8_t)sc;
                 }
             }
@@ -302,7 +321,39 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualP
             if (orow < p.cols && rin < p.rows)
                 stg_v4(p.ccodes + orow * p.ld_ccodes + (rin >> 1), tout[row * OCH + (ch ^ ((row >> T::OSH) & (OCH - 1)))]);
         }
+        if constexpr (STRIP) {
+            if (last) {                                      // the strip's scales: k + 1 words per output row
+                const int64_t kb0 = (int64_t)band * strip * 4;
+                if constexpr (MMA) {
+                    // the 4 K-blocks of one tile are 4 contiguous bytes of an MMA atom row slot
+                    for (uint32_t idx = tid; idx < TC * (k + 1); idx += 256) {
+                        const uint32_t a = idx / TC, row = idx % TC;
+                        const int64_t orow = c0 + row, kb = kb0 + 4 * a;
+                        if (orow < p.cols && kb * 32 < p.rows) {
+                            uint8_t *dst = p.cscales + mma_scale_off(orow, kb, p.c_katoms);
+                            const uint32_t w = ssc[row * SPITCH + a];
+                            if ((kb + 4) * 32 <= p.rows) {
+                                *reinterpret_cast<uint32_t *>(dst) = w;
+                            } else {                         // ragged last tile: valid K-blocks only
+                                for (int j = 0; j < 4 && (kb + j) * 32 < p.rows; ++j) dst[j] = (uint8_t)(w >> (8 * j));
+                            }
+                        }
+                    }
+                } else {
+                    // row-major: consecutive threads write consecutive bytes of one output row
+                    const uint32_t nb = 4 * (k + 1);
+                    const uint8_t *sb = reinterpret_cast<const uint8_t *>(ssc);
+                    for (uint32_t idx = tid; idx < TC * nb; idx += 256) {
+                        const uint32_t row = idx / nb, j = idx - row * nb;
+                        const int64_t orow = c0 + row, kb = kb0 + j;
+                        if (orow < p.cols && kb * 32 < p.rows) p.cscales[orow * p.ld_cscales + kb] = sb[4 * row * SPITCH + j];
+                    }
+                }
+            }
+        }
         __syncthreads();                                     // the load after next overwrites this buffer
+        S = Sn;
+        k = kn;
     }
 }
 
@@ -745,18 +796,40 @@ cudaError_t launch_quantize(const void *x, int64_t rows, int64_t cols, int64_t l
     }
 }
 
+// Tiles per strip of the column-only RNE quantizer: the L in {1, 2, 4, 8}
+// that minimises (strips of the busiest CTA) x L x (time per tile at L), over
+// the L that still fill the persistent grid.  Time per tile relative to L = 1,
+// measured on B200 with a 186,400 x 2880 bf16 tensor: 0.88 (L = 2), 0.815
+// (4), 0.805 (8).
+static uint32_t strip_len(uint64_t tiles_r, uint64_t tiles_c, uint64_t grid) {
+    static const uint32_t cost[4] = {1000, 880, 815, 805};
+    uint32_t best = 1;
+    uint64_t best_t = ((tiles_r * tiles_c + grid - 1) / grid) * cost[0];
+    for (int i = 1; i < 4; ++i) {
+        const uint64_t L = 1ull << i, strips = (tiles_r + L - 1) / L * tiles_c;
+        if (strips < grid) break;
+        const uint64_t t = (strips + grid - 1) / grid * L * cost[i];
+        if (t < best_t) { best_t = t; best = (uint32_t)L; }
+    }
+    return best;
+}
+
 template <class T, int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
 static cudaError_t launch_dual_t(DualParams p, cudaStream_t s) {
     p.tiles_c = (uint32_t)((p.cols + T::TC - 1) / T::TC);
-    const uint64_t tiles = (uint64_t)((p.rows + T::TR - 1) / T::TR) * p.tiles_c;
+    const uint64_t tiles_r = (uint64_t)((p.rows + T::TR - 1) / T::TR);
+    const uint64_t tiles = tiles_r * p.tiles_c;
     if (tiles > 0xFFFFFFFFull - 0x7FFFFFFFull) return cudaErrorInvalidValue;   // tile index fits 32 bits
+    p.tiles_r = (uint32_t)tiles_r;
     auto kern = quant_dual_kernel<T, CRHT, SR, MMA, DO_ROW, DO_COL>;
     // RNE is memory-bound: a persistent grid at full occupancy keeps the next
     // tile's load in flight.  SR is ALU-bound: one CTA per tile lets the
     // hardware scheduler balance the tail.
     const uint64_t cap = SR ? 0x7FFFFFFFull
                             : (uint64_t)num_sms() * (uint64_t)resident_ctas(reinterpret_cast<const void *>(kern), 256);
-    return launch_pdl(kern, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(256), 0, s, p, (uint32_t)tiles);
+    p.strip = (!SR && DO_COL && !DO_ROW && tiles > 0) ? strip_len(tiles_r, p.tiles_c, cap) : 1u;
+    const uint64_t strips = (tiles_r + p.strip - 1) / p.strip * p.tiles_c;
+    return launch_pdl(kern, dim3((unsigned)(strips < cap ? strips : cap)), dim3(256), 0, s, p, (uint32_t)strips);
 }
 
 // 1D-column quantization: the column-only dual kernel on 128 x 64 tiles.

@@ -228,15 +228,17 @@ def test_sweep_2gib_sampled_rows():
             assert np.array_equal(host(q.codes[r0:r0 + 32]), codes)
             assert np.array_equal(host(q.scales[r0:r0 + 32]), scales)
         del q
-    qc = mx.mxfp4_quantize(x, mx.LAYOUT_1D_COL, 32, mx.ROUND_SR, 42)
-    g = np.random.default_rng(10)
-    for c0 in list(g.integers(0, cols // 8, 4) * 8) + [cols - 8]:
-        xs = host(x[:, c0:c0 + 8])
-        codes, scales = oracle.quantize(np.ascontiguousarray(xs), oracle.LAYOUT_1D_COL, 32, oracle.ROUND_SR, 42,
-                                        elem_offset=int(c0) * rows)
-        assert np.array_equal(host(qc.codes[c0:c0 + 8]), codes)
-        assert np.array_equal(host(qc.scales[c0:c0 + 8]), scales)
-    del qc, x
+    for rnd in (mx.ROUND_SR, mx.ROUND_RNE):     # RNE walks strips of 8 row tiles; the last tile holds 64 rows
+        qc = mx.mxfp4_quantize(x, mx.LAYOUT_1D_COL, 32, rnd, 42)
+        g = np.random.default_rng(10)
+        for c0 in list(g.integers(0, cols // 8, 4) * 8) + [cols - 8]:
+            xs = host(x[:, c0:c0 + 8])
+            codes, scales = oracle.quantize(np.ascontiguousarray(xs), oracle.LAYOUT_1D_COL, 32, rnd, 42,
+                                            elem_offset=int(c0) * rows)
+            assert np.array_equal(host(qc.codes[c0:c0 + 8]), codes)
+            assert np.array_equal(host(qc.scales[c0:c0 + 8]), scales)
+        del qc
+    del x
     torch.cuda.empty_cache()
 
 

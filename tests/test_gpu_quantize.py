@@ -58,6 +58,22 @@ def test_quantize_bit_exact(layout, rht, rnd, scale_layout):
             assert np.array_equal(from_mma(st, cols, rows), expand_2d(ref[1].T, cols))
 
 
+@pytest.mark.parametrize("scale_layout", [mx.SCALES_ROWMAJOR, mx.SCALES_MMA])
+@pytest.mark.parametrize("rht", [0, 32])
+def test_column_quantizer_strips(rht, scale_layout):
+    """1D-column RNE on 65,632 x 1080: 513 row tiles of 128 (the last holds 96
+    rows, so 3 of its 4 K-blocks), 17 column tiles of 64 (the last holds 56
+    columns).  With 148 SMs the launcher walks strips of 8 vertically adjacent
+    tiles whose scales leave together, so the last strip is one ragged tile;
+    codes and scales must be bit-exact."""
+    rows, cols = 65632, 1080
+    x = synth.student_t_bf16((rows, cols), seed=12)
+    q = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_COL, rht, mx.ROUND_RNE, 42, 0, scale_layout)
+    codes, scales = oracle.quantize(x, oracle.LAYOUT_1D_COL, rht, oracle.ROUND_RNE, 42)[:2]
+    assert np.array_equal(host(q.codes), codes)
+    assert np.array_equal(_scales_rowmajor(q, mx.LAYOUT_1D_COL, scales, rows, cols), scales)
+
+
 @pytest.mark.parametrize("rht", [0, 32])
 @pytest.mark.parametrize("layout", LAYOUTS)
 def test_every_bf16_pattern(layout, rht):
