@@ -84,6 +84,91 @@ __device__ __forceinline__ uint32_t quantize32(const float *v, uint4 &out, uint6
         out, g0, k0, k1, rule);
 }
 
+// Packed two-lane fp32 arithmetic (sm_100a `.f32x2`): each lane is rounded
+// to nearest even exactly as the scalar operation, subnormals kept.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// The same butterfly as fwht<D> on 32 values held as 16 pairs
+// P[m] = (v[m], v[m + 16]).  Stages h = 1, 2, 4, 8 act on both 16-element
+// halves at once (the two lanes of a pair), with the same operations in the
+// same order; for D = 32 the last stage (h = 16) combines the two lanes of
+// each pair.  Bit-identical to fwht<D> on v (both halves for D = 16).
+template <int D>
+__device__ __forceinline__ void fwht_pairs(float2 *P) {
+    static_assert(D == 16 || D == 32, "RHT size");
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            if ((m & h) == 0) {
+                const float2 a = P[m], b = P[m + h];
+                P[m] = add2(a, b);
+                P[m + h] = sub2(a, b);
+            }
+        }
+    }
+    if constexpr (D == 32) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) P[m] = make_float2(__fadd_rn(P[m].x, P[m].y), __fsub_rn(P[m].x, P[m].y));
+    }
+}
+
+// The same for 32 fp32 values held as 16 pairs P[m] = (v[m], v[m + 16]),
+// scaled with packed two-lane multiplies (each lane rounded as the scalar
+// product): groups 0, 1 are the low lanes of P[0..15], groups 2, 3 the high.
+template <bool SR>
+__device__ __forceinline__ uint32_t quantize32_pairs(float2 *P, uint4 &out, uint64_t g0, uint32_t k0, uint32_t k1,
+                                                     int rule) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) amax = amax_nan(amax_nan(amax, P[m].x), P[m].y);
+    const uint32_t code = scale_code_rule(amax, rule);
+    if (code == 0xFFu) {
+        out = make_uint4(0, 0, 0, 0);
+        return code;
+    }
+    const float inv = inv_scale_from_code(code);
+    if (rule == 2) {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) P[m] = mul2(mul2(P[m], make_float2(0.75f, 0.75f)), make_float2(inv, inv));
+    } else {
+#pragma unroll
+        for (int m = 0; m < 16; ++m) P[m] = mul2(P[m], make_float2(inv, inv));
+    }
+    const uint64_t blk = g0 >> 2;  // g0 % 4 == 0
+    uint32_t p[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = q < 2 ? P[8 * q + j].x : P[8 * (q - 2) + j].y;
+        if constexpr (SR) p[q] = e2m1x8_sr(w, blk + 2 * q, k0, k1);
+        else p[q] = e2m1x8_rn(w);
+    }
+    out = make_uint4(p[0], p[1], p[2], p[3]);
+    return code;
+}
+
 // The same for 32 bf16 values packed in four uint4 (no transform): amax on
 // the packed pairs, each group unpacked when it is encoded, so that the block
 // occupies 16 registers rather than 32.
@@ -273,23 +358,23 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualP
                 const int64_t orow = c0 + c, rin = r0 + 32 * b;
                 if (orow < p.cols && rin < p.rows) {
                     const uint16_t *col = tile + 32 * b * PITCH + c;
-                    float v[32];
+                    float2 P[16];                    // (v[m], v[m + 16]): packed two-lane arithmetic
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int m = 0; m < 16; ++m) {
                         // bf16 -> fp32 with the RHT sign: adding 2^31 flips bit 31
-                        const uint32_t u = (uint32_t)col[i * PITCH] * 65536u + (CRHT ? p.sgn_bit[i % 32] : 0u);
-                        v[i] = __uint_as_float(u);
+                        const uint32_t u0 = (uint32_t)col[m * PITCH] * 65536u + (CRHT ? p.sgn_bit[m] : 0u);
+                        const uint32_t u1 = (uint32_t)col[(m + 16) * PITCH] * 65536u + (CRHT ? p.sgn_bit[m + 16] : 0u);
+                        P[m] = make_float2(__uint_as_float(u0), __uint_as_float(u1));
                     }
                     if constexpr (CRHT) {
                         const float cn = rht_norm<CRHT>();
+                        fwht_pairs<CRHT>(P);
 #pragma unroll
-                        for (int s = 0; s < 32; s += CRHT) fwht<CRHT>(v + s);
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], cn);
+                        for (int m = 0; m < 16; ++m) P[m] = mul2(P[m], make_float2(cn, cn));
                     }
                     uint4 q;
                     const uint64_t g0 = (uint64_t)(orow * p.rows + rin) + p.c_offset;
-                    const uint32_t sc = quantize32<SR>(v, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
+                    const uint32_t sc = quantize32_pairs<SR>(P, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
                     tout[c * OCH + (b ^ ((c >> T::OSH) & (OCH - 1)))] = q;
                     const int64_t kb = rin >> 5;
                     if constexpr (STRIP) reinterpret_cast<uint8_t *>(ssc)[4 * (c * SPITCH + (MULTI ? k : 0u)) + b] = (uint8_t)sc;
