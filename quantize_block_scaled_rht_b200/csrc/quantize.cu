@@ -278,7 +278,7 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 // form keeps a strip's scale bytes in shared memory and writes them when the
 // strip ends: each output row then receives 4 * strip contiguous bytes from
 // one CTA instead of 4-byte pieces from `strip` CTAs at different times (the
-// scattered partial-sector writes cost about a quarter of the kernel's time
+// scattered partial-sector writes cost 30% of the kernel's time
 // on a 1 GiB tensor).  The dual form runs strips of one tile.
 // ---------------------------------------------------------------------------
 template <int TR_, int TC_>
