@@ -133,6 +133,23 @@ __device__ __forceinline__ void fwht_pairs(float2 *P) {
     }
 }
 
+// fwht<D> on v[0..31] (each D-element segment) followed by the product with
+// c, through the packed pairs (v[m], v[m + 16]); bit-identical to the scalar
+// loops.
+template <int D>
+__device__ __forceinline__ void fwht32_scaled(float *v, float c) {
+    float2 P[16];
+#pragma unroll
+    for (int m = 0; m < 16; ++m) P[m] = make_float2(v[m], v[m + 16]);
+    fwht_pairs<D>(P);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+        P[m] = mul2(P[m], make_float2(c, c));
+        v[m] = P[m].x;
+        v[m + 16] = P[m].y;
+    }
+}
+
 // The same for 32 fp32 values held as 16 pairs P[m] = (v[m], v[m + 16]),
 // scaled with packed two-lane multiplies (each lane rounded as the scalar
 // product): groups 0, 1 are the low lanes of P[0..15], groups 2, 3 the high.
@@ -189,13 +206,7 @@ __device__ __forceinline__ void unpack_row32(const uint32_t *w, float *v, const 
         v[2 * j] = bf16lo(u);
         v[2 * j + 1] = bf16hi(u);
     }
-    if constexpr (RHT) {
-#pragma unroll
-        for (int s = 0; s < 32; s += RHT) fwht<RHT>(v + s);
-        const float c = rht_norm<RHT>();
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], c);
-    }
+    if constexpr (RHT) fwht32_scaled<RHT>(v, rht_norm<RHT>());
 }
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
@@ -610,11 +621,7 @@ __device__ __forceinline__ void decode32(const uint4 q, uint32_t scode, float *v
 template <int RHT>
 __device__ __forceinline__ void inverse_rht32(float *v, const uint32_t *sgn_pair) {
     if constexpr (RHT) {
-        const float c = rht_norm<RHT>();
-#pragma unroll
-        for (int s = 0; s < 32; s += RHT) fwht<RHT>(v + s);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(v[i], c);
+        fwht32_scaled<RHT>(v, rht_norm<RHT>());
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             v[2 * j] = __uint_as_float(__float_as_uint(v[2 * j]) ^ (sgn_pair[j] << 16));
