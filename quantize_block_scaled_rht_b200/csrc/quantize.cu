@@ -6,9 +6,11 @@
 // stochastic rounding).  "Training an MoE LLM in MXFP4" (ALTO), abstract:
 // 1D blocks for activations/gradients, 2D blocks for weights.
 //
-// All kernels are HBM-bound streaming kernels (2 B read + 0.5 B + 1/32 B
-// written per element): 128-bit loads/stores, in-register Hadamard butterflies,
-// and shared-memory staging only where a transpose is needed.
+// Streaming kernels (2 B read + 0.5 B + 1/32 B written per element):
+// 128-bit loads/stores, in-register Hadamard butterflies on packed two-lane
+// fp32, and shared-memory staging only where a transpose is needed.  Under
+// RNE they are bound by HBM; stochastic rounding adds the integer work of
+// Philox4x32-10 and the exact rounding decision, which then bounds them.
 #include <cstdint>
 #include <map>
 #include <mutex>
