@@ -252,7 +252,7 @@ def run_reference(args, rank):
     import oracle
     x, w, dy = rank_inputs(0)
     # calibrate on the smallest sample, then pick the sub-problem for the budget
-    budget_s = 120.0
+    budget_s = args.ref_budget_s
     n_total = args.steps + args.warmup
     ladder = [(32, 256, 512), (32, 512, 1024), (32, 1024, 2048), (64, 1440, 2880), (64, HIDDEN, INTER)]
     dt0, fl0 = oracle_sample(x, w, dy, *ladder[0])
@@ -535,6 +535,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-budget-s", type=float, default=120.0,
+                    help="reference arm: host seconds the warm-up and timed samples may take together")
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-mib", type=int, default=256)
