@@ -64,7 +64,7 @@ KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 NCU_TRAFFIC = {
     "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "cfcae9425fa80c24",
              "bytes": {"fprop": 52.26e6, "dgrad": 23.36e6, "wgrad": 29.88e6}},
-    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "9dee2b6ed63a9620",
+    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "b9c5a4ffd3c6011a",
               "bytes": {"quant_x_dual": 23.62e6, "quant_w_2d": 33.43e6, "quant_dy_dual_sr": 48.71e6},
               # thread instructions per element (ncu smsp__inst_executed x 32 / elements)
               "inst_per_elem": {"quant_dy_dual_sr": 77.1}},

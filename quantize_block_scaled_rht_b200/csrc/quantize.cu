@@ -292,7 +292,8 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 // strip ends: each output row then receives 4 * strip contiguous bytes from
 // one CTA instead of 4-byte pieces from `strip` CTAs at different times (the
 // scattered partial-sector writes cost 30% of the kernel's time
-// on a 1 GiB tensor).  The dual form runs strips of one tile.
+// on a 1 GiB tensor).  The dual form and stochastic rounding run strips of
+// one tile (SR launches one CTA per tile).
 // ---------------------------------------------------------------------------
 template <int TR_, int TC_>
 struct DualTile {
