@@ -58,9 +58,9 @@ KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# the ncu --set full capture of one bench step summarised in
-# profiles/expert_step_kernels_ncu_full.md.  The figures hold only for the
-# kernel sources they were taken from: a changed source gives traffic null.
+# ncu captures of the kernels of one bench step (one kernel per capture).  The
+# figures hold only for the kernel sources they were taken from: a changed
+# source gives traffic null.
 NCU_TRAFFIC = {
     "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "cfcae9425fa80c24",
              "bytes": {"fprop": 52.26e6, "dgrad": 23.36e6, "wgrad": 29.88e6}},

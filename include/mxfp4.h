@@ -94,7 +94,7 @@ MXFP4_API const char *mxfp4_status_string(int status);
 
 /* ABI version (major * 100 + minor).  1.01 added mxfp4_gemm_bf16 and
  * mxfp4_grouped_gemm_bf16; 1.02 mxfp4_gemm_mxfp4; 1.03
- * mxfp4_grouped_gemm_wgrad_bf16. */
+ * mxfp4_grouped_gemm_wgrad_bf16; 1.04 mxfp4_scales_to_mma. */
 MXFP4_API int mxfp4_version(void);
 
 /*
@@ -111,6 +111,29 @@ MXFP4_API int mxfp4_version(void);
  */
 MXFP4_API int64_t mxfp4_mma_scales_bytes(int64_t rows, int64_t k);
 MXFP4_API int64_t mxfp4_mma_scale_offset(int64_t row, int64_t kb, int64_t k);
+
+/*
+ * mxfp4_scales_to_mma -- canonical row-major E8M0 scales to the GEMM-ready
+ * layout above, on the device.  ("MXFP4" (aiwiki.ai), "Use in models /
+ * gpt-oss": one scale byte per 32-element block, stored apart from the
+ * codes.)  For a caller that holds canonical scales -- from mxfp4_quantize
+ * with MXFP4_SCALES_ROWMAJOR, or from elsewhere -- and wants to call the
+ * GEMMs, which read only the GEMM-ready layout.
+ *
+ * scales: DEVICE, row-major with row stride ld_scales bytes:
+ *   two_d = 0: [rows, k/32], one scale per row and K-block (1D blocks);
+ *   two_d = 1: [rows/32, k/32], one scale per 32x32 tile (2D blocks, as
+ *              mxfp4_quantize writes for MXFP4_LAYOUT_2D); each tile's scale
+ *              is repeated on its 32 rows in the output.
+ * mma_scales: DEVICE, mxfp4_mma_scales_bytes(rows, k) bytes, 4-byte aligned,
+ *   fully overwritten (pad rows and pad K-blocks zero).  The two buffers must
+ *   not overlap.
+ * Requirements: rows > 0; k > 0, k % 32 == 0; rows % 32 == 0 when two_d;
+ * ld_scales >= k / 32.  Reads 1 byte per block (1D) or per tile (2D), writes
+ * the GEMM-ready bytes once: about 1/32 byte per element of the operand.
+ */
+MXFP4_API int mxfp4_scales_to_mma(const uint8_t *scales, int64_t ld_scales, int64_t rows, int64_t k, int two_d,
+                                  uint8_t *mma_scales, void *stream);
 
 /*
  * mxfp4_quantize -- bf16 tensor x[rows, cols] to MXFP4 codes and E8M0 scales.

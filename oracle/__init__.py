@@ -312,3 +312,11 @@ def nvfp4_gemm_entries(a_codes, a_scales, a_amax: float, b_codes, b_scales, b_am
                                ctypes.byref(c), ctypes.byref(s))
         out_c[i], out_s[i] = c.value, s.value
     return out_c, out_s
+
+
+def f32_to_bf16(values) -> np.ndarray:
+    """The oracle's fp32 -> bf16 rounding (nearest even) of each value, as bit
+    patterns; used for bf16 outputs of dequantize."""
+    L = lib()
+    v = np.ascontiguousarray(values, np.float32).ravel()
+    return np.fromiter((L.orc_f32_to_bf16(float(x)) for x in v), dtype=np.uint16, count=v.size)

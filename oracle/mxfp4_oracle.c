@@ -210,7 +210,8 @@ uint16_t orc_f32_to_bf16(float f)
     memcpy(&u, &f, 4);
     if (isnan(f)) return (uint16_t)((u >> 16) | 0x0040u);
     uint32_t lsb = (u >> 16) & 1u;
-    u += 0x7FFFu + lsb;
+    if (MUT(27)) u += 0x8000u;                 /* ties away from zero */
+    else if (!MUT(28)) u += 0x7FFFu + lsb;     /* MUT(28): truncation */
     return (uint16_t)(u >> 16);
 }
 
@@ -490,8 +491,12 @@ int orc_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales
     for (int64_t orow = 0; orow < orows; ++orow) {
         float y[32];
         for (int64_t b = 0; b < ocols / 32; ++b) {
-            uint8_t sc = layout == ORC_LAYOUT_2D ? scales[(orow / 32) * ld_scales + b]
-                                                 : scales[orow * ld_scales + b];
+            /* MUT(29) reads a 2D tile's scale at the 1D row index (clamped to
+             * the tile-row count, so the mistake stays inside the array). */
+            int64_t srow = layout == ORC_LAYOUT_2D
+                               ? (MUT(29) ? (orow < rows / 32 ? orow : rows / 32 - 1) : orow / 32)
+                               : orow;
+            uint8_t sc = scales[srow * ld_scales + b];
             double X = orc_e8m0_decode(sc);
             for (int i = 0; i < 32; ++i) {
                 double v = orc_e2m1_decode(orc_get_nibble(codes + orow * ld_codes, b * 32 + i));
@@ -501,7 +506,7 @@ int orc_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales
                 for (int s = 0; s < 32; s += rht) orc_rht_inverse(y + s, rht, smask);
             for (int i = 0; i < 32; ++i) {
                 int64_t ocol = b * 32 + i;
-                int64_t r = transposed ? ocol : orow;
+                int64_t r = transposed ? (MUT(30) ? ocol ^ 1 : ocol) : orow;   /* MUT(30): nibble slip */
                 int64_t c = transposed ? orow : ocol;
                 out_f32[r * ld_out + c] = y[i];
                 if (out_bf16) out_bf16[r * ld_out + c] = orc_f32_to_bf16(y[i]);

@@ -44,7 +44,7 @@ ABI_FUNCTIONS = (
     "mxfp4_gemm_bf16", "mxfp4_grouped_gemm_bf16", "mxfp4_gemm_mxfp4", "mxfp4_grouped_gemm_wgrad",
     "mxfp4_grouped_gemm_wgrad_bf16", "mxfp4_nvfp4_quantize", "mxfp4_nvfp4_dequantize", "mxfp4_nvfp4_gemm",
     "mxfp4_get_error",
-    "mxfp4_set_wait_limit_ns", "mxfp4_wait_probe",
+    "mxfp4_set_wait_limit_ns", "mxfp4_wait_probe", "mxfp4_scales_to_mma",
 )
 
 
@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.mxfp4_nvfp4_dequantize.restype = i32
         L.mxfp4_nvfp4_gemm.argtypes = [vp, i64, vp, vp, vp, i64, vp, vp, i64, i64, i64, vp, i64, vp]
         L.mxfp4_nvfp4_gemm.restype = i32
+        L.mxfp4_scales_to_mma.argtypes = [vp, i64, i64, i64, i32, vp, vp]
+        L.mxfp4_scales_to_mma.restype = i32
         L.mxfp4_get_error.argtypes = [vp]
         L.mxfp4_get_error.restype = i32
         L.mxfp4_set_wait_limit_ns.argtypes = [u64]
@@ -142,6 +144,31 @@ def mma_scales_bytes(rows: int, k: int) -> int:
 
 def mma_scale_offset(row: int, kb: int, k: int) -> int:
     return int(lib().mxfp4_mma_scale_offset(row, kb, k))
+
+
+def _check_operand(codes: torch.Tensor, scales: torch.Tensor, rows: int, K: int, what: str, groups: int = 1,
+                   scale_bytes=None) -> None:
+    """Host-side check of one GEMM operand before its pointers cross the ABI:
+    the C library cannot see buffer sizes, so a row-major scale tensor passed
+    where the GEMM-ready layout is read (32x smaller for 2D weights) is caught
+    here instead of becoming reads past the allocation."""
+    if codes.dtype != torch.uint8 or scales.dtype != torch.uint8:
+        raise ValueError(f"{what}: codes and scales must be uint8 tensors")
+    if codes.shape[-1] * 2 < K:
+        raise ValueError(f"{what}: codes hold {codes.shape[-1] * 2} elements per row, K = {K}")
+    need = groups * (scale_bytes or mma_scales_bytes)(rows, K)
+    if scales.dim() != 1 or scales.numel() < need:
+        raise ValueError(f"{what}: scales must be the GEMM-ready (SCALES_MMA) layout, a 1-D tensor of at least "
+                         f"{need} bytes; got shape {tuple(scales.shape)} (quantize with scale_layout=SCALES_MMA "
+                         f"or convert with mxfp4_scales_to_mma)")
+    if codes.device != scales.device:
+        raise ValueError(f"{what}: codes and scales on different devices")
+
+
+def _check_same_device(*ts: torch.Tensor) -> None:
+    devs = {t.device for t in ts if t is not None}
+    if len(devs) > 1:
+        raise ValueError(f"GEMM operands on different devices: {sorted(map(str, devs))}")
 
 
 @dataclass
@@ -246,6 +273,9 @@ def mxfp4_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Ten
                K: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """C[M, N] = A[M, K] B[N, K]^T in FP32; scales in the GEMM-ready (MMA) layout."""
     M, N = a_codes.shape[0], b_codes.shape[0]
+    _check_operand(a_codes, a_scales, M, K, "A")
+    _check_operand(b_codes, b_scales, N, K, "B")
+    _check_same_device(a_codes, b_codes, out)
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=a_codes.device)
     rc = lib().mxfp4_gemm(_ptr(a_codes), a_codes.stride(0), _ptr(a_scales), _ptr(b_codes), b_codes.stride(0),
@@ -260,6 +290,9 @@ def mxfp4_grouped_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, group_offs
     """Per group g: C[rows of g] = A[rows of g] B_g^T.  b_codes is [G, N, K/2]."""
     a_rows = a_codes.shape[0]
     G = group_sizes.numel()
+    _check_operand(a_codes, a_scales, a_rows, K, "A")
+    _check_operand(b_codes, b_scales, N, K, "B", groups=G)
+    _check_same_device(a_codes, b_codes, group_offsets, group_sizes, out)
     if out is None:
         out = torch.empty((a_rows, N), dtype=torch.float32, device=a_codes.device)
     rc = lib().mxfp4_grouped_gemm(_ptr(a_codes), a_codes.stride(0), _ptr(a_scales), a_rows, _ptr(group_offsets),
@@ -273,6 +306,9 @@ def mxfp4_gemm_bf16(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torc
                     K: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """mxfp4_gemm with the FP32 accumulators rounded to a bf16 output."""
     M, N = a_codes.shape[0], b_codes.shape[0]
+    _check_operand(a_codes, a_scales, M, K, "A")
+    _check_operand(b_codes, b_scales, N, K, "B")
+    _check_same_device(a_codes, b_codes, out)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
     if out.dtype != torch.bfloat16:
@@ -289,6 +325,8 @@ def mxfp4_gemm_mxfp4(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: tor
     """mxfp4_gemm with C requantized to MXFP4 (1D row blocks, reference scale
     rule, RNE) in the epilogue; returns C as a Quantized [M, N]."""
     M, N = a_codes.shape[0], b_codes.shape[0]
+    _check_operand(a_codes, a_scales, M, K, "A")
+    _check_operand(b_codes, b_scales, N, K, "B")
     dev = a_codes.device
     if out is None:
         out = Quantized(torch.empty((M, N // 2), dtype=torch.uint8, device=dev), _scale_tensor(M, N, scale_layout, dev),
@@ -307,6 +345,9 @@ def mxfp4_grouped_gemm_bf16(a_codes: torch.Tensor, a_scales: torch.Tensor, group
     """mxfp4_grouped_gemm with a bf16 output."""
     a_rows = a_codes.shape[0]
     G = group_sizes.numel()
+    _check_operand(a_codes, a_scales, a_rows, K, "A")
+    _check_operand(b_codes, b_scales, N, K, "B", groups=G)
+    _check_same_device(a_codes, b_codes, group_offsets, group_sizes, out)
     if out is None:
         out = torch.empty((a_rows, N), dtype=torch.bfloat16, device=a_codes.device)
     if out.dtype != torch.bfloat16:
@@ -326,6 +367,9 @@ def mxfp4_grouped_gemm_wgrad(a_codes: torch.Tensor, a_scales: torch.Tensor, b_co
     int32 tensor of G + 1 offsets along K; returns [G * M, N] FP32."""
     M, N = a_codes.shape[0], b_codes.shape[0]
     G = group_offsets.numel() - 1
+    _check_operand(a_codes, a_scales, M, K, "A")
+    _check_operand(b_codes, b_scales, N, K, "B")
+    _check_same_device(a_codes, b_codes, group_offsets, out)
     if out is None:
         out = torch.empty((G * M, N), dtype=torch.float32, device=a_codes.device)
     rc = lib().mxfp4_grouped_gemm_wgrad(_ptr(a_codes), a_codes.stride(0), _ptr(a_scales), _ptr(b_codes),
@@ -341,6 +385,9 @@ def mxfp4_grouped_gemm_wgrad_bf16(a_codes: torch.Tensor, a_scales: torch.Tensor,
     """mxfp4_grouped_gemm_wgrad with a bf16 output; returns [G * M, N] bf16."""
     M, N = a_codes.shape[0], b_codes.shape[0]
     G = group_offsets.numel() - 1
+    _check_operand(a_codes, a_scales, M, K, "A")
+    _check_operand(b_codes, b_scales, N, K, "B")
+    _check_same_device(a_codes, b_codes, group_offsets, out)
     if out is None:
         out = torch.empty((G * M, N), dtype=torch.bfloat16, device=a_codes.device)
     if out.dtype != torch.bfloat16:
@@ -410,12 +457,37 @@ def mxfp4_nvfp4_gemm(a: NvQuantized, b: NvQuantized, out: Optional[torch.Tensor]
                      stream=None) -> torch.Tensor:
     """C = A B^T for NVFP4 operands quantized with SCALES_MMA."""
     M, N, K = a.rows, b.rows, a.k
+    if a.scale_layout != SCALES_MMA or b.scale_layout != SCALES_MMA or b.k != K:
+        raise ValueError("mxfp4_nvfp4_gemm: both operands need SCALES_MMA scales and the same K")
+    _check_operand(a.codes, a.scales, M, K, "A", scale_bytes=nv_mma_scales_bytes)
+    _check_operand(b.codes, b.scales, N, K, "B", scale_bytes=nv_mma_scales_bytes)
+    _check_same_device(a.codes, b.codes, a.amax, b.amax, out)
     if out is None:
         out = torch.empty((M, N), dtype=torch.float32, device=a.codes.device)
     rc = lib().mxfp4_nvfp4_gemm(_ptr(a.codes), a.codes.stride(0), _ptr(a.scales), _ptr(a.amax), _ptr(b.codes),
                                 b.codes.stride(0), _ptr(b.scales), _ptr(b.amax), M, N, K, _ptr(out), out.stride(0),
                                 _stream(stream))
     _check(rc, "mxfp4_nvfp4_gemm")
+    return out
+
+
+def mxfp4_scales_to_mma(scales: torch.Tensor, rows: int, k: int, two_d: bool = False,
+                        out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Canonical row-major scales ([rows, k/32], or [rows/32, k/32] tile scales
+    with two_d) to the GEMM-ready layout the GEMMs read (see
+    mxfp4_scales_to_mma in include/mxfp4.h)."""
+    if scales.dtype != torch.uint8 or scales.dim() != 2:
+        raise ValueError("scales must be a 2-D uint8 tensor (canonical row-major)")
+    want = ((rows // 32) if two_d else rows, k // 32)
+    if tuple(scales.shape) != want or scales.stride(1) != 1:
+        raise ValueError(f"scales must be {want} row-major; got {tuple(scales.shape)}")
+    if out is None:
+        out = torch.empty(mma_scales_bytes(rows, k), dtype=torch.uint8, device=scales.device)
+    if out.dim() != 1 or out.numel() < mma_scales_bytes(rows, k):
+        raise ValueError("out must be a 1-D uint8 tensor of mma_scales_bytes(rows, k) bytes")
+    rc = lib().mxfp4_scales_to_mma(_ptr(scales), scales.stride(0), rows, k, 1 if two_d else 0, _ptr(out),
+                                   _stream(stream))
+    _check(rc, "mxfp4_scales_to_mma")
     return out
 
 

@@ -51,6 +51,8 @@ cudaError_t launch_nvfp4_dequantize(const uint8_t *codes, int64_t ld_codes, cons
 int launch_nvfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const float *a_amax,
                       const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, const float *b_amax, int64_t M,
                       int64_t N, int64_t K, float *c, int64_t ldc, cudaStream_t s);
+cudaError_t launch_scales_to_mma(const uint8_t *src, int64_t ld_src, int64_t rows, int64_t k, int two_d,
+                                 uint8_t *dst, cudaStream_t s);
 int get_error(cudaStream_t s);
 int launch_wait_probe(int arrive, cudaStream_t s);
 uint64_t set_wait_limit(uint64_t ns);
@@ -74,7 +76,7 @@ const char *mxfp4_status_string(int status) {
     }
 }
 
-int mxfp4_version(void) { return 103; }
+int mxfp4_version(void) { return 104; }
 
 int64_t mxfp4_mma_scales_bytes(int64_t rows, int64_t k) {
     if (rows <= 0 || k <= 0) return 0;
@@ -152,6 +154,10 @@ int mxfp4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
     if (!aligned16(x) || (ld_x % 8)) return MXFP4_ERR_ALIGNMENT;
     if (row_codes && (!aligned16(row_codes) || (ld_row_codes % 16))) return MXFP4_ERR_ALIGNMENT;
     if (col_codes && (!aligned16(col_codes) || (ld_col_codes % 16))) return MXFP4_ERR_ALIGNMENT;
+    // GEMM-ready scales are written in 4- and 16-byte pieces
+    if (scale_layout == MXFP4_SCALES_MMA &&
+        ((row_codes && !aligned16(row_scales)) || (col_codes && !aligned16(col_scales))))
+        return MXFP4_ERR_ALIGNMENT;
     const cudaError_t e = mxfp4::launch_quantize_dual(
         x, rows, cols, ld_x, col_rht_size, rounding, seed, row_elem_offset, col_elem_offset, row_codes, ld_row_codes,
         row_scales, ld_row_scales, col_codes, ld_col_codes, col_scales, ld_col_scales, scale_layout,
@@ -347,6 +353,19 @@ int mxfp4_nvfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scale
     if (M > (int64_t)1 << 31) return MXFP4_ERR_UNSUPPORTED;
     return mxfp4::launch_nvfp4_gemm(a_codes, lda, a_scales, a_amax, b_codes, ldb, b_scales, b_amax, M, N, K, c, ldc,
                                     static_cast<cudaStream_t>(stream));
+}
+
+int mxfp4_scales_to_mma(const uint8_t *scales, int64_t ld_scales, int64_t rows, int64_t k, int two_d,
+                        uint8_t *mma_scales, void *stream) {
+    if (!scales || !mma_scales) return MXFP4_ERR_INVALID_ARG;
+    if (rows <= 0 || k <= 0 || (k % 32) || (two_d != 0 && two_d != 1)) return MXFP4_ERR_INVALID_ARG;
+    if (two_d && (rows % 32)) return MXFP4_ERR_INVALID_ARG;
+    if (ld_scales < k / 32) return MXFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(mma_scales) & 3u) != 0) return MXFP4_ERR_ALIGNMENT;
+    if (rows > (int64_t)1 << 40 || k > (int64_t)1 << 40) return MXFP4_ERR_UNSUPPORTED;
+    const cudaError_t e = mxfp4::launch_scales_to_mma(scales, ld_scales, rows, k, two_d, mma_scales,
+                                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
 }
 
 int mxfp4_get_error(void *stream) { return mxfp4::get_error(static_cast<cudaStream_t>(stream)); }

@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_layout_helpers():
     assert mx.status_string(mx.MXFP4_OK) == "MXFP4_OK"
     assert mx.status_string(mx.MXFP4_ERR_TIMEOUT) == "MXFP4_ERR_TIMEOUT"
-    assert mx.lib().mxfp4_version() == 103
+    assert mx.lib().mxfp4_version() == 104
     # 128 rows x 4 K-blocks per 512-byte atom
     assert mx.mma_scales_bytes(128, 128) == 512
     assert mx.mma_scales_bytes(129, 2880) == 2 * 23 * 512
@@ -85,3 +85,60 @@ def test_invalid_arguments_rejected_without_gpu():
     # grouped: too many groups
     assert L.mxfp4_grouped_gemm(fake, 32, fake, 128, fake, fake, 5000, fake, 32, fake, 128, 64, fake, 128,
                                 None) == 3
+
+
+def test_dual_quantize_rejects_misaligned_mma_scales_without_gpu():
+    """GEMM-ready scales are written in 4- and 16-byte pieces: an offset scale
+    pointer is an alignment error before launch, not a misaligned store."""
+    L = mx.lib()
+    fake = ctypes.c_void_p(0x10000)
+    off = ctypes.c_void_p(0x10004)
+    args = lambda rs, cs: (fake, 64, 64, 64, 0, 0, 0, 0, 0, fake, 32, rs, 2, fake, 32, cs, 2, mx.SCALES_MMA, None)
+    assert L.mxfp4_quantize_dual(*args(off, fake)) == mx.MXFP4_ERR_ALIGNMENT
+    assert L.mxfp4_quantize_dual(*args(fake, off)) == mx.MXFP4_ERR_ALIGNMENT
+    # row-major scales are single bytes: any address is fine (the check passes
+    # and the call would launch, so only the failing forms are called here)
+
+
+def test_scales_to_mma_rejects_invalid_arguments_without_gpu():
+    L = mx.lib()
+    fake = ctypes.c_void_p(0x10000)
+    assert L.mxfp4_scales_to_mma(None, 4, 128, 128, 0, fake, None) == mx.MXFP4_ERR_INVALID_ARG
+    assert L.mxfp4_scales_to_mma(fake, 4, 128, 96 + 8, 0, fake, None) == mx.MXFP4_ERR_INVALID_ARG   # k % 32
+    assert L.mxfp4_scales_to_mma(fake, 4, 48, 128, 1, fake, None) == mx.MXFP4_ERR_INVALID_ARG       # 2D rows % 32
+    assert L.mxfp4_scales_to_mma(fake, 3, 128, 128, 0, fake, None) == mx.MXFP4_ERR_INVALID_ARG      # ld < k/32
+    assert L.mxfp4_scales_to_mma(fake, 4, 128, 128, 2, fake, None) == mx.MXFP4_ERR_INVALID_ARG      # two_d flag
+    assert L.mxfp4_scales_to_mma(fake, 4, 128, 128, 0, ctypes.c_void_p(0x10002), None) == mx.MXFP4_ERR_ALIGNMENT
+
+
+def test_gemm_wrappers_reject_rowmajor_scales_before_the_abi():
+    """The binding checks scale sizes the C library cannot see: row-major scales
+    (or too-short codes) raise ValueError before any pointer is taken."""
+    import torch
+    M, N, K = 256, 192, 512
+    a = torch.zeros((M, K // 2), dtype=torch.uint8)
+    b = torch.zeros((N, K // 2), dtype=torch.uint8)
+    a_rm = torch.zeros((M, K // 32), dtype=torch.uint8)
+    b_rm = torch.zeros((N, K // 32), dtype=torch.uint8)
+    b_2d = torch.zeros((N // 32, K // 32), dtype=torch.uint8)
+    a_mma = torch.zeros(mx.mma_scales_bytes(M, K), dtype=torch.uint8)
+    b_mma = torch.zeros(mx.mma_scales_bytes(N, K), dtype=torch.uint8)
+    for fn in (mx.mxfp4_gemm, mx.mxfp4_gemm_bf16, mx.mxfp4_gemm_mxfp4):
+        with pytest.raises(ValueError, match="SCALES_MMA"):
+            fn(a, a_rm, b, b_mma, K)
+        with pytest.raises(ValueError, match="SCALES_MMA"):
+            fn(a, a_mma, b, b_2d, K)
+        with pytest.raises(ValueError, match="elements per row"):
+            fn(a[:, :100], a_mma, b, b_mma, K)
+    G = 4
+    offs = torch.zeros(G + 1, dtype=torch.int32)
+    sizes = torch.zeros(G, dtype=torch.int32)
+    bg = torch.zeros((G, N, K // 2), dtype=torch.uint8)
+    for fn in (mx.mxfp4_grouped_gemm, mx.mxfp4_grouped_gemm_bf16):
+        with pytest.raises(ValueError, match="SCALES_MMA"):       # one expert's scales for G experts
+            fn(a, a_mma, offs, sizes, bg, b_mma, N, K)
+        with pytest.raises(ValueError, match="SCALES_MMA"):
+            fn(a, a_rm, offs, sizes, bg, torch.zeros(G * mx.mma_scales_bytes(N, K), dtype=torch.uint8), N, K)
+    for fn in (mx.mxfp4_grouped_gemm_wgrad, mx.mxfp4_grouped_gemm_wgrad_bf16):
+        with pytest.raises(ValueError, match="SCALES_MMA"):
+            fn(a, a_mma, b, b_rm, offs, K)

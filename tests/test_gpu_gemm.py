@@ -462,3 +462,44 @@ def test_grouped_wgrad_bf16(sizes):
     torch.cuda.synchronize()
     assert mx.mxfp4_get_error() == mx.MXFP4_OK
     assert torch.equal(c16.view(torch.int16), c32.to(torch.bfloat16).view(torch.int16))
+
+
+@pytest.mark.parametrize("rows,k,two_d", [(256, 2880, False), (130, 320, False), (1, 64, False),
+                                          (192, 2880, True), (96, 576, True)])
+def test_scales_to_mma_matches_host_permutation(rows, k, two_d):
+    """mxfp4_scales_to_mma writes every valid (row, K-block) byte where the
+    GEMM-ready layout puts it (2D tile scales repeated on their 32 rows) and
+    zero in every pad byte."""
+    g = np.random.default_rng(rows + k)
+    srows = rows // 32 if two_d else rows
+    canon = g.integers(0, 256, size=(srows, k // 32), dtype=np.uint8)
+    out = dev_u8(np.full(mx.mma_scales_bytes(rows, k), 0xA5, np.uint8))
+    mx.mxfp4_scales_to_mma(dev_u8(canon), rows, k, two_d=two_d, out=out)
+    got = host(out)
+    per_row = expand_2d(canon, rows) if two_d else canon
+    assert np.array_equal(got, to_mma(per_row, k))   # to_mma zero-fills the pads
+
+
+def test_gemm_from_canonical_2d_weight_scales():
+    """A caller holding canonical scales (1D row-major for X, 2D tile scales for
+    W) converts them with mxfp4_scales_to_mma and gets the same products as
+    from the quantizer's GEMM-ready scales, bit for bit."""
+    T, H, I = 256, 576, 384
+    x = synth.activations_with_outliers(T, H, seed=2)
+    w = synth.normal_bf16((I, H), 3, 0.02)
+    qx_rm = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_ROW)
+    qw_rm = mx.mxfp4_quantize(dev_bf16(w), mx.LAYOUT_2D, transposed_copy=True)
+    qx = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    qw = mx.mxfp4_quantize(dev_bf16(w), mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA, transposed_copy=True)
+    sx = mx.mxfp4_scales_to_mma(qx_rm.scales, T, H)
+    sw = mx.mxfp4_scales_to_mma(qw_rm.scales, I, H, two_d=True)
+    swt = mx.mxfp4_scales_to_mma(qw_rm.scales_t, H, I, two_d=True)
+    c_ref = host(mx.mxfp4_gemm(qx.codes, qx.scales, qw.codes, qw.scales, H))
+    c = host(mx.mxfp4_gemm(qx_rm.codes, sx, qw_rm.codes, sw, H))
+    assert np.array_equal(c.view(np.uint32), c_ref.view(np.uint32))
+    # dgrad-style product through the transposed copy and its converted tile scales
+    dy = synth.normal_bf16((T, I), 4, 1e-3)
+    qdy = mx.mxfp4_quantize(dev_bf16(dy), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    d_ref = host(mx.mxfp4_gemm(qdy.codes, qdy.scales, qw.codes_t, qw.scales_t, I))
+    d = host(mx.mxfp4_gemm(qdy.codes, qdy.scales, qw_rm.codes_t, swt, I))
+    assert np.array_equal(d.view(np.uint32), d_ref.view(np.uint32))

@@ -45,10 +45,15 @@ MUTANTS = {
     24: "E4M3 rounding ties to the odd code",
     25: "NVFP4 GEMM drops the per-tensor scales",
     26: "NVFP4 element divisor without the tensor scale",
+    27: "bf16 output rounding ties away from zero",
+    28: "bf16 output truncated instead of rounded",
+    29: "2D dequantize reads the tile scale at the 1D row index",
+    30: "1D-column dequantize swaps the two elements of each byte",
 }
 
 PIN_FILES = ["test_oracle_format.py", "test_oracle_gemm.py", "test_oracle_quantize.py", "test_oracle_rht.py",
-             "test_oracle_sr.py", "test_oracle_scale_rules.py", "test_oracle_nvfp4.py", "test_oracle_philox.py"]
+             "test_oracle_sr.py", "test_oracle_scale_rules.py", "test_oracle_nvfp4.py", "test_oracle_philox.py",
+             "test_oracle_bf16.py"]
 
 
 @pytest.fixture(scope="module")
