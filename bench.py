@@ -164,8 +164,13 @@ class ClockSampler:
 class ExpertStep:
     """Device buffers and the enqueue order of one step (all on the current stream)."""
 
-    def __init__(self, mx, torch, x_bits, w_bits, dy_bits, device):
+    def __init__(self, mx, torch, x_bits, w_bits, dy_bits, device, rank=0, world=1, dw_allreduce=False):
         self.mx, self.torch = mx, torch
+        # data-parallel token split: this rank holds tokens [rank * T, (rank + 1) * T)
+        # of a global batch of world * T; its quantizations are its slice of the
+        # whole batch's (global SR indices), and dW is summed over ranks
+        self.row0, self.total_rows = rank * TOKENS, world * TOKENS
+        self.world, self.dw_allreduce = world, dw_allreduce
         bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(device)
         self.x, self.w, self.dy = bf(x_bits), bf(w_bits), bf(dy_bits)
         T, H, I = TOKENS, HIDDEN, INTER
@@ -182,6 +187,8 @@ class ExpertStep:
 
     def ops(self):
         mx = self.mx
+        if self.world > 1:
+            return self.dp_ops()
         return [
             # X: row blocks (fprop) and blocks along tokens with RHT-32 (wgrad), one read
             ("quant_x_dual", lambda: mx.mxfp4_quantize_dual(self.x, 32, mx.ROUND_RNE, SR_SEED, 0, 0, mx.SCALES_MMA,
@@ -198,6 +205,51 @@ class ExpertStep:
             ("wgrad", lambda: mx.mxfp4_gemm(self.qdyt.codes, self.qdyt.scales, self.qxt.codes, self.qxt.scales,
                                             TOKENS, out=self.dw)),
         ]
+
+
+    def dp_ops(self):
+        """The step of one data-parallel rank: the token-slice forms of the dual
+        quantizers (global SR indices), wgrad before dgrad, and with
+        dw_allreduce the FP32 all-reduce (sum) of dW over ranks on a side stream,
+        overlapping dgrad; the step ends when both have finished."""
+        mx, torch = self.mx, self.torch
+        import torch.distributed as dist
+        if not hasattr(self, "comm_stream"):
+            self.comm_stream = torch.cuda.Stream()
+            self.ev_dw, self.ev_comm = torch.cuda.Event(), torch.cuda.Event()
+
+        def allreduce_start():
+            main = torch.cuda.current_stream()
+            self.ev_dw.record(main)
+            self.comm_stream.wait_event(self.ev_dw)
+            with torch.cuda.stream(self.comm_stream):
+                dist.all_reduce(self.dw, op=dist.ReduceOp.SUM)
+                self.ev_comm.record(self.comm_stream)
+
+        def allreduce_join():
+            torch.cuda.current_stream().wait_event(self.ev_comm)
+
+        ops = [
+            ("quant_x_dual", lambda: mx.mxfp4_quantize_dual_rows(self.x, self.row0, self.total_rows, 32, mx.ROUND_RNE,
+                                                                 SR_SEED, mx.SCALES_MMA, out_row=self.qx,
+                                                                 out_col=self.qxt)),
+            ("quant_w_2d", lambda: mx.mxfp4_quantize(self.w, mx.LAYOUT_2D, 0, mx.ROUND_RNE, 0, 0, mx.SCALES_MMA,
+                                                     out=self.qw)),
+            ("fprop", lambda: mx.mxfp4_gemm(self.qx.codes, self.qx.scales, self.qw.codes, self.qw.scales, HIDDEN,
+                                            out=self.y)),
+            ("quant_dy_dual_sr", lambda: mx.mxfp4_quantize_dual_rows(self.dy, self.row0, self.total_rows, 32,
+                                                                     mx.ROUND_SR, SR_SEED, mx.SCALES_MMA,
+                                                                     out_row=self.qdy, out_col=self.qdyt)),
+            ("wgrad", lambda: mx.mxfp4_gemm(self.qdyt.codes, self.qdyt.scales, self.qxt.codes, self.qxt.scales,
+                                            TOKENS, out=self.dw)),
+        ]
+        if self.dw_allreduce:
+            ops.append(("dw_allreduce_start", allreduce_start))
+        ops.append(("dgrad", lambda: mx.mxfp4_gemm(self.qdy.codes, self.qdy.scales, self.qw.codes_t,
+                                                   self.qw.scales_t, INTER, out=self.dx)))
+        if self.dw_allreduce:
+            ops.append(("dw_allreduce_join", allreduce_join))
+        return ops
 
 
 def rank_inputs(rank: int):
@@ -540,6 +592,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-mib", type=int, default=256)
+    ap.add_argument("--dw-allreduce", action="store_true",
+                    help="N > 1: the data-parallel training step -- the token split of a global batch with an FP32 "
+                         "NCCL all-reduce (sum) of dW every step; without it the ranks run independent steps")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the grouped-MoE GEMM and quantizer-sweep measurements (1-GPU runs only)")
     args = ap.parse_args()
@@ -566,7 +621,8 @@ def main():
     peaks = load_peaks()
 
     x, w, dy = rank_inputs(rank)
-    step = ExpertStep(mx, torch, x, w, dy, device)
+    dp_kw = dict(rank=rank, world=world, dw_allreduce=args.dw_allreduce and world > 1)
+    step = ExpertStep(mx, torch, x, w, dy, device, **dp_kw)
     ops = step.ops()
     flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
@@ -640,6 +696,10 @@ def main():
     gemm_ms = 0.0
     quant_ms, quant_bytes = 0.0, 0.0
     for j, n in enumerate(names):
+        if n.startswith("dw_allreduce"):
+            # the collective's issue (start) and the wait for it after dgrad (join)
+            kernels[n] = {"us": avg_ms[j] * 1e3, "bytes": step.dw.numel() * 4}
+            continue
         if n in GEMMS:
             m_, n_, k_ = GEMMS[n]
             tf = 2 * m_ * n_ * k_ / (avg_ms[j] / 1e3) / 1e12
@@ -690,7 +750,7 @@ def main():
     # read them has finished, its outputs only after their download.
     e2e = None
     if args.e2e_steps > 0:
-        sets = [step, ExpertStep(mx, torch, x, w, dy, device)]
+        sets = [step, ExpertStep(mx, torch, x, w, dy, device, **dp_kw)]
         set_ops = [st.ops() for st in sets]
         hx = step.x.cpu().pin_memory()
         hw = step.w.cpu().pin_memory()
@@ -769,7 +829,9 @@ def main():
                 "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "mxfp4 e2m1/e8m0 operands, fp32 accumulate", "data": "synthetic",
                 "config": {"workload": WORKLOAD, "tokens_per_gpu": TOKENS, "hidden": HIDDEN, "intermediate": INTER,
-                           "parallelism": f"dp{world} (independent tokens per rank, no collective)",
+                           "parallelism": (f"dp{world} (token split of a {world * TOKENS}-token batch; FP32 NCCL "
+                                           f"all-reduce of dW every step, overlapping dgrad)" if dp_kw["dw_allreduce"]
+                                           else f"dp{world} (independent tokens per rank, no collective)"),
                            "l2": f"flushed between timed steps ({args.flush_mib} MiB write, outside step events)"},
                 "roofline": roofline, "roofline_quantize": roofline_q, "roofline_sr_dual": roofline_sr,
                 "kernels": kernels,

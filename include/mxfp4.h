@@ -94,7 +94,8 @@ MXFP4_API const char *mxfp4_status_string(int status);
 
 /* ABI version (major * 100 + minor).  1.01 added mxfp4_gemm_bf16 and
  * mxfp4_grouped_gemm_bf16; 1.02 mxfp4_gemm_mxfp4; 1.03
- * mxfp4_grouped_gemm_wgrad_bf16; 1.04 mxfp4_scales_to_mma. */
+ * mxfp4_grouped_gemm_wgrad_bf16; 1.04 mxfp4_scales_to_mma; 1.05
+ * mxfp4_quantize_dual_rows. */
 MXFP4_API int mxfp4_version(void);
 
 /*
@@ -204,6 +205,36 @@ MXFP4_API int mxfp4_quantize_dual(const void *x, int64_t rows, int64_t cols, int
                                   uint8_t *col_codes, int64_t ld_col_codes,
                                   uint8_t *col_scales, int64_t ld_col_scales,
                                   int scale_layout, void *stream);
+
+/*
+ * mxfp4_quantize_dual_rows -- mxfp4_quantize_dual of the row slice
+ * [row0, row0 + rows) of a [total_rows, cols] tensor, producing exactly the
+ * slice's part of the whole tensor's quantization.  For data-parallel
+ * training that splits tokens across ranks (the ALTO recipe trains
+ * GPT-OSS-20B, "Training an MoE LLM in MXFP4", abstract): each rank quantizes
+ * its own tokens, and its codes and scales equal the whole batch's, stochastic
+ * rounding included.
+ *
+ * x points at the slice's first row ([rows, cols], ld_x).  Row output: rows
+ * [rows, cols/2] with SR indices row0 * cols + (r * cols + c), as
+ * mxfp4_quantize_dual with row_elem_offset = row0 * cols.  Column output: the
+ * whole tensor's column view is [cols, total_rows]; the slice is its column
+ * range [row0, row0 + rows), written as [cols, rows/2] (ld_col_codes) with SR
+ * indices c * total_rows + row0 + r -- which no single element offset can
+ * express.  Column blocks of 32 tokens never straddle two slices because
+ * row0 and total_rows are multiples of 32.  The RHT (col_rht_size) runs along
+ * tokens within each block, as in mxfp4_quantize_dual.
+ *
+ * Requirements: as mxfp4_quantize_dual, plus 0 <= row0, row0 % 32 == 0,
+ * total_rows % 32 == 0, row0 + rows <= total_rows.
+ */
+MXFP4_API int mxfp4_quantize_dual_rows(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int64_t row0,
+                                       int64_t total_rows, int col_rht_size, int rounding, uint64_t seed,
+                                       uint8_t *row_codes, int64_t ld_row_codes,
+                                       uint8_t *row_scales, int64_t ld_row_scales,
+                                       uint8_t *col_codes, int64_t ld_col_codes,
+                                       uint8_t *col_scales, int64_t ld_col_scales,
+                                       int scale_layout, void *stream);
 
 /*
  * mxfp4_dequantize -- MXFP4 codes and scales back to a [rows, cols] tensor.

@@ -76,6 +76,10 @@ def lib():
         L.orc_quantize.argtypes = [ctypes.c_void_p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                    ctypes.c_uint64, ctypes.c_uint64, u8p, i64, u8p, i64, ctypes.c_void_p, i64]
         L.orc_quantize.restype = ctypes.c_int
+        L.orc_quantize_view.argtypes = [ctypes.c_void_p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_uint64, ctypes.c_uint64, i64, u8p, i64, u8p, i64,
+                                        ctypes.c_void_p, i64]
+        L.orc_quantize_view.restype = ctypes.c_int
         L.orc_dequantize.argtypes = [u8p, i64, u8p, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_uint64,
                                      fp, ctypes.c_void_p, i64]
         L.orc_dequantize.restype = ctypes.c_int
@@ -173,11 +177,15 @@ def scale_code_rule(amax: float, rule: int) -> int:
 
 
 def quantize(x_bf16: np.ndarray, layout: int, rht: int = 0, rnd: int = ROUND_RNE, seed: int = 0,
-             elem_offset: int = 0, transposed_copy: bool = False, scale_rule: int = SCALE_FLOOR):
+             elem_offset: int = 0, transposed_copy: bool = False, scale_rule: int = SCALE_FLOOR,
+             sr_ld: int = 0):
     """Quantize a bf16 tensor given as uint16 bit patterns [rows, cols].
 
     Returns (codes, scales) or (codes, scales, codes_t) in the canonical
-    layouts described in the C file (row-major scales).
+    layouts described in the C file (row-major scales).  sr_ld (with
+    elem_offset) places the tensor as a slice of a larger one for the SR
+    stream: the row length of the whole tensor's quantized output view
+    (0 = this tensor's own).
     """
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     rows, cols = x.shape
@@ -191,10 +199,10 @@ def quantize(x_bf16: np.ndarray, layout: int, rht: int = 0, rnd: int = ROUND_RNE
         codes = np.zeros((rows, cols // 2), np.uint8)
         scales = np.zeros((rows, cols // 32), np.uint8)
     codes_t = np.zeros((cols, rows // 2), np.uint8) if (layout == LAYOUT_2D and transposed_copy) else None
-    rc = lib().orc_quantize(x.ctypes.data, rows, cols, cols, layout, rht, rnd, scale_rule, seed, elem_offset,
-                            _ptr(codes, ctypes.c_uint8), codes.shape[1], _ptr(scales, ctypes.c_uint8),
-                            scales.shape[1], codes_t.ctypes.data if codes_t is not None else None,
-                            codes_t.shape[1] if codes_t is not None else 0)
+    rc = lib().orc_quantize_view(x.ctypes.data, rows, cols, cols, layout, rht, rnd, scale_rule, seed, elem_offset,
+                                 sr_ld, _ptr(codes, ctypes.c_uint8), codes.shape[1], _ptr(scales, ctypes.c_uint8),
+                                 scales.shape[1], codes_t.ctypes.data if codes_t is not None else None,
+                                 codes_t.shape[1] if codes_t is not None else 0)
     if rc != 0:
         raise ValueError("oracle: shape not defined for this layout")
     return (codes, scales, codes_t) if codes_t is not None else (codes, scales)

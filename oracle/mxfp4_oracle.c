@@ -395,10 +395,34 @@ uint32_t orc_get_nibble(const uint8_t *row, int64_t pos)
  * linear index in the output view plus elem_offset.  Returns 0, or -1 on a
  * shape the format does not define.
  */
+int orc_quantize_view(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
+                      int layout, int rht, int rnd, int rule, uint64_t seed, uint64_t elem_offset,
+                      int64_t sr_ld, uint8_t *codes, int64_t ld_codes, uint8_t *scales, int64_t ld_scales,
+                      uint8_t *codes_t, int64_t ld_codes_t);
+
 int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
                  int layout, int rht, int rnd, int rule, uint64_t seed, uint64_t elem_offset,
                  uint8_t *codes, int64_t ld_codes, uint8_t *scales, int64_t ld_scales,
                  uint8_t *codes_t, int64_t ld_codes_t)
+{
+    return orc_quantize_view(x, rows, cols, ld_x, layout, rht, rnd, rule, seed, elem_offset, 0,
+                             codes, ld_codes, scales, ld_scales, codes_t, ld_codes_t);
+}
+
+/*
+ * As orc_quantize, for a tensor that is a slice of a larger one (R8: the SR
+ * index is the element's position in the quantized output view of the WHOLE
+ * tensor).  sr_ld is the row length of that whole output view (0: this
+ * tensor's own, ocols); with elem_offset the index of the slice's first
+ * element there, element (orow, ocol) of the slice draws index
+ * orow * sr_ld + ocol + elem_offset.  A slice of tokens (rows of x) in the
+ * 1D-column layout is a column range of the output view: sr_ld = the whole
+ * tensor's rows, elem_offset = the slice's first row.
+ */
+int orc_quantize_view(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
+                      int layout, int rht, int rnd, int rule, uint64_t seed, uint64_t elem_offset,
+                      int64_t sr_ld, uint8_t *codes, int64_t ld_codes, uint8_t *scales, int64_t ld_scales,
+                      uint8_t *codes_t, int64_t ld_codes_t)
 {
     if (rht != 0 && rht != 16 && rht != 32) return -1;
     if (rule < ORC_SCALE_FLOOR || rule > ORC_SCALE_PRESCALE_34) return -1;
@@ -409,6 +433,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
         int transposed = layout == ORC_LAYOUT_1D_COL;
         int64_t orows = transposed ? cols : rows;
         int64_t ocols = transposed ? rows : cols;
+        int64_t gld = sr_ld ? sr_ld : ocols;            /* row length of the whole output view */
         if (ocols % 32) return -1;
         #pragma omp parallel for schedule(static)
         for (int64_t orow = 0; orow < orows; ++orow) {
@@ -421,7 +446,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
                     int64_t r = transposed ? ocol : orow;
                     int64_t c = transposed ? orow : ocol;
                     y[i] = orc_bf16_to_f32(x[r * ld_x + c]);
-                    g[i] = (uint64_t)(MUT(17) ? r * cols + c : orow * ocols + ocol) + (MUT(12) ? 0 : elem_offset);
+                    g[i] = (uint64_t)(MUT(17) ? r * cols + c : orow * gld + ocol) + (MUT(12) ? 0 : elem_offset);
                 }
                 if (rht)
                     for (int s = 0; s < 32; s += rht) orc_rht_forward(y + s, rht, smask);
@@ -446,7 +471,7 @@ int orc_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld_x,
                     for (int j = 0; j < 32; ++j) {
                         int64_t c = bc * 32 + j;
                         y[i * 32 + j] = orc_bf16_to_f32(x[r * ld_x + c]);
-                        g[i * 32 + j] = (uint64_t)(r * cols + c) + elem_offset;
+                        g[i * 32 + j] = (uint64_t)(r * (sr_ld ? sr_ld : cols) + c) + elem_offset;
                     }
                     if (rht)
                         for (int s = 0; s < 32; s += rht) orc_rht_forward(y + i * 32 + s, rht, smask);

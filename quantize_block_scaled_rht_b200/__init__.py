@@ -45,6 +45,7 @@ ABI_FUNCTIONS = (
     "mxfp4_grouped_gemm_wgrad_bf16", "mxfp4_nvfp4_quantize", "mxfp4_nvfp4_dequantize", "mxfp4_nvfp4_gemm",
     "mxfp4_get_error",
     "mxfp4_set_wait_limit_ns", "mxfp4_wait_probe", "mxfp4_scales_to_mma",
+    "mxfp4_quantize_dual_rows",
 )
 
 
@@ -78,6 +79,9 @@ def lib() -> ctypes.CDLL:
         L.mxfp4_quantize_dual.argtypes = [vp, i64, i64, i64, i32, i32, u64, u64, u64, vp, i64, vp, i64, vp, i64,
                                           vp, i64, i32, vp]
         L.mxfp4_quantize_dual.restype = i32
+        L.mxfp4_quantize_dual_rows.argtypes = [vp, i64, i64, i64, i64, i64, i32, i32, u64, vp, i64, vp, i64, vp,
+                                               i64, vp, i64, i32, vp]
+        L.mxfp4_quantize_dual_rows.restype = i32
         L.mxfp4_dequantize.argtypes = [vp, i64, vp, i64, i32, i64, i64, i32, i32, u64, vp, i64, i32, vp]
         L.mxfp4_dequantize.restype = i32
         L.mxfp4_gemm.argtypes = [vp, i64, vp, vp, i64, vp, i64, i64, i64, vp, i64, vp]
@@ -250,6 +254,37 @@ def mxfp4_quantize_dual(x: torch.Tensor, col_rht_size: int = 0, rounding: int = 
         ld(r), _ptr(c.codes) if c else None, c.codes.stride(0) if c else 0, _ptr(c.scales) if c else None, ld(c),
         scale_layout, _stream(stream))
     _check(rc, "mxfp4_quantize_dual")
+    return r, c
+
+
+def mxfp4_quantize_dual_rows(x: torch.Tensor, row0: int, total_rows: int, col_rht_size: int = 0,
+                             rounding: int = ROUND_RNE, seed: int = 0, scale_layout: int = SCALES_ROWMAJOR,
+                             row: bool = True, col: bool = True, stream=None, out_row: Optional[Quantized] = None,
+                             out_col: Optional[Quantized] = None, scale_rule: int = SCALE_FLOOR):
+    """mxfp4_quantize_dual of rows [row0, row0 + x.shape[0]) of a tensor with
+    total_rows rows: the slice's part of the whole tensor's quantization, SR
+    included (see mxfp4_quantize_dual_rows in include/mxfp4.h).  The column
+    output is [cols, rows/2], the slice's columns of the whole [cols,
+    total_rows] view."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a 2-D bfloat16 tensor")
+    rows, cols = x.shape
+    dev = x.device
+    if row and out_row is None:
+        out_row = Quantized(torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev),
+                            _scale_tensor(rows, cols, scale_layout, dev), rows, cols, LAYOUT_1D_ROW, scale_layout)
+    if col and out_col is None:
+        out_col = Quantized(torch.empty((cols, rows // 2), dtype=torch.uint8, device=dev),
+                            _scale_tensor(cols, rows, scale_layout, dev), cols, rows, LAYOUT_1D_COL, scale_layout)
+    r = out_row if row else None
+    c = out_col if col else None
+    ld = lambda q: (q.scales.shape[1] if q.scales.dim() == 2 else 0) if q is not None else 0
+    rc = lib().mxfp4_quantize_dual_rows(
+        _ptr(x), rows, cols, x.stride(0), row0, total_rows, col_rht_size, rounding | scale_rule,
+        seed & 0xFFFFFFFFFFFFFFFF, _ptr(r.codes) if r else None, r.codes.stride(0) if r else 0,
+        _ptr(r.scales) if r else None, ld(r), _ptr(c.codes) if c else None, c.codes.stride(0) if c else 0,
+        _ptr(c.scales) if c else None, ld(c), scale_layout, _stream(stream))
+    _check(rc, "mxfp4_quantize_dual_rows")
     return r, c
 
 

@@ -16,7 +16,7 @@ cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int6
                                  uint64_t seed, uint64_t row_offset, uint64_t col_offset, uint8_t *rcodes,
                                  int64_t ld_rcodes, uint8_t *rscales, int64_t ld_rscales, uint8_t *ccodes,
                                  int64_t ld_ccodes, uint8_t *cscales, int64_t ld_cscales, int scale_layout,
-                                 cudaStream_t s);
+                                 int64_t col_sr_ld, cudaStream_t s);
 cudaError_t launch_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
                               int scale_layout, int64_t rows, int64_t cols, int layout, int rht, uint64_t seed,
                               void *out, int64_t ld_out, int out_dtype, cudaStream_t s);
@@ -76,7 +76,7 @@ const char *mxfp4_status_string(int status) {
     }
 }
 
-int mxfp4_version(void) { return 104; }
+int mxfp4_version(void) { return 105; }
 
 int64_t mxfp4_mma_scales_bytes(int64_t rows, int64_t k) {
     if (rows <= 0 || k <= 0) return 0;
@@ -132,11 +132,42 @@ int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int 
     return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
 }
 
+static int quantize_dual_impl(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int col_rht_size,
+                              int rounding, uint64_t seed, uint64_t row_elem_offset, uint64_t col_elem_offset,
+                              int64_t col_sr_ld, uint8_t *row_codes, int64_t ld_row_codes, uint8_t *row_scales,
+                              int64_t ld_row_scales, uint8_t *col_codes, int64_t ld_col_codes, uint8_t *col_scales,
+                              int64_t ld_col_scales, int scale_layout, void *stream);
+
 int mxfp4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int col_rht_size, int rounding,
                         uint64_t seed, uint64_t row_elem_offset, uint64_t col_elem_offset, uint8_t *row_codes,
                         int64_t ld_row_codes, uint8_t *row_scales, int64_t ld_row_scales, uint8_t *col_codes,
                         int64_t ld_col_codes, uint8_t *col_scales, int64_t ld_col_scales, int scale_layout,
                         void *stream) {
+    return quantize_dual_impl(x, rows, cols, ld_x, col_rht_size, rounding, seed, row_elem_offset, col_elem_offset,
+                              rows, row_codes, ld_row_codes, row_scales, ld_row_scales, col_codes, ld_col_codes,
+                              col_scales, ld_col_scales, scale_layout, stream);
+}
+
+int mxfp4_quantize_dual_rows(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int64_t row0,
+                             int64_t total_rows, int col_rht_size, int rounding, uint64_t seed, uint8_t *row_codes,
+                             int64_t ld_row_codes, uint8_t *row_scales, int64_t ld_row_scales, uint8_t *col_codes,
+                             int64_t ld_col_codes, uint8_t *col_scales, int64_t ld_col_scales, int scale_layout,
+                             void *stream) {
+    if (row0 < 0 || (row0 % 32) || total_rows <= 0 || (total_rows % 32) || rows > total_rows - row0)
+        return MXFP4_ERR_INVALID_ARG;
+    if (cols > 0 && row0 > ((int64_t)1 << 62) / cols) return MXFP4_ERR_UNSUPPORTED;
+    // row output: rows of the whole tensor, offset row0 * cols; column output:
+    // columns of the whole tensor's [cols, total_rows] view from column row0
+    return quantize_dual_impl(x, rows, cols, ld_x, col_rht_size, rounding, seed, (uint64_t)(row0 * cols),
+                              (uint64_t)row0, total_rows, row_codes, ld_row_codes, row_scales, ld_row_scales,
+                              col_codes, ld_col_codes, col_scales, ld_col_scales, scale_layout, stream);
+}
+
+static int quantize_dual_impl(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int col_rht_size,
+                              int rounding, uint64_t seed, uint64_t row_elem_offset, uint64_t col_elem_offset,
+                              int64_t col_sr_ld, uint8_t *row_codes, int64_t ld_row_codes, uint8_t *row_scales,
+                              int64_t ld_row_scales, uint8_t *col_codes, int64_t ld_col_codes, uint8_t *col_scales,
+                              int64_t ld_col_scales, int scale_layout, void *stream) {
     if (!x || (!row_codes && !col_codes)) return MXFP4_ERR_INVALID_ARG;
     if ((row_codes && !row_scales) || (col_codes && !col_scales)) return MXFP4_ERR_INVALID_ARG;
     if (rows <= 0 || cols <= 0 || (rows % 32) || (cols % 32)) return MXFP4_ERR_INVALID_ARG;
@@ -160,7 +191,7 @@ int mxfp4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
         return MXFP4_ERR_ALIGNMENT;
     const cudaError_t e = mxfp4::launch_quantize_dual(
         x, rows, cols, ld_x, col_rht_size, rounding, seed, row_elem_offset, col_elem_offset, row_codes, ld_row_codes,
-        row_scales, ld_row_scales, col_codes, ld_col_codes, col_scales, ld_col_scales, scale_layout,
+        row_scales, ld_row_scales, col_codes, ld_col_codes, col_scales, ld_col_scales, scale_layout, col_sr_ld,
         static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? MXFP4_OK : MXFP4_ERR_CUDA;
 }

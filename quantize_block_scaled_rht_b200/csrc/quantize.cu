@@ -316,6 +316,7 @@ struct DualParams {
     uint32_t seed_lo, seed_hi;
     int scale_rule;                        // MXFP4_SCALE_* >> 4
     uint64_t r_offset, c_offset;           // SR stream index of each output's first element
+    int64_t c_sr_ld;                       // row length of the column output's SR view (the whole tensor's rows)
     uint32_t tiles_c, tiles_r;             // column tiles, row tiles
     uint32_t strip;                        // tiles per strip (1 unless column-only; at most 8)
     uint32_t sgn_bit[32];                  // RHT sign of element i (mod the RHT size) as bit 31
@@ -387,7 +388,7 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualP
                         for (int m = 0; m < 16; ++m) P[m] = mul2(P[m], make_float2(cn, cn));
                     }
                     uint4 q;
-                    const uint64_t g0 = (uint64_t)(orow * p.rows + rin) + p.c_offset;
+                    const uint64_t g0 = (uint64_t)(orow * p.c_sr_ld + rin) + p.c_offset;
                     const uint32_t sc = quantize32_pairs<SR>(P, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
                     tout[c * OCH + (b ^ ((c >> T::OSH) & (OCH - 1)))] = q;
                     const int64_t kb = rin >> 5;
@@ -938,6 +939,7 @@ static cudaError_t launch_col_dual(const QuantParams &q, cudaStream_t s) {
     p.seed_lo = q.seed_lo; p.seed_hi = q.seed_hi;
     p.scale_rule = q.scale_rule;
     p.c_offset = q.elem_offset;
+    p.c_sr_ld = q.rows;
     for (int i = 0; i < 32; ++i) p.sgn_bit[i] = q.sgn_bit[i];
     return launch_dual_t<DualCol, RHT, SR, MMA, false, true>(p, s);
 }
@@ -959,7 +961,7 @@ cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int6
                                  uint64_t seed, uint64_t row_offset, uint64_t col_offset, uint8_t *rcodes,
                                  int64_t ld_rcodes, uint8_t *rscales, int64_t ld_rscales, uint8_t *ccodes,
                                  int64_t ld_ccodes, uint8_t *cscales, int64_t ld_cscales, int scale_layout,
-                                 cudaStream_t s) {
+                                 int64_t col_sr_ld, cudaStream_t s) {
     DualParams p{};
     p.x = static_cast<const uint16_t *>(x);
     p.rows = rows; p.cols = cols; p.ld_x = ld_x;
@@ -969,6 +971,7 @@ cudaError_t launch_quantize_dual(const void *x, int64_t rows, int64_t cols, int6
     p.c_katoms = mma_katoms(rows);
     p.seed_lo = (uint32_t)seed; p.seed_hi = (uint32_t)(seed >> 32);
     p.r_offset = row_offset; p.c_offset = col_offset;
+    p.c_sr_ld = col_sr_ld > 0 ? col_sr_ld : rows;
     uint32_t pair_unused[16];
     fill_signs(col_rht ? rht_sign_mask_hd(seed) : 0u, col_rht, pair_unused, p.sgn_bit);
     const bool sr = (rounding & 0x0F) == MXFP4_ROUND_SR, mma = scale_layout == MXFP4_SCALES_MMA;

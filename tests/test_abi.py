@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 def test_status_strings_and_layout_helpers():
     assert mx.status_string(mx.MXFP4_OK) == "MXFP4_OK"
     assert mx.status_string(mx.MXFP4_ERR_TIMEOUT) == "MXFP4_ERR_TIMEOUT"
-    assert mx.lib().mxfp4_version() == 104
+    assert mx.lib().mxfp4_version() == 105
     # 128 rows x 4 K-blocks per 512-byte atom
     assert mx.mma_scales_bytes(128, 128) == 512
     assert mx.mma_scales_bytes(129, 2880) == 2 * 23 * 512
@@ -142,3 +142,14 @@ def test_gemm_wrappers_reject_rowmajor_scales_before_the_abi():
     for fn in (mx.mxfp4_grouped_gemm_wgrad, mx.mxfp4_grouped_gemm_wgrad_bf16):
         with pytest.raises(ValueError, match="SCALES_MMA"):
             fn(a, a_mma, b, b_rm, offs, K)
+
+
+def test_quantize_dual_rows_rejects_bad_slices_without_gpu():
+    L = mx.lib()
+    fake = ctypes.c_void_p(0x10000)
+    call = lambda row0, total, rows=64: L.mxfp4_quantize_dual_rows(fake, rows, 64, 64, row0, total, 32, 1, 42, fake,
+                                                                   32, fake, 2, fake, 32, fake, 2, 0, None)
+    assert call(16, 256) == mx.MXFP4_ERR_INVALID_ARG        # slice start off a 32-token boundary
+    assert call(0, 240) == mx.MXFP4_ERR_INVALID_ARG         # whole tensor not a multiple of 32 rows
+    assert call(224, 256) == mx.MXFP4_ERR_INVALID_ARG       # slice past the end
+    assert call(-32, 256) == mx.MXFP4_ERR_INVALID_ARG

@@ -220,6 +220,32 @@ def test_dual_single_outputs_and_offsets():
     assert np.array_equal(host(qc.codes), oracle.quantize(x, oracle.LAYOUT_1D_COL, 32, oracle.ROUND_SR, 5, 8)[0])
 
 
+@pytest.mark.parametrize("scale_layout", [mx.SCALES_ROWMAJOR, mx.SCALES_MMA])
+@pytest.mark.parametrize("rnd", [mx.ROUND_RNE, mx.ROUND_SR])
+def test_dual_rows_token_slices_equal_the_whole(rnd, scale_layout):
+    """Data-parallel token split: each slice quantized with
+    mxfp4_quantize_dual_rows equals its part of the whole tensor's dual
+    quantization (row blocks: its rows; column blocks along tokens with RHT-32:
+    its token columns), bit for bit, SR included; and both equal the oracle
+    run on the slice with the whole view's row length."""
+    T, C = 384, 320
+    x = synth.student_t_bf16((T, C), seed=77)
+    xd = dev_bf16(x)
+    wr, wc = mx.mxfp4_quantize_dual(xd, 32, rnd, 42)
+    wrc, wrs, wcc, wcs = host(wr.codes), host(wr.scales), host(wc.codes), host(wc.scales)
+    for t0, n in ((0, 128), (128, 96), (224, 160)):
+        qr, qc = mx.mxfp4_quantize_dual_rows(xd[t0:t0 + n], t0, T, 32, rnd, 42, scale_layout=scale_layout)
+        assert np.array_equal(host(qr.codes), wrc[t0:t0 + n])
+        assert np.array_equal(host(qc.codes), wcc[:, t0 // 2:(t0 + n) // 2])
+        sr_, sc = host(qr.scales), host(qc.scales)
+        if scale_layout == mx.SCALES_MMA:
+            sr_, sc = from_mma(sr_, n, C), from_mma(sc, C, n)
+        assert np.array_equal(sr_, wrs[t0:t0 + n]) and np.array_equal(sc, wcs[:, t0 // 32:(t0 + n) // 32])
+        part = np.ascontiguousarray(x[t0:t0 + n])
+        oc, os_ = oracle.quantize(part, oracle.LAYOUT_1D_COL, 32, rnd, 42, elem_offset=t0, sr_ld=T)
+        assert np.array_equal(host(qc.codes), oc) and np.array_equal(sc, os_)
+
+
 RULES = [(mx.SCALE_ROUNDUP, oracle.SCALE_ROUNDUP), (mx.SCALE_PRESCALE_34, oracle.SCALE_PRESCALE_34)]
 
 

@@ -126,6 +126,30 @@ def test_sharded_sr_with_offsets_equals_whole(layout):
         assert np.array_equal(w, np.concatenate([pa, pb], axis=0))
 
 
+@pytest.mark.parametrize("rnd", [oracle.ROUND_RNE, oracle.ROUND_SR])
+def test_token_slices_of_column_layout_equal_the_whole(rnd):
+    """A slice of tokens (rows of x) quantized along tokens is a column range of
+    the whole tensor's output view: with the whole view's row length (sr_ld =
+    total tokens) and the slice's first token as offset, every slice draws the
+    whole tensor's SR words (reading R8), so the slices' codes and scales are the
+    whole's, bit for bit.  Row blocks of the same slice need only the offset."""
+    x = synth.student_t_bf16((256, 96), seed=23)
+    whole_c, whole_s = oracle.quantize(x, oracle.LAYOUT_1D_COL, 32, rnd, seed=42)
+    whole_rc, whole_rs = oracle.quantize(x, oracle.LAYOUT_1D_ROW, 0, rnd, seed=42)
+    for t0, n in ((0, 64), (64, 128), (192, 64)):
+        part = np.ascontiguousarray(x[t0:t0 + n])
+        c, s = oracle.quantize(part, oracle.LAYOUT_1D_COL, 32, rnd, seed=42, elem_offset=t0, sr_ld=256)
+        assert np.array_equal(c, whole_c[:, t0 // 2:(t0 + n) // 2])
+        assert np.array_equal(s, whole_s[:, t0 // 32:(t0 + n) // 32])
+        rc, rs = oracle.quantize(part, oracle.LAYOUT_1D_ROW, 0, rnd, seed=42, elem_offset=t0 * 96)
+        assert np.array_equal(rc, whole_rc[t0:t0 + n]) and np.array_equal(rs, whole_rs[t0:t0 + n])
+    if rnd == oracle.ROUND_SR:
+        # without the whole view's row length the slice draws other words
+        c, _ = oracle.quantize(np.ascontiguousarray(x[64:192]), oracle.LAYOUT_1D_COL, 32, rnd, seed=42,
+                               elem_offset=64)
+        assert not np.array_equal(c, whole_c[:, 32:96])
+
+
 @pytest.mark.parametrize("rht", [16, 32])
 def test_dequantize_inverts_rht(rht):
     x = synth.normal_bf16((32, 64), 5)
