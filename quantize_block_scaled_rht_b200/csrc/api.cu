@@ -4,6 +4,7 @@
 #include <cstdint>
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 
@@ -60,6 +61,16 @@ uint64_t set_wait_limit(uint64_t ns);
 
 namespace {
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// An NVTX range around each entry point that enqueues work, so a profiler's
+// timeline shows the library call that launched each kernel.  Without a tool
+// attached NVTX calls return at once.
+struct Range {
+    explicit Range(const char *name) { nvtxRangePushA(name); }
+    ~Range() { nvtxRangePop(); }
+    Range(const Range &) = delete;
+    Range &operator=(const Range &) = delete;
+};
 }  // namespace
 
 extern "C" {
@@ -99,6 +110,7 @@ int mxfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int 
                    uint64_t seed, uint64_t elem_offset, uint8_t *codes, int64_t ld_codes, uint8_t *scales,
                    int64_t ld_scales, int scale_layout, uint8_t *codes_t, int64_t ld_codes_t, uint8_t *scales_t,
                    int64_t ld_scales_t, void *stream) {
+    Range range_("mxfp4_quantize");
     if (!x || !codes || !scales) return MXFP4_ERR_INVALID_ARG;
     if (rows <= 0 || cols <= 0) return MXFP4_ERR_INVALID_ARG;
     if (layout != MXFP4_LAYOUT_1D_ROW && layout != MXFP4_LAYOUT_1D_COL && layout != MXFP4_LAYOUT_2D)
@@ -143,6 +155,7 @@ int mxfp4_quantize_dual(const void *x, int64_t rows, int64_t cols, int64_t ld_x,
                         int64_t ld_row_codes, uint8_t *row_scales, int64_t ld_row_scales, uint8_t *col_codes,
                         int64_t ld_col_codes, uint8_t *col_scales, int64_t ld_col_scales, int scale_layout,
                         void *stream) {
+    Range range_("mxfp4_quantize_dual");
     return quantize_dual_impl(x, rows, cols, ld_x, col_rht_size, rounding, seed, row_elem_offset, col_elem_offset,
                               rows, row_codes, ld_row_codes, row_scales, ld_row_scales, col_codes, ld_col_codes,
                               col_scales, ld_col_scales, scale_layout, stream);
@@ -153,6 +166,7 @@ int mxfp4_quantize_dual_rows(const void *x, int64_t rows, int64_t cols, int64_t 
                              int64_t ld_row_codes, uint8_t *row_scales, int64_t ld_row_scales, uint8_t *col_codes,
                              int64_t ld_col_codes, uint8_t *col_scales, int64_t ld_col_scales, int scale_layout,
                              void *stream) {
+    Range range_("mxfp4_quantize_dual_rows");
     if (row0 < 0 || (row0 % 32) || total_rows <= 0 || (total_rows % 32) || rows > total_rows - row0)
         return MXFP4_ERR_INVALID_ARG;
     if (cols > 0 && row0 > ((int64_t)1 << 62) / cols) return MXFP4_ERR_UNSUPPORTED;
@@ -199,6 +213,7 @@ static int quantize_dual_impl(const void *x, int64_t rows, int64_t cols, int64_t
 int mxfp4_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
                      int scale_layout, int64_t rows, int64_t cols, int layout, int rht_size, uint64_t seed,
                      void *out, int64_t ld_out, int out_dtype, void *stream) {
+    Range range_("mxfp4_dequantize");
     if (!codes || !scales || !out) return MXFP4_ERR_INVALID_ARG;
     if (rows <= 0 || cols <= 0) return MXFP4_ERR_INVALID_ARG;
     if (layout != MXFP4_LAYOUT_1D_ROW && layout != MXFP4_LAYOUT_1D_COL && layout != MXFP4_LAYOUT_2D)
@@ -241,6 +256,7 @@ static int check_gemm_common(const uint8_t *a_codes, int64_t lda, const uint8_t 
 
 int mxfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes, int64_t ldb,
                const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, float *c, int64_t ldc, void *stream) {
+    Range range_("mxfp4_gemm");
     if (M <= 0) return MXFP4_ERR_INVALID_ARG;
     const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc);
     if (rc != MXFP4_OK) return rc;
@@ -253,6 +269,7 @@ int mxfp4_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_sca
                        const int32_t *group_offsets, const int32_t *group_sizes, int num_groups,
                        const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K, float *c,
                        int64_t ldc, void *stream) {
+    Range range_("mxfp4_grouped_gemm");
     if (!group_offsets || !group_sizes) return MXFP4_ERR_INVALID_ARG;
     if (num_groups <= 0 || a_rows <= 0) return MXFP4_ERR_INVALID_ARG;
     if (num_groups > 1024) return MXFP4_ERR_UNSUPPORTED;
@@ -266,6 +283,7 @@ int mxfp4_grouped_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_sca
 int mxfp4_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
                     int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint16_t *c, int64_t ldc,
                     void *stream) {
+    Range range_("mxfp4_gemm_bf16");
     if (M <= 0) return MXFP4_ERR_INVALID_ARG;
     const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc, 2);
     if (rc != MXFP4_OK) return rc;
@@ -277,6 +295,7 @@ int mxfp4_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales
 int mxfp4_gemm_mxfp4(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
                      int64_t ldb, const uint8_t *b_scales, int64_t M, int64_t N, int64_t K, uint8_t *c_codes,
                      int64_t ld_c_codes, uint8_t *c_scales, int64_t ld_c_scales, int c_scale_layout, void *stream) {
+    Range range_("mxfp4_gemm_mxfp4");
     if (!a_codes || !a_scales || !b_codes || !b_scales || !c_codes || !c_scales) return MXFP4_ERR_INVALID_ARG;
     if (M <= 0 || N <= 0 || K <= 0 || (N % 32) || (K % 32)) return MXFP4_ERR_INVALID_ARG;
     if (c_scale_layout != MXFP4_SCALES_ROWMAJOR && c_scale_layout != MXFP4_SCALES_MMA) return MXFP4_ERR_INVALID_ARG;
@@ -296,6 +315,7 @@ int mxfp4_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *
                             const int32_t *group_offsets, const int32_t *group_sizes, int num_groups,
                             const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, int64_t N, int64_t K,
                             uint16_t *c, int64_t ldc, void *stream) {
+    Range range_("mxfp4_grouped_gemm_bf16");
     if (!group_offsets || !group_sizes) return MXFP4_ERR_INVALID_ARG;
     if (num_groups <= 0 || a_rows <= 0) return MXFP4_ERR_INVALID_ARG;
     if (num_groups > 1024) return MXFP4_ERR_UNSUPPORTED;
@@ -309,6 +329,7 @@ int mxfp4_grouped_gemm_bf16(const uint8_t *a_codes, int64_t lda, const uint8_t *
 int mxfp4_grouped_gemm_wgrad(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const uint8_t *b_codes,
                              int64_t ldb, const uint8_t *b_scales, const int32_t *group_offsets, int num_groups,
                              int64_t M, int64_t N, int64_t K, float *c, int64_t ldc, void *stream) {
+    Range range_("mxfp4_grouped_gemm_wgrad");
     if (!group_offsets || num_groups <= 0 || M <= 0) return MXFP4_ERR_INVALID_ARG;
     if (num_groups > 1024) return MXFP4_ERR_UNSUPPORTED;
     const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc);
@@ -323,6 +344,7 @@ int mxfp4_grouped_gemm_wgrad_bf16(const uint8_t *a_codes, int64_t lda, const uin
                                   const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales,
                                   const int32_t *group_offsets, int num_groups, int64_t M, int64_t N, int64_t K,
                                   uint16_t *c, int64_t ldc, void *stream) {
+    Range range_("mxfp4_grouped_gemm_wgrad_bf16");
     if (!group_offsets || num_groups <= 0 || M <= 0) return MXFP4_ERR_INVALID_ARG;
     if (num_groups > 1024) return MXFP4_ERR_UNSUPPORTED;
     const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc, 2);
@@ -336,6 +358,7 @@ int mxfp4_grouped_gemm_wgrad_bf16(const uint8_t *a_codes, int64_t lda, const uin
 int mxfp4_nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x, int layout, int rounding,
                          uint64_t seed, uint64_t elem_offset, float *tensor_amax, uint8_t *codes, int64_t ld_codes,
                          uint8_t *scales, int64_t ld_scales, int scale_layout, void *stream) {
+    Range range_("mxfp4_nvfp4_quantize");
     if (!x || !codes || !scales || !tensor_amax) return MXFP4_ERR_INVALID_ARG;
     if (rows <= 0 || cols <= 0) return MXFP4_ERR_INVALID_ARG;
     if (layout != MXFP4_LAYOUT_1D_ROW && layout != MXFP4_LAYOUT_1D_COL) return MXFP4_ERR_INVALID_ARG;
@@ -359,6 +382,7 @@ int mxfp4_nvfp4_quantize(const void *x, int64_t rows, int64_t cols, int64_t ld_x
 int mxfp4_nvfp4_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t *scales, int64_t ld_scales,
                            int scale_layout, const float *tensor_amax, int64_t rows, int64_t cols, int layout,
                            float *out, int64_t ld_out, void *stream) {
+    Range range_("mxfp4_nvfp4_dequantize");
     if (!codes || !scales || !tensor_amax || !out) return MXFP4_ERR_INVALID_ARG;
     if (rows <= 0 || cols <= 0 || rows % 16 || cols % 16) return MXFP4_ERR_INVALID_ARG;
     if (layout != MXFP4_LAYOUT_1D_ROW && layout != MXFP4_LAYOUT_1D_COL) return MXFP4_ERR_INVALID_ARG;
@@ -378,6 +402,7 @@ int mxfp4_nvfp4_dequantize(const uint8_t *codes, int64_t ld_codes, const uint8_t
 int mxfp4_nvfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scales, const float *a_amax,
                      const uint8_t *b_codes, int64_t ldb, const uint8_t *b_scales, const float *b_amax, int64_t M,
                      int64_t N, int64_t K, float *c, int64_t ldc, void *stream) {
+    Range range_("mxfp4_nvfp4_gemm");
     if (M <= 0 || !a_amax || !b_amax) return MXFP4_ERR_INVALID_ARG;
     const int rc = check_gemm_common(a_codes, lda, a_scales, b_codes, ldb, b_scales, N, K, c, ldc);
     if (rc != MXFP4_OK) return rc;
@@ -388,6 +413,7 @@ int mxfp4_nvfp4_gemm(const uint8_t *a_codes, int64_t lda, const uint8_t *a_scale
 
 int mxfp4_scales_to_mma(const uint8_t *scales, int64_t ld_scales, int64_t rows, int64_t k, int two_d,
                         uint8_t *mma_scales, void *stream) {
+    Range range_("mxfp4_scales_to_mma");
     if (!scales || !mma_scales) return MXFP4_ERR_INVALID_ARG;
     if (rows <= 0 || k <= 0 || (k % 32) || (two_d != 0 && two_d != 1)) return MXFP4_ERR_INVALID_ARG;
     if (two_d && (rows % 32)) return MXFP4_ERR_INVALID_ARG;
@@ -404,6 +430,7 @@ int mxfp4_get_error(void *stream) { return mxfp4::get_error(static_cast<cudaStre
 uint64_t mxfp4_set_wait_limit_ns(uint64_t limit_ns) { return mxfp4::set_wait_limit(limit_ns); }
 
 int mxfp4_wait_probe(int arrive, void *stream) {
+    Range range_("mxfp4_wait_probe");
     return mxfp4::launch_wait_probe(arrive, static_cast<cudaStream_t>(stream));
 }
 
