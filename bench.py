@@ -472,45 +472,88 @@ def grouped_bench(mx, torch, device, peaks, reps=10):
     return out
 
 
-def sweep_bench(mx, torch, device, peaks, nbytes=1 << 30, reps=5):
-    """Quantize and dequantize (bf16 out) of a 1 GiB bf16 tensor [186368 x 2880]
-    of Student-t(3) values with 0.1% outliers x100 (drawn on the device), every
-    layout x RHT size x rounding.  Algorithmic bytes per element: 2 read + 0.5
-    + 1/32 written (1D; 2D: + 1/1024), and the reverse for dequantize.  The
-    tensor exceeds L2, so no flush is needed between launches."""
-    rows, cols = synth.sweep_shape(nbytes, 2880)
+def _timed_flushed(torch, fn, reps, flush):
+    """Median time (ms) of `reps` launches, L2 flushed before each (outside the
+    events), events on the current stream."""
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    return float(np.median([a.elapsed_time(b) for a, b in ts]))
+
+
+SWEEP_MIB = (64, 128, 256, 512, 1024, 2048)
+SWEEP_COLS = (2880, 5760)
+
+
+def sweep_bench(mx, torch, device, peaks, sizes_mib=SWEEP_MIB, widths=SWEEP_COLS, reps=5):
+    """The quantizer bandwidth sweep: bf16 tensors of 64 MiB to 2 GiB with rows
+    of 2880 and of 5760 elements (rows rounded down to a multiple of 32) of
+    Student-t(3) values with 0.1% outliers x100 (drawn on the device, seed 7);
+    every layout x RHT size x rounding, quantize and then dequantize (bf16
+    out).  Algorithmic bytes per element: 2 read + 0.5 + 1/32 written (1D;
+    2D: + 1/1024), and the reverse for dequantize.  L2 is flushed before every
+    launch, so the tensors that fit in L2 are timed from HBM too.  Each mode
+    maps to [quantize GB/s, fraction of HBM, dequantize GB/s, fraction]."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    hbm = peaks["hbm"]
+    table = {}
+    worst = {}
+    for cols in widths:
+        for mib in sizes_mib:
+            rows, _ = synth.sweep_shape(mib << 20, cols)
+            x = synth.student_t_bf16_device(rows, cols, seed=7, device=device)
+            n = rows * cols
+            out = torch.empty_like(x)
+            res = {}
+            for layout, lname in ((mx.LAYOUT_1D_ROW, "row"), (mx.LAYOUT_1D_COL, "col"), (mx.LAYOUT_2D, "2d")):
+                sbytes = 1 / 1024 if layout == mx.LAYOUT_2D else 1 / 32
+                for rht in (0, 16, 32):
+                    for rnd, rname in ((mx.ROUND_RNE, "rne"), (mx.ROUND_SR, "sr")):
+                        q = mx.mxfp4_quantize(x, layout, rht, rnd, 42)
+                        tq = _timed_flushed(torch, lambda: mx.mxfp4_quantize(x, layout, rht, rnd, 42, out=q), reps,
+                                            flush)
+                        td = _timed_flushed(torch, lambda: mx.mxfp4_dequantize(q.codes, q.scales, rows, cols, layout,
+                                                                               rht, 42, out=out), reps, flush)
+                        gq = n * (2 + 0.5 + sbytes) / (tq / 1e3) / 1e9
+                        gd = n * (2 + 0.5 + sbytes) / (td / 1e3) / 1e9
+                        key = f"{lname}_rht{rht}_{rname}"
+                        res[key] = [round(gq), round(gq / hbm, 3), round(gd), round(gd / hbm, 3)]
+                        w = worst.setdefault(key, [1e9, 1e9])
+                        w[0], w[1] = min(w[0], gq / hbm), min(w[1], gd / hbm)
+                        del q
+            table[f"{mib}MiB_x{cols}"] = {"shape": f"{rows} x {cols}", "modes": res}
+            del x, out
+            torch.cuda.empty_cache()
+    # the scale-rule variants cost no extra traffic; measured on the 1D-row and
+    # 2D RNE paths at 1 GiB x 2880
+    rows, cols = synth.sweep_shape(1 << 30, 2880)
     x = synth.student_t_bf16_device(rows, cols, seed=7, device=device)
     n = rows * cols
-    res = {}
-    out = torch.empty_like(x)
-    for layout, lname in ((mx.LAYOUT_1D_ROW, "row"), (mx.LAYOUT_1D_COL, "col"), (mx.LAYOUT_2D, "2d")):
-        sbytes = 1 / 1024 if layout == mx.LAYOUT_2D else 1 / 32
-        for rht in (0, 16, 32):
-            for rnd, rname in ((mx.ROUND_RNE, "rne"), (mx.ROUND_SR, "sr")):
-                q = mx.mxfp4_quantize(x, layout, rht, rnd, 42)
-                tq = _timed(torch, lambda: mx.mxfp4_quantize(x, layout, rht, rnd, 42, out=q), reps)
-                td = _timed(torch, lambda: mx.mxfp4_dequantize(q.codes, q.scales, rows, cols, layout, rht, 42,
-                                                               out=out), reps)
-                gq = n * (2 + 0.5 + sbytes) / (tq / 1e3) / 1e9
-                gd = n * (2 + 0.5 + sbytes) / (td / 1e3) / 1e9
-                res[f"{lname}_rht{rht}_{rname}"] = {"quant_GBps": round(gq), "quant_frac_hbm": round(gq / peaks["hbm"], 3),
-                                                    "dequant_GBps": round(gd),
-                                                    "dequant_frac_hbm": round(gd / peaks["hbm"], 3)}
-                del q
-    # the scale-rule variants cost no extra traffic; measured on the 1D-row and 2D RNE paths
+    rules = {}
     for layout, lname in ((mx.LAYOUT_1D_ROW, "row"), (mx.LAYOUT_2D, "2d")):
         sbytes = 1 / 1024 if layout == mx.LAYOUT_2D else 1 / 32
         for rule, rname in ((mx.SCALE_ROUNDUP, "roundup"), (mx.SCALE_PRESCALE_34, "prescale34")):
             q = mx.mxfp4_quantize(x, layout, 0, mx.ROUND_RNE, 42, scale_rule=rule)
-            tq = _timed(torch, lambda: mx.mxfp4_quantize(x, layout, 0, mx.ROUND_RNE, 42, out=q, scale_rule=rule), reps)
+            tq = _timed_flushed(torch, lambda: mx.mxfp4_quantize(x, layout, 0, mx.ROUND_RNE, 42, out=q,
+                                                                 scale_rule=rule), reps, flush)
             gq = n * (2 + 0.5 + sbytes) / (tq / 1e3) / 1e9
-            res[f"{lname}_rht0_rne_{rname}"] = {"quant_GBps": round(gq), "quant_frac_hbm": round(gq / peaks["hbm"], 3)}
+            rules[f"{lname}_rht0_rne_{rname}"] = [round(gq), round(gq / hbm, 3)]
             del q
     if mx.mxfp4_get_error() != mx.MXFP4_OK:
         raise RuntimeError("device-side error in the sweep")
-    del x, out
+    del x, flush
     torch.cuda.empty_cache()
-    return {"tensor": f"{rows} x {cols} bf16 ({nbytes >> 20} MiB)", "modes": res,
+    return {"sizes": table, "scale_rules_1GiB_x2880": rules,
+            "worst_frac_over_sizes": {k: [round(a, 3), round(b, 3)] for k, (a, b) in worst.items()},
+            "columns": "mode: [quantize GB/s, fraction of HBM, dequantize GB/s, fraction of HBM]",
             "note": "SR modes are bound by the integer work of Philox4x32-10 and the exact SR decision, not HBM"}
 
 

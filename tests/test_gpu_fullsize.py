@@ -38,7 +38,7 @@ def expert_step():
     import bench
     x, w, dy = bench.rank_inputs(0)
     step = bench.ExpertStep(mx, torch, x, w, dy, torch.device("cuda"))
-    for _, fn in step.ops():
+    for _, fn in step.overlapped_ops():      # the schedule the bench times
         fn()
     torch.cuda.synchronize()
     assert mx.mxfp4_get_error() == mx.MXFP4_OK
@@ -136,6 +136,52 @@ def test_grouped_moe_gate_up_sampled(moe):
         ref, s = oracle.gemm_entries(ca, sa, cw, sw, K, pairs, 0, 1)
         got = np.array([c[m, nn] for m, nn in pairs], np.float64)
         assert_gemm_close(got, ref, s)
+
+
+def test_expert_dgrad_full_tensor(expert_step):
+    """Every entry of the dgrad output (4096 x 2880, K = 5760, the longest
+    reduction of the step) against the oracle's fp64 GEMM of the oracle's own
+    quantization of dY (row blocks, SR) and of W (2D, transposed copy)."""
+    x, w, dy, st = expert_step
+    T, H, I = synth.TOKENS, synth.HIDDEN, synth.INTERMEDIATE
+    _, sw, cwt = oracle.quantize(w, oracle.LAYOUT_2D, transposed_copy=True)
+    cdy, sdy = oracle.quantize(dy, oracle.LAYOUT_1D_ROW, 0, oracle.ROUND_SR, synth.SR_SEED)
+    ref, s = oracle.gemm(cdy, sdy, cwt, sw, I, 0, 2)
+    worst = assert_gemm_close(host(st.dx), ref, s)
+    assert worst < 1e-5
+
+
+def test_grouped_moe_down_sampled(moe):
+    """The MoE down projection at full size: 16384 tokens routed top-4 of 32
+    experts (65,536 routed rows, groups padded to 128), 2880 -> 2880 per
+    expert, activations 1D row RNE, weights 2D RNE, FP32 out; every expert
+    sampled (rows including its first and last, random columns)."""
+    d = moe
+    E, H = synth.EXPERTS, synth.HIDDEN
+    qa = mx.mxfp4_quantize(dev_bf16(d["a"]), mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
+    wq = [mx.mxfp4_quantize(dev_bf16(d["w_down"][e]), mx.LAYOUT_2D, scale_layout=mx.SCALES_MMA) for e in range(E)]
+    offsets = torch.from_numpy(d["offsets"]).cuda()
+    sizes = torch.from_numpy(d["sizes"]).cuda()
+    c = mx.mxfp4_grouped_gemm(qa.codes, qa.scales, offsets, sizes, torch.stack([q.codes for q in wq]),
+                              torch.cat([q.scales for q in wq]), H, H)
+    assert mx.mxfp4_get_error() == mx.MXFP4_OK
+    c = host(c)
+    del wq
+    ca, sa = oracle.quantize(d["a"], oracle.LAYOUT_1D_ROW)
+    g = np.random.default_rng(7)
+    checked = 0
+    for e in range(E):
+        o, n = int(d["offsets"][e]), int(d["sizes"][e])
+        if n == 0:
+            continue
+        cw, sw = oracle.quantize(d["w_down"][e], oracle.LAYOUT_2D)
+        rs = np.unique(np.concatenate([g.integers(0, n, 12), [0, n - 1]]))
+        pairs = [(int(o + r), int(cc)) for r in rs for cc in list(g.integers(0, H, 8)) + [0, H - 1]]
+        ref, s = oracle.gemm_entries(ca, sa, cw, sw, H, pairs, 0, 1)
+        got = np.array([c[m, nn] for m, nn in pairs], np.float64)
+        assert_gemm_close(got, ref, s)
+        checked += 1
+    assert checked >= 16
 
 
 def test_grouped_moe_backward_sampled(moe):
