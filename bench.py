@@ -185,31 +185,6 @@ class ExpertStep:
         self.qxt = Q(u8(H, T // 2), u8(msb(H, T)), H, T, mx.LAYOUT_1D_COL, mx.SCALES_MMA)
         self.y, self.dx, self.dw = f32(T, I), f32(T, H), f32(I, H)
 
-    def overlapped_ops(self):
-        """The same six launches with the dY quantizer on a side stream: it
-        depends only on dY, and its integer-bound work runs beside the X and W
-        quantizers (latency- and tail-bound at these sizes).  The GEMMs start
-        after both streams join, so they run alone on the SMs."""
-        torch = self.torch
-        if not hasattr(self, "side"):
-            self.side = torch.cuda.Stream()
-            self.ev_fork, self.ev_dy = torch.cuda.Event(), torch.cuda.Event()
-        named = dict(self.ops())
-
-        def fork():
-            self.ev_fork.record(torch.cuda.current_stream())
-            self.side.wait_event(self.ev_fork)
-            with torch.cuda.stream(self.side):
-                named["quant_dy_dual_sr"]()
-                self.ev_dy.record(self.side)
-
-        def join():
-            torch.cuda.current_stream().wait_event(self.ev_dy)
-
-        return [("fork_quant_dy_dual_sr", fork), ("quant_x_dual", named["quant_x_dual"]),
-                ("quant_w_2d", named["quant_w_2d"]), ("join", join), ("fprop", named["fprop"]),
-                ("dgrad", named["dgrad"]), ("wgrad", named["wgrad"])]
-
     def ops(self):
         mx = self.mx
         if self.world > 1:
@@ -663,8 +638,10 @@ def main():
     ap.add_argument("--dw-allreduce", action="store_true",
                     help="N > 1: the data-parallel training step -- the token split of a global batch with an FP32 "
                          "NCCL all-reduce (sum) of dW every step; without it the ranks run independent steps")
-    ap.add_argument("--serial-step", action="store_true",
-                    help="run the step's six launches in one stream (no quantizer overlap)")
+    ap.add_argument("--ncu-case", default=None,
+                    help="profiling case for one ncu capture: run the step once to build the operands, then the named "
+                         "launch of the step (fprop, dgrad, wgrad, quant_x_dual, quant_w_2d, quant_dy_dual_sr) "
+                         "--steps times, and exit without timing or a JSON line")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the grouped-MoE GEMM and quantizer-sweep measurements (1-GPU runs only)")
     args = ap.parse_args()
@@ -694,15 +671,27 @@ def main():
     dp_kw = dict(rank=rank, world=world, dw_allreduce=args.dw_allreduce and world > 1)
     step = ExpertStep(mx, torch, x, w, dy, device, **dp_kw)
     ops = step.ops()
-    # the timed step overlaps the dY quantizer with the X and W quantizers (one
-    # GPU, independent steps); the breakdown pass runs the launches one by one
-    overlap = world == 1 and not args.serial_step
-    step_ops = step.overlapped_ops() if overlap else ops
+    if args.ncu_case is not None:
+        named = dict(ops)
+        if args.ncu_case not in named:
+            ap.error(f"--ncu-case must be one of {sorted(named)}")
+        for _, fn in ops:
+            fn()
+        torch.cuda.synchronize()
+        for _ in range(args.steps):
+            named[args.ncu_case]()
+        torch.cuda.synchronize()
+        if mx.mxfp4_get_error() != mx.MXFP4_OK:
+            raise RuntimeError("device-side error in the profiling case")
+        print(f"ncu case {args.ncu_case}: {args.steps} launches after one step", flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
-        for _, fn in step_ops:
+        for _, fn in ops:
             fn()
     torch.cuda.synchronize()
     if mx.mxfp4_get_error() != mx.MXFP4_OK:
@@ -722,7 +711,7 @@ def main():
             flush.zero_()                               # L2 flush between timed steps (outside the step)
             e = evs[i]
             e[0].record(stream)
-            for j, (_, fn) in enumerate(ops if per_op else step_ops):
+            for j, (_, fn) in enumerate(ops):
                 fn()
                 if per_op:
                     e[j + 1].record(stream)
@@ -825,7 +814,7 @@ def main():
     e2e = None
     if args.e2e_steps > 0:
         sets = [step, ExpertStep(mx, torch, x, w, dy, device, **dp_kw)]
-        set_ops = [st.overlapped_ops() if overlap else st.ops() for st in sets]
+        set_ops = [st.ops() for st in sets]
         hx = step.x.cpu().pin_memory()
         hw = step.w.cpu().pin_memory()
         hdy = step.dy.cpu().pin_memory()
@@ -912,8 +901,6 @@ def main():
                 "quantize_GBps": quant_gbs, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": KERNELS_PER_STEP * K, "clocks": clocks, "wall_s_timed_region": t_wall,
                 "breakdown": f"per-kernel figures from {KB} further steps with an event after every kernel",
-                "step_schedule": ("dY quantizer on a side stream beside the X and W quantizers, GEMMs after the join"
-                                  if overlap else "six launches in one stream"),
                 **extras}
         print(json.dumps(line), flush=True)
     if world > 1:

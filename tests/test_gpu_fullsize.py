@@ -38,7 +38,7 @@ def expert_step():
     import bench
     x, w, dy = bench.rank_inputs(0)
     step = bench.ExpertStep(mx, torch, x, w, dy, torch.device("cuda"))
-    for _, fn in step.overlapped_ops():      # the schedule the bench times
+    for _, fn in step.ops():
         fn()
     torch.cuda.synchronize()
     assert mx.mxfp4_get_error() == mx.MXFP4_OK
