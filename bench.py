@@ -671,6 +671,25 @@ def main():
     dp_kw = dict(rank=rank, world=world, dw_allreduce=args.dw_allreduce and world > 1)
     step = ExpertStep(mx, torch, x, w, dy, device, **dp_kw)
     ops = step.ops()
+    if args.ncu_case is not None and args.ncu_case.startswith("sweep:"):
+        # sweep:<row|col|2d>:<rht>:<rne|sr>:<quant|dequant>:<MiB>[:<cols>] -- one
+        # quantizer-sweep launch on a tensor of that size (drawn on the device)
+        _, lname, rht, rname, what, mib, *rest = args.ncu_case.split(":")
+        layout = {"row": mx.LAYOUT_1D_ROW, "col": mx.LAYOUT_1D_COL, "2d": mx.LAYOUT_2D}[lname]
+        rnd = {"rne": mx.ROUND_RNE, "sr": mx.ROUND_SR}[rname]
+        rows, cols = synth.sweep_shape(int(mib) << 20, int(rest[0]) if rest else 2880)
+        xs = synth.student_t_bf16_device(rows, cols, seed=7, device=device)
+        q = mx.mxfp4_quantize(xs, layout, int(rht), rnd, 42)
+        out = torch.empty_like(xs)
+        fn = ((lambda: mx.mxfp4_quantize(xs, layout, int(rht), rnd, 42, out=q)) if what == "quant" else
+              (lambda: mx.mxfp4_dequantize(q.codes, q.scales, rows, cols, layout, int(rht), 42, out=out)))
+        for _ in range(args.steps):
+            fn()
+        torch.cuda.synchronize()
+        if mx.mxfp4_get_error() != mx.MXFP4_OK:
+            raise RuntimeError("device-side error in the profiling case")
+        print(f"ncu case {args.ncu_case}: {rows} x {cols}, {args.steps} launches", flush=True)
+        return
     if args.ncu_case is not None:
         named = dict(ops)
         if args.ncu_case not in named:
