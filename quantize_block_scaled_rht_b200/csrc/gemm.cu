@@ -128,8 +128,16 @@ struct Shared {
     uint64_t drain;
     uint32_t tmem_base;
     volatile int abort;
+    int drain_failed;    // set in both CTAs by the leader when a bounded drain wait ran out
     int ntiles;
 };
+
+// Mark the pair's drain as failed, in this CTA and in its peer (rank ^ 1).
+__device__ __forceinline__ void mark_drain_failed(Shared *sh, uint32_t rank) {
+    sh->drain_failed = 1;
+    const uint32_t peer = mapa_shared(smem_u32(&sh->drain_failed), rank ^ 1u);
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(peer), "r"(1u) : "memory");
+}
 
 // Bounded wait: true once the phase of `parity` has completed; false if the
 // CTA aborted or the wait ran past the limit (which records the timeout and
@@ -318,6 +326,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         for (int b = 0; b < 2; ++b) { mbar_init(&sh->tmem_full[b], 1); mbar_init(&sh->tmem_empty[b], 2 * EPI_WARPS); }
         mbar_init(&sh->drain, 1);
         sh->abort = 0;
+        sh->drain_failed = 0;
         fence_barrier_init();
         fence_proxy_async_smem();
         prefetch_tmap(&tma_a);
@@ -423,8 +432,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             }
             if (rank == 0) {
                 // drain: the last load of every armed stage (both CTAs' bytes) has landed
+                bool drained = true;
                 for (int i = 0; i < STAGES; ++i)
-                    if (armed & (1u << i)) wait_phase(&sh->full[i], (armed_par >> i) & 1u, sh, limit, true);
+                    if (armed & (1u << i))
+                        drained &= wait_phase(&sh->full[i], (armed_par >> i) & 1u, sh, limit, true);
+                if (!drained && issuer) mark_drain_failed(sh, rank);
             }
             if (sh->abort) aborted_any = true;
         }
@@ -469,7 +481,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             if (issued) {
                 // drain: all MMAs / copies of this thread complete before TMEM or smem go away
                 tc_commit_pair_elect(&sh->drain);
-                wait_phase(&sh->drain, 0, sh, limit, true);
+                if (!wait_phase(&sh->drain, 0, sh, limit, true) && lane == 0) mark_drain_failed(sh, rank);
             }
             if (sh->abort) aborted_any = true;
         }
@@ -665,11 +677,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         __syncwarp();
         if (sh->abort) aborted_any = true;
     }
-    // After an abort, loads issued by this CTA may still be landing in its
-    // shared memory with nobody waiting for them: give them time to finish.
-    if (aborted_any) spin_ns(200000);
+    (void)aborted_any;
     __syncthreads();
     cluster_sync();   // neither CTA leaves while the pair may still touch its smem or TMEM
+    // The leader's drain waited (bounded) for every load of both CTAs and for
+    // its MMAs; only if such a wait ran out can a copy or an MMA still be in
+    // flight: then give it time before the shared and tensor memory go away.
+    if (sh->drain_failed) spin_ns(200000);
+    __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc_pair(tmem, TMEM_COLS);
