@@ -622,6 +622,83 @@ __device__ __forceinline__ void decode32(const uint4 q, uint32_t scode, float *v
     for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(e2m1_value((w[i >> 3] >> (4 * (i & 7))) & 0xFu), X);
 }
 
+// E2M1 decode by table lookup.  For a block with scale code sc < 0xFF every
+// decoded value mag(c) * 2^(sc - 127) is exact in fp32 and has zero low 16
+// bits: at most two significant bits, the smallest nonzero value 2^-128 is the
+// subnormal 0x00200000, and products of 2^128 or more are Inf.  So its bf16
+// pattern is exactly its fp32 high half, and the fp32 value is that half
+// shifted up.  The eight magnitudes' half-words are computed once per block
+// (eight exact products) and split into a table of low bytes and one of high
+// bytes (two registers each); byte permutes look up four codes at a time and
+// interleave the bytes into bf16 pairs; one multiply per pair moves the two
+// sign bits (bit 3 of each nibble) to bits 15 and 31.
+struct DecodeTable {
+    uint32_t lo0, lo1, hi0, hi1;    // byte m of {lo1:lo0} / {hi1:hi0}: low / high byte of magnitude m's bf16
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ DecodeTable decode_table(uint32_t sc) {
+    const float X = scale_from_code(sc);
+    uint32_t h[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) h[m] = __float_as_uint(__fmul_rn(e2m1_value((uint32_t)m), X)) >> 16;
+    const uint32_t p01 = prmt(h[0], h[1], 0x5140u), p23 = prmt(h[2], h[3], 0x5140u);
+    const uint32_t p45 = prmt(h[4], h[5], 0x5140u), p67 = prmt(h[6], h[7], 0x5140u);
+    DecodeTable t;
+    t.lo0 = prmt(p01, p23, 0x5410u);
+    t.hi0 = prmt(p01, p23, 0x7632u);
+    t.lo1 = prmt(p45, p67, 0x5410u);
+    t.hi1 = prmt(p45, p67, 0x7632u);
+    return t;
+}
+
+// Four codes (the nibbles of the low 16 bits of g) -> two bf16 pairs.
+__device__ __forceinline__ void decode4_bf16(const DecodeTable &t, uint32_t g, uint32_t &p01, uint32_t &p23) {
+    const uint32_t sel = g & 0x7777u;
+    const uint32_t lb = prmt(t.lo0, t.lo1, sel), hb = prmt(t.hi0, t.hi1, sel);
+    p01 = prmt(lb, hb, 0x5140u) | (((g & 0x0088u) * 0x01001000u) & 0x80008000u);
+    p23 = prmt(lb, hb, 0x7362u) | (((g & 0x8800u) * 0x00010010u) & 0x80008000u);
+}
+
+// 32 codes of one block -> 16 bf16 pairs (pair p = elements 2p, 2p + 1),
+// exactly the nearest bf16 of the fp32 decode (which is exact); a NaN scale
+// gives NaN pairs.
+__device__ __forceinline__ void decode32_bf16(const uint4 q, uint32_t sc, uint32_t *pairs) {
+    if (sc == 0xFFu) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pairs[i] = 0x7FFF7FFFu;
+        return;
+    }
+    const DecodeTable t = decode_table(sc);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        decode4_bf16(t, w[j], pairs[4 * j], pairs[4 * j + 1]);
+        decode4_bf16(t, w[j] >> 16, pairs[4 * j + 2], pairs[4 * j + 3]);
+    }
+}
+
+// The same as fp32 values (NaN scale: the quiet NaN 0x7FFFFFFF).
+__device__ __forceinline__ void decode32_f32(const uint4 q, uint32_t sc, float *v) {
+    uint32_t pr[16];
+    decode32_bf16(q, sc, pr);
+    if (sc == 0xFFu) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(0x7FFFFFFFu);
+        return;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        v[2 * i] = __uint_as_float(pr[i] << 16);
+        v[2 * i + 1] = __uint_as_float(pr[i] & 0xFFFF0000u);
+    }
+}
+
 template <int RHT>
 __device__ __forceinline__ void inverse_rht32(float *v, const uint32_t *sgn_pair) {
     if constexpr (RHT) {
@@ -636,6 +713,46 @@ __device__ __forceinline__ void inverse_rht32(float *v, const uint32_t *sgn_pair
 
 // SMODE: 0 = row-major per row [rows, cols/32], 1 = row-major 2D tiles
 // [rows/32, cols/32], 2 = MMA layout per row.
+template <int SMODE>
+__device__ __forceinline__ uint32_t dequant_scale(const DequantParams &p, int64_t r, int64_t kb) {
+    if constexpr (SMODE == 0) return p.scales[r * p.ld_scales + kb];
+    else if constexpr (SMODE == 1) return p.scales[(r >> 5) * p.ld_scales + kb];
+    else return p.scales[mma_scale_off(r, kb, p.katoms)];
+}
+
+template <int RHT, bool F32>
+__device__ __forceinline__ void dequant_block_store(const DequantParams &p, int64_t r, int64_t kb, uint4 q,
+                                                    uint32_t sc) {
+    if constexpr (RHT == 0 && !F32) {
+        // no transform, bf16 out: the looked-up pairs are the output
+        uint32_t pr[16];
+        decode32_bf16(q, sc, pr);
+        uint16_t *dst = reinterpret_cast<uint16_t *>(p.out) + r * p.ld_out + (kb << 5);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) stg_v4(dst + 8 * i, make_uint4(pr[4 * i], pr[4 * i + 1], pr[4 * i + 2], pr[4 * i + 3]));
+        return;
+    }
+    float v[32];
+    decode32_f32(q, sc, v);
+    inverse_rht32<RHT>(v, p.sgn_pair);
+    if constexpr (F32) {
+        float *dst = reinterpret_cast<float *>(p.out) + r * p.ld_out + (kb << 5);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            stg_v4(dst + 4 * i, make_uint4(__float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
+                                           __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3])));
+    } else {
+        uint16_t *dst = reinterpret_cast<uint16_t *>(p.out) + r * p.ld_out + (kb << 5);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            stg_v4(dst + 8 * i, make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                                           pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7])));
+    }
+}
+
+// One 32-element block per thread and grid-stride step, two steps per loop
+// iteration: both blocks' code and scale loads are issued before either is
+// decoded, so each thread keeps two loads in flight.
 template <int RHT, bool F32, int SMODE>
 __global__ void __launch_bounds__(256) dequant_row_kernel(const DequantParams p) {
     pdl_wait();
@@ -647,48 +764,53 @@ __global__ void __launch_bounds__(256) dequant_row_kernel(const DequantParams p)
     const int64_t b0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t dr = stride / nb, dk = stride - dr * nb;
     int64_t rr = b0 / nb, kk = b0 - rr * nb;
-    for (int64_t b = b0; b < total; b += stride) {
-        const int64_t r = rr, kb = kk;
+    auto step = [&](int64_t &r_, int64_t &k_) {
+        r_ = rr;
+        k_ = kk;
         rr += dr;
         kk += dk;
         if (kk >= nb) { kk -= nb; ++rr; }
-        const uint4 q = ldg_nc_v4(p.codes + r * p.ld_codes + (kb << 4));
-        uint32_t sc;
-        if constexpr (SMODE == 0) sc = p.scales[r * p.ld_scales + kb];
-        else if constexpr (SMODE == 1) sc = p.scales[(r >> 5) * p.ld_scales + kb];
-        else sc = p.scales[mma_scale_off(r, kb, p.katoms)];
-        float v[32];
-        decode32(q, sc, v);
-        inverse_rht32<RHT>(v, p.sgn_pair);
-        if constexpr (F32) {
-            float *dst = reinterpret_cast<float *>(p.out) + r * p.ld_out + (kb << 5);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                stg_v4(dst + 4 * i, make_uint4(__float_as_uint(v[4 * i]), __float_as_uint(v[4 * i + 1]),
-                                               __float_as_uint(v[4 * i + 2]), __float_as_uint(v[4 * i + 3])));
-        } else {
-            uint16_t *dst = reinterpret_cast<uint16_t *>(p.out) + r * p.ld_out + (kb << 5);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                stg_v4(dst + 8 * i, make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                                               pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7])));
-        }
+    };
+    for (int64_t b = b0; b < total; b += 2 * stride) {
+        int64_t r1, k1, r2, k2;
+        step(r1, k1);
+        step(r2, k2);
+        const bool second = b + stride < total;
+        const uint4 q1 = ldg_nc_v4(p.codes + r1 * p.ld_codes + (k1 << 4));
+        const uint4 q2 = second ? ldg_nc_v4(p.codes + r2 * p.ld_codes + (k2 << 4)) : make_uint4(0, 0, 0, 0);
+        const uint32_t s1 = dequant_scale<SMODE>(p, r1, k1);
+        const uint32_t s2 = second ? dequant_scale<SMODE>(p, r2, k2) : 0u;
+        dequant_block_store<RHT, F32>(p, r1, k1, q1, s1);
+        if (second) dequant_block_store<RHT, F32>(p, r2, k2, q2, s2);
     }
 }
 
 // Transposed-view codes [cols, rows/2] back to out[rows, cols].  A tile is
 // 64 code rows (= output columns) x 8 blocks (= 256 output rows): the codes
 // are staged with coalesced 16-byte cp.async loads into a two-tile ring, the
-// next tile's load in flight while this one is decoded (persistent grid);
-// warp w decodes block w, lane l the output columns 2l and 2l+1, so each
-// output row is written as one contiguous 128-byte (bf16) or 256-byte (fp32)
-// warp store.
+// next tile's load in flight while this one is decoded (persistent grid).
+// Warp w decodes block w, lane l the output columns 2l and 2l+1, one column at
+// a time (decode, inverse RHT, then 32 values written down the column of a
+// per-warp 32-row shared tile), so only one 32-value block is live in
+// registers.  The warp then writes the tile's rows to global memory with
+// 16-byte stores, 128 (bf16) or 256 (fp32) contiguous bytes per row.  The
+// fp32 tile swaps word pairs of columns 32..63 so that the column writes of
+// lanes l and l + 16 fall in different banks.
+template <bool F32>
+__host__ __device__ constexpr int dequant_col_row_bytes() { return COL_TC * (F32 ? 4 : 2); }
+template <bool F32>
+__host__ __device__ constexpr int dequant_col_smem() { return (int)sizeof(uint4) * 2 * COL_TC * 8 + 8 * 32 * dequant_col_row_bytes<F32>(); }
+
 template <int RHT, bool F32, bool MMA>
 __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p) {
     pdl_wait();
     pdl_trigger();
-    __shared__ __align__(16) uint4 tin[2][COL_TC][8];              // 2 x 8 KB of codes
+    extern __shared__ __align__(16) uint8_t dyn_smem[];
+    constexpr int ROWB = dequant_col_row_bytes<F32>();               // staged bytes per output row
+    constexpr int CH = ROWB / 16;                                    // 16-byte chunks per row
+    uint4 (*tin)[COL_TC][8] = reinterpret_cast<uint4 (*)[COL_TC][8]>(dyn_smem);   // 2 x 8 KB of codes
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint8_t *stage = dyn_smem + sizeof(uint4) * 2 * COL_TC * 8 + warp * 32 * ROWB;
     const int64_t tiles_r = (p.rows + COL_TR - 1) / COL_TR;
     const int64_t tiles_c = (p.cols + COL_TC - 1) / COL_TC;
     const int64_t ntiles = tiles_r * tiles_c;
@@ -719,66 +841,74 @@ __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p)
         __syncthreads();
         const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
         const int64_t r0 = tr * COL_TR, c0 = tc * COL_TC;
-        const int64_t rb = r0 + 32 * warp, oc = c0 + 2 * lane;
-        if (rb < p.rows && oc < p.cols) {
-            const int64_t kb = rb >> 5;
-            uint32_t s0, s1;
-            if constexpr (MMA) {
-                s0 = p.scales[mma_scale_off(oc, kb, p.katoms)];
-                s1 = p.scales[mma_scale_off(oc + 1, kb, p.katoms)];
-            } else {
-                s0 = p.scales[oc * p.ld_scales + kb];
-                s1 = p.scales[(oc + 1) * p.ld_scales + kb];
+        const int64_t rb = r0 + 32 * warp;
+        if (rb < p.rows) {
+          const int64_t kb = rb >> 5;
+          if constexpr (RHT == 0 && !F32) {
+            // no transform, bf16 out: both columns' looked-up pairs at once, one
+            // 32-bit word (columns 2l, 2l + 1) per row of the staged tile
+            const int64_t oc = c0 + 2 * lane;
+            if (oc < p.cols) {                 // cols is even: oc + 1 < cols too
+                const uint32_t s0 = MMA ? p.scales[mma_scale_off(oc, kb, p.katoms)] : p.scales[oc * p.ld_scales + kb];
+                const uint32_t s1 =
+                    MMA ? p.scales[mma_scale_off(oc + 1, kb, p.katoms)] : p.scales[(oc + 1) * p.ld_scales + kb];
+                uint32_t pa[16], pb[16];
+                decode32_bf16(tin[buf][2 * lane][warp], s0, pa);
+                decode32_bf16(tin[buf][2 * lane + 1][warp], s1, pb);
+                uint32_t *w = reinterpret_cast<uint32_t *>(stage) + lane;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    w[(2 * i) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x5410u);
+                    w[(2 * i + 1) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x7632u);
+                }
             }
-            if constexpr (RHT == 0) {
-                // no transform: decode and store one row pair at a time, so
-                // that only the packed codes stay in registers
-                const uint4 q0 = tin[buf][2 * lane][warp], q1 = tin[buf][2 * lane + 1][warp];
-                const uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
-                const float X0 = scale_from_code(s0), X1 = scale_from_code(s1);
+          } else {
+#pragma unroll 1
+            for (int j = 0; j < 2; ++j) {      // one column at a time: one 32-value block live
+                const int c = 2 * lane + j;
+                const int64_t oc = c0 + c;
+                if (oc < p.cols) {
+                    const uint32_t sc = MMA ? p.scales[mma_scale_off(oc, kb, p.katoms)] : p.scales[oc * p.ld_scales + kb];
+                    float v[32];
+                    decode32_f32(tin[buf][c][warp], sc, v);
+                    if constexpr (RHT) {
+                        fwht32_scaled<RHT>(v, rht_norm<RHT>());
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float a = s0 == 0xFFu ? __uint_as_float(0x7FFFFFFFu)
-                                                : __fmul_rn(e2m1_value((w0[i >> 3] >> (4 * (i & 7))) & 0xFu), X0);
-                    const float b = s1 == 0xFFu ? __uint_as_float(0x7FFFFFFFu)
-                                                : __fmul_rn(e2m1_value((w1[i >> 3] >> (4 * (i & 7))) & 0xFu), X1);
-                    const int64_t gr = rb + i;
-                    if constexpr (F32) {
-                        float2 *dst = reinterpret_cast<float2 *>(reinterpret_cast<float *>(p.out) + gr * p.ld_out + oc);
-                        *dst = make_float2(a, b);
-                    } else {
-                        uint32_t *dst =
-                            reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(p.out) + gr * p.ld_out + oc);
-                        *dst = pack_bf16x2(a, b);
+                        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ p.sgn_bit[i % RHT]);
                     }
-                }
-            } else {
-                float v0[32], v1[32];
-                decode32(tin[buf][2 * lane][warp], s0, v0);
-                decode32(tin[buf][2 * lane + 1][warp], s1, v1);
-                if constexpr (RHT) {
-                    const float c = rht_norm<RHT>();
-#pragma unroll
-                    for (int s = 0; s < 32; s += RHT) { fwht<RHT>(v0 + s); fwht<RHT>(v1 + s); }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const uint32_t fl = p.sgn_bit[i % RHT];
-                        v0[i] = __uint_as_float(__float_as_uint(__fmul_rn(v0[i], c)) ^ fl);
-                        v1[i] = __uint_as_float(__float_as_uint(__fmul_rn(v1[i], c)) ^ fl);
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int64_t gr = rb + i;
                     if constexpr (F32) {
-                        float2 *dst = reinterpret_cast<float2 *>(reinterpret_cast<float *>(p.out) + gr * p.ld_out + oc);
-                        *dst = make_float2(v0[i], v1[i]);
+                        const int wpos = c ^ ((c >> 5) & 1);            // bank-spreading word swap
+                        uint32_t *col = reinterpret_cast<uint32_t *>(stage) + wpos;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) col[i * (ROWB / 4)] = __float_as_uint(v[i]);
                     } else {
-                        uint32_t *dst = reinterpret_cast<uint32_t *>(reinterpret_cast<uint16_t *>(p.out) + gr * p.ld_out + oc);
-                        *dst = pack_bf16x2(v0[i], v1[i]);
+                        uint16_t *col = reinterpret_cast<uint16_t *>(stage) + c;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            uint16_t h;    // nearest-even bf16
+                            asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(v[i]));
+                            col[i * (ROWB / 2)] = h;
+                        }
                     }
                 }
             }
+          }
+            __syncwarp();
+            // 32 rows of ROWB bytes: lane-contiguous 16-byte chunks of each row
+#pragma unroll
+            for (int idx = lane; idx < 32 * CH; idx += 32) {
+                const int row = idx / CH, ch = idx - row * CH;
+                const int64_t col0 = c0 + ch * (16 / (F32 ? 4 : 2));
+                if (col0 < p.cols) {
+                    uint4 w = *reinterpret_cast<const uint4 *>(stage + row * ROWB + ch * 16);
+                    if constexpr (F32) {
+                        if (ch >= CH / 2) w = make_uint4(w.y, w.x, w.w, w.z);   // undo the word swap
+                    }
+                    uint8_t *dst = static_cast<uint8_t *>(p.out) + ((rb + row) * p.ld_out + col0) * (F32 ? 4 : 2);
+                    stg_v4(dst, w);
+                }
+            }
+            __syncwarp();
         }
         __syncthreads();
     }
@@ -801,16 +931,31 @@ static int num_sms() {
 
 // Resident CTAs per SM of a kernel (persistent grids are SMs x this).
 // Cached per kernel; the value depends only on the kernel and block size.
-static int resident_ctas(const void *kern, int threads) {
+static int resident_ctas(const void *kern, int threads, size_t dyn_smem = 0) {
     static std::mutex mu;
     static std::map<const void *, int> cache;
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(kern);
     if (it != cache.end()) return it->second;
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, 0) != cudaSuccess || occ <= 0) occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, dyn_smem) != cudaSuccess || occ <= 0)
+        occ = 1;
     cache[kern] = occ;
     return occ;
+}
+
+// Dynamic shared memory above the 48 KB default: the opt-in, once per kernel
+// and device.
+static cudaError_t allow_dyn_smem(const void *kern, int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, bool> done;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({kern, dev})) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[{kern, dev}] = true;
+    return e;
 }
 
 static void fill_signs(uint32_t mask, int rht, uint32_t *pair, uint32_t *bit) {
@@ -990,9 +1135,12 @@ static cudaError_t launch_dequant_t(int layout, int smode, const DequantParams &
         // persistent at full occupancy: each CTA keeps its next tile's load in flight
         const int64_t tiles = ((p.rows + COL_TR - 1) / COL_TR) * ((p.cols + COL_TC - 1) / COL_TC);
         auto kern = smode == 2 ? dequant_col_kernel<RHT, F32, true> : dequant_col_kernel<RHT, F32, false>;
-        const int64_t cap = (int64_t)num_sms() * resident_ctas(reinterpret_cast<const void *>(kern), 256);
+        constexpr int smem = dequant_col_smem<F32>();
+        const cudaError_t ea = allow_dyn_smem(reinterpret_cast<const void *>(kern), smem);
+        if (ea != cudaSuccess) return ea;
+        const int64_t cap = (int64_t)num_sms() * resident_ctas(reinterpret_cast<const void *>(kern), 256, smem);
         const unsigned g = (unsigned)(tiles < cap ? tiles : cap);
-        return launch_pdl(kern, dim3(g), dim3(256), 0, s, p);
+        return launch_pdl(kern, dim3(g), dim3(256), (size_t)smem, s, p);
     } else {
         const unsigned g = (unsigned)grid_for(p.rows * (p.cols / 32), 256);
         if (smode == 0) return launch_pdl(dequant_row_kernel<RHT, F32, 0>, dim3(g), dim3(256), 0, s, p);
