@@ -112,6 +112,13 @@ __device__ __forceinline__ float amax_nan(float acc, float v) {
     asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(acc), "f"(fabsf(v)));
     return r;
 }
+// Two values at once: the three-input max of sm_100 (the same result as two
+// nested max.NaN).
+__device__ __forceinline__ float amax_nan2(float acc, float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(acc), "f"(fabsf(a)), "f"(fabsf(b)));
+    return r;
+}
 
 // E8M0 scale code of a block from its amax (NaN or Inf -> 0xFF; 0 -> 0):
 // clamp(floor(log2 amax) - 2 + 127, 0, 254).  For a normal amax the biased

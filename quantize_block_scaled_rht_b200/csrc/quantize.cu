@@ -41,6 +41,30 @@ struct QuantParams {
     uint32_t sgn_bit[32];                  // RHT sign of element i (mod the RHT size) as bit 31
 };
 
+// Packed two-lane fp32 arithmetic (sm_100a `.f32x2`): each lane is rounded
+// to nearest even exactly as the scalar operation, subnormals kept.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
 // ---------------------------------------------------------------------------
 // Per-block quantization core: the scale code from the block's amax, then the
 // four groups of 8 values (unscaled, from get8(q, w)) scaled and encoded into
@@ -76,7 +100,7 @@ __device__ __forceinline__ uint32_t quantize32(const float *v, uint4 &out, uint6
                                            int rule) {
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) amax = amax_nan(amax, v[i]);
+    for (int i = 0; i < 32; i += 2) amax = amax_nan2(amax, v[i], v[i + 1]);
     return quantize_groups<SR>(
         amax,
         [&](int q, float *w) {
@@ -84,30 +108,6 @@ __device__ __forceinline__ uint32_t quantize32(const float *v, uint4 &out, uint6
             for (int j = 0; j < 8; ++j) w[j] = v[8 * q + j];
         },
         out, g0, k0, k1, rule);
-}
-
-// Packed two-lane fp32 arithmetic (sm_100a `.f32x2`): each lane is rounded
-// to nearest even exactly as the scalar operation, subnormals kept.
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
-}
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    float2 d;
-    asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
-        "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
-        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-    return d;
 }
 
 // The same butterfly as fwht<D> on 32 values held as 16 pairs
@@ -155,12 +155,18 @@ __device__ __forceinline__ void fwht32_scaled(float *v, float c) {
 // The same for 32 fp32 values held as 16 pairs P[m] = (v[m], v[m + 16]),
 // scaled with packed two-lane multiplies (each lane rounded as the scalar
 // product): groups 0, 1 are the low lanes of P[0..15], groups 2, 3 the high.
-template <bool SR>
-__device__ __forceinline__ uint32_t quantize32_pairs(float2 *P, uint4 &out, uint64_t g0, uint32_t k0, uint32_t k1,
-                                                     int rule) {
+__device__ __forceinline__ float amax_pairs(const float2 *P) {
     float amax = 0.0f;
 #pragma unroll
-    for (int m = 0; m < 16; ++m) amax = amax_nan(amax_nan(amax, P[m].x), P[m].y);
+    for (int m = 0; m < 16; ++m) amax = amax_nan2(amax, P[m].x, P[m].y);
+    return amax;
+}
+
+// The block's scale from a given amax (a 2D tile's, or the block's own) and
+// the elements from the pairs.
+template <bool SR>
+__device__ __forceinline__ uint32_t quantize32_pairs_amax(float2 *P, float amax, uint4 &out, uint64_t g0,
+                                                          uint32_t k0, uint32_t k1, int rule) {
     const uint32_t code = scale_code_rule(amax, rule);
     if (code == 0xFFu) {
         out = make_uint4(0, 0, 0, 0);
@@ -188,6 +194,12 @@ __device__ __forceinline__ uint32_t quantize32_pairs(float2 *P, uint4 &out, uint
     return code;
 }
 
+template <bool SR>
+__device__ __forceinline__ uint32_t quantize32_pairs(float2 *P, uint4 &out, uint64_t g0, uint32_t k0, uint32_t k1,
+                                                     int rule) {
+    return quantize32_pairs_amax<SR>(P, amax_pairs(P), out, g0, k0, k1, rule);
+}
+
 // The same for 32 bf16 values packed in four uint4 (no transform): amax on
 // the packed pairs, each group unpacked when it is encoded, so that the block
 // occupies 16 registers rather than 32.
@@ -199,6 +211,23 @@ __device__ __forceinline__ uint32_t quantize32_bf16(const uint4 *u, uint4 &out, 
 }
 
 // Unpack 16 bf16x2 words to 32 fp32 values, with RHT sign flips and butterfly.
+// A row block of 32 bf16 values (w[j]: elements 2j, 2j + 1) as the pairs
+// P[m] = (v[m], v[m + 16]) of the packed butterfly, sign-flipped, transformed
+// and normalised; the same values as unpack_row32.
+template <int RHT>
+__device__ __forceinline__ void unpack_row32_pairs(const uint32_t *w, float2 *P, const QuantParams &p) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t a = w[j] ^ p.sgn_pair[j], b = w[j + 8] ^ p.sgn_pair[j + 8];
+        P[2 * j] = make_float2(bf16lo(a), bf16lo(b));
+        P[2 * j + 1] = make_float2(bf16hi(a), bf16hi(b));
+    }
+    const float c = rht_norm<RHT>();
+    fwht_pairs<RHT>(P);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) P[m] = mul2(P[m], make_float2(c, c));
+}
+
 template <int RHT>
 __device__ __forceinline__ void unpack_row32(const uint32_t *w, float *v, const QuantParams &p) {
 #pragma unroll
@@ -246,11 +275,18 @@ __global__ void __launch_bounds__(256) quant_row_kernel(const QuantParams p) {
             const uint4 t = ldg_nc_v4(src + 8 * q);
             w[4 * q] = t.x; w[4 * q + 1] = t.y; w[4 * q + 2] = t.z; w[4 * q + 3] = t.w;
         }
-        float v[32];
-        unpack_row32<RHT>(w, v, p);
         uint4 packed;
         const uint64_t g0 = (uint64_t)(r * p.cols + (kb << 5)) + p.elem_offset;
-        const uint32_t code = quantize32<SR>(v, packed, g0, p.seed_lo, p.seed_hi, p.scale_rule);
+        uint32_t code;
+        if constexpr (RHT) {
+            float2 P[16];
+            unpack_row32_pairs<RHT>(w, P, p);
+            code = quantize32_pairs<SR>(P, packed, g0, p.seed_lo, p.seed_hi, p.scale_rule);
+        } else {
+            float v[32];
+            unpack_row32<0>(w, v, p);
+            code = quantize32<SR>(v, packed, g0, p.seed_lo, p.seed_hi, p.scale_rule);
+        }
         stg_v4(p.codes + r * p.ld_codes + (kb << 4), packed);
         if constexpr (MMA) p.scales[mma_scale_off(r, kb, p.katoms)] = (uint8_t)code;
         else p.scales[r * p.ld_scales + kb] = (uint8_t)code;
@@ -720,6 +756,20 @@ __device__ __forceinline__ uint32_t dequant_scale(const DequantParams &p, int64_
     else return p.scales[mma_scale_off(r, kb, p.katoms)];
 }
 
+// One 32-value block decoded, inverse-transformed and rounded to 16 bf16
+// pairs (pair j = elements 2j, 2j + 1); the RHT signs are applied to the
+// rounded pairs (sgn_pair[j] holds them at bits 15 and 31), which equals
+// flipping the fp32 values first since rounding to nearest is symmetric.
+template <int RHT>
+__device__ __forceinline__ void column_rht_bf16(const uint4 q, uint32_t sc, const uint32_t *sgn_pair,
+                                                uint32_t *pairs) {
+    float v[32];
+    decode32_f32(q, sc, v);
+    fwht32_scaled<RHT>(v, rht_norm<RHT>());
+#pragma unroll
+    for (int j = 0; j < 16; ++j) pairs[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]) ^ sgn_pair[j];
+}
+
 template <int RHT, bool F32>
 __device__ __forceinline__ void dequant_block_store(const DequantParams &p, int64_t r, int64_t kb, uint4 q,
                                                     uint32_t sc) {
@@ -802,7 +852,7 @@ template <bool F32>
 __host__ __device__ constexpr int dequant_col_smem() { return (int)sizeof(uint4) * 2 * COL_TC * 8 + 8 * 32 * dequant_col_row_bytes<F32>(); }
 
 template <int RHT, bool F32, bool MMA>
-__global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p) {
+__global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 1)) dequant_col_kernel(const DequantParams p) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ __align__(16) uint8_t dyn_smem[];
@@ -844,8 +894,9 @@ __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p)
         const int64_t rb = r0 + 32 * warp;
         if (rb < p.rows) {
           const int64_t kb = rb >> 5;
-          if constexpr (RHT == 0 && !F32) {
-            // no transform, bf16 out: both columns' looked-up pairs at once, one
+          if constexpr (!F32) {
+            // bf16 out: each column as 16 bf16 pairs along its rows (looked up,
+            // or transformed, rounded and sign-flipped as pairs), then one
             // 32-bit word (columns 2l, 2l + 1) per row of the staged tile
             const int64_t oc = c0 + 2 * lane;
             if (oc < p.cols) {                 // cols is even: oc + 1 < cols too
@@ -853,8 +904,13 @@ __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p)
                 const uint32_t s1 =
                     MMA ? p.scales[mma_scale_off(oc + 1, kb, p.katoms)] : p.scales[(oc + 1) * p.ld_scales + kb];
                 uint32_t pa[16], pb[16];
-                decode32_bf16(tin[buf][2 * lane][warp], s0, pa);
-                decode32_bf16(tin[buf][2 * lane + 1][warp], s1, pb);
+                if constexpr (RHT == 0) {
+                    decode32_bf16(tin[buf][2 * lane][warp], s0, pa);
+                    decode32_bf16(tin[buf][2 * lane + 1][warp], s1, pb);
+                } else {
+                    column_rht_bf16<RHT>(tin[buf][2 * lane][warp], s0, p.sgn_pair, pa);
+                    column_rht_bf16<RHT>(tin[buf][2 * lane + 1][warp], s1, p.sgn_pair, pb);
+                }
                 uint32_t *w = reinterpret_cast<uint32_t *>(stage) + lane;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -863,8 +919,9 @@ __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p)
                 }
             }
           } else {
+            // fp32 out: one column at a time, one 32-value block live
 #pragma unroll 1
-            for (int j = 0; j < 2; ++j) {      // one column at a time: one 32-value block live
+            for (int j = 0; j < 2; ++j) {
                 const int c = 2 * lane + j;
                 const int64_t oc = c0 + c;
                 if (oc < p.cols) {
@@ -876,20 +933,10 @@ __global__ void __launch_bounds__(256) dequant_col_kernel(const DequantParams p)
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ p.sgn_bit[i % RHT]);
                     }
-                    if constexpr (F32) {
-                        const int wpos = c ^ ((c >> 5) & 1);            // bank-spreading word swap
-                        uint32_t *col = reinterpret_cast<uint32_t *>(stage) + wpos;
+                    const int wpos = c ^ ((c >> 5) & 1);                // bank-spreading word swap
+                    uint32_t *col = reinterpret_cast<uint32_t *>(stage) + wpos;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) col[i * (ROWB / 4)] = __float_as_uint(v[i]);
-                    } else {
-                        uint16_t *col = reinterpret_cast<uint16_t *>(stage) + c;
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            uint16_t h;    // nearest-even bf16
-                            asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(h) : "f"(v[i]));
-                            col[i * (ROWB / 2)] = h;
-                        }
-                    }
+                    for (int i = 0; i < 32; ++i) col[i * (ROWB / 4)] = __float_as_uint(v[i]);
                 }
             }
           }
