@@ -62,10 +62,10 @@ KERNELS_PER_STEP = len(QUANT_OPS) + len(GEMMS)
 # figures hold only for the kernel sources they were taken from: a changed
 # source gives traffic null.
 NCU_TRAFFIC = {
-    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "cfcae9425fa80c24",
-             "bytes": {"fprop": 52.26e6, "dgrad": 23.36e6, "wgrad": 29.88e6}},
-    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "b9c5a4ffd3c6011a",
-              "bytes": {"quant_x_dual": 23.62e6, "quant_w_2d": 33.43e6, "quant_dy_dual_sr": 48.71e6},
+    "gemm": {"sources": ("gemm.cu", "ptx.cuh", "common.cuh"), "sha1": "aa4d623082758f27",
+             "bytes": {"fprop": 47.95e6, "dgrad": 21.68e6, "wgrad": 26.51e6}},
+    "quant": {"sources": ("quantize.cu", "common.cuh"), "sha1": "6b8b7b9db3e2f390",
+              "bytes": {"quant_x_dual": 23.63e6, "quant_w_2d": 33.27e6, "quant_dy_dual_sr": 47.34e6},
               # thread instructions per element (ncu smsp__inst_executed x 32 / elements)
               "inst_per_elem": {"quant_dy_dual_sr": 77.1}},
 }
