@@ -852,7 +852,7 @@ template <bool F32>
 __host__ __device__ constexpr int dequant_col_smem() { return (int)sizeof(uint4) * 2 * COL_TC * 8 + 8 * 32 * dequant_col_row_bytes<F32>(); }
 
 template <int RHT, bool F32, bool MMA>
-__global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 1)) dequant_col_kernel(const DequantParams p) {
+__global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kernel(const DequantParams p) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ __align__(16) uint8_t dyn_smem[];
