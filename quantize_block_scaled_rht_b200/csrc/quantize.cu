@@ -494,6 +494,226 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualP
 }
 
 // ---------------------------------------------------------------------------
+// 1D-column quantizer (blocks of 32 along rows; output [cols, rows / 2]).  A
+// CTA streams 256 x 64 bf16 tiles (32 KB, unpadded) through a three-deep
+// cp.async ring.  Warp w owns row block w of a tile, lane l the column pair
+// (2l, 2l + 1): each of its 32 shared loads is one bf16x2 word of a row (a
+// warp reads one 128-byte row, conflict-free), and the two columns travel as
+// the two lanes of packed fp32 pairs through the sign flip, the butterfly,
+// the normalisation and the scaling, one f32x2 instruction per two elements.
+// Every lane takes the same operations in the same order as the scalar
+// reference, so the results are bit-identical.  Codes are staged per tile as
+// 64 output rows of 128 bytes (16-byte pieces swizzled by column pair) and
+// leave as 128-byte runs; scale bytes are staged per strip of
+// vertically adjacent tiles and leave as 8 bytes per tile and output row in
+// one run.
+// ---------------------------------------------------------------------------
+constexpr int CQ_TR = 256, CQ_TC = 64, CQ_STAGES = 3, CQ_MAX_STRIP = 8;
+constexpr int CQ_TILE_BYTES = CQ_TR * CQ_TC * 2;                       // 32 KB of bf16
+constexpr int CQ_OUT_BYTES = CQ_TC * (CQ_TR / 2);                      // 8 KB of codes
+constexpr int CQ_SPITCH = 2 * CQ_MAX_STRIP + 1;                        // scale words per output row (+1: banks)
+constexpr int CQ_SCALE_BYTES = CQ_TC * CQ_SPITCH * 4;                 // a strip's scale bytes
+constexpr int CQ_SMEM = CQ_STAGES * CQ_TILE_BYTES + CQ_OUT_BYTES + CQ_SCALE_BYTES;
+
+// Butterfly stages h = 1 .. D/2 over the 32 rows of a column pair (both
+// lanes at once); D = 16 transforms the two 16-row halves separately.
+template <int D>
+__device__ __forceinline__ void fwht_col_pairs(float2 *P) {
+#pragma unroll
+    for (int h = 1; h < D; h <<= 1) {
+#pragma unroll
+        for (int m = 0; m < 32; ++m) {
+            if ((m & h) == 0) {
+                const float2 a = P[m], b = P[m + h];
+                P[m] = add2(a, b);
+                P[m + h] = sub2(a, b);
+            }
+        }
+    }
+}
+
+// Codes of one column (lane HI of the pairs) of scaled values: four groups of
+// eight rows, each one 32-bit word of nibbles.
+template <bool SR, bool HI>
+__device__ __forceinline__ uint4 encode_col_lane(const float2 *P, uint64_t g0, uint32_t k0, uint32_t k1) {
+    const uint64_t blk = g0 >> 2;    // g0 % 4 == 0
+    uint32_t q[4];
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        float w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) w[j] = HI ? P[8 * g + j].y : P[8 * g + j].x;
+        if constexpr (SR) q[g] = e2m1x8_sr(w, blk + 2 * g, k0, k1);
+        else q[g] = e2m1x8_rn(w);
+    }
+    return make_uint4(q[0], q[1], q[2], q[3]);
+}
+
+template <int RHT, bool SR, bool MMA>
+__global__ void __launch_bounds__(256, 2) quant_col_kernel(const DualParams p, const uint32_t nstrips) {
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ __align__(16) uint8_t cq_smem[];
+    uint8_t *ring = cq_smem;
+    uint4 *tout = reinterpret_cast<uint4 *>(cq_smem + CQ_STAGES * CQ_TILE_BYTES);
+    uint32_t *ssc = reinterpret_cast<uint32_t *>(cq_smem + CQ_STAGES * CQ_TILE_BYTES + CQ_OUT_BYTES);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t strip = p.strip;
+    // The CTA's tiles in order: strips S = blockIdx.x + j * gridDim.x, tile k
+    // of each (row band (S / tiles_c) * strip + k, column band S % tiles_c).
+    // A strip index past nstrips stays past it under next().
+    auto strip_tiles = [&](uint32_t S) -> uint32_t {
+        const uint32_t t0 = (S / p.tiles_c) * strip;
+        return t0 + strip <= p.tiles_r ? strip : (t0 < p.tiles_r ? p.tiles_r - t0 : strip);
+    };
+    auto next = [&](uint32_t &S, uint32_t &k) {
+        if (k + 1 < strip_tiles(S)) {
+            ++k;
+        } else {
+            S += gridDim.x;
+            k = 0;
+        }
+    };
+    auto load = [&](uint32_t S, uint32_t k, int buf) {
+        if (S < nstrips) {
+            const uint32_t band = S / p.tiles_c;
+            const int64_t r0 = (int64_t)(band * strip + k) * CQ_TR, c0 = (int64_t)(S - band * p.tiles_c) * CQ_TC;
+            const int ch = tid & 7, row = tid >> 3;          // rows row + 32 i, 16-byte chunk ch
+            const int64_t gc = c0 + 8 * ch;
+            const uint16_t *src = p.x + (r0 + row) * p.ld_x + gc;
+            uint8_t *dst = ring + buf * CQ_TILE_BYTES + row * 128 + 16 * ch;
+            if (r0 + CQ_TR <= p.rows && c0 + CQ_TC <= p.cols) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cp_async16(dst + i * 32 * 128, src + (int64_t)i * 32 * p.ld_x);
+            } else if (gc < p.cols) {                          // cols % 8 == 0: a chunk is whole or absent
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (r0 + row + 32 * i < p.rows) cp_async16(dst + i * 32 * 128, src + (int64_t)i * 32 * p.ld_x);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    uint32_t S = blockIdx.x, k = 0;
+    uint32_t S1 = S, k1 = k;
+    next(S1, k1);
+    uint32_t S2 = S1, k2 = k1;
+    next(S2, k2);
+    load(S, k, 0);
+    load(S1, k1, 1);
+    for (int it = 0; S < nstrips; ++it) {
+        load(S2, k2, (it + 2) % CQ_STAGES);                  // two tiles in flight while this one is quantized
+        asm volatile("cp.async.wait_group 2;" ::: "memory");
+        __syncthreads();
+        const uint32_t band = S / p.tiles_c;
+        const int64_t r0 = (int64_t)(band * strip + k) * CQ_TR, c0 = (int64_t)(S - band * p.tiles_c) * CQ_TC;
+        const int64_t rin = r0 + 32 * warp, oc = c0 + 2 * lane;
+        if (rin < p.rows && oc < p.cols) {
+            const uint32_t *src =
+                reinterpret_cast<const uint32_t *>(ring + (it % CQ_STAGES) * CQ_TILE_BYTES) + warp * 32 * 32 + lane;
+            float2 P[32];                            // (column oc, column oc + 1) at row rin + m
+#pragma unroll
+            for (int m = 0; m < 32; ++m) {
+                // bf16 -> fp32 with the RHT sign: adding 2^31 flips bit 31
+                const uint32_t u = src[m * 32];
+                const uint32_t sg = RHT ? p.sgn_bit[m] : 0u;
+                P[m] = make_float2(__uint_as_float(u * 65536u + sg), __uint_as_float((u & 0xFFFF0000u) ^ sg));
+            }
+            if constexpr (RHT != 0) {
+                const float cn = rht_norm<RHT>();
+                fwht_col_pairs<RHT>(P);
+#pragma unroll
+                for (int m = 0; m < 32; ++m) P[m] = mul2(P[m], make_float2(cn, cn));
+            }
+            float alo = 0.0f, ahi = 0.0f;
+#pragma unroll
+            for (int m = 0; m < 32; m += 2) {
+                alo = amax_nan2(alo, P[m].x, P[m + 1].x);
+                ahi = amax_nan2(ahi, P[m].y, P[m + 1].y);
+            }
+            const uint32_t slo = scale_code_rule(alo, p.scale_rule), shi = scale_code_rule(ahi, p.scale_rule);
+            // a NaN block (code 0xFF) stores zero codes; its lane is scaled by 1
+            const float2 inv = make_float2(slo == 0xFFu ? 1.0f : inv_scale_from_code(slo),
+                                           shi == 0xFFu ? 1.0f : inv_scale_from_code(shi));
+            if (p.scale_rule == 2) {
+#pragma unroll
+                for (int m = 0; m < 32; ++m) P[m] = mul2(mul2(P[m], make_float2(0.75f, 0.75f)), inv);
+            } else {
+#pragma unroll
+                for (int m = 0; m < 32; ++m) P[m] = mul2(P[m], inv);
+            }
+            const uint64_t g0 = (uint64_t)(oc * p.c_sr_ld + rin) + p.c_offset;
+            uint4 qlo = encode_col_lane<SR, false>(P, g0, p.seed_lo, p.seed_hi);
+            uint4 qhi = encode_col_lane<SR, true>(P, g0 + (uint64_t)p.c_sr_ld, p.seed_lo, p.seed_hi);
+            if (slo == 0xFFu) qlo = make_uint4(0, 0, 0, 0);
+            if (shi == 0xFFu) qhi = make_uint4(0, 0, 0, 0);
+            const int c = 2 * lane, sw = warp ^ (lane & 7);
+            tout[c * 8 + sw] = qlo;
+            tout[(c + 1) * 8 + sw] = qhi;
+            uint8_t *sb = reinterpret_cast<uint8_t *>(ssc);
+            sb[4 * (c * CQ_SPITCH + 2 * k) + warp] = (uint8_t)slo;
+            sb[4 * ((c + 1) * CQ_SPITCH + 2 * k) + warp] = (uint8_t)shi;
+        }
+        __syncthreads();                                     // tile read; codes and scales staged
+        const uint32_t ntiles = strip_tiles(S);
+        const bool last = k + 1 == ntiles;
+        // codes: 64 output rows x 8 chunks of 16 bytes; 8 lanes write one row's 128 bytes
+#pragma unroll
+        for (int pass = 0; pass < 2; ++pass) {
+            const int row = (tid >> 3) + 32 * pass, ch = tid & 7;
+            const int64_t orow = c0 + row, rb = r0 + 32 * ch;
+            if (orow < p.cols && rb < p.rows)
+                stg_v4(p.ccodes + orow * p.ld_ccodes + (rb >> 1), tout[row * 8 + (ch ^ ((row >> 1) & 7))]);
+        }
+        if (last) {                                          // the strip's scales: 8 K-blocks per tile and output row
+            const int64_t kb0 = (int64_t)band * strip * 8, nkb = p.rows >> 5;
+            const uint8_t *sb = reinterpret_cast<const uint8_t *>(ssc);
+            if constexpr (MMA) {
+                // 4-byte pieces (one MMA atom row slot each); consecutive
+                // threads take consecutive rows, 16 bytes apart in an atom
+                for (uint32_t idx = tid; idx < CQ_TC * 2u * ntiles; idx += 256) {
+                    const uint32_t a = idx / CQ_TC, row = idx % CQ_TC;
+                    const int64_t orow = c0 + row, kb = kb0 + 4 * a;
+                    if (orow < p.cols && kb < nkb) {
+                        uint8_t *dst = p.cscales + mma_scale_off(orow, kb, p.c_katoms);
+                        const uint32_t w = ssc[row * CQ_SPITCH + a];
+                        if (kb + 4 <= nkb) *reinterpret_cast<uint32_t *>(dst) = w;
+                        else for (int j = 0; j < 4 && kb + j < nkb; ++j) dst[j] = (uint8_t)(w >> (8 * j));
+                    }
+                }
+            } else if (((reinterpret_cast<uintptr_t>(p.cscales) | (uintptr_t)p.ld_cscales) & 3u) == 0) {
+                // row-major, word-aligned rows: consecutive threads write
+                // consecutive words of one output row
+                const uint32_t nw = 2u * ntiles;
+                for (uint32_t idx = tid; idx < CQ_TC * nw; idx += 256) {
+                    const uint32_t row = idx / nw, a = idx - row * nw;
+                    const int64_t orow = c0 + row, kb = kb0 + 4 * a;
+                    if (orow < p.cols && kb < nkb) {
+                        uint8_t *dst = p.cscales + orow * p.ld_cscales + kb;
+                        const uint32_t w = ssc[row * CQ_SPITCH + a];
+                        if (kb + 4 <= nkb) *reinterpret_cast<uint32_t *>(dst) = w;
+                        else for (int j = 0; j < 4 && kb + j < nkb; ++j) dst[j] = (uint8_t)(w >> (8 * j));
+                    }
+                }
+            } else {
+                // row-major, any alignment: consecutive threads write
+                // consecutive bytes of one output row
+                const uint32_t nb = 8u * ntiles;
+                for (uint32_t idx = tid; idx < CQ_TC * nb; idx += 256) {
+                    const uint32_t row = idx / nb, j = idx - row * nb;
+                    const int64_t orow = c0 + row, kb = kb0 + j;
+                    if (orow < p.cols && kb < nkb) p.cscales[orow * p.ld_cscales + kb] = sb[4 * row * CQ_SPITCH + j];
+                }
+            }
+        }
+        S = S1; k = k1;
+        S1 = S2; k1 = k2;
+        next(S2, k2);
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // 2D 32x32 blocks.  A CTA streams tiles of 8 blocks through a double-buffered
 // shared-memory ring (cp.async of whole tile rows, so the global reads are
 // coalesced): 32 x 256 (one block row) without the transposed copy, 128 x 64
@@ -749,13 +969,6 @@ __device__ __forceinline__ void inverse_rht32(float *v, const uint32_t *sgn_pair
 
 // SMODE: 0 = row-major per row [rows, cols/32], 1 = row-major 2D tiles
 // [rows/32, cols/32], 2 = MMA layout per row.
-template <int SMODE>
-__device__ __forceinline__ uint32_t dequant_scale(const DequantParams &p, int64_t r, int64_t kb) {
-    if constexpr (SMODE == 0) return p.scales[r * p.ld_scales + kb];
-    else if constexpr (SMODE == 1) return p.scales[(r >> 5) * p.ld_scales + kb];
-    else return p.scales[mma_scale_off(r, kb, p.katoms)];
-}
-
 // One 32-value block decoded, inverse-transformed and rounded to 16 bf16
 // pairs (pair j = elements 2j, 2j + 1); the RHT signs are applied to the
 // rounded pairs (sgn_pair[j] holds them at bits 15 and 31), which equals
@@ -768,6 +981,12 @@ __device__ __forceinline__ void column_rht_bf16(const uint4 q, uint32_t sc, cons
     fwht32_scaled<RHT>(v, rht_norm<RHT>());
 #pragma unroll
     for (int j = 0; j < 16; ++j) pairs[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]) ^ sgn_pair[j];
+}
+template <int SMODE>
+__device__ __forceinline__ uint32_t dequant_scale(const DequantParams &p, int64_t r, int64_t kb) {
+    if constexpr (SMODE == 0) return p.scales[r * p.ld_scales + kb];
+    else if constexpr (SMODE == 1) return p.scales[(r >> 5) * p.ld_scales + kb];
+    else return p.scales[mma_scale_off(r, kb, p.katoms)];
 }
 
 template <int RHT, bool F32>
@@ -875,13 +1094,31 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
+    // the bf16 path's two scale bytes (columns 2l, 2l + 1 of row block w) of a
+    // tile, loaded one tile ahead so that their latency hides behind a tile
+    auto scale_pair = [&](int64_t tt, uint32_t &s0, uint32_t &s1) {
+        s0 = s1 = 0xFFu;
+        if (tt < ntiles) {
+            const int64_t tr = tt / tiles_c, tc = tt - tr * tiles_c;
+            const int64_t rb = tr * COL_TR + 32 * warp, oc = tc * COL_TC + 2 * lane;
+            if (rb < p.rows && oc < p.cols) {
+                const int64_t kb = rb >> 5;
+                s0 = MMA ? p.scales[mma_scale_off(oc, kb, p.katoms)] : p.scales[oc * p.ld_scales + kb];
+                s1 = MMA ? p.scales[mma_scale_off(oc + 1, kb, p.katoms)] : p.scales[(oc + 1) * p.ld_scales + kb];
+            }
+        }
+    };
     int64_t t = blockIdx.x;
     if (t < ntiles) load(t, 0);
+    uint32_t sa = 0xFFu, sb = 0xFFu;
+    if constexpr (!F32) scale_pair(t, sa, sb);
     for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
         // the buffer refilled here was read in the previous iteration, which
         // ended with a barrier
         const int buf = it & 1;
         const int64_t tn = t + gridDim.x;
+        uint32_t sa_n = 0xFFu, sb_n = 0xFFu;
+        if constexpr (!F32) scale_pair(tn, sa_n, sb_n);
         if (tn < ntiles) {
             load(tn, buf ^ 1);
             asm volatile("cp.async.wait_group 1;" ::: "memory");
@@ -895,27 +1132,32 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
         if (rb < p.rows) {
           const int64_t kb = rb >> 5;
           if constexpr (!F32) {
-            // bf16 out: each column as 16 bf16 pairs along its rows (looked up,
-            // or transformed, rounded and sign-flipped as pairs), then one
-            // 32-bit word (columns 2l, 2l + 1) per row of the staged tile
+            // bf16 out: one 32-bit word (columns 2l, 2l + 1) per row of the
+            // staged tile
             const int64_t oc = c0 + 2 * lane;
             if (oc < p.cols) {                 // cols is even: oc + 1 < cols too
-                const uint32_t s0 = MMA ? p.scales[mma_scale_off(oc, kb, p.katoms)] : p.scales[oc * p.ld_scales + kb];
-                const uint32_t s1 =
-                    MMA ? p.scales[mma_scale_off(oc + 1, kb, p.katoms)] : p.scales[(oc + 1) * p.ld_scales + kb];
-                uint32_t pa[16], pb[16];
-                if constexpr (RHT == 0) {
-                    decode32_bf16(tin[buf][2 * lane][warp], s0, pa);
-                    decode32_bf16(tin[buf][2 * lane + 1][warp], s1, pb);
-                } else {
-                    column_rht_bf16<RHT>(tin[buf][2 * lane][warp], s0, p.sgn_pair, pa);
-                    column_rht_bf16<RHT>(tin[buf][2 * lane + 1][warp], s1, p.sgn_pair, pb);
-                }
                 uint32_t *w = reinterpret_cast<uint32_t *>(stage) + lane;
+                if constexpr (RHT == 0) {
+                    // each column as 16 looked-up bf16 pairs along its rows
+                    uint32_t pa[16], pb[16];
+                    decode32_bf16(tin[buf][2 * lane][warp], sa, pa);
+                    decode32_bf16(tin[buf][2 * lane + 1][warp], sb, pb);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    w[(2 * i) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x5410u);
-                    w[(2 * i + 1) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x7632u);
+                    for (int i = 0; i < 16; ++i) {
+                        w[(2 * i) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x5410u);
+                        w[(2 * i + 1) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x7632u);
+                    }
+                } else {
+                    // each column decoded, transformed, rounded and
+                    // sign-flipped as 16 bf16 pairs along its rows
+                    uint32_t pa[16], pb[16];
+                    column_rht_bf16<RHT>(tin[buf][2 * lane][warp], sa, p.sgn_pair, pa);
+                    column_rht_bf16<RHT>(tin[buf][2 * lane + 1][warp], sb, p.sgn_pair, pb);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        w[(2 * i) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x5410u);
+                        w[(2 * i + 1) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x7632u);
+                    }
                 }
             }
           } else {
@@ -958,6 +1200,8 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
             __syncwarp();
         }
         __syncthreads();
+        sa = sa_n;
+        sb = sb_n;
     }
 }
 
@@ -1120,7 +1364,27 @@ static cudaError_t launch_dual_t(DualParams p, cudaStream_t s) {
     return launch_pdl(kern, dim3((unsigned)(strips < cap ? strips : cap)), dim3(256), 0, s, p, (uint32_t)strips);
 }
 
-// 1D-column quantization: the column-only dual kernel on 128 x 64 tiles.
+// Column output only: the column quantizer on 256 x 64 tiles, persistent at
+// full occupancy (two CTAs per SM), strips as long as the grid stays full.
+template <int RHT, bool SR, bool MMA>
+static cudaError_t launch_col_t(DualParams p, cudaStream_t s) {
+    p.tiles_c = (uint32_t)((p.cols + CQ_TC - 1) / CQ_TC);
+    const uint64_t tiles_r = (uint64_t)((p.rows + CQ_TR - 1) / CQ_TR);
+    if (tiles_r * p.tiles_c > 0xFFFFFFFFull - 0x7FFFFFFFull) return cudaErrorInvalidValue;
+    p.tiles_r = (uint32_t)tiles_r;
+    auto kern = quant_col_kernel<RHT, SR, MMA>;
+    const cudaError_t ea = allow_dyn_smem(reinterpret_cast<const void *>(kern), CQ_SMEM);
+    if (ea != cudaSuccess) return ea;
+    const uint64_t cap =
+        (uint64_t)num_sms() * (uint64_t)resident_ctas(reinterpret_cast<const void *>(kern), 256, CQ_SMEM);
+    p.strip = tiles_r * p.tiles_c > 0 ? strip_len(tiles_r, p.tiles_c, cap) : 1u;
+    if (p.strip > 4) p.strip = 4;
+    const uint64_t strips = (tiles_r + p.strip - 1) / p.strip * p.tiles_c;
+    return launch_pdl(kern, dim3((unsigned)(strips < cap ? strips : cap)), dim3(256), (size_t)CQ_SMEM, s, p,
+                      (uint32_t)strips);
+}
+
+// 1D-column quantization through the column quantizer.
 template <int RHT, bool SR, bool MMA>
 static cudaError_t launch_col_dual(const QuantParams &q, cudaStream_t s) {
     DualParams p{};
@@ -1133,13 +1397,13 @@ static cudaError_t launch_col_dual(const QuantParams &q, cudaStream_t s) {
     p.c_offset = q.elem_offset;
     p.c_sr_ld = q.rows;
     for (int i = 0; i < 32; ++i) p.sgn_bit[i] = q.sgn_bit[i];
-    return launch_dual_t<DualCol, RHT, SR, MMA, false, true>(p, s);
+    return launch_col_t<RHT, SR, MMA>(p, s);
 }
 
 template <int CRHT, bool SR, bool MMA>
 static cudaError_t launch_dual_o(bool do_row, bool do_col, const DualParams &p, cudaStream_t s) {
     if (do_row && do_col) return launch_dual_t<DualBoth, CRHT, SR, MMA, true, true>(p, s);
-    if (do_col) return launch_dual_t<DualCol, CRHT, SR, MMA, false, true>(p, s);
+    if (do_col) return launch_col_t<CRHT, SR, MMA>(p, s);
     return launch_dual_t<DualBoth, CRHT, SR, MMA, true, false>(p, s);
 }
 

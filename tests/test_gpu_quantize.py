@@ -61,8 +61,8 @@ def test_quantize_bit_exact(layout, rht, rnd, scale_layout):
 @pytest.mark.parametrize("scale_layout", [mx.SCALES_ROWMAJOR, mx.SCALES_MMA])
 @pytest.mark.parametrize("rht", [0, 32])
 def test_column_quantizer_strips(rht, scale_layout):
-    """1D-column RNE on 65,632 x 1080: 513 row tiles of 128 (the last holds 96
-    rows, so 3 of its 4 K-blocks), 17 column tiles of 64 (the last holds 56
+    """1D-column RNE on 65,632 x 1080: 257 row tiles of 256 (the last holds 96
+    rows, so 3 of its 8 K-blocks), 17 column tiles of 64 (the last holds 56
     columns).  With 148 SMs the launcher walks strips of 8 vertically adjacent
     tiles whose scales leave together, so the last strip is one ragged tile;
     codes and scales must be bit-exact."""
