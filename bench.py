@@ -817,7 +817,7 @@ def main():
         n_sms = torch.cuda.get_device_properties(device).multi_processor_count
         ach = ipe * TOKENS * INTER / (kernels["quant_dy_dual_sr"]["us"] / 1e6) / 1e12
         peak_i = n_sms * 4 * 32 * clocks["sm_mhz"] * 1e6 / 1e12
-        roofline_sr = {"bound": "alu", "kernel": "quant_dual_kernel (dY: row SR + column RHT-32 SR)",
+        roofline_sr = {"bound": "alu", "kernel": "quant_dual_sr_kernel (dY: row SR + column RHT-32 SR)",
                        "achieved": ach, "peak": peak_i, "unit": "T thread-instructions/s", "frac": ach / peak_i,
                        "traffic": ncu_traffic("quant", ["quant_dy_dual_sr"]),
                        "peak_note": f"issue rate {n_sms} SMs x 4 schedulers x 32 lanes x {clocks['sm_mhz']:.0f} MHz "

@@ -307,41 +307,8 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
 
 
 // ---------------------------------------------------------------------------
-// Dual output: 1D-row blocks (no RHT) and 1D-column blocks (optional RHT along
-// rows) of the same tensor from one read.  The recipe quantizes activations
-// and gradients both ways (row blocks for fprop/dgrad, blocks along tokens for
-// wgrad).  A CTA streams TR x TC bf16 tiles through a double-buffered
-// shared-memory ring (cp.async; the row pitch is padded by 16 bytes, which
-// keeps both access patterns below conflict-free).  Each thread does one
-// column job and one row job through one inlined quantizer body:
-//   column job: thread (column c, row block b) reads 32 rows of column c and
-//     applies the RHT; the 16 bytes of transposed codes are staged in shared
-//     memory so that each output row leaves as TR/2 contiguous bytes;
-//   row job: thread (row r, column block b) reads 64 bytes of its row and
-//     stores 16 bytes of codes.
-// Either output may be disabled (DO_ROW / DO_COL); the column-only form with
-// tall 128 x 64 tiles is the 1D-column quantizer.
-//
-// Tiles are visited in strips of `strip` vertically adjacent tiles (same
-// columns, consecutive row bands), a CTA taking whole strips.  The column-only
-// form keeps a strip's scale bytes in shared memory and writes them when the
-// strip ends: each output row then receives 4 * strip contiguous bytes from
-// one CTA instead of 4-byte pieces from `strip` CTAs at different times (the
-// scattered partial-sector writes cost 30% of the kernel's time
-// on a 1 GiB tensor).  The dual form and stochastic rounding run strips of
-// one tile (SR launches one CTA per tile).
+// Parameters of the column quantizer and of the dual (row + column) quantizer.
 // ---------------------------------------------------------------------------
-template <int TR_, int TC_>
-struct DualTile {
-    static constexpr int TR = TR_, TC = TC_;          // tile rows, tile columns (TR * TC = 8192)
-    static constexpr int PITCH = TC + 8;              // bf16 per smem row
-    static constexpr int OCH = TR / 32;               // 16-byte code chunks per column output row
-    static constexpr int OSH = OCH == 4 ? 1 : 2;      // swizzle of those chunks (conflict-free staging)
-    static_assert(TR * TC == 8192 && (OCH == 2 || OCH == 4), "tile shape");
-};
-using DualBoth = DualTile<64, 128>;                  // row + column outputs
-using DualCol = DualTile<128, 64>;                   // column output only
-
 struct DualParams {
     const uint16_t *x;
     int64_t rows, cols, ld_x;
@@ -354,144 +321,9 @@ struct DualParams {
     uint64_t r_offset, c_offset;           // SR stream index of each output's first element
     int64_t c_sr_ld;                       // row length of the column output's SR view (the whole tensor's rows)
     uint32_t tiles_c, tiles_r;             // column tiles, row tiles
-    uint32_t strip;                        // tiles per strip (1 unless column-only; at most 8)
+    uint32_t strip;                        // column quantizer: tiles per strip (at most 8)
     uint32_t sgn_bit[32];                  // RHT sign of element i (mod the RHT size) as bit 31
 };
-
-// SR instantiations get up to 80 registers (3 CTAs per SM): the column block
-// (32 transformed values) and the Philox state together do not fit in 64.
-template <class T, int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
-__global__ void __launch_bounds__(256, SR ? 3 : 4) quant_dual_kernel(const DualParams p, const uint32_t nstrips) {
-    pdl_wait();
-    pdl_trigger();
-    constexpr int TR = T::TR, TC = T::TC, PITCH = T::PITCH, OCH = T::OCH;
-    constexpr bool STRIP = DO_COL && !DO_ROW;          // column scales staged per strip
-    constexpr int SPITCH = 9;                          // words per output row: 8 tiles x 4 bytes, +1 against bank conflicts
-    static_assert(!STRIP || OCH == 4, "one 4-byte scale word per output row and tile");
-    __shared__ __align__(16) uint16_t tin[2][TR * PITCH];
-    __shared__ __align__(16) uint4 tout[DO_COL ? TC * OCH : 1];   // column codes: TC rows x TR/2 bytes
-    __shared__ __align__(16) uint32_t ssc[STRIP ? TC * SPITCH : 1];
-    constexpr bool MULTI = STRIP && !SR;                // strips of several tiles (SR and dual: one tile)
-    const int tid = threadIdx.x;
-    const uint32_t strip = MULTI ? p.strip : 1u;
-    // tile k of strip S: row band (S / tiles_c) * strip + k, column band S % tiles_c
-    auto load = [&](uint32_t S, uint32_t k, int buf) {
-        const int64_t r0 = ((int64_t)(S / p.tiles_c) * strip + (MULTI ? k : 0u)) * TR, c0 = (int64_t)(S % p.tiles_c) * TC;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int idx = tid + 256 * i, row = idx / (TC / 8), ch = idx % (TC / 8);
-            const int64_t gr = r0 + row, gc = c0 + 8 * ch;
-            if (gr < p.rows && gc < p.cols) cp_async16(tin[buf] + row * PITCH + 8 * ch, p.x + gr * p.ld_x + gc);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-    uint32_t S = blockIdx.x, k = 0;
-    if (S < nstrips) load(S, 0, 0);
-    for (int it = 0; S < nstrips; ++it) {
-        // the next tile's load is in flight while this one is quantized
-        const int buf = it & 1;
-        const uint32_t band = S / p.tiles_c, tr = MULTI ? band * strip + k : band;
-        const bool last = !MULTI || k + 1 == strip || tr + 1 >= p.tiles_r;   // last tile of this strip
-        const uint32_t Sn = last ? S + gridDim.x : S, kn = (MULTI && !last) ? k + 1 : 0u;
-        if (Sn < nstrips) {
-            load(Sn, kn, buf ^ 1);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        } else {
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        }
-        __syncthreads();
-        const uint16_t *tile = tin[buf];
-        const int64_t r0 = (int64_t)tr * TR, c0 = (int64_t)(S - band * p.tiles_c) * TC;
-
-        {
-            if constexpr (DO_COL) {                          // column c, rows 32b .. 32b+31
-                const int c = tid % TC, b = tid / TC;
-                const int64_t orow = c0 + c, rin = r0 + 32 * b;
-                if (orow < p.cols && rin < p.rows) {
-                    const uint16_t *col = tile + 32 * b * PITCH + c;
-                    float2 P[16];                    // (v[m], v[m + 16]): packed two-lane arithmetic
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        // bf16 -> fp32 with the RHT sign: adding 2^31 flips bit 31
-                        const uint32_t u0 = (uint32_t)col[m * PITCH] * 65536u + (CRHT ? p.sgn_bit[m] : 0u);
-                        const uint32_t u1 = (uint32_t)col[(m + 16) * PITCH] * 65536u + (CRHT ? p.sgn_bit[m + 16] : 0u);
-                        P[m] = make_float2(__uint_as_float(u0), __uint_as_float(u1));
-                    }
-                    if constexpr (CRHT) {
-                        const float cn = rht_norm<CRHT>();
-                        fwht_pairs<CRHT>(P);
-#pragma unroll
-                        for (int m = 0; m < 16; ++m) P[m] = mul2(P[m], make_float2(cn, cn));
-                    }
-                    uint4 q;
-                    const uint64_t g0 = (uint64_t)(orow * p.c_sr_ld + rin) + p.c_offset;
-                    const uint32_t sc = quantize32_pairs<SR>(P, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
-                    tout[c * OCH + (b ^ ((c >> T::OSH) & (OCH - 1)))] = q;
-                    const int64_t kb = rin >> 5;
-                    if constexpr (STRIP) reinterpret_cast<uint8_t *>(ssc)[4 * (c * SPITCH + (MULTI ? k : 0u)) + b] = (uint8_t)sc;
-                    else if constexpr (MMA) p.cscales[mma_scale_off(orow, kb, p.c_katoms)] = (uint8_t)sc;
-                    else p.cscales[orow * p.ld_cscales + kb] = (uint8_t)sc;
-                }
-            }
-            if constexpr (DO_ROW) {                          // row r, columns 32b .. 32b+31
-                const int r = tid % TR, b = tid / TR;
-                const int64_t orow = r0 + r, gc = c0 + 32 * b;
-                if (orow < p.rows && gc < p.cols) {
-                    const uint4 *s4 = reinterpret_cast<const uint4 *>(tile + r * PITCH + 32 * b);
-                    const uint4 u[4] = {s4[0], s4[1], s4[2], s4[3]};
-                    uint4 q;
-                    const uint64_t g0 = (uint64_t)(orow * p.cols + gc) + p.r_offset;
-                    const uint32_t sc = quantize32_bf16<SR>(u, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
-                    const int64_t kb = gc >> 5;
-                    stg_v4(p.rcodes + orow * p.ld_rcodes + kb * 16, q);
-                    if constexpr (MMA) p.rscales[mma_scale_off(orow, kb, p.r_katoms)] = (uint8_t)sc;
-                    else p.rscales[orow * p.ld_rscales + kb] = (uint8_t)sc;
-                }
-            }
-        }
-        if constexpr (DO_COL) {
-            __syncthreads();
-            // column codes: TC output rows x OCH chunks of 16 bytes, one chunk per thread
-            const int row = tid / OCH, ch = tid % OCH;
-            const int64_t orow = c0 + row, rin = r0 + 32 * ch;
-            if (orow < p.cols && rin < p.rows)
-                stg_v4(p.ccodes + orow * p.ld_ccodes + (rin >> 1), tout[row * OCH + (ch ^ ((row >> T::OSH) & (OCH - 1)))]);
-        }
-        if constexpr (STRIP) {
-            if (last) {                                      // the strip's scales: k + 1 words per output row
-                const int64_t kb0 = (int64_t)band * strip * 4;
-                if constexpr (MMA) {
-                    // the 4 K-blocks of one tile are 4 contiguous bytes of an MMA atom row slot
-                    for (uint32_t idx = tid; idx < TC * (k + 1); idx += 256) {
-                        const uint32_t a = idx / TC, row = idx % TC;
-                        const int64_t orow = c0 + row, kb = kb0 + 4 * a;
-                        if (orow < p.cols && kb * 32 < p.rows) {
-                            uint8_t *dst = p.cscales + mma_scale_off(orow, kb, p.c_katoms);
-                            const uint32_t w = ssc[row * SPITCH + a];
-                            if ((kb + 4) * 32 <= p.rows) {
-                                *reinterpret_cast<uint32_t *>(dst) = w;
-                            } else {                         // ragged last tile: valid K-blocks only
-                                for (int j = 0; j < 4 && (kb + j) * 32 < p.rows; ++j) dst[j] = (uint8_t)(w >> (8 * j));
-                            }
-                        }
-                    }
-                } else {
-                    // row-major: consecutive threads write consecutive bytes of one output row
-                    const uint32_t nb = 4 * (k + 1);
-                    const uint8_t *sb = reinterpret_cast<const uint8_t *>(ssc);
-                    for (uint32_t idx = tid; idx < TC * nb; idx += 256) {
-                        const uint32_t row = idx / nb, j = idx - row * nb;
-                        const int64_t orow = c0 + row, kb = kb0 + j;
-                        if (orow < p.cols && kb * 32 < p.rows) p.cscales[orow * p.ld_cscales + kb] = sb[4 * row * SPITCH + j];
-                    }
-                }
-            }
-        }
-        __syncthreads();                                     // the load after next overwrites this buffer
-        S = Sn;
-        k = kn;
-    }
-}
 
 // ---------------------------------------------------------------------------
 // 1D-column quantizer (blocks of 32 along rows; output [cols, rows / 2]).  A
@@ -547,6 +379,52 @@ __device__ __forceinline__ uint4 encode_col_lane(const float2 *P, uint64_t g0, u
         else q[g] = e2m1x8_rn(w);
     }
     return make_uint4(q[0], q[1], q[2], q[3]);
+}
+
+// One column-pair job: rows rin .. rin + 31 of output rows (columns) oc and
+// oc + 1, lane word m at src[m * wstride] of a staged tile (bf16 of column oc
+// in the low half).  The codes of each column (16 bytes) and its scale code;
+// a NaN block (scale code 0xFF) gets zero codes.
+template <int RHT, bool SR>
+__device__ __forceinline__ void col_pair_job(const uint32_t *src, int wstride, const DualParams &p, int64_t oc,
+                                             int64_t rin, uint4 &qlo, uint4 &qhi, uint32_t &slo, uint32_t &shi) {
+    float2 P[32];                            // (column oc, column oc + 1) at row rin + m
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
+        // bf16 -> fp32 with the RHT sign: adding 2^31 flips bit 31
+        const uint32_t u = src[m * wstride];
+        const uint32_t sg = RHT ? p.sgn_bit[m] : 0u;
+        P[m] = make_float2(__uint_as_float(u * 65536u + sg), __uint_as_float((u & 0xFFFF0000u) ^ sg));
+    }
+    if constexpr (RHT != 0) {
+        const float cn = rht_norm<RHT>();
+        fwht_col_pairs<RHT>(P);
+#pragma unroll
+        for (int m = 0; m < 32; ++m) P[m] = mul2(P[m], make_float2(cn, cn));
+    }
+    float alo = 0.0f, ahi = 0.0f;
+#pragma unroll
+    for (int m = 0; m < 32; m += 2) {
+        alo = amax_nan2(alo, P[m].x, P[m + 1].x);
+        ahi = amax_nan2(ahi, P[m].y, P[m + 1].y);
+    }
+    slo = scale_code_rule(alo, p.scale_rule);
+    shi = scale_code_rule(ahi, p.scale_rule);
+    // a NaN block's lane is scaled by 1 and its codes replaced by zeros
+    const float2 inv = make_float2(slo == 0xFFu ? 1.0f : inv_scale_from_code(slo),
+                                   shi == 0xFFu ? 1.0f : inv_scale_from_code(shi));
+    if (p.scale_rule == 2) {
+#pragma unroll
+        for (int m = 0; m < 32; ++m) P[m] = mul2(mul2(P[m], make_float2(0.75f, 0.75f)), inv);
+    } else {
+#pragma unroll
+        for (int m = 0; m < 32; ++m) P[m] = mul2(P[m], inv);
+    }
+    const uint64_t g0 = (uint64_t)(oc * p.c_sr_ld + rin) + p.c_offset;
+    qlo = encode_col_lane<SR, false>(P, g0, p.seed_lo, p.seed_hi);
+    qhi = encode_col_lane<SR, true>(P, g0 + (uint64_t)p.c_sr_ld, p.seed_lo, p.seed_hi);
+    if (slo == 0xFFu) qlo = make_uint4(0, 0, 0, 0);
+    if (shi == 0xFFu) qhi = make_uint4(0, 0, 0, 0);
 }
 
 template <int RHT, bool SR, bool MMA>
@@ -611,42 +489,9 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const DualParams p, c
         if (rin < p.rows && oc < p.cols) {
             const uint32_t *src =
                 reinterpret_cast<const uint32_t *>(ring + (it % CQ_STAGES) * CQ_TILE_BYTES) + warp * 32 * 32 + lane;
-            float2 P[32];                            // (column oc, column oc + 1) at row rin + m
-#pragma unroll
-            for (int m = 0; m < 32; ++m) {
-                // bf16 -> fp32 with the RHT sign: adding 2^31 flips bit 31
-                const uint32_t u = src[m * 32];
-                const uint32_t sg = RHT ? p.sgn_bit[m] : 0u;
-                P[m] = make_float2(__uint_as_float(u * 65536u + sg), __uint_as_float((u & 0xFFFF0000u) ^ sg));
-            }
-            if constexpr (RHT != 0) {
-                const float cn = rht_norm<RHT>();
-                fwht_col_pairs<RHT>(P);
-#pragma unroll
-                for (int m = 0; m < 32; ++m) P[m] = mul2(P[m], make_float2(cn, cn));
-            }
-            float alo = 0.0f, ahi = 0.0f;
-#pragma unroll
-            for (int m = 0; m < 32; m += 2) {
-                alo = amax_nan2(alo, P[m].x, P[m + 1].x);
-                ahi = amax_nan2(ahi, P[m].y, P[m + 1].y);
-            }
-            const uint32_t slo = scale_code_rule(alo, p.scale_rule), shi = scale_code_rule(ahi, p.scale_rule);
-            // a NaN block (code 0xFF) stores zero codes; its lane is scaled by 1
-            const float2 inv = make_float2(slo == 0xFFu ? 1.0f : inv_scale_from_code(slo),
-                                           shi == 0xFFu ? 1.0f : inv_scale_from_code(shi));
-            if (p.scale_rule == 2) {
-#pragma unroll
-                for (int m = 0; m < 32; ++m) P[m] = mul2(mul2(P[m], make_float2(0.75f, 0.75f)), inv);
-            } else {
-#pragma unroll
-                for (int m = 0; m < 32; ++m) P[m] = mul2(P[m], inv);
-            }
-            const uint64_t g0 = (uint64_t)(oc * p.c_sr_ld + rin) + p.c_offset;
-            uint4 qlo = encode_col_lane<SR, false>(P, g0, p.seed_lo, p.seed_hi);
-            uint4 qhi = encode_col_lane<SR, true>(P, g0 + (uint64_t)p.c_sr_ld, p.seed_lo, p.seed_hi);
-            if (slo == 0xFFu) qlo = make_uint4(0, 0, 0, 0);
-            if (shi == 0xFFu) qhi = make_uint4(0, 0, 0, 0);
+            uint4 qlo, qhi;
+            uint32_t slo, shi;
+            col_pair_job<RHT, SR>(src, 32, p, oc, rin, qlo, qhi, slo, shi);
             const int c = 2 * lane, sw = warp ^ (lane & 7);
             tout[c * 8 + sw] = qlo;
             tout[(c + 1) * 8 + sw] = qhi;
@@ -714,6 +559,211 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const DualParams p, c
 }
 
 // ---------------------------------------------------------------------------
+// Dual output: 1D-row blocks (no RHT) and 1D-column blocks (optional RHT along
+// rows) of the same tensor from one read.  The recipe quantizes activations
+// and gradients both ways (row blocks for fprop and dgrad, blocks along
+// tokens for wgrad).  Under round-to-nearest (SR runs the kernel below) a CTA
+// streams 128 x 64 bf16 tiles through a three-deep cp.async ring (rows padded
+// to 144 bytes, which keeps both access patterns conflict-free), and its
+// warps specialise:
+//   warps 0-3, column jobs: warp w takes row block w, lane l the column pair
+//     (2l, 2l + 1) as packed fp32 lanes, as in the column quantizer; the
+//     codes are staged so that each output row leaves as 64 contiguous bytes;
+//   warps 4-7, row jobs: thread r takes row r of the tile, both of its 32-
+//     element blocks (64 bytes each from shared memory), 32 bytes of codes.
+// The two halves carry about the same instruction count per tile.
+// ---------------------------------------------------------------------------
+constexpr int DQ_TR = 128, DQ_TC = 64, DQ_STAGES = 3;
+constexpr int DQ_PITCH = DQ_TC * 2 + 16;                               // staged bytes per tile row
+constexpr int DQ_TILE_BYTES = DQ_TR * DQ_PITCH;                        // 18 KB
+constexpr int DQ_OUT_BYTES = DQ_TC * (DQ_TR / 2);                      // 4 KB of column codes
+constexpr int DQ_SMEM = DQ_STAGES * DQ_TILE_BYTES + DQ_OUT_BYTES;
+
+template <int CRHT, bool MMA>
+__global__ void __launch_bounds__(256, 2) quant_dual_kernel(const DualParams p, const uint32_t ntiles) {
+    pdl_wait();
+    pdl_trigger();
+    extern __shared__ __align__(16) uint8_t dq_smem[];
+    uint8_t *ring = dq_smem;
+    uint4 *tout = reinterpret_cast<uint4 *>(dq_smem + DQ_STAGES * DQ_TILE_BYTES);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    auto load = [&](uint32_t t, int buf) {
+        if (t < ntiles) {
+            const uint32_t tr = t / p.tiles_c;
+            const int64_t r0 = (int64_t)tr * DQ_TR, c0 = (int64_t)(t - tr * p.tiles_c) * DQ_TC;
+            const int ch = tid & 7, row = tid >> 3;            // rows row + 32 i, 16-byte chunk ch
+            const int64_t gc = c0 + 8 * ch;
+            const uint16_t *src = p.x + (r0 + row) * p.ld_x + gc;
+            uint8_t *dst = ring + buf * DQ_TILE_BYTES + row * DQ_PITCH + 16 * ch;
+            if (r0 + DQ_TR <= p.rows && c0 + DQ_TC <= p.cols) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) cp_async16(dst + i * 32 * DQ_PITCH, src + (int64_t)i * 32 * p.ld_x);
+            } else if (gc < p.cols) {                            // cols % 32 == 0: a chunk is whole or absent
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    if (r0 + row + 32 * i < p.rows) cp_async16(dst + i * 32 * DQ_PITCH, src + (int64_t)i * 32 * p.ld_x);
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    uint32_t t = blockIdx.x;
+    load(t, 0);
+    load(t + gridDim.x, 1);
+    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+        // two tiles in flight while this one is quantized; the buffer loaded
+        // here was read in the previous iteration, before its barrier
+        load(t + 2 * gridDim.x, (it + 2) % DQ_STAGES);
+        asm volatile("cp.async.wait_group 2;" ::: "memory");
+        __syncthreads();
+        const uint32_t tr = t / p.tiles_c;
+        const int64_t r0 = (int64_t)tr * DQ_TR, c0 = (int64_t)(t - tr * p.tiles_c) * DQ_TC;
+        const uint8_t *tile = ring + (it % DQ_STAGES) * DQ_TILE_BYTES;
+        if (warp < 4) {                                          // column pair (2 lane, 2 lane + 1), row block warp
+            const int64_t rin = r0 + 32 * warp, oc = c0 + 2 * lane;
+            if (rin < p.rows && oc < p.cols) {
+                const uint32_t *src = reinterpret_cast<const uint32_t *>(tile + 32 * warp * DQ_PITCH) + lane;
+                uint4 qlo, qhi;
+                uint32_t slo, shi;
+                col_pair_job<CRHT, false>(src, DQ_PITCH / 4, p, oc, rin, qlo, qhi, slo, shi);
+                const int c = 2 * lane, sw = warp ^ (lane & 3);
+                tout[c * 4 + sw] = qlo;
+                tout[(c + 1) * 4 + sw] = qhi;
+                const int64_t kb = rin >> 5;
+                if constexpr (MMA) {
+                    p.cscales[mma_scale_off(oc, kb, p.c_katoms)] = (uint8_t)slo;
+                    p.cscales[mma_scale_off(oc + 1, kb, p.c_katoms)] = (uint8_t)shi;
+                } else {
+                    p.cscales[oc * p.ld_cscales + kb] = (uint8_t)slo;
+                    p.cscales[(oc + 1) * p.ld_cscales + kb] = (uint8_t)shi;
+                }
+            }
+        } else {                                                 // row r, both 32-element blocks
+            const int r = tid - 128;
+            const int64_t orow = r0 + r;
+            if (orow < p.rows) {
+                const uint4 *s4 = reinterpret_cast<const uint4 *>(tile + r * DQ_PITCH);
+#pragma unroll 1
+                for (int b = 0; b < 2; ++b) {
+                    const int64_t gc = c0 + 32 * b;
+                    if (gc < p.cols) {
+                        const uint4 u[4] = {s4[4 * b], s4[4 * b + 1], s4[4 * b + 2], s4[4 * b + 3]};
+                        uint4 q;
+                        const uint64_t g0 = (uint64_t)(orow * p.cols + gc) + p.r_offset;
+                        const uint32_t sc = quantize32_bf16<false>(u, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
+                        const int64_t kb = gc >> 5;
+                        stg_v4(p.rcodes + orow * p.ld_rcodes + kb * 16, q);
+                        if constexpr (MMA) p.rscales[mma_scale_off(orow, kb, p.r_katoms)] = (uint8_t)sc;
+                        else p.rscales[orow * p.ld_rscales + kb] = (uint8_t)sc;
+                    }
+                }
+            }
+        }
+        __syncthreads();                                         // tile read; column codes staged
+        {   // column codes: 64 output rows x 4 chunks of 16 bytes, 4 lanes per row
+            const int row = tid >> 2, ch = tid & 3;
+            const int64_t orow = c0 + row, rb = r0 + 32 * ch;
+            if (orow < p.cols && rb < p.rows)
+                stg_v4(p.ccodes + orow * p.ld_ccodes + (rb >> 1), tout[row * 4 + (ch ^ ((row >> 1) & 3))]);
+        }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// The dual quantizer under stochastic rounding, where Philox4x32-10 and the
+// SR decision bound the kernel by integer issue rather than by HBM: more warps
+// per SM matter more than wide jobs.  A CTA takes one 64 x 128 tile (rows
+// padded by 16 bytes) and each thread does one column job, 32 rows of one
+// column held as the pairs (v[m], v[m + 16]) of the packed butterfly, and one
+// row job, 32 columns of one row; 80 registers, three CTAs per SM.
+constexpr int DS_TR = 64, DS_TC = 128, DS_PITCH = DS_TC + 8;          // bf16 per staged row
+
+template <int CRHT, bool MMA>
+__global__ void __launch_bounds__(256, 3) quant_dual_sr_kernel(const DualParams p, const uint32_t ntiles) {
+    pdl_wait();
+    pdl_trigger();
+    __shared__ __align__(16) uint16_t tin[2][DS_TR * DS_PITCH];
+    __shared__ __align__(16) uint4 tout[DS_TC * 2];         // column codes: 128 output rows x 32 bytes
+    const int tid = threadIdx.x;
+    auto load = [&](uint32_t t, int buf) {
+        const int64_t r0 = (int64_t)(t / p.tiles_c) * DS_TR, c0 = (int64_t)(t % p.tiles_c) * DS_TC;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int idx = tid + 256 * i, row = idx / (DS_TC / 8), ch = idx % (DS_TC / 8);
+            const int64_t gr = r0 + row, gc = c0 + 8 * ch;
+            if (gr < p.rows && gc < p.cols) cp_async16(tin[buf] + row * DS_PITCH + 8 * ch, p.x + gr * p.ld_x + gc);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    uint32_t t = blockIdx.x;
+    if (t < ntiles) load(t, 0);
+    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+        // the next tile's load is in flight while this one is quantized
+        const int buf = it & 1;
+        const uint32_t tn = t + gridDim.x;
+        if (tn < ntiles) {
+            load(tn, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
+        const uint16_t *tile = tin[buf];
+        const int64_t r0 = (int64_t)(t / p.tiles_c) * DS_TR, c0 = (int64_t)(t % p.tiles_c) * DS_TC;
+        {                                                    // column c, rows 32b .. 32b + 31
+            const int c = tid % DS_TC, b = tid / DS_TC;
+            const int64_t orow = c0 + c, rin = r0 + 32 * b;
+            if (orow < p.cols && rin < p.rows) {
+                const uint16_t *col = tile + 32 * b * DS_PITCH + c;
+                float2 P[16];                        // (v[m], v[m + 16]): packed two-lane arithmetic
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    // bf16 -> fp32 with the RHT sign: adding 2^31 flips bit 31
+                    const uint32_t u0 = (uint32_t)col[m * DS_PITCH] * 65536u + (CRHT ? p.sgn_bit[m] : 0u);
+                    const uint32_t u1 = (uint32_t)col[(m + 16) * DS_PITCH] * 65536u + (CRHT ? p.sgn_bit[m + 16] : 0u);
+                    P[m] = make_float2(__uint_as_float(u0), __uint_as_float(u1));
+                }
+                if constexpr (CRHT) {
+                    const float cn = rht_norm<CRHT>();
+                    fwht_pairs<CRHT>(P);
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) P[m] = mul2(P[m], make_float2(cn, cn));
+                }
+                uint4 q;
+                const uint64_t g0 = (uint64_t)(orow * p.c_sr_ld + rin) + p.c_offset;
+                const uint32_t sc = quantize32_pairs<true>(P, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
+                tout[c * 2 + (b ^ ((c >> 2) & 1))] = q;
+                const int64_t kb = rin >> 5;
+                if constexpr (MMA) p.cscales[mma_scale_off(orow, kb, p.c_katoms)] = (uint8_t)sc;
+                else p.cscales[orow * p.ld_cscales + kb] = (uint8_t)sc;
+            }
+        }
+        {                                                    // row r, columns 32b .. 32b + 31
+            const int r = tid % DS_TR, b = tid / DS_TR;
+            const int64_t orow = r0 + r, gc = c0 + 32 * b;
+            if (orow < p.rows && gc < p.cols) {
+                const uint4 *s4 = reinterpret_cast<const uint4 *>(tile + r * DS_PITCH + 32 * b);
+                const uint4 u[4] = {s4[0], s4[1], s4[2], s4[3]};
+                uint4 q;
+                const uint64_t g0 = (uint64_t)(orow * p.cols + gc) + p.r_offset;
+                const uint32_t sc = quantize32_bf16<true>(u, q, g0, p.seed_lo, p.seed_hi, p.scale_rule);
+                const int64_t kb = gc >> 5;
+                stg_v4(p.rcodes + orow * p.ld_rcodes + kb * 16, q);
+                if constexpr (MMA) p.rscales[mma_scale_off(orow, kb, p.r_katoms)] = (uint8_t)sc;
+                else p.rscales[orow * p.ld_rscales + kb] = (uint8_t)sc;
+            }
+        }
+        __syncthreads();
+        {   // column codes: 128 output rows x 2 chunks of 16 bytes, one chunk per thread
+            const int row = tid >> 1, ch = tid & 1;
+            const int64_t orow = c0 + row, rin = r0 + 32 * ch;
+            if (orow < p.cols && rin < p.rows)
+                stg_v4(p.ccodes + orow * p.ld_ccodes + (rin >> 1), tout[row * 2 + (ch ^ ((row >> 2) & 1))]);
+        }
+        __syncthreads();                                     // the load after next overwrites this buffer
+    }
+}
+
+// ---------------------------------------------------------------------------
 // 2D 32x32 blocks.  A CTA streams tiles of 8 blocks through a double-buffered
 // shared-memory ring (cp.async of whole tile rows, so the global reads are
 // coalesced): 32 x 256 (one block row) without the transposed copy, 128 x 64
@@ -733,8 +783,9 @@ struct Q2Tile {
     static constexpr int CHUNKS = COLS / 8;           // 16-byte chunks per row
 };
 
+
 template <int RHT, bool SR, bool MMA, bool TRANS>
-__global__ void __launch_bounds__(256, 3) quant_2d_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(256, SR ? 3 : 4) quant_2d_kernel(const QuantParams p) {
     pdl_wait();
     pdl_trigger();
     using T = Q2Tile<TRANS>;
@@ -778,33 +829,37 @@ __global__ void __launch_bounds__(256, 3) quant_2d_kernel(const QuantParams p) {
                 const uint4 u = s4[q];
                 w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
             }
-            float v[32];
-            unpack_row32<RHT>(w, v, p);
-            float amax = 0.0f;
+            // the block's amax is the warp max of the lanes' row maxima
+            auto warp_amax = [](float amax) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) amax = amax_nan(amax, v[i]);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float other = __shfl_xor_sync(0xFFFFFFFFu, amax, o);
-                asm("max.NaN.f32 %0, %0, %1;" : "+f"(amax) : "f"(other));
-            }
-            const uint32_t code = scale_code_rule(amax, p.scale_rule);
-            uint4 packed = make_uint4(0, 0, 0, 0);
-            if (code != 0xFFu) {
-                const float inv = inv_scale_from_code(code);
-                scale_block32(v, inv, p.scale_rule);
-                uint32_t pk[4];
-                if constexpr (!SR) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) pk[q] = e2m1x8_rn(v + 8 * q);
-                } else {
-                    const uint64_t blk = ((uint64_t)(r * p.cols + c0) + p.elem_offset) >> 2;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        pk[q] = e2m1x8_sr(v + 8 * q, blk + 2 * q, p.seed_lo, p.seed_hi);
-                    }
+                for (int o = 16; o > 0; o >>= 1) {
+                    const float other = __shfl_xor_sync(0xFFFFFFFFu, amax, o);
+                    asm("max.NaN.f32 %0, %0, %1;" : "+f"(amax) : "f"(other));
                 }
-                packed = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                return amax;
+            };
+            uint4 packed;
+            uint32_t code;
+            const uint64_t g0 = (uint64_t)(r * p.cols + c0) + p.elem_offset;
+            if constexpr (RHT) {
+                // the row stays in the packed butterfly's pairs through scaling and rounding
+                float2 P[16];
+                unpack_row32_pairs<RHT>(w, P, p);
+                code = quantize32_pairs_amax<SR>(P, warp_amax(amax_pairs(P)), packed, g0, p.seed_lo, p.seed_hi,
+                                                 p.scale_rule);
+            } else {
+                float v[32];
+                unpack_row32<0>(w, v, p);
+                float amax = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) amax = amax_nan2(amax, v[i], v[i + 1]);
+                code = quantize_groups<SR>(
+                    warp_amax(amax),
+                    [&](int q, float *u) {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) u[j] = v[8 * q + j];
+                    },
+                    packed, g0, p.seed_lo, p.seed_hi, p.scale_rule);
             }
             stg_v4(p.codes + r * p.ld_codes + (c0 >> 1), packed);
             if constexpr (MMA) {
@@ -1277,7 +1332,7 @@ static cudaError_t launch_quant_t(int layout, bool trans, const QuantParams &p, 
     if (layout == MXFP4_LAYOUT_1D_ROW) {
         return launch_pdl(quant_row_kernel<RHT, SR, MMA>, dim3((unsigned)grid_for(p.rows * (p.cols / 32), 256)), dim3(256), 0, s, p);
     } else if (layout == MXFP4_LAYOUT_1D_COL) {
-        return launch_col_dual<RHT, SR, MMA>(p, s);      // the dual kernel, column output only
+        return launch_col_dual<RHT, SR, MMA>(p, s);      // the column quantizer
     } else {
         const int br = trans ? Q2Tile<true>::BR : Q2Tile<false>::BR;
         const int64_t tiles = ((p.rows / 32 + br - 1) / br) * ((p.cols / 32 + 8 / br - 1) / (8 / br));
@@ -1346,22 +1401,35 @@ static uint32_t strip_len(uint64_t tiles_r, uint64_t tiles_c, uint64_t grid) {
     return best;
 }
 
-template <class T, int CRHT, bool SR, bool MMA, bool DO_ROW, bool DO_COL>
+// Both outputs under SR: one CTA per 64 x 128 tile (the hardware scheduler
+// balances the tail of an issue-bound kernel).
+template <int CRHT, bool MMA>
+static cudaError_t launch_dual_sr(DualParams p, cudaStream_t s) {
+    p.tiles_c = (uint32_t)((p.cols + DS_TC - 1) / DS_TC);
+    const uint64_t tiles = (uint64_t)((p.rows + DS_TR - 1) / DS_TR) * p.tiles_c;
+    if (tiles > 0x7FFFFFFFull) return cudaErrorInvalidValue;
+    return launch_pdl(quant_dual_sr_kernel<CRHT, MMA>, dim3((unsigned)tiles), dim3(256), 0, s, p, (uint32_t)tiles);
+}
+
+// Both outputs: under RNE the dual quantizer, persistent at full occupancy.
+template <int CRHT, bool SR, bool MMA>
 static cudaError_t launch_dual_t(DualParams p, cudaStream_t s) {
-    p.tiles_c = (uint32_t)((p.cols + T::TC - 1) / T::TC);
-    const uint64_t tiles_r = (uint64_t)((p.rows + T::TR - 1) / T::TR);
-    const uint64_t tiles = tiles_r * p.tiles_c;
-    if (tiles > 0xFFFFFFFFull - 0x7FFFFFFFull) return cudaErrorInvalidValue;   // tile index fits 32 bits
-    p.tiles_r = (uint32_t)tiles_r;
-    auto kern = quant_dual_kernel<T, CRHT, SR, MMA, DO_ROW, DO_COL>;
-    // RNE is memory-bound: a persistent grid at full occupancy keeps the next
-    // tile's load in flight.  SR is ALU-bound: one CTA per tile lets the
-    // hardware scheduler balance the tail.
-    const uint64_t cap = SR ? 0x7FFFFFFFull
-                            : (uint64_t)num_sms() * (uint64_t)resident_ctas(reinterpret_cast<const void *>(kern), 256);
-    p.strip = (!SR && DO_COL && !DO_ROW && tiles > 0) ? strip_len(tiles_r, p.tiles_c, cap) : 1u;
-    const uint64_t strips = (tiles_r + p.strip - 1) / p.strip * p.tiles_c;
-    return launch_pdl(kern, dim3((unsigned)(strips < cap ? strips : cap)), dim3(256), 0, s, p, (uint32_t)strips);
+    if constexpr (SR) {
+        return launch_dual_sr<CRHT, MMA>(p, s);
+    } else {
+        p.tiles_c = (uint32_t)((p.cols + DQ_TC - 1) / DQ_TC);
+        const uint64_t tiles_r = (uint64_t)((p.rows + DQ_TR - 1) / DQ_TR);
+        const uint64_t tiles = tiles_r * p.tiles_c;
+        if (tiles > 0xFFFFFFFFull - 0x7FFFFFFFull) return cudaErrorInvalidValue;   // tile index fits 32 bits
+        p.tiles_r = (uint32_t)tiles_r;
+        auto kern = quant_dual_kernel<CRHT, MMA>;
+        const cudaError_t ea = allow_dyn_smem(reinterpret_cast<const void *>(kern), DQ_SMEM);
+        if (ea != cudaSuccess) return ea;
+        const uint64_t cap =
+            (uint64_t)num_sms() * (uint64_t)resident_ctas(reinterpret_cast<const void *>(kern), 256, DQ_SMEM);
+        return launch_pdl(kern, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(256), (size_t)DQ_SMEM, s, p,
+                          (uint32_t)tiles);
+    }
 }
 
 // Column output only: the column quantizer on 256 x 64 tiles, persistent at
@@ -1402,9 +1470,19 @@ static cudaError_t launch_col_dual(const QuantParams &q, cudaStream_t s) {
 
 template <int CRHT, bool SR, bool MMA>
 static cudaError_t launch_dual_o(bool do_row, bool do_col, const DualParams &p, cudaStream_t s) {
-    if (do_row && do_col) return launch_dual_t<DualBoth, CRHT, SR, MMA, true, true>(p, s);
+    if (do_row && do_col) return launch_dual_t<CRHT, SR, MMA>(p, s);
     if (do_col) return launch_col_t<CRHT, SR, MMA>(p, s);
-    return launch_dual_t<DualBoth, CRHT, SR, MMA, true, false>(p, s);
+    // row output only: the row quantizer (no RHT) with the row output's offset
+    QuantParams q{};
+    q.x = p.x;
+    q.rows = p.rows; q.cols = p.cols; q.ld_x = p.ld_x;
+    q.codes = p.rcodes; q.ld_codes = p.ld_rcodes;
+    q.scales = p.rscales; q.ld_scales = p.ld_rscales; q.katoms = p.r_katoms;
+    q.seed_lo = p.seed_lo; q.seed_hi = p.seed_hi;
+    q.scale_rule = p.scale_rule;
+    q.elem_offset = p.r_offset;
+    return launch_pdl(quant_row_kernel<0, SR, MMA>, dim3((unsigned)grid_for(q.rows * (q.cols / 32), 256)), dim3(256),
+                      0, s, q);
 }
 
 template <int CRHT>
