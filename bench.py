@@ -447,6 +447,22 @@ def grouped_bench(mx, torch, device, peaks, reps=10):
     return out
 
 
+class L2Flush:
+    """Evicts L2 between timed launches, outside their events: writes a buffer
+    larger than L2, then reads a second one, so that the lines left in L2 are
+    clean.  After a write alone the timed launch also pays for writing the
+    flush's 126 MB of dirty lines back to HBM (the sweep's 256 MiB row
+    quantizer measured 0.85 of HBM that way, 0.99 with the read)."""
+
+    def __init__(self, torch, device, mib=256):
+        self.w = torch.empty(mib << 20, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(mib << 20, dtype=torch.uint8, device=device)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.amax()
+
+
 def _timed_flushed(torch, fn, reps, flush):
     """Median time (ms) of `reps` launches, L2 flushed before each (outside the
     events), events on the current stream."""
@@ -454,7 +470,7 @@ def _timed_flushed(torch, fn, reps, flush):
     torch.cuda.synchronize()
     ts = []
     for _ in range(reps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         fn()
@@ -477,7 +493,7 @@ def sweep_bench(mx, torch, device, peaks, sizes_mib=SWEEP_MIB, widths=SWEEP_COLS
     2D: + 1/1024), and the reverse for dequantize.  L2 is flushed before every
     launch, so the tensors that fit in L2 are timed from HBM too.  Each mode
     maps to [quantize GB/s, fraction of HBM, dequantize GB/s, fraction]."""
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(torch, device)
     hbm = peaks["hbm"]
     table = {}
     worst = {}
@@ -546,7 +562,7 @@ def bf16_out_bench(mx, torch, device, peaks, reps=20):
     c32 = torch.empty((TOKENS, INTER), dtype=torch.float32, device=device)
     c16 = torch.empty((TOKENS, INTER), dtype=torch.bfloat16, device=device)
     cq = mx.mxfp4_gemm_mxfp4(qa.codes, qa.scales, qw.codes, qw.scales, HIDDEN, scale_layout=mx.SCALES_MMA)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(torch, device)
     res = {}
     for name, fn in (("fp32_out", lambda: mx.mxfp4_gemm(qa.codes, qa.scales, qw.codes, qw.scales, HIDDEN, out=c32)),
                      ("bf16_out", lambda: mx.mxfp4_gemm_bf16(qa.codes, qa.scales, qw.codes, qw.scales, HIDDEN,
@@ -557,7 +573,7 @@ def bf16_out_bench(mx, torch, device, peaks, reps=20):
         torch.cuda.synchronize()
         ts = []
         for _ in range(reps):
-            flush.zero_()
+            flush()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
             fn()
@@ -595,14 +611,14 @@ def nvfp4_bench(mx, torch, device, peaks, reps=10):
     qa = mx.mxfp4_nvfp4_quantize(a, scale_layout=mx.SCALES_MMA)
     qw = mx.mxfp4_nvfp4_quantize(w, scale_layout=mx.SCALES_MMA)
     c = torch.empty((TOKENS, INTER), dtype=torch.float32, device=device)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(torch, device)
 
     # time the GEMM alone: events around the launch, the flush before them
     mx.mxfp4_nvfp4_gemm(qa, qw, out=c)
     torch.cuda.synchronize()
     ts = []
     for _ in range(reps):
-        flush.zero_()
+        flush()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         mx.mxfp4_nvfp4_gemm(qa, qw, out=c)
@@ -706,7 +722,7 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         return
-    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=device)
+    flush = L2Flush(torch, device, args.flush_mib)
     stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
@@ -727,7 +743,7 @@ def main():
         without them)."""
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ops + 1 if per_op else 2)] for _ in range(n)]
         for i in range(n):
-            flush.zero_()                               # L2 flush between timed steps (outside the step)
+            flush()                                     # L2 flush between timed steps (outside the step)
             e = evs[i]
             e[0].record(stream)
             for j, (_, fn) in enumerate(ops):
@@ -914,7 +930,8 @@ def main():
                            "parallelism": (f"dp{world} (token split of a {world * TOKENS}-token batch; FP32 NCCL "
                                            f"all-reduce of dW every step, overlapping dgrad)" if dp_kw["dw_allreduce"]
                                            else f"dp{world} (independent tokens per rank, no collective)"),
-                           "l2": f"flushed between timed steps ({args.flush_mib} MiB write, outside step events)"},
+                           "l2": f"flushed between timed steps, outside the step events: a {args.flush_mib} MiB write, then a "
+                                 f"{args.flush_mib} MiB read of another buffer (clean lines left in L2)"},
                 "roofline": roofline, "roofline_quantize": roofline_q, "roofline_sr_dual": roofline_sr,
                 "kernels": kernels,
                 "quantize_GBps": quant_gbs, "cpu_baseline": cpu, "e2e": e2e,

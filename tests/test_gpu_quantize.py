@@ -59,17 +59,20 @@ def test_quantize_bit_exact(layout, rht, rnd, scale_layout):
 
 
 @pytest.mark.parametrize("scale_layout", [mx.SCALES_ROWMAJOR, mx.SCALES_MMA])
-@pytest.mark.parametrize("rht", [0, 32])
-def test_column_quantizer_strips(rht, scale_layout):
-    """1D-column RNE on 65,632 x 1080: 257 row tiles of 256 (the last holds 96
-    rows, so 3 of its 8 K-blocks), 17 column tiles of 64 (the last holds 56
-    columns).  With 148 SMs the launcher walks strips of 8 vertically adjacent
-    tiles whose scales leave together, so the last strip is one ragged tile;
-    codes and scales must be bit-exact."""
+@pytest.mark.parametrize("rht,rnd", [(0, mx.ROUND_RNE), (32, mx.ROUND_RNE), (32, mx.ROUND_SR)])
+def test_column_quantizer_strips(rht, rnd, scale_layout):
+    """1D-column quantization of 65,632 x 1080: 257 row tiles of 256 (the last
+    holds 96 rows, so 3 of its 8 K-blocks), 17 column tiles of 64 (the last
+    holds 56 columns).  With 148 SMs the launcher walks strips of 4 vertically
+    adjacent tiles whose scales leave together, so the last strip is one
+    ragged tile; the scale rows (2051 bytes) are not word-aligned, so the
+    row-major scales leave byte by byte.  Codes and scales must be bit-exact,
+    under SR too (each element's stream index is its position in the
+    transposed view)."""
     rows, cols = 65632, 1080
     x = synth.student_t_bf16((rows, cols), seed=12)
-    q = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_COL, rht, mx.ROUND_RNE, 42, 0, scale_layout)
-    codes, scales = oracle.quantize(x, oracle.LAYOUT_1D_COL, rht, oracle.ROUND_RNE, 42)[:2]
+    q = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_COL, rht, rnd, 42, 0, scale_layout)
+    codes, scales = oracle.quantize(x, oracle.LAYOUT_1D_COL, rht, rnd, 42)[:2]
     assert np.array_equal(host(q.codes), codes)
     assert np.array_equal(_scales_rowmajor(q, mx.LAYOUT_1D_COL, scales, rows, cols), scales)
 
