@@ -54,7 +54,7 @@ extern "C" {
 #define MXFP4_OK 0
 #define MXFP4_ERR_INVALID_ARG 1   /* null pointer, bad enum, shape outside the format */
 #define MXFP4_ERR_ALIGNMENT 2     /* pointer or leading dimension not 16-byte aligned */
-#define MXFP4_ERR_UNSUPPORTED 3   /* valid MXFP4 shape this build has no kernel for */
+#define MXFP4_ERR_UNSUPPORTED 3   /* valid MXFP4 shape the library has no kernel for */
 #define MXFP4_ERR_CUDA 4          /* a CUDA runtime/driver call failed */
 #define MXFP4_ERR_TIMEOUT 5       /* a bounded device-side wait ran out (see mxfp4_get_error) */
 
