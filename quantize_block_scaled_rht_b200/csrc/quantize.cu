@@ -305,6 +305,26 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
 }
 
+// Row and column of tile t in a grid of `cols` tile columns, for a
+// persistent CTA's sequence t0, t0 + step, t0 + 2 step, ...: 32-bit divisions
+// when the walk starts, then additions only.  (A 64-bit division per tile cost
+// the 2D quantizer about 4.5 of its 13.9 instructions per element.)
+struct TileStep {
+    uint32_t step, dr, dc, cols;
+    __device__ __forceinline__ TileStep(uint32_t step_, uint32_t cols_)
+        : step(step_), dr(step_ / cols_), dc(step_ % cols_), cols(cols_) {}
+};
+struct TileWalk {
+    uint32_t t, r, c;
+    __device__ __forceinline__ TileWalk(uint32_t t0, uint32_t cols) : t(t0), r(t0 / cols), c(t0 % cols) {}
+    __device__ __forceinline__ void next(const TileStep &st) {
+        t += st.step;
+        r += st.dr;
+        c += st.dc;
+        if (c >= st.cols) { c -= st.cols; ++r; }
+    }
+};
+
 
 // ---------------------------------------------------------------------------
 // Parameters of the column quantizer and of the dual (row + column) quantizer.
@@ -437,25 +457,30 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const DualParams p, c
     uint32_t *ssc = reinterpret_cast<uint32_t *>(cq_smem + CQ_STAGES * CQ_TILE_BYTES + CQ_OUT_BYTES);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t strip = p.strip;
-    // The CTA's tiles in order: strips S = blockIdx.x + j * gridDim.x, tile k
-    // of each (row band (S / tiles_c) * strip + k, column band S % tiles_c).
-    // A strip index past nstrips stays past it under next().
-    auto strip_tiles = [&](uint32_t S) -> uint32_t {
-        const uint32_t t0 = (S / p.tiles_c) * strip;
+    // The CTA's tiles in order: strips S = blockIdx.x + j * gridDim.x (row band
+    // w.r, column band w.c of the strip grid), tile k of each of its len tiles
+    // (row band w.r * strip + k).  A strip index past nstrips stays past it.
+    struct Pos {
+        TileWalk w;
+        uint32_t k, len;
+    };
+    auto strip_len_of = [&](uint32_t band) -> uint32_t {
+        const uint32_t t0 = band * strip;
         return t0 + strip <= p.tiles_r ? strip : (t0 < p.tiles_r ? p.tiles_r - t0 : strip);
     };
-    auto next = [&](uint32_t &S, uint32_t &k) {
-        if (k + 1 < strip_tiles(S)) {
-            ++k;
+    const TileStep st(gridDim.x, p.tiles_c);
+    auto advance = [&](Pos &q) {
+        if (q.k + 1 < q.len) {
+            ++q.k;
         } else {
-            S += gridDim.x;
-            k = 0;
+            q.w.next(st);
+            q.k = 0;
+            q.len = strip_len_of(q.w.r);
         }
     };
-    auto load = [&](uint32_t S, uint32_t k, int buf) {
-        if (S < nstrips) {
-            const uint32_t band = S / p.tiles_c;
-            const int64_t r0 = (int64_t)(band * strip + k) * CQ_TR, c0 = (int64_t)(S - band * p.tiles_c) * CQ_TC;
+    auto load = [&](const Pos &q, int buf) {
+        if (q.w.t < nstrips) {
+            const int64_t r0 = (int64_t)(q.w.r * strip + q.k) * CQ_TR, c0 = (int64_t)q.w.c * CQ_TC;
             const int ch = tid & 7, row = tid >> 3;          // rows row + 32 i, 16-byte chunk ch
             const int64_t gc = c0 + 8 * ch;
             const uint16_t *src = p.x + (r0 + row) * p.ld_x + gc;
@@ -472,19 +497,20 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const DualParams p, c
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
 
-    uint32_t S = blockIdx.x, k = 0;
-    uint32_t S1 = S, k1 = k;
-    next(S1, k1);
-    uint32_t S2 = S1, k2 = k1;
-    next(S2, k2);
-    load(S, k, 0);
-    load(S1, k1, 1);
-    for (int it = 0; S < nstrips; ++it) {
-        load(S2, k2, (it + 2) % CQ_STAGES);                  // two tiles in flight while this one is quantized
+    Pos cur{TileWalk(blockIdx.x, p.tiles_c), 0u, 0u};
+    cur.len = strip_len_of(cur.w.r);
+    Pos n1 = cur;
+    advance(n1);
+    Pos n2 = n1;
+    advance(n2);
+    load(cur, 0);
+    load(n1, 1);
+    for (int it = 0; cur.w.t < nstrips; ++it) {
+        load(n2, (it + 2) % CQ_STAGES);                      // two tiles in flight while this one is quantized
         asm volatile("cp.async.wait_group 2;" ::: "memory");
         __syncthreads();
-        const uint32_t band = S / p.tiles_c;
-        const int64_t r0 = (int64_t)(band * strip + k) * CQ_TR, c0 = (int64_t)(S - band * p.tiles_c) * CQ_TC;
+        const uint32_t band = cur.w.r, k = cur.k;
+        const int64_t r0 = (int64_t)(band * strip + k) * CQ_TR, c0 = (int64_t)cur.w.c * CQ_TC;
         const int64_t rin = r0 + 32 * warp, oc = c0 + 2 * lane;
         if (rin < p.rows && oc < p.cols) {
             const uint32_t *src =
@@ -500,7 +526,7 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const DualParams p, c
             sb[4 * ((c + 1) * CQ_SPITCH + 2 * k) + warp] = (uint8_t)shi;
         }
         __syncthreads();                                     // tile read; codes and scales staged
-        const uint32_t ntiles = strip_tiles(S);
+        const uint32_t ntiles = cur.len;
         const bool last = k + 1 == ntiles;
         // codes: 64 output rows x 8 chunks of 16 bytes; 8 lanes write one row's 128 bytes
 #pragma unroll
@@ -551,9 +577,9 @@ __global__ void __launch_bounds__(256, 2) quant_col_kernel(const DualParams p, c
                 }
             }
         }
-        S = S1; k = k1;
-        S1 = S2; k1 = k2;
-        next(S2, k2);
+        cur = n1;
+        n1 = n2;
+        advance(n2);
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
@@ -587,10 +613,9 @@ __global__ void __launch_bounds__(256, 2) quant_dual_kernel(const DualParams p, 
     uint8_t *ring = dq_smem;
     uint4 *tout = reinterpret_cast<uint4 *>(dq_smem + DQ_STAGES * DQ_TILE_BYTES);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    auto load = [&](uint32_t t, int buf) {
-        if (t < ntiles) {
-            const uint32_t tr = t / p.tiles_c;
-            const int64_t r0 = (int64_t)tr * DQ_TR, c0 = (int64_t)(t - tr * p.tiles_c) * DQ_TC;
+    auto load = [&](const TileWalk &w, int buf) {
+        if (w.t < ntiles) {
+            const int64_t r0 = (int64_t)w.r * DQ_TR, c0 = (int64_t)w.c * DQ_TC;
             const int ch = tid & 7, row = tid >> 3;            // rows row + 32 i, 16-byte chunk ch
             const int64_t gc = c0 + 8 * ch;
             const uint16_t *src = p.x + (r0 + row) * p.ld_x + gc;
@@ -606,17 +631,20 @@ __global__ void __launch_bounds__(256, 2) quant_dual_kernel(const DualParams p, 
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    uint32_t t = blockIdx.x;
-    load(t, 0);
-    load(t + gridDim.x, 1);
-    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+    const TileStep st(gridDim.x, p.tiles_c);
+    TileWalk cur(blockIdx.x, p.tiles_c), w1 = cur, w2 = cur;
+    w1.next(st);
+    w2.next(st);
+    w2.next(st);
+    load(cur, 0);
+    load(w1, 1);
+    for (int it = 0; cur.t < ntiles; ++it) {
         // two tiles in flight while this one is quantized; the buffer loaded
         // here was read in the previous iteration, before its barrier
-        load(t + 2 * gridDim.x, (it + 2) % DQ_STAGES);
+        load(w2, (it + 2) % DQ_STAGES);
         asm volatile("cp.async.wait_group 2;" ::: "memory");
         __syncthreads();
-        const uint32_t tr = t / p.tiles_c;
-        const int64_t r0 = (int64_t)tr * DQ_TR, c0 = (int64_t)(t - tr * p.tiles_c) * DQ_TC;
+        const int64_t r0 = (int64_t)cur.r * DQ_TR, c0 = (int64_t)cur.c * DQ_TC;
         const uint8_t *tile = ring + (it % DQ_STAGES) * DQ_TILE_BYTES;
         if (warp < 4) {                                          // column pair (2 lane, 2 lane + 1), row block warp
             const int64_t rin = r0 + 32 * warp, oc = c0 + 2 * lane;
@@ -665,6 +693,9 @@ __global__ void __launch_bounds__(256, 2) quant_dual_kernel(const DualParams p, 
             if (orow < p.cols && rb < p.rows)
                 stg_v4(p.ccodes + orow * p.ld_ccodes + (rb >> 1), tout[row * 4 + (ch ^ ((row >> 1) & 3))]);
         }
+        cur = w1;
+        w1 = w2;
+        w2.next(st);
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
@@ -793,10 +824,10 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_2d_kernel(const QuantPa
     __shared__ __align__(16) uint8_t tb[8][16][32];   // per warp: byte j of row r at [j][r]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t nbr = p.rows >> 5, nbc = p.cols >> 5;
-    const int64_t tiles_c = (nbc + T::BC - 1) / T::BC;
-    const int64_t ntiles = ((nbr + T::BR - 1) / T::BR) * tiles_c;
-    auto load = [&](int64_t t, int buf) {
-        const int64_t r0 = (t / tiles_c) * T::ROWS, c0 = (t % tiles_c) * T::COLS;
+    const uint32_t tiles_c = (uint32_t)((nbc + T::BC - 1) / T::BC);
+    const uint32_t ntiles = (uint32_t)((nbr + T::BR - 1) / T::BR) * tiles_c;   // the launcher checks it fits
+    auto load = [&](const TileWalk &w, int buf) {
+        const int64_t r0 = (int64_t)w.r * T::ROWS, c0 = (int64_t)w.c * T::COLS;
 #pragma unroll
         for (int i = 0; i < T::ROWS * T::CHUNKS / 256; ++i) {
             const int idx = tid + 256 * i, row = idx / T::CHUNKS, ch = idx % T::CHUNKS;
@@ -805,21 +836,22 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_2d_kernel(const QuantPa
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    int64_t t = blockIdx.x;
-    if (t < ntiles) load(t, 0);
-    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+    const TileStep st(gridDim.x, tiles_c);
+    TileWalk cur(blockIdx.x, tiles_c), nxt = cur;
+    nxt.next(st);
+    if (cur.t < ntiles) load(cur, 0);
+    for (int it = 0; cur.t < ntiles; ++it) {
         const int buf = it & 1;
-        const int64_t tn = t + gridDim.x;
-        if (tn < ntiles) {
-            load(tn, buf ^ 1);
+        if (nxt.t < ntiles) {
+            load(nxt, buf ^ 1);
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
         const int wr = warp / T::BC, wc = warp % T::BC;   // this warp's block within the tile
-        const int64_t br = (t / tiles_c) * T::BR + wr;
-        const int64_t bc = (t % tiles_c) * T::BC + wc;
+        const int64_t br = (int64_t)cur.r * T::BR + wr;
+        const int64_t bc = (int64_t)cur.c * T::BC + wc;
         if (br < nbr && bc < nbc) {
             const int64_t r = (br << 5) + lane, c0 = bc << 5;
             const uint4 *s4 = reinterpret_cast<const uint4 *>(tin[buf] + (32 * wr + lane) * T::PITCH + 32 * wc);
@@ -902,6 +934,8 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_2d_kernel(const QuantPa
             }
         }
         __syncthreads();                     // the load after next overwrites this buffer
+        cur = nxt;
+        nxt.next(st);
     }
 }
 
@@ -1204,12 +1238,11 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
     uint4 (*tin)[COL_TC][8] = reinterpret_cast<uint4 (*)[COL_TC][8]>(dyn_smem);   // 2 x 8 KB of codes
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint8_t *stage = dyn_smem + sizeof(uint4) * 2 * COL_TC * 8 + warp * 32 * ROWB;
-    const int64_t tiles_r = (p.rows + COL_TR - 1) / COL_TR;
-    const int64_t tiles_c = (p.cols + COL_TC - 1) / COL_TC;
-    const int64_t ntiles = tiles_r * tiles_c;
-    auto load = [&](int64_t t, int buf) {
-        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
-        const int64_t r0 = tr * COL_TR, c0 = tc * COL_TC;
+    const uint32_t tiles_r = (uint32_t)((p.rows + COL_TR - 1) / COL_TR);
+    const uint32_t tiles_c = (uint32_t)((p.cols + COL_TC - 1) / COL_TC);
+    const uint32_t ntiles = tiles_r * tiles_c;                         // the launcher checks it fits
+    auto load = [&](const TileWalk &w, int buf) {
+        const int64_t r0 = (int64_t)w.r * COL_TR, c0 = (int64_t)w.c * COL_TC;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
             const int row = (tid >> 3) + 32 * i, ch = tid & 7;
@@ -1220,11 +1253,10 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
     };
     // the bf16 path's two scale bytes (columns 2l, 2l + 1 of row block w) of a
     // tile, loaded one tile ahead so that their latency hides behind a tile
-    auto scale_pair = [&](int64_t tt, uint32_t &s0, uint32_t &s1) {
+    auto scale_pair = [&](const TileWalk &w, uint32_t &s0, uint32_t &s1) {
         s0 = s1 = 0xFFu;
-        if (tt < ntiles) {
-            const int64_t tr = tt / tiles_c, tc = tt - tr * tiles_c;
-            const int64_t rb = tr * COL_TR + 32 * warp, oc = tc * COL_TC + 2 * lane;
+        if (w.t < ntiles) {
+            const int64_t rb = (int64_t)w.r * COL_TR + 32 * warp, oc = (int64_t)w.c * COL_TC + 2 * lane;
             if (rb < p.rows && oc < p.cols) {
                 const int64_t kb = rb >> 5;
                 s0 = MMA ? p.scales[mma_scale_off(oc, kb, p.katoms)] : p.scales[oc * p.ld_scales + kb];
@@ -1232,26 +1264,27 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
             }
         }
     };
-    int64_t t = blockIdx.x;
-    if (t < ntiles) load(t, 0);
+    const TileStep st(gridDim.x, tiles_c);
+    TileWalk cur(blockIdx.x, tiles_c);
+    if (cur.t < ntiles) load(cur, 0);
     uint32_t sa = 0xFFu, sb = 0xFFu;
-    if constexpr (!F32) scale_pair(t, sa, sb);
-    for (int it = 0; t < ntiles; t += gridDim.x, ++it) {
+    if constexpr (!F32) scale_pair(cur, sa, sb);
+    for (int it = 0; cur.t < ntiles; ++it) {
         // the buffer refilled here was read in the previous iteration, which
         // ended with a barrier
         const int buf = it & 1;
-        const int64_t tn = t + gridDim.x;
+        TileWalk nxt = cur;
+        nxt.next(st);
         uint32_t sa_n = 0xFFu, sb_n = 0xFFu;
-        if constexpr (!F32) scale_pair(tn, sa_n, sb_n);
-        if (tn < ntiles) {
-            load(tn, buf ^ 1);
+        if constexpr (!F32) scale_pair(nxt, sa_n, sb_n);
+        if (nxt.t < ntiles) {
+            load(nxt, buf ^ 1);
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
-        const int64_t tr = t / tiles_c, tc = t - tr * tiles_c;
-        const int64_t r0 = tr * COL_TR, c0 = tc * COL_TC;
+        const int64_t r0 = (int64_t)cur.r * COL_TR, c0 = (int64_t)cur.c * COL_TC;
         const int64_t rb = r0 + 32 * warp;
         if (rb < p.rows) {
           const int64_t kb = rb >> 5;
@@ -1326,6 +1359,7 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
         __syncthreads();
         sa = sa_n;
         sb = sb_n;
+        cur.next(st);
     }
 }
 
@@ -1405,6 +1439,7 @@ static cudaError_t launch_quant_t(int layout, bool trans, const QuantParams &p, 
     } else {
         const int br = trans ? Q2Tile<true>::BR : Q2Tile<false>::BR;
         const int64_t tiles = ((p.rows / 32 + br - 1) / br) * ((p.cols / 32 + 8 / br - 1) / (8 / br));
+        if (tiles > 0xFFFFFFFFll - 0x7FFFFFFFll) return cudaErrorInvalidValue;   // tile index fits 32 bits
         auto kern = trans ? quant_2d_kernel<RHT, SR, MMA, true> : quant_2d_kernel<RHT, SR, MMA, false>;
         // persistent for RNE (memory-bound), one CTA per tile for SR (ALU-bound)
         const int64_t cap = SR ? 0x7FFFFFFFll
@@ -1592,6 +1627,7 @@ static cudaError_t launch_dequant_t(int layout, int smode, const DequantParams &
     if (layout == MXFP4_LAYOUT_1D_COL) {
         // persistent at full occupancy: each CTA keeps its next tile's load in flight
         const int64_t tiles = ((p.rows + COL_TR - 1) / COL_TR) * ((p.cols + COL_TC - 1) / COL_TC);
+        if (tiles > 0xFFFFFFFFll - 0x7FFFFFFFll) return cudaErrorInvalidValue;   // tile index fits 32 bits
         auto kern = smode == 2 ? dequant_col_kernel<RHT, F32, true> : dequant_col_kernel<RHT, F32, false>;
         constexpr int smem = dequant_col_smem<F32>();
         const cudaError_t ea = allow_dyn_smem(reinterpret_cast<const void *>(kern), smem);
