@@ -1044,6 +1044,29 @@ __device__ __forceinline__ void decode32_f32(const uint4 q, uint32_t sc, float *
     }
 }
 
+// One block decoded and inverse-transformed before the sign flip: v = c_d
+// H_d (decode(code) 2^e) per d-segment.  For scale codes 27..246 (e = code -
+// 127 in [-100, 119]) the butterfly runs on the unscaled magnitudes
+// {0, 0.5, ..., 6}: every partial sum is a multiple of 0.5 below 2^8, exact in
+// fp32, and so is its image under 2^e in the scaled butterfly (no overflow:
+// 192 2^119 < FLT_MAX; below the normal range sums of multiples of 2^-149 are
+// exact too).  The normalisation then multiplies by K = fp32(c_d 2^e), exact
+// for these e, and RN(S K) equals the scaled path's RN(c_d (S 2^e)) because
+// both round the same real number.  The decode table is the constant one of
+// scale code 127, so the per-block table products disappear.  Other codes
+// (tiny or huge scales, NaN) take the scaled path.
+template <int RHT>
+__device__ __forceinline__ void decode_inverse_fwht32(const uint4 q, uint32_t sc, float *v) {
+    if (sc - 27u <= 219u) {
+        decode32_f32(q, 127u, v);
+        const float K = __uint_as_float(__float_as_uint(rht_norm<RHT>()) + ((sc - 127u) << 23));
+        fwht32_scaled<RHT>(v, K);
+    } else {
+        decode32_f32(q, sc, v);
+        fwht32_scaled<RHT>(v, rht_norm<RHT>());
+    }
+}
+
 template <int RHT>
 __device__ __forceinline__ void inverse_rht32(float *v, const uint32_t *sgn_pair) {
     if constexpr (RHT) {
@@ -1066,8 +1089,7 @@ template <int RHT>
 __device__ __forceinline__ void column_rht_bf16(const uint4 q, uint32_t sc, const uint32_t *sgn_pair,
                                                 uint32_t *pairs) {
     float v[32];
-    decode32_f32(q, sc, v);
-    fwht32_scaled<RHT>(v, rht_norm<RHT>());
+    decode_inverse_fwht32<RHT>(q, sc, v);
 #pragma unroll
     for (int j = 0; j < 16; ++j) pairs[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]) ^ sgn_pair[j];
 }
@@ -1092,8 +1114,12 @@ __device__ __forceinline__ void dequant_block_store(const DequantParams &p, int6
         return;
     }
     float v[32];
-    decode32_f32(q, sc, v);
-    inverse_rht32<RHT>(v, p.sgn_pair);
+    decode_inverse_fwht32<RHT>(q, sc, v);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        v[2 * j] = __uint_as_float(__float_as_uint(v[2 * j]) ^ (p.sgn_pair[j] << 16));
+        v[2 * j + 1] = __uint_as_float(__float_as_uint(v[2 * j + 1]) ^ (p.sgn_pair[j] & 0x80000000u));
+    }
     if constexpr (F32) {
         float *dst = reinterpret_cast<float *>(p.out) + r * p.ld_out + (kb << 5);
 #pragma unroll
@@ -1161,7 +1187,7 @@ __device__ __forceinline__ void dequant_warp_store(const uint4 *slot, uint8_t *d
 // its own block) write half sectors per instruction, which held a 1:4
 // read:write stream to 4.0 TB/s against 5.5 TB/s coalesced.
 template <int RHT, bool F32, int SMODE>
-__global__ void __launch_bounds__(256) dequant_row_kernel(const DequantParams p) {
+__global__ void __launch_bounds__(256, RHT ? 3 : (F32 ? 2 : 4)) dequant_row_kernel(const DequantParams p) {
     pdl_wait();
     pdl_trigger();
     __shared__ __align__(16) uint4 stage_all[RHT == 0 ? 8 : 1][RHT == 0 ? 32 * (F32 ? 8 : 4) : 1];
@@ -1326,11 +1352,12 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                 if (oc < p.cols) {
                     const uint32_t sc = MMA ? p.scales[mma_scale_off(oc, kb, p.katoms)] : p.scales[oc * p.ld_scales + kb];
                     float v[32];
-                    decode32_f32(tin[buf][c][warp], sc, v);
                     if constexpr (RHT) {
-                        fwht32_scaled<RHT>(v, rht_norm<RHT>());
+                        decode_inverse_fwht32<RHT>(tin[buf][c][warp], sc, v);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ p.sgn_bit[i % RHT]);
+                    } else {
+                        decode32_f32(tin[buf][c][warp], sc, v);
                     }
                     const int wpos = c ^ ((c >> 5) & 1);                // bank-spreading word swap
                     uint32_t *col = reinterpret_cast<uint32_t *>(stage) + wpos;

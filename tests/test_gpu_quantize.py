@@ -155,6 +155,39 @@ def test_dequantize_matches_oracle(layout, rht, out_dtype):
         assert np.array_equal(got[~nan], b16[~nan])
 
 
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rht", [16, 32])
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_dequantize_rht_every_scale_code(layout, rht, out_dtype):
+    """The inverse RHT over random codes with every scale code 0..255: the
+    dequantizers transform scale codes 27..246 in the unscaled domain and the
+    others (subnormal, overflowing and NaN scales) directly; both must equal
+    the oracle's scaled butterfly bit for bit (NaN positions equal)."""
+    rows, cols = {mx.LAYOUT_1D_ROW: (256, 320), mx.LAYOUT_1D_COL: (320, 256), mx.LAYOUT_2D: (512, 512)}[layout]
+    rng = np.random.default_rng(900 + layout * 10 + rht)
+    if layout == mx.LAYOUT_1D_COL:
+        codes = rng.integers(0, 256, size=(cols, rows // 2), dtype=np.uint8)
+        sshape = (cols, rows // 32)
+    else:
+        codes = rng.integers(0, 256, size=(rows, cols // 2), dtype=np.uint8)
+        sshape = (rows // 32, cols // 32) if layout == mx.LAYOUT_2D else (rows, cols // 32)
+    n = sshape[0] * sshape[1]
+    scales = rng.permutation(np.arange(n) % 256).astype(np.uint8).reshape(sshape)
+    assert len(np.unique(scales)) == 256
+    f32, b16 = oracle.dequantize(codes, scales, rows, cols, layout, rht, 5)
+    out = mx.mxfp4_dequantize(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), rows, cols,
+                              layout, rht, 5, out_dtype=out_dtype)
+    got = host(out)
+    if out_dtype == torch.float32:
+        assert np.array_equal(np.isnan(got), np.isnan(f32))
+        ok = ~np.isnan(f32)
+        assert np.array_equal(got[ok].view(np.uint32), f32[ok].view(np.uint32))
+    else:
+        nan = np.isnan(synth.bf16_to_f32(b16))
+        assert np.array_equal(np.isnan(synth.bf16_to_f32(got)), nan)
+        assert np.array_equal(got[~nan], b16[~nan])
+
+
 def test_dequantize_mma_scales():
     rows, cols = 200, 256
     x = synth.normal_bf16((rows, cols), 4)
