@@ -1448,10 +1448,18 @@ static void fill_signs(uint32_t mask, int rht, uint32_t *pair, uint32_t *bit) {
     }
 }
 
+// Grid of the grid-stride row kernels: about 14 items per thread, between 4
+// and 32 CTAs per SM.  Small tensors then run as resident CTAs that each loop
+// several times (a 64 MiB row quantize: 0.63 -> 0.70 of HBM against one item
+// per thread), large ones oversubscribed (1 GiB: 0.96 against 0.88 with 4
+// CTAs per SM).
 static int64_t grid_for(int64_t items, int threads) {
-    int64_t g = (items + threads - 1) / threads;
-    const int64_t cap = (int64_t)num_sms() * 32;
-    return g < 1 ? 1 : (g > cap ? cap : g);
+    const int64_t g = (items + threads - 1) / threads;
+    const int64_t lo = (int64_t)num_sms() * 4, hi = (int64_t)num_sms() * 32;
+    int64_t want = (items + (int64_t)threads * 14 - 1) / ((int64_t)threads * 14);
+    want = want < lo ? lo : (want > hi ? hi : want);
+    const int64_t grid = g < want ? g : want;
+    return grid < 1 ? 1 : grid;
 }
 
 template <int RHT, bool SR, bool MMA>
