@@ -952,6 +952,7 @@ struct DequantParams {
     int64_t ld_out;
     uint32_t sgn_pair[16];
     uint32_t sgn_bit[32];                  // RHT sign of element i (mod the RHT size) as bit 31
+    uint32_t sgn_word[32];                 // the same sign at bits 15 and 31 (both halves of a bf16 pair)
 };
 
 
@@ -1066,6 +1067,65 @@ __device__ __forceinline__ void decode_inverse_fwht32(const uint4 q, uint32_t sc
         fwht32_scaled<RHT>(v, rht_norm<RHT>());
     }
 }
+
+// Two blocks a and b of the unscaled domain at once, as f16 pairs P[i] =
+// (a_i low, b_i high).  The decoded magnitudes {0, 0.5, ..., 6} and every
+// partial sum of the butterfly (multiples of 0.5 below 2^8) are exact in f16
+// as in fp32, so the packed f16 butterfly, taken in the same stage order
+// and pairing as the fp32 one, gives the same values, zeros' signs included.
+// The decode is the hardware E2M1 -> f16 conversion of bytes whose low
+// nibble is a code of a and high nibble the code of b at the same index.
+__device__ __forceinline__ void e2m1x2x4_f16x2(uint32_t w, uint32_t &h0, uint32_t &h1, uint32_t &h2, uint32_t &h3) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3) : "r"(w));
+}
+__device__ __forceinline__ uint32_t hadd2_rn(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t hsub2_rn(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ float2 f16x2_to_f32(uint32_t p) {
+    float2 r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tcvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
+        : "=f"(r.x), "=f"(r.y) : "r"(p));
+    return r;
+}
+template <int RHT>
+__device__ __forceinline__ void decode_pair_fwht_f16(const uint4 qa, const uint4 qb, uint32_t *P) {
+    const uint32_t wa[4] = {qa.x, qa.y, qa.z, qa.w}, wb[4] = {qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        // bytes (a_{8k+2m}, b_{8k+2m}) and (a_{8k+2m+1}, b_{8k+2m+1}), m = 0..3
+        const uint32_t ev = (wa[k] & 0x0F0F0F0Fu) | ((wb[k] << 4) & 0xF0F0F0F0u);
+        const uint32_t od = ((wa[k] >> 4) & 0x0F0F0F0Fu) | (wb[k] & 0xF0F0F0F0u);
+        e2m1x2x4_f16x2(ev, P[8 * k], P[8 * k + 2], P[8 * k + 4], P[8 * k + 6]);
+        e2m1x2x4_f16x2(od, P[8 * k + 1], P[8 * k + 3], P[8 * k + 5], P[8 * k + 7]);
+    }
+#pragma unroll
+    for (int h = 1; h < RHT; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (!(i & h)) {
+                const uint32_t x = P[i], y = P[i + h];
+                P[i] = hadd2_rn(x, y);
+                P[i + h] = hsub2_rn(x, y);
+            }
+        }
+    }
+}
+// K = fp32(c_d 2^e) of a scale code in the unscaled-domain range 27..246.
+template <int RHT>
+__device__ __forceinline__ float unscaled_norm(uint32_t sc) {
+    return __uint_as_float(__float_as_uint(rht_norm<RHT>()) + ((sc - 127u) << 23));
+}
+__device__ __forceinline__ bool unscaled_ok(uint32_t sc) { return sc - 27u <= 219u; }
 
 template <int RHT>
 __device__ __forceinline__ void inverse_rht32(float *v, const uint32_t *sgn_pair) {
@@ -1329,6 +1389,18 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                     for (int i = 0; i < 16; ++i) {
                         w[(2 * i) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x5410u);
                         w[(2 * i + 1) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x7632u);
+                    }
+                } else if (unscaled_ok(sa) && unscaled_ok(sb)) {
+                    // both columns at once in the unscaled domain: row i of
+                    // the pair is one f16 pair, then one fp32 pair scaled by
+                    // (K_a, K_b), rounded to the bf16 pair of the staged word
+                    uint32_t P[32];
+                    decode_pair_fwht_f16<RHT>(tin[buf][2 * lane][warp], tin[buf][2 * lane + 1][warp], P);
+                    const float2 K2 = make_float2(unscaled_norm<RHT>(sa), unscaled_norm<RHT>(sb));
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float2 f = mul2(f16x2_to_f32(P[i]), K2);
+                        w[i * (ROWB / 4)] = pack_bf16x2(f.x, f.y) ^ p.sgn_word[i];
                     }
                 } else {
                     // each column decoded, transformed, rounded and
@@ -1693,6 +1765,7 @@ cudaError_t launch_dequantize(const uint8_t *codes, int64_t ld_codes, const uint
     p.rows = rows; p.cols = cols; p.out = out; p.ld_out = ld_out;
     p.katoms = mma_katoms(layout == MXFP4_LAYOUT_1D_COL ? rows : cols);
     fill_signs(rht ? rht_sign_mask_hd(seed) : 0u, rht, p.sgn_pair, p.sgn_bit);
+    for (int i = 0; i < 32; ++i) p.sgn_word[i] = p.sgn_bit[i] | (p.sgn_bit[i] >> 16);
     const int smode = scale_layout == MXFP4_SCALES_MMA ? 2 : (layout == MXFP4_LAYOUT_2D ? 1 : 0);
     const bool f32 = out_dtype == MXFP4_OUT_F32;
     switch (rht) {
