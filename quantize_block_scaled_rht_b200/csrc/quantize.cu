@@ -1323,6 +1323,10 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
     constexpr int CH = ROWB / 16;                                    // 16-byte chunks per row
     uint4 (*tin)[COL_TC][8] = reinterpret_cast<uint4 (*)[COL_TC][8]>(dyn_smem);   // 2 x 8 KB of codes
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // chunk ch of staged code row `row` sits at ch ^ ((row >> 1) & 7): the
+    // lanes of a warp read block `warp` of rows 2l, 2l + 1 (256 bytes apart),
+    // which this spreads over all banks
+    const int wsw = warp ^ (lane & 7);
     uint8_t *stage = dyn_smem + sizeof(uint4) * 2 * COL_TC * 8 + warp * 32 * ROWB;
     const uint32_t tiles_r = (uint32_t)((p.rows + COL_TR - 1) / COL_TR);
     const uint32_t tiles_c = (uint32_t)((p.cols + COL_TC - 1) / COL_TC);
@@ -1333,7 +1337,8 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
         for (int i = 0; i < 2; ++i) {
             const int row = (tid >> 3) + 32 * i, ch = tid & 7;
             const int64_t crow = c0 + row, rin = r0 + 32 * ch;
-            if (crow < p.cols && rin < p.rows) cp_async16(&tin[buf][row][ch], p.codes + crow * p.ld_codes + (rin >> 1));
+            if (crow < p.cols && rin < p.rows)
+                cp_async16(&tin[buf][row][ch ^ ((row >> 1) & 7)], p.codes + crow * p.ld_codes + (rin >> 1));
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
@@ -1383,8 +1388,8 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                 if constexpr (RHT == 0) {
                     // each column as 16 looked-up bf16 pairs along its rows
                     uint32_t pa[16], pb[16];
-                    decode32_bf16(tin[buf][2 * lane][warp], sa, pa);
-                    decode32_bf16(tin[buf][2 * lane + 1][warp], sb, pb);
+                    decode32_bf16(tin[buf][2 * lane][wsw], sa, pa);
+                    decode32_bf16(tin[buf][2 * lane + 1][wsw], sb, pb);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         w[(2 * i) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x5410u);
@@ -1395,7 +1400,7 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                     // the pair is one f16 pair, then one fp32 pair scaled by
                     // (K_a, K_b), rounded to the bf16 pair of the staged word
                     uint32_t P[32];
-                    decode_pair_fwht_f16<RHT>(tin[buf][2 * lane][warp], tin[buf][2 * lane + 1][warp], P);
+                    decode_pair_fwht_f16<RHT>(tin[buf][2 * lane][wsw], tin[buf][2 * lane + 1][wsw], P);
                     const float2 K2 = make_float2(unscaled_norm<RHT>(sa), unscaled_norm<RHT>(sb));
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -1406,8 +1411,8 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                     // each column decoded, transformed, rounded and
                     // sign-flipped as 16 bf16 pairs along its rows
                     uint32_t pa[16], pb[16];
-                    column_rht_bf16<RHT>(tin[buf][2 * lane][warp], sa, p.sgn_pair, pa);
-                    column_rht_bf16<RHT>(tin[buf][2 * lane + 1][warp], sb, p.sgn_pair, pb);
+                    column_rht_bf16<RHT>(tin[buf][2 * lane][wsw], sa, p.sgn_pair, pa);
+                    column_rht_bf16<RHT>(tin[buf][2 * lane + 1][wsw], sb, p.sgn_pair, pb);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         w[(2 * i) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x5410u);
@@ -1425,11 +1430,11 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                     const uint32_t sc = MMA ? p.scales[mma_scale_off(oc, kb, p.katoms)] : p.scales[oc * p.ld_scales + kb];
                     float v[32];
                     if constexpr (RHT) {
-                        decode_inverse_fwht32<RHT>(tin[buf][c][warp], sc, v);
+                        decode_inverse_fwht32<RHT>(tin[buf][c][wsw], sc, v);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ p.sgn_bit[i % RHT]);
                     } else {
-                        decode32_f32(tin[buf][c][warp], sc, v);
+                        decode32_f32(tin[buf][c][wsw], sc, v);
                     }
                     const int wpos = c ^ ((c >> 5) & 1);                // bank-spreading word swap
                     uint32_t *col = reinterpret_cast<uint32_t *>(stage) + wpos;
