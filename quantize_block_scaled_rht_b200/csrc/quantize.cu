@@ -1195,6 +1195,37 @@ __device__ __forceinline__ void dequant_block_store(const DequantParams &p, int6
     }
 }
 
+// A lane's two blocks with the inverse RHT, both scale codes in the
+// unscaled-domain range: transformed together as f16 pairs; block 1's bf16
+// output words (pair j = elements 2j, 2j + 1, RHT signs applied) go straight
+// to the lane's slot, block 2's are returned in w2.
+template <int RHT>
+__device__ __forceinline__ void rht_pair_stage(uint4 q1, uint32_t s1, uint4 q2, uint32_t s2, const uint32_t *sgn_pair,
+                                               uint4 *slot, int lane, uint32_t *w2) {
+    uint32_t P[32];
+    decode_pair_fwht_f16<RHT>(q1, q2, P);
+    const float2 K2 = make_float2(unscaled_norm<RHT>(s1), unscaled_norm<RHT>(s2));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t a[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const int j = 4 * i + m;
+            const float2 f0 = mul2(f16x2_to_f32(P[2 * j]), K2), f1 = mul2(f16x2_to_f32(P[2 * j + 1]), K2);
+            a[m] = pack_bf16x2(f0.x, f1.x) ^ sgn_pair[j];
+            w2[j] = pack_bf16x2(f0.y, f1.y) ^ sgn_pair[j];
+        }
+        slot[4 * lane + (i ^ ((lane >> 1) & 3))] = make_uint4(a[0], a[1], a[2], a[3]);
+    }
+}
+
+// A block's 16 bf16 output words into a lane's slot (layout as below).
+__device__ __forceinline__ void stage_words_bf16(const uint32_t *w, uint4 *slot, int lane) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        slot[4 * lane + (i ^ ((lane >> 1) & 3))] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+}
+
 // One block's output words without a transform (16 bf16 pairs or 32 fp32)
 // into a lane's slot of the warp's staging area: 16-byte unit q of lane l at
 // unit 4l + (q ^ ((l >> 1) & 3)) (bf16; fp32: 8l + (q ^ (l & 7))), so that
@@ -1247,12 +1278,13 @@ __device__ __forceinline__ void dequant_warp_store(const uint4 *slot, uint8_t *d
 // its own block) write half sectors per instruction, which held a 1:4
 // read:write stream to 4.0 TB/s against 5.5 TB/s coalesced.
 template <int RHT, bool F32, int SMODE>
-__global__ void __launch_bounds__(256, RHT ? 3 : (F32 ? 2 : 4)) dequant_row_kernel(const DequantParams p) {
+__global__ void __launch_bounds__(256, RHT ? (F32 ? 3 : 2) : (F32 ? 2 : 4)) dequant_row_kernel(const DequantParams p) {
     pdl_wait();
     pdl_trigger();
-    __shared__ __align__(16) uint4 stage_all[RHT == 0 ? 8 : 1][RHT == 0 ? 32 * (F32 ? 8 : 4) : 1];
+    constexpr bool STAGED = RHT == 0 || !F32;
+    __shared__ __align__(16) uint4 stage_all[STAGED ? 8 : 1][STAGED ? 32 * (F32 ? 8 : 4) : 1];
     const int lane = threadIdx.x & 31;
-    uint4 *slot = stage_all[RHT == 0 ? threadIdx.x >> 5 : 0];
+    uint4 *slot = stage_all[STAGED ? threadIdx.x >> 5 : 0];
     const int64_t nb = p.cols >> 5;
     const int64_t total = p.rows * nb;
     // (row, block) of the flat index b, stepped by the grid stride without a
@@ -1273,27 +1305,72 @@ __global__ void __launch_bounds__(256, RHT ? 3 : (F32 ? 2 : 4)) dequant_row_kern
     // the warp's lanes hold consecutive flat indices: it runs the loop as a
     // whole while any lane has a block
     const int64_t wb0 = b0 - lane;
-    for (int64_t b = b0, wb = wb0; wb < total; b += 2 * stride, wb += 2 * stride) {
+    auto load_block = [&](bool has, int64_t r_, int64_t k_, uint4 &q, uint32_t &sc) {
+        q = has ? ldg_nc_v4(p.codes + r_ * p.ld_codes + (k_ << 4)) : make_uint4(0, 0, 0, 0);
+        sc = has ? dequant_scale<SMODE>(p, r_, k_) : 0u;
+    };
+    if constexpr (RHT != 0 && !F32) {
+        // bf16 with the inverse RHT: both blocks transformed together, then
+        // staged and stored like the blocks without it.  At two CTAs per SM
+        // the next iteration's blocks are loaded before this one's are
+        // processed, so each lane keeps four loads in flight.
         int64_t r1, k1, r2, k2;
         step(r1, k1);
         step(r2, k2);
-        const bool first = b < total, second = b + stride < total;
-        const uint4 q1 = first ? ldg_nc_v4(p.codes + r1 * p.ld_codes + (k1 << 4)) : make_uint4(0, 0, 0, 0);
-        const uint4 q2 = second ? ldg_nc_v4(p.codes + r2 * p.ld_codes + (k2 << 4)) : make_uint4(0, 0, 0, 0);
-        const uint32_t s1 = first ? dequant_scale<SMODE>(p, r1, k1) : 0u;
-        const uint32_t s2 = second ? dequant_scale<SMODE>(p, r2, k2) : 0u;
-        if constexpr (RHT == 0) {
-            if (first) dequant_block_stage<F32>(q1, s1, slot, lane);
-            dequant_warp_store<F32>(slot, first ? out_at(r1, k1) : nullptr, lane);
-            if (wb + stride < total) {
-                if (second) dequant_block_stage<F32>(q2, s2, slot, lane);
-                dequant_warp_store<F32>(slot, second ? out_at(r2, k2) : nullptr, lane);
+        uint4 q1, q2;
+        uint32_t s1, s2;
+        load_block(b0 < total, r1, k1, q1, s1);
+        load_block(b0 + stride < total, r2, k2, q2, s2);
+        for (int64_t b = b0, wb = wb0; wb < total; b += 2 * stride, wb += 2 * stride) {
+            const bool first = b < total, second = b + stride < total;
+            int64_t nr1, nk1, nr2, nk2;
+            step(nr1, nk1);
+            step(nr2, nk2);
+            uint4 nq1, nq2;
+            uint32_t ns1, ns2;
+            load_block(b + 2 * stride < total, nr1, nk1, nq1, ns1);
+            load_block(b + 3 * stride < total, nr2, nk2, nq2, ns2);
+            const bool pair = unscaled_ok(s1) && unscaled_ok(s2);
+            uint32_t w2[16];
+            if (pair) {
+                rht_pair_stage<RHT>(q1, s1, q2, s2, p.sgn_pair, slot, lane, w2);
+            } else {
+                uint32_t w1[16];
+                column_rht_bf16<RHT>(q1, s1, p.sgn_pair, w1);
+                stage_words_bf16(w1, slot, lane);
             }
-        } else {
-            // with the inverse RHT the kernel is bound by its arithmetic: the
-            // staging costs more issue slots than its coalescing gains
-            if (first) dequant_block_store<RHT, F32>(p, r1, k1, q1, s1);
-            if (second) dequant_block_store<RHT, F32>(p, r2, k2, q2, s2);
+            dequant_warp_store<false>(slot, first ? out_at(r1, k1) : nullptr, lane);
+            if (wb + stride < total) {
+                if (!pair) column_rht_bf16<RHT>(q2, s2, p.sgn_pair, w2);
+                stage_words_bf16(w2, slot, lane);
+                dequant_warp_store<false>(slot, second ? out_at(r2, k2) : nullptr, lane);
+            }
+            r1 = nr1; k1 = nk1; r2 = nr2; k2 = nk2;
+            q1 = nq1; q2 = nq2; s1 = ns1; s2 = ns2;
+        }
+    } else {
+        for (int64_t b = b0, wb = wb0; wb < total; b += 2 * stride, wb += 2 * stride) {
+            int64_t r1, k1, r2, k2;
+            step(r1, k1);
+            step(r2, k2);
+            const bool first = b < total, second = b + stride < total;
+            uint4 q1, q2;
+            uint32_t s1, s2;
+            load_block(first, r1, k1, q1, s1);
+            load_block(second, r2, k2, q2, s2);
+            if constexpr (RHT == 0) {
+                if (first) dequant_block_stage<F32>(q1, s1, slot, lane);
+                dequant_warp_store<F32>(slot, first ? out_at(r1, k1) : nullptr, lane);
+                if (wb + stride < total) {
+                    if (second) dequant_block_stage<F32>(q2, s2, slot, lane);
+                    dequant_warp_store<F32>(slot, second ? out_at(r2, k2) : nullptr, lane);
+                }
+            } else {
+                // fp32 with the inverse RHT: bound by its arithmetic, each
+                // lane stores its own blocks
+                if (first) dequant_block_store<RHT, F32>(p, r1, k1, q1, s1);
+                if (second) dequant_block_store<RHT, F32>(p, r2, k2, q2, s2);
+            }
         }
     }
 }
