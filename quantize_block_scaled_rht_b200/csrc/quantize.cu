@@ -822,26 +822,51 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_2d_kernel(const QuantPa
     using T = Q2Tile<TRANS>;
     __shared__ __align__(16) uint16_t tin[2][T::ROWS * T::PITCH];
     __shared__ __align__(16) uint8_t tb[8][16][32];   // per warp: byte j of row r at [j][r]
+    // round-to-nearest without the RHT or the transposed copy: the codes (32 rows
+    // x 8 blocks of 16 bytes, block b of row r at b ^ (r & 7)), stored
+    // row-contiguously during the next tile, after its first barrier
+    constexpr bool STAGE = !TRANS && !SR && RHT == 0;
+    __shared__ __align__(16) uint4 ocodes[STAGE ? 2 : 1][STAGE ? 32 * 8 : 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t nbr = p.rows >> 5, nbc = p.cols >> 5;
+    auto flush = [&](const TileWalk &w, int ob) {
+        if constexpr (STAGE) {
+            const int row = tid >> 3, ch = tid & 7;
+            const int64_t br = w.r, bc = (int64_t)w.c * T::BC + ch;
+            if (br < nbr && bc < nbc)
+                stg_v4(p.codes + ((br << 5) + row) * p.ld_codes + (bc << 4), ocodes[ob][row * 8 + (ch ^ (row & 7))]);
+        }
+    };
     const uint32_t tiles_c = (uint32_t)((nbc + T::BC - 1) / T::BC);
     const uint32_t ntiles = (uint32_t)((nbr + T::BR - 1) / T::BR) * tiles_c;   // the launcher checks it fits
     auto load = [&](const TileWalk &w, int buf) {
+        // thread tid copies 16-byte chunk ch of rows row0 + RSTEP i
+        constexpr int RSTEP = 256 / T::CHUNKS;
+        static_assert(256 % T::CHUNKS == 0 && T::ROWS % RSTEP == 0, "tile copy shape");
+        const int row0 = tid / T::CHUNKS, ch = tid % T::CHUNKS;
         const int64_t r0 = (int64_t)w.r * T::ROWS, c0 = (int64_t)w.c * T::COLS;
+        const uint16_t *src = p.x + (r0 + row0) * p.ld_x + c0 + 8 * ch;
+        uint16_t *dst = tin[buf] + row0 * T::PITCH + 8 * ch;
+        if (r0 + T::ROWS <= p.rows && c0 + T::COLS <= p.cols) {
 #pragma unroll
-        for (int i = 0; i < T::ROWS * T::CHUNKS / 256; ++i) {
-            const int idx = tid + 256 * i, row = idx / T::CHUNKS, ch = idx % T::CHUNKS;
-            const int64_t gr = r0 + row, gc = c0 + 8 * ch;
-            if (gr < p.rows && gc < p.cols) cp_async16(tin[buf] + row * T::PITCH + 8 * ch, p.x + gr * p.ld_x + gc);
+            for (int i = 0; i < T::ROWS / RSTEP; ++i)
+                cp_async16(dst + i * RSTEP * T::PITCH, src + (int64_t)i * RSTEP * p.ld_x);
+        } else if (c0 + 8 * ch < p.cols) {
+#pragma unroll
+            for (int i = 0; i < T::ROWS / RSTEP; ++i)
+                if (r0 + row0 + i * RSTEP < p.rows)
+                    cp_async16(dst + i * RSTEP * T::PITCH, src + (int64_t)i * RSTEP * p.ld_x);
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     const TileStep st(gridDim.x, tiles_c);
-    TileWalk cur(blockIdx.x, tiles_c), nxt = cur;
+    TileWalk cur(blockIdx.x, tiles_c), nxt = cur, prv = cur;
     nxt.next(st);
     if (cur.t < ntiles) load(cur, 0);
+    int last = 0;
     for (int it = 0; cur.t < ntiles; ++it) {
         const int buf = it & 1;
+        last = buf;
         if (nxt.t < ntiles) {
             load(nxt, buf ^ 1);
             asm volatile("cp.async.wait_group 1;" ::: "memory");
@@ -849,6 +874,7 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_2d_kernel(const QuantPa
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
+        if (it > 0) flush(prv, buf ^ 1);                 // the previous tile's codes
         const int wr = warp / T::BC, wc = warp % T::BC;   // this warp's block within the tile
         const int64_t br = (int64_t)cur.r * T::BR + wr;
         const int64_t bc = (int64_t)cur.c * T::BC + wc;
@@ -893,7 +919,8 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_2d_kernel(const QuantPa
                     },
                     packed, g0, p.seed_lo, p.seed_hi, p.scale_rule);
             }
-            stg_v4(p.codes + r * p.ld_codes + (c0 >> 1), packed);
+            if constexpr (STAGE) ocodes[buf][lane * 8 + (wc ^ (lane & 7))] = packed;
+            else stg_v4(p.codes + r * p.ld_codes + (c0 >> 1), packed);
             if constexpr (MMA) {
                 p.scales[mma_scale_off(r, bc, p.katoms)] = (uint8_t)code;
             } else {
@@ -934,9 +961,11 @@ __global__ void __launch_bounds__(256, SR ? 3 : 4) quant_2d_kernel(const QuantPa
             }
         }
         __syncthreads();                     // the load after next overwrites this buffer
+        prv = cur;
         cur = nxt;
         nxt.next(st);
     }
+    if (prv.t < ntiles) flush(prv, last);               // the last tile's codes
 }
 
 // ---------------------------------------------------------------------------
