@@ -1854,10 +1854,18 @@ static cudaError_t launch_dequant_t(int layout, int smode, const DequantParams &
         const unsigned g = (unsigned)(tiles < cap ? tiles : cap);
         return launch_pdl(kern, dim3(g), dim3(256), (size_t)smem, s, p);
     } else {
-        const unsigned g = (unsigned)grid_for(p.rows * (p.cols / 32), 256);
-        if (smode == 0) return launch_pdl(dequant_row_kernel<RHT, F32, 0>, dim3(g), dim3(256), 0, s, p);
-        else if (smode == 1) return launch_pdl(dequant_row_kernel<RHT, F32, 1>, dim3(g), dim3(256), 0, s, p);
-        else return launch_pdl(dequant_row_kernel<RHT, F32, 2>, dim3(g), dim3(256), 0, s, p);
+        auto kern = smode == 0 ? dequant_row_kernel<RHT, F32, 0>
+                               : (smode == 1 ? dequant_row_kernel<RHT, F32, 1> : dequant_row_kernel<RHT, F32, 2>);
+        const int64_t items = p.rows * (p.cols / 32);
+        int64_t g = grid_for(items, 256);
+        if constexpr (RHT != 0 && !F32) {
+            // the software-pipelined loop: one wave of resident CTAs, each
+            // carrying its prefetch across all of its iterations
+            const int64_t cap = (int64_t)num_sms() * resident_ctas(reinterpret_cast<const void *>(kern), 256, 0);
+            const int64_t need = (items + 255) / 256;
+            g = need < cap ? need : cap;
+        }
+        return launch_pdl(kern, dim3((unsigned)(g < 1 ? 1 : g)), dim3(256), 0, s, p);
     }
     return cudaGetLastError();
 }
