@@ -1660,8 +1660,9 @@ static cudaError_t launch_quant_t(int layout, bool trans, const QuantParams &p, 
         if (tiles > 0xFFFFFFFFll - 0x7FFFFFFFll) return cudaErrorInvalidValue;   // tile index fits 32 bits
         auto kern = trans ? quant_2d_kernel<RHT, SR, MMA, true> : quant_2d_kernel<RHT, SR, MMA, false>;
         // persistent for RNE (memory-bound), one CTA per tile for SR (ALU-bound)
-        const int64_t cap = SR ? 0x7FFFFFFFll
-                               : (int64_t)num_sms() * resident_ctas(reinterpret_cast<const void *>(kern), 256);
+        int64_t cap = SR ? 0x7FFFFFFFll
+                         : (int64_t)num_sms() * resident_ctas(reinterpret_cast<const void *>(kern), 256);
+        if (tiles < 4 * cap) cap = tiles;                   // small tensors: one CTA per tile
         return launch_pdl(kern, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(256), 0, s, p);
     }
     return cudaGetLastError();
@@ -1747,8 +1748,9 @@ static cudaError_t launch_dual_t(DualParams p, cudaStream_t s) {
         auto kern = quant_dual_kernel<CRHT, MMA>;
         const cudaError_t ea = allow_dyn_smem(reinterpret_cast<const void *>(kern), DQ_SMEM);
         if (ea != cudaSuccess) return ea;
-        const uint64_t cap =
+        uint64_t cap =
             (uint64_t)num_sms() * (uint64_t)resident_ctas(reinterpret_cast<const void *>(kern), 256, DQ_SMEM);
+        if (tiles < 4 * cap) cap = tiles;                   // small tensors: one CTA per tile
         return launch_pdl(kern, dim3((unsigned)(tiles < cap ? tiles : cap)), dim3(256), (size_t)DQ_SMEM, s, p,
                           (uint32_t)tiles);
     }
