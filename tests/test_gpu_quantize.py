@@ -188,6 +188,50 @@ def test_dequantize_rht_every_scale_code(layout, rht, out_dtype):
         assert np.array_equal(got[~nan], b16[~nan])
 
 
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rht", [16, 32])
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_dequantize_rht_signed_zeros(layout, rht, out_dtype):
+    """Blocks built to make the inverse butterfly produce exact zeros: all
+    codes +-0 (codes 0 and 8), a +-0 first half with +-0.5 after it, and +-0
+    / +-0.5 throughout.  The sign of an exact zero depends on the butterfly's
+    order and pairing, which the dequantizers must follow exactly; every
+    output bit pattern, zero signs included, must equal the oracle's."""
+    rows, cols = {mx.LAYOUT_1D_ROW: (256, 320), mx.LAYOUT_1D_COL: (320, 256), mx.LAYOUT_2D: (512, 512)}[layout]
+    rng = np.random.default_rng(1700 + layout * 10 + rht)
+    if layout == mx.LAYOUT_1D_COL:
+        shape, sshape = (cols, rows // 2), (cols, rows // 32)
+    else:
+        shape = (rows, cols // 2)
+        sshape = (rows // 32, cols // 32) if layout == mx.LAYOUT_2D else (rows, cols // 32)
+    nblk = shape[0] * shape[1] // 16
+    nib = rng.choice(np.array([0, 8], dtype=np.uint8), size=(nblk, 32))     # every element +-0
+    kind = rng.integers(0, 3, size=nblk)
+    small = rng.choice(np.array([0, 1, 8, 9], dtype=np.uint8), size=(nblk, 32))   # +-0, +-0.5
+    nib[kind == 1, 16:] = small[kind == 1, 16:]
+    nib[kind == 2] = small[kind == 2]
+    codes = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8).reshape(shape)
+    # scale codes mostly in the unscaled-domain range, some outside it (no NaN)
+    scales = rng.integers(100, 150, size=sshape).astype(np.uint8)
+    edge = rng.random(sshape) < 0.1
+    scales[edge] = rng.choice(np.array([0, 1, 20, 26, 247, 254], dtype=np.uint8), size=int(edge.sum()))
+    f32, b16 = oracle.dequantize(codes, scales, rows, cols, layout, rht, 11)
+    assert (f32 == 0).mean() > 0.2
+    out = mx.mxfp4_dequantize(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), rows, cols,
+                              layout, rht, 11, out_dtype=out_dtype)
+    got = host(out)
+    # scale code 254 overflows the scaled butterfly (Inf - Inf): NaN payloads
+    # differ between the device and the host, so NaNs compare by position
+    if out_dtype == torch.float32:
+        nan = np.isnan(f32)
+        assert np.array_equal(np.isnan(got), nan)
+        assert np.array_equal(got[~nan].view(np.uint32), f32[~nan].view(np.uint32))
+    else:
+        nan = np.isnan(synth.bf16_to_f32(b16))
+        assert np.array_equal(np.isnan(synth.bf16_to_f32(got)), nan)
+        assert np.array_equal(got[~nan], b16[~nan])
+
+
 def test_dequantize_mma_scales():
     rows, cols = 200, 256
     x = synth.normal_bf16((rows, cols), 4)
