@@ -816,7 +816,7 @@ struct Q2Tile {
 
 
 template <int RHT, bool SR, bool MMA, bool TRANS>
-__global__ void __launch_bounds__(256, SR ? 3 : 4) quant_2d_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(256, SR ? 3 : (RHT != 0 || TRANS ? 5 : 4)) quant_2d_kernel(const QuantParams p) {
     pdl_wait();
     pdl_trigger();
     using T = Q2Tile<TRANS>;
