@@ -232,13 +232,17 @@ def test_dequantize_rht_signed_zeros(layout, rht, out_dtype):
         assert np.array_equal(got[~nan], b16[~nan])
 
 
-def test_dequantize_mma_scales():
+@pytest.mark.parametrize("rht", [0, 16, 32])
+def test_dequantize_mma_scales(rht):
+    """Row dequantize reading GEMM-ready scales, with and without the inverse
+    RHT (the RHT path's pipelined loop is its own instantiation per scale
+    layout)."""
     rows, cols = 200, 256
     x = synth.normal_bf16((rows, cols), 4)
-    q = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_ROW, 0, mx.ROUND_RNE, 0, 0, mx.SCALES_MMA)
-    out = mx.mxfp4_dequantize(q.codes, q.scales, rows, cols, mx.LAYOUT_1D_ROW, scale_layout=mx.SCALES_MMA)
-    codes, scales = oracle.quantize(x, oracle.LAYOUT_1D_ROW)
-    _, b16 = oracle.dequantize(codes, scales, rows, cols, oracle.LAYOUT_1D_ROW)
+    q = mx.mxfp4_quantize(dev_bf16(x), mx.LAYOUT_1D_ROW, rht, mx.ROUND_RNE, 3, 0, mx.SCALES_MMA)
+    out = mx.mxfp4_dequantize(q.codes, q.scales, rows, cols, mx.LAYOUT_1D_ROW, rht, 3, scale_layout=mx.SCALES_MMA)
+    codes, scales = oracle.quantize(x, oracle.LAYOUT_1D_ROW, rht, oracle.ROUND_RNE, 3)[:2]
+    _, b16 = oracle.dequantize(codes, scales, rows, cols, oracle.LAYOUT_1D_ROW, rht, 3)
     assert np.array_equal(host(out), b16)
 
 
