@@ -1406,34 +1406,48 @@ __global__ void __launch_bounds__(256, RHT ? (F32 ? 3 : 2) : (F32 ? 2 : 4)) dequ
 
 // Transposed-view codes [cols, rows/2] back to out[rows, cols].  A tile is
 // 64 code rows (= output columns) x 8 blocks (= 256 output rows): the codes
-// are staged with coalesced 16-byte cp.async loads into a two-tile ring, the
-// next tile's load in flight while this one is decoded (persistent grid).
-// Warp w decodes block w, lane l the output columns 2l and 2l+1, one column at
-// a time (decode, inverse RHT, then 32 values written down the column of a
-// per-warp 32-row shared tile), so only one 32-value block is live in
-// registers.  The warp then writes the tile's rows to global memory with
-// 16-byte stores, 128 (bf16) or 256 (fp32) contiguous bytes per row.  The
-// fp32 tile swaps word pairs of columns 32..63 so that the column writes of
-// lanes l and l + 16 fall in different banks.
+// are staged with coalesced 16-byte cp.async loads into a two-tile ring (three
+// for bf16 with the RHT), the next tiles' loads in flight while this one is
+// decoded (persistent grid).  Warp w decodes block w, lane l the output
+// columns 2l and 2l+1 (bf16: both at once; fp32: one at a time, so that one
+// 32-value block is live) and writes its 32 values per column down a per-warp
+// 32-row shared tile, which the warp then writes to global memory with
+// 16-byte stores, 128 (bf16) or 256 (fp32) contiguous bytes per row.  bf16
+// with the RHT skips the tile: a lane's row word goes straight to its output
+// row, 128 contiguous bytes per warp store.  The fp32 tile swaps word pairs of
+// columns 32..63 so that the column writes of lanes l and l + 16 fall in
+// different banks.
 template <bool F32>
 __host__ __device__ constexpr int dequant_col_row_bytes() { return COL_TC * (F32 ? 4 : 2); }
-template <bool F32>
-__host__ __device__ constexpr int dequant_col_smem() { return (int)sizeof(uint4) * 2 * COL_TC * 8 + 8 * 32 * dequant_col_row_bytes<F32>(); }
+// bf16 output with the inverse RHT stores each row word directly (the
+// transposing tile is only for the other outputs) and spends the shared
+// memory saved on a three-tile code ring.
+template <int RHT, bool F32>
+__host__ __device__ constexpr bool dequant_col_direct() { return RHT != 0 && !F32; }
+template <int RHT, bool F32>
+__host__ __device__ constexpr int dequant_col_stages() { return dequant_col_direct<RHT, F32>() ? 3 : 2; }
+template <int RHT, bool F32>
+__host__ __device__ constexpr int dequant_col_smem() {
+    return (int)sizeof(uint4) * dequant_col_stages<RHT, F32>() * COL_TC * 8 +
+           (dequant_col_direct<RHT, F32>() ? 0 : 8 * 32 * dequant_col_row_bytes<F32>());
+}
 
 template <int RHT, bool F32, bool MMA>
-__global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kernel(const DequantParams p) {
+__global__ void __launch_bounds__(256, (F32 || RHT) ? 2 : 4) dequant_col_kernel(const DequantParams p) {
     pdl_wait();
     pdl_trigger();
     extern __shared__ __align__(16) uint8_t dyn_smem[];
     constexpr int ROWB = dequant_col_row_bytes<F32>();               // staged bytes per output row
     constexpr int CH = ROWB / 16;                                    // 16-byte chunks per row
-    uint4 (*tin)[COL_TC][8] = reinterpret_cast<uint4 (*)[COL_TC][8]>(dyn_smem);   // 2 x 8 KB of codes
+    constexpr bool DIRECT = dequant_col_direct<RHT, F32>();
+    constexpr int NST = dequant_col_stages<RHT, F32>();
+    uint4 (*tin)[COL_TC][8] = reinterpret_cast<uint4 (*)[COL_TC][8]>(dyn_smem);   // NST x 8 KB of codes
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     // chunk ch of staged code row `row` sits at ch ^ ((row >> 1) & 7): the
     // lanes of a warp read block `warp` of rows 2l, 2l + 1 (256 bytes apart),
     // which this spreads over all banks
     const int wsw = warp ^ (lane & 7);
-    uint8_t *stage = dyn_smem + sizeof(uint4) * 2 * COL_TC * 8 + warp * 32 * ROWB;
+    uint8_t *stage = dyn_smem + sizeof(uint4) * NST * COL_TC * 8 + warp * 32 * ROWB;   // unless DIRECT
     const uint32_t tiles_r = (uint32_t)((p.rows + COL_TR - 1) / COL_TR);
     const uint32_t tiles_c = (uint32_t)((p.cols + COL_TC - 1) / COL_TC);
     const uint32_t ntiles = tiles_r * tiles_c;                         // the launcher checks it fits
@@ -1462,20 +1476,28 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
         }
     };
     const TileStep st(gridDim.x, tiles_c);
-    TileWalk cur(blockIdx.x, tiles_c);
+    TileWalk cur(blockIdx.x, tiles_c), w1 = cur, w2 = cur;           // this tile, the next two
+    w1.next(st);
     if (cur.t < ntiles) load(cur, 0);
+    if constexpr (NST == 3) {
+        w2 = w1;
+        w2.next(st);
+        load(w1, 1);                                                  // tiles past the end load nothing
+    }
     uint32_t sa = 0xFFu, sb = 0xFFu;
     if constexpr (!F32) scale_pair(cur, sa, sb);
     for (int it = 0; cur.t < ntiles; ++it) {
-        // the buffer refilled here was read in the previous iteration, which
-        // ended with a barrier
-        const int buf = it & 1;
-        TileWalk nxt = cur;
-        nxt.next(st);
+        // NST - 1 tiles in flight while this one is decoded; the buffer
+        // refilled here was read in an earlier iteration, before a barrier
+        // every warp has passed
+        const int buf = it % NST;
         uint32_t sa_n = 0xFFu, sb_n = 0xFFu;
-        if constexpr (!F32) scale_pair(nxt, sa_n, sb_n);
-        if (nxt.t < ntiles) {
-            load(nxt, buf ^ 1);
+        if constexpr (!F32) scale_pair(w1, sa_n, sb_n);
+        if constexpr (NST == 3) {
+            load(w2, (it + 2) % 3);
+            asm volatile("cp.async.wait_group 2;" ::: "memory");
+        } else if (w1.t < ntiles) {
+            load(w1, buf ^ 1);
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -1486,11 +1508,14 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
         if (rb < p.rows) {
           const int64_t kb = rb >> 5;
           if constexpr (!F32) {
-            // bf16 out: one 32-bit word (columns 2l, 2l + 1) per row of the
-            // staged tile
+            // bf16 out: one 32-bit word (columns 2l, 2l + 1) per row, into
+            // the staged tile, or with the RHT straight to the output row
+            // (a warp's store then covers 128 contiguous bytes)
             const int64_t oc = c0 + 2 * lane;
             if (oc < p.cols) {                 // cols is even: oc + 1 < cols too
-                uint32_t *w = reinterpret_cast<uint32_t *>(stage) + lane;
+                uint32_t *w = DIRECT ? reinterpret_cast<uint32_t *>(static_cast<uint16_t *>(p.out) + rb * p.ld_out + oc)
+                                     : reinterpret_cast<uint32_t *>(stage) + lane;
+                const int64_t RW = DIRECT ? p.ld_out / 2 : ROWB / 4;   // 32-bit words between rows
                 if constexpr (RHT == 0) {
                     // each column as 16 looked-up bf16 pairs along its rows
                     uint32_t pa[16], pb[16];
@@ -1498,8 +1523,8 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                     decode32_bf16(tin[buf][2 * lane + 1][wsw], sb, pb);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        w[(2 * i) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x5410u);
-                        w[(2 * i + 1) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x7632u);
+                        w[(2 * i) * RW] = prmt(pa[i], pb[i], 0x5410u);
+                        w[(2 * i + 1) * RW] = prmt(pa[i], pb[i], 0x7632u);
                     }
                 } else if (unscaled_ok(sa) && unscaled_ok(sb)) {
                     // both columns at once in the unscaled domain: row i of
@@ -1511,7 +1536,7 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const float2 f = mul2(f16x2_to_f32(P[i]), K2);
-                        w[i * (ROWB / 4)] = pack_bf16x2(f.x, f.y) ^ p.sgn_word[i];
+                        w[i * RW] = pack_bf16x2(f.x, f.y) ^ p.sgn_word[i];
                     }
                 } else {
                     // each column decoded, transformed, rounded and
@@ -1521,8 +1546,8 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                     column_rht_bf16<RHT>(tin[buf][2 * lane + 1][wsw], sb, p.sgn_pair, pb);
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        w[(2 * i) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x5410u);
-                        w[(2 * i + 1) * (ROWB / 4)] = prmt(pa[i], pb[i], 0x7632u);
+                        w[(2 * i) * RW] = prmt(pa[i], pb[i], 0x5410u);
+                        w[(2 * i + 1) * RW] = prmt(pa[i], pb[i], 0x7632u);
                     }
                 }
             }
@@ -1549,6 +1574,7 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                 }
             }
           }
+          if constexpr (!DIRECT) {
             __syncwarp();
             // 32 rows of ROWB bytes: lane-contiguous 16-byte chunks of each row
 #pragma unroll
@@ -1565,12 +1591,20 @@ __global__ void __launch_bounds__(256, F32 ? 2 : (RHT ? 3 : 4)) dequant_col_kern
                 }
             }
             __syncwarp();
+          }
         }
         __syncthreads();
         sa = sa_n;
         sb = sb_n;
-        cur.next(st);
+        cur = w1;
+        if constexpr (NST == 3) {
+            w1 = w2;
+            w2.next(st);
+        } else {
+            w1.next(st);
+        }
     }
+    if constexpr (NST == 3) asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -1849,7 +1883,7 @@ static cudaError_t launch_dequant_t(int layout, int smode, const DequantParams &
         const int64_t tiles = ((p.rows + COL_TR - 1) / COL_TR) * ((p.cols + COL_TC - 1) / COL_TC);
         if (tiles > 0xFFFFFFFFll - 0x7FFFFFFFll) return cudaErrorInvalidValue;   // tile index fits 32 bits
         auto kern = smode == 2 ? dequant_col_kernel<RHT, F32, true> : dequant_col_kernel<RHT, F32, false>;
-        constexpr int smem = dequant_col_smem<F32>();
+        constexpr int smem = dequant_col_smem<RHT, F32>();
         const cudaError_t ea = allow_dyn_smem(reinterpret_cast<const void *>(kern), smem);
         if (ea != cudaSuccess) return ea;
         const int64_t cap = (int64_t)num_sms() * resident_ctas(reinterpret_cast<const void *>(kern), 256, smem);
