@@ -887,14 +887,14 @@ __global__ void __launch_bounds__(256, SR ? 3 : (RHT != 0 || TRANS ? 5 : 4)) qua
                 const uint4 u = s4[q];
                 w[4 * q] = u.x; w[4 * q + 1] = u.y; w[4 * q + 2] = u.z; w[4 * q + 3] = u.w;
             }
-            // the block's amax is the warp max of the lanes' row maxima
+            // the block's amax is the warp max of the lanes' row maxima.  A
+            // lane's maximum is +0, positive or the canonical NaN 0x7FFFFFFF,
+            // so the unsigned maximum of the bit patterns is the NaN-
+            // propagating float maximum, bit for bit, in one reduction
             auto warp_amax = [](float amax) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    const float other = __shfl_xor_sync(0xFFFFFFFFu, amax, o);
-                    asm("max.NaN.f32 %0, %0, %1;" : "+f"(amax) : "f"(other));
-                }
-                return amax;
+                uint32_t r;
+                asm("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(__float_as_uint(amax)));
+                return __uint_as_float(r);
             };
             uint4 packed;
             uint32_t code;
