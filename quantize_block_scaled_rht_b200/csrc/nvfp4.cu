@@ -121,8 +121,35 @@ __device__ __forceinline__ uint32_t nv_block(float *v, const NvTensor &t, uint64
 #pragma unroll
         for (int i = 0; i < 16; ++i) v[i] = copysignf(0.0f, v[i]);
     } else {
+        // The quotients v / X rounded to nearest even.  With y = RN(1/X),
+        // q = RN(|v| y) is within one ulp of |v| / X, the residual |v| - q X
+        // is exact by FMA, and RN(q + (|v| - q X) y) is the correctly rounded
+        // quotient (Markstein's FMA division, "Computation of elementary
+        // functions on the IBM RISC System/6000 processor", 1990); the sign
+        // goes back on exactly.  The residual must not underflow and the
+        // reciprocal must be normal, so the block takes this path only when
+        // X lies in [2^-100, 2^100] and every nonzero |v| is at least 2^-100
+        // (the quotients are below 16 here); otherwise each element is
+        // divided with the IEEE division.
+        bool tiny = !(X >= 0x1p-100f && X <= 0x1p100f);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(v[i], X);
+        for (int i = 0; i < 16; ++i) {
+            const float a = fabsf(v[i]);
+            tiny |= a != 0.0f && a < 0x1p-100f;
+        }
+        if (!tiny) {
+            const float y = __frcp_rn(X);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float a = fabsf(v[i]);
+                const float q = __fmul_rn(a, y);
+                const float r = __fmaf_rn(-q, X, a);
+                v[i] = copysignf(__fmaf_rn(r, y, q), v[i]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[i] = __fdiv_rn(v[i], X);
+        }
     }
     if constexpr (!SR) {
         out = make_uint2(e2m1x8_rn(v), e2m1x8_rn(v + 8));
