@@ -182,14 +182,28 @@ __global__ void __launch_bounds__(256) nv_quant_row_kernel(const NvParams p) {
     const int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t dr = stride / nb, dk = stride - dr * nb;
     int64_t rr = i0 / nb, kk = i0 - rr * nb;
+    // the next step's 32 bytes are loaded before this step's block is
+    // quantized, so each thread keeps a load in flight through its compute
+    uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
+    if (i0 < n) {
+        const uint16_t *src = p.x + rr * p.ld_x + 16 * kk;
+        u0 = nv_ldg_v4(src);
+        u1 = nv_ldg_v4(src + 8);
+    }
     for (int64_t i = i0; i < n; i += stride) {
         const int64_t r = rr, kb = kk;
         rr += dr;
         kk += dk;
         if (kk >= nb) { kk -= nb; ++rr; }
-        const uint16_t *src = p.x + r * p.ld_x + 16 * kb;
-        const uint4 u0 = nv_ldg_v4(src), u1 = nv_ldg_v4(src + 8);
+        uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+        if (i + stride < n) {
+            const uint16_t *src = p.x + rr * p.ld_x + 16 * kk;
+            n0 = nv_ldg_v4(src);
+            n1 = nv_ldg_v4(src + 8);
+        }
         const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+        u0 = n0;
+        u1 = n1;
         float v[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) { v[2 * j] = bf16lo(w[j]); v[2 * j + 1] = bf16hi(w[j]); }
