@@ -421,6 +421,29 @@ def test_nvfp4_every_bf16_pattern_and_specials():
     assert float(z.amax.item()) == 0.0 and not host(z.codes).any() and not host(z.scales).any()
 
 
+@pytest.mark.parametrize("k", [-120, -106, -100, -94, 0, 94, 100, 106, 112])
+def test_nvfp4_division_at_extreme_scales(k):
+    """The element division by the block's X takes an FMA-corrected
+    reciprocal when X lies in [2^-100, 2^100] and every nonzero element is at
+    least 2^-100, the IEEE division otherwise.  Tensors scaled by 2^k put
+    their blocks on both sides of those limits (k = -106 and below: tiny
+    elements and divisors; 94 and above: divisors near the top), with a spread
+    of block magnitudes and exact zeros; codes and scales must match the
+    oracle bit for bit under RNE and SR, in both layouts."""
+    rows, cols = 64, 256
+    base = synth.student_t_bf16((rows, cols), seed=700 + k)
+    f = synth.bf16_to_f32(base).astype(np.float64)
+    f *= np.exp2(np.random.default_rng(701).integers(-6, 7, size=(rows, 1)).astype(np.float64))   # row spread
+    f[3, :40] = 0.0
+    x = synth.bf16_bits((f * 2.0 ** k).astype(np.float32))
+    for layout in (mx.LAYOUT_1D_ROW, mx.LAYOUT_1D_COL):
+        for rnd in (mx.ROUND_RNE, mx.ROUND_SR):
+            q = mx.mxfp4_nvfp4_quantize(dev_bf16(x), layout, rnd, 13)
+            codes, scales, _ = oracle.nvfp4_quantize(x, layout, rnd, 13)
+            assert np.array_equal(host(q.codes), codes), (layout, rnd)
+            assert np.array_equal(host(q.scales), scales), (layout, rnd)
+
+
 @pytest.mark.parametrize("layout", [mx.LAYOUT_1D_ROW, mx.LAYOUT_1D_COL])
 def test_nvfp4_dequantize_matches_oracle(layout):
     rows, cols = 96, 160
